@@ -1,0 +1,457 @@
+"""Benchmark of the CSA2 decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stack20]
+    python bench.py --impl reference ...      # the CPU oracle, same metric
+
+A step is one decode step of the workload through the C-ABI: FP4 append of
+the new token of every sequence, then every layer of the static mode schedule
+(Full / Reindex indexer where scheduled, Reuse otherwise) followed by sparse +
+window attention. Default workload: the 20-layer decoder stack, 8 sequences
+x 1 query, 65536 FP4 entries each (Full at 0 and 10, Reindex at 5 and 15,
+Reuse elsewhere, Top-K 2048, 64 heads, window 512).
+
+Metric: decode query-steps per second per layer = batch * queries * layers /
+step time, with the achieved HBM bandwidth of the step's algorithmic bytes.
+Timing: the step is captured once in a CUDA graph; each of the K timed steps
+is preceded by a 256 MiB L2 flush and bracketed by CUDA events on the
+launching stream; a barrier and a device synchronize bracket the whole timed
+loop; the reported time is the max over ranks. Multi-GPU runs give every rank
+its own independent batch of sequences (weak scaling, no collective on the
+data path).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode query-steps/s per layer; achieved HBM TB/s vs ~8 TB/s peak"
+UNIT = "query-steps/s/layer"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="stack20")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method must move / compute)
+# ---------------------------------------------------------------------------
+def algorithmic(recipe, lens, schedule):
+    """(bytes, flops) of one step, and (bytes, flops) of one attention launch."""
+    nq, h, d = recipe.nq, recipe.h, 512
+    n_vis = [int(l) for l in lens.tolist()]
+    by = fl = 0.0
+    rows_app = recipe.append if recipe.chunked else recipe.batch
+    by += rows_app * (d * 2 + d // 2 + d // 16)
+    attn_by = attn_fl = 0.0
+    for mode, src in schedule:
+        if mode == "full":
+            for qi in range(nq):
+                n = n_vis[qi // recipe.q_per_seq]
+                by += n * recipe.di
+                fl += 2.0 * recipe.hi * recipe.di * n
+        elif mode == "reindex":
+            by += nq * recipe.p * (recipe.di + 4)
+            fl += 2.0 * nq * recipe.hi * recipe.di * recipe.p
+        rows = recipe.k + recipe.w
+        a_by = nq * (recipe.k * (d // 2 + d // 16 + 4) + recipe.w * d + 2 * 2 * h * d)
+        a_fl = 4.0 * nq * h * rows * d
+        by += a_by
+        fl += a_fl
+        attn_by, attn_fl = a_by, a_fl
+    return by, fl, attn_by, attn_fl
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("hbm_gbs", 6650.0), j.get("bf16_tflops", 1590.0), j.get("bf16_tflops_sustained", 1400.0), \
+            "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(os.path.join(ROOT, "sparse_fp4_kv_b200", "csrc"))):
+        with open(os.path.join(ROOT, "sparse_fp4_kv_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary, if it was
+    taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(f"{kernel}:{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler
+# ---------------------------------------------------------------------------
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(recipe, layers, seq=0):
+    """Time the oracle's step for one sequence over `layers` (cache build and
+    input generation excluded). Returns (seconds, query-layers processed)."""
+    import numpy as np
+    import torch
+    import oracle
+    import oracle.stack as ostack
+    sched = ostack.schedule(recipe.modes)
+    cache = ostack.SeqCache(recipe, seq)
+    qis = [seq * recipe.q_per_seq + j for j in range(recipe.q_per_seq)]
+    inputs = {}
+    for l in layers:
+        inputs[l] = (recipe.qidx(l).numpy(), recipe.weights(l).numpy(), recipe.q(l, rows=qis),
+                     recipe.swa(l, seqs=[seq])[0].numpy())
+    wb, we = recipe.swa_window()
+    ql = recipe.q_limit()
+    scale = 1.0 / math.sqrt(512.0)
+    topk, pool = {}, {}
+    t0 = time.perf_counter()
+    for l in layers:
+        mode, src = sched[l]
+        qidx, w, q, swa = inputs[l]
+        for j, qi in enumerate(qis):
+            if mode == "full":
+                lim = int(ql[qi]) if ql is not None else cache.n
+                topk[(l, qi)], pool[(l, qi)] = oracle.index_full(qidx[qi], w[qi], cache.kidx, cache.page_table,
+                                                                 cache.page_size, lim, recipe.k, recipe.p)
+            elif mode == "reindex":
+                topk[(l, qi)] = oracle.index_reindex(qidx[qi], w[qi], cache.kidx, cache.page_table, cache.page_size,
+                                                     pool[(src, qi)], recipe.k)
+            else:
+                topk[(l, qi)] = topk[(src, qi)]
+            oracle.sparse_attn(ostack.bf16_bits(q[j]), cache.codes, cache.scales, cache.page_table, cache.page_size,
+                               topk[(l, qi)], swa[int(wb[qi]):int(we[qi])], scale)
+    return time.perf_counter() - t0, len(qis) * len(layers)
+
+
+def reference_layers(recipe):
+    """Layers of the bounded oracle sample: from layer 0 up to the first
+    Reindex layer (so every mode is exercised), capped at 6."""
+    modes = recipe.modes
+    end = modes.find("R")
+    end = len(modes) if end < 0 else end + 1
+    return list(range(min(end, 6)))
+
+
+def run_reference(args):
+    from sparse_fp4_kv_b200.workloads import RECIPES
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    recipe = RECIPES[args.workload]
+    layers = reference_layers(recipe)
+    times = []
+    n_units = 0
+    for i in range(args.warmup + args.steps):
+        dt, n_units = oracle_sample(recipe, layers)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n_units * len(times) / total
+    sample = (f"sequence 0 of {recipe.name}, layers {layers[0]}..{layers[-1]} "
+              f"({''.join(recipe.modes[l] for l in layers)}), {recipe.q_per_seq} quer"
+              f"{'y' if recipe.q_per_seq == 1 else 'ies'}, single-threaded C oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": recipe.name, "sample_layers": layers},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from cuda.bindings import driver as cu
+
+    from sparse_fp4_kv_b200 import build
+    build.build()
+    from sparse_fp4_kv_b200 import binding as B
+    from sparse_fp4_kv_b200.stack import Csa2Decoder
+    from sparse_fp4_kv_b200.workloads import RECIPES
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    base = RECIPES[args.workload]
+    recipe = base.scaled(seed=base.seed + 1000 * rank) if world > 1 else base
+    dec = Csa2Decoder(recipe, dev)
+    by, fl, attn_by, attn_fl = algorithmic(recipe, dec.lens, dec.schedule)
+
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # external timing events around every attention launch inside the graph
+    def new_event():
+        err, ev = cu.cuEventCreate(cu.CUevent_flags.CU_EVENT_DEFAULT)
+        assert err == cu.CUresult.CUDA_SUCCESS
+        return ev
+
+    attn_layers = list(range(recipe.layers))
+    ev_pairs = [(new_event(), new_event()) for _ in attn_layers]
+    ext = cu.CUevent_record_flags.CU_EVENT_RECORD_EXTERNAL
+
+    def step_with_events(s):
+        dec.append(s)
+        h = cu.CUstream(s.cuda_stream)
+        for i, l in enumerate(attn_layers):
+            mode, src = dec.schedule[l]
+            # the indexer call of the layer, then the timed attention launch
+            r = dec.r
+            if mode == "full":
+                B.csa2_index_full(dec.qidx[l], dec.w[l], r.q_per_seq, dec.q_limit, dec.n_max, dec.kv, r.k,
+                                  r.p if dec.pool[l] is not None else 0, dec.topk[l], dec.pool[l], dec.ws_full, s)
+            elif mode == "reindex":
+                B.csa2_index_reindex(dec.qidx[l], dec.w[l], r.q_per_seq, dec.pool[src], dec.kv, r.k, dec.topk[l],
+                                     dec.ws_reindex, s)
+            cu.cuEventRecordWithFlags(ev_pairs[i][0], h, ext)
+            B.csa2_sparse_attn_decode(dec.q[l], r.q_per_seq, dec.kv, dec.topk_of(l), dec.swa[l], dec.swa[l].shape[1],
+                                      dec.swa_begin, dec.swa_end, r.w, dec.scale, dec.o[l], dec.lse[l], dec.ws_attn,
+                                      s)
+            cu.cuEventRecordWithFlags(ev_pairs[i][1], h, ext)
+
+    # eager warm-up (first calls set kernel attributes), then capture
+    with torch.cuda.stream(stream):
+        step_with_events(stream)
+    stream.synchronize()
+    if B.csa2_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step_with_events(stream)
+    stream.synchronize()
+
+    def timed_steps(g, n, record):
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        per_step, attn = [], []
+        for i in range(n):
+            with torch.cuda.stream(stream):
+                flush.fill_(i & 0xFF)
+                st[i].record(stream)
+                g.replay()
+                en[i].record(stream)
+            en[i].synchronize()
+            per_step.append(st[i].elapsed_time(en[i]))
+            if record:
+                for a, b in ev_pairs:
+                    err, ms = cu.cuEventElapsedTime(a, b)
+                    attn.append(ms)
+        return per_step, attn
+
+    launches_per_step = count_launches(dec, recipe)
+    for _ in range(args.warmup):
+        timed_steps(graph, 1, False)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    per_step, attn = timed_steps(graph, args.steps, True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    if B.csa2_device_status(stream) != 0:
+        raise RuntimeError("device error during the timed steps")
+    total_ms = sum(per_step)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    units = recipe.nq * recipe.layers * world
+    value = units / (ms * 1e-3)
+
+    # e2e: host buffers in pinned memory, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, dec, stream, flush, graph_fn=step_with_events, world=world, dev=dev)
+
+    hbm_gbs, bf16_burst, bf16_sust, peak_kind = peaks()
+    attn_ms = statistics.mean(attn) if attn else float("nan")
+    achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
+    kernel = f"k_sparse_attn<{recipe.h}>"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16+e4m3 tensor-core, f32 accumulate", "data": "synthetic",
+        "config": {"workload": recipe.name, "batch": recipe.batch, "queries_per_seq": recipe.q_per_seq,
+                   "layers": recipe.layers, "modes": recipe.modes, "entries": int(dec.n_max),
+                   "topk": recipe.k, "pool": recipe.p, "heads": recipe.h, "window": recipe.w,
+                   "indexer": f"{recipe.hi}x{recipe.di}", "l2": "256 MiB flush before every timed step",
+                   "graph": "one CUDA graph per step", "parallelism": f"dp{world} (independent sequences)"},
+        "hbm_tbs": by / (ms * 1e-3) / 1e12,
+        "algorithmic_bytes_per_step": by, "algorithmic_flops_per_step": fl,
+        "roofline": {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": bf16_sust,
+                     "unit": "TFLOP/s", "frac": achieved_tf / bf16_sust,
+                     "peak_source": f"{peak_kind} bf16 dense sustained (f16 runs at the bf16 rate)",
+                     "launch_us": attn_ms * 1e3, "flops_per_launch": attn_fl, "bytes_per_launch": attn_by,
+                     "hbm_frac": attn_by / (attn_ms * 1e-3) / (hbm_gbs * 1e9),
+                     "traffic": recorded_traffic(kernel, recipe.name)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        layers = list(range(recipe.layers))
+        dt, n = oracle_sample(recipe, layers)
+        line["cpu_baseline"] = {
+            "value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"sequence 0, layers {layers[0]}..{layers[-1]} of {recipe.name}, single-threaded C oracle "
+                      f"({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def count_launches(dec, recipe):
+    """Kernels of this library launched by one step (the memset of the Full
+    layer's histograms is a runtime call, not counted)."""
+    from sparse_fp4_kv_b200 import binding as B
+    n = 1  # append
+    for mode, _ in dec.schedule:
+        if mode == "full":
+            n += 5
+        elif mode == "reindex":
+            n += 2
+        n += 1 + (1 if B.csa2_sparse_attn_workspace_size(recipe.nq, recipe.h, recipe.k, recipe.w) > 0 else 0)
+    return n
+
+
+def run_e2e(args, dec, stream, flush, graph_fn, world, dev):
+    """Same metric through the C-ABI with host buffers: every step copies its
+    inputs (new latent rows, per-layer queries, indexer queries and weights)
+    from pinned host memory to the device and reads every layer's output back."""
+    import torch
+    r = dec.r
+    ins = [dec.x_new] + dec.q + dec.qidx + dec.w
+    host_in = [t.cpu().pin_memory() for t in ins]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in dec.o]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for d_t, h_t in zip(ins, host_in):
+            d_t.copy_(h_t, non_blocking=True)
+        graph_fn(stream)
+        for h_t, o in zip(host_out, dec.o):
+            h_t.copy_(o, non_blocking=True)
+    stream.synchronize()
+    times = []
+    for i in range(args.warmup + args.steps):
+        st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            flush.fill_(i & 0xFF)
+            st.record(stream)
+            g.replay()
+            en.record(stream)
+        en.synchronize()
+        if i >= args.warmup:
+            times.append(st.elapsed_time(en))
+    total = sum(times)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    ms = total / len(times)
+    del g
+    return {"value": r.nq * r.layers * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

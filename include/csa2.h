@@ -1,0 +1,197 @@
+/*
+ * csa2.h -- C ABI of libcsa2.so, the B200 (sm_100a) CSA2 sparse FP4-KV
+ * decode path.
+ *
+ * What the path computes (web pages on DeepSeek V4.1-Flash; they give no
+ * formulas, the readings taken are stated per call):
+ *   [P3] "DeepSeek V4.1-Flash Cuts KV Cache by 437x With New CED and CSA2
+ *        Architecture" (ainewsfeed.tech): paragraphs "CSA2 tackles storage"
+ *        (one global KV shared by all layers, cross-layer Top-K reuse),
+ *        "CSA2 assigns each layer one of three static operating modes"
+ *        (Full / Reindex / Reuse, hierarchical indexer pool) and
+ *        "V4.1-Flash also uses FP4 quantization" (FP4 global KV, FP8 SWA KV,
+ *        values restored at runtime for computation).
+ *   [P4] "DeepSeek V4.1 Flash Architecture Breakdown: KV Cache Compressed to
+ *        1/437 of First Generation" (nashnova.com): sections "How does the
+ *        cache compress along three dimensions at once?" (three modes, pool
+ *        built by the first Full layer) and "How are cache precision and
+ *        storage arranged?" (FP4 E2M1 main KV, FP8 sliding-window KV).
+ *
+ * Conventions for every call:
+ *   - Every pointer argument except the descriptor structs themselves is a
+ *     DEVICE pointer owned by the caller. The library allocates and frees
+ *     nothing, never synchronises, and enqueues all work on `stream`.
+ *   - Arguments are checked on the host before any launch; a failed check
+ *     returns CSA2_ERR_INVALID_ARG / CSA2_ERR_UNSUPPORTED /
+ *     CSA2_ERR_WORKSPACE and launches nothing. A launch failure returns
+ *     CSA2_ERR_CUDA. Conditions only the device can see (an id or page
+ *     outside the cache, a timed-out wait) skip the offending access and set
+ *     a sticky device error word, read and cleared by csa2_device_status().
+ *   - Layouts are dense row-major. Device pointers must be 16-byte aligned.
+ *   - Entry ids are logical positions within a sequence; -1 marks an empty
+ *     slot in every id list.
+ *   - Reuse mode is not a call: a Reuse layer passes its source layer's
+ *     Top-k list to csa2_sparse_attn_decode.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment      */
+    CSA2_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d != 512) */
+    CSA2_ERR_WORKSPACE = 3,    /* workspace missing or too small            */
+    CSA2_ERR_CUDA = 4,         /* a CUDA call or kernel launch failed       */
+    CSA2_ERR_DEVICE = 5        /* the device error word was set            */
+} csa2_status;
+
+/* Latent width of the global KV (the pages leave it open; this library
+ * fixes it at 512) and the FP4 scale block (one E4M3 scale per 16 values). */
+#define CSA2_D 512
+#define CSA2_BLOCK 16
+
+/*
+ * The global KV cache shared by all layers ([P3] "CSA2 tackles storage").
+ * One physical row per entry:
+ *   codes  [rows_cap][d/2]  FP4 E2M1, two per byte, element 2i in the low
+ *                           nibble of byte i                    (256 B/row)
+ *   scales [rows_cap][d/16] E4M3 scale of each block of 16 values (32 B/row)
+ *   kidx   [rows_cap][di]   E4M3 indexer key, one per entry, shared by all
+ *                           indexer heads                    (di = 64 or 128)
+ * Logical entry t of sequence b lives in physical row
+ *   page_table[b * max_pages + t / page_size] * page_size + t % page_size.
+ * A contiguous per-sequence cache is the case max_pages = 1, page_size =
+ * per-sequence capacity, page_table[b] = b. page_size must be a multiple of
+ * 32, and of 128 when it exceeds 128. seq_len[b] is the number of valid
+ * entries of sequence b (device array).
+ */
+typedef struct {
+    uint8_t *codes;
+    uint8_t *scales;
+    const uint8_t *kidx;
+    const int32_t *page_table;
+    const int32_t *seq_len;
+    int64_t rows_cap;
+    int32_t d;
+    int32_t di;
+    int32_t page_size;
+    int32_t max_pages;
+    int32_t batch;
+    int32_t reserved;
+} csa2_kv_desc;
+
+/*
+ * FP4 quantise + append ([P3] "V4.1-Flash also uses FP4 quantization";
+ * [P4] "How are cache precision and storage arranged?": E2M1 main KV).
+ * x_bf16 [n][d] bf16 rows. Row i is stored at logical position pos[i] of
+ * sequence seq[i] (device arrays). For each block of 16 values:
+ *   amax = max|x|;  s = E4M3_RNE_satfinite(amax / 6)   (binary32 division)
+ *   c_i  = 0 if value(s) == 0 else E2M1_RNE_satfinite(x_i / value(s))
+ * Rounding is to nearest with ties to the even mantissa; a NaN element gives
+ * a signed zero code and does not enter amax. Rows whose (seq, pos) falls
+ * outside the page table or the cache are skipped and set the device error
+ * word. seq_len is not updated (the caller owns it).
+ */
+csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq,
+                            const int64_t *pos, const csa2_kv_desc *kv,
+                            cudaStream_t stream);
+
+/*
+ * Full-mode indexer ([P3] modes paragraph: Full "reads the entire context,
+ * generates complete KV and index data, and selects Top-K"; [P4]: the first
+ * Full layer builds the candidate pool of the hierarchical indexer).
+ * nq queries; query i belongs to sequence i / q_per_seq.
+ *   qidx [nq][hi][di] E4M3, w [nq][hi] f32.
+ *   q_limit [nq]: number of entries query i may see (entries 0..q_limit-1);
+ *   NULL means seq_len of its sequence. n_max >= every such limit.
+ * Score of entry t (reading of the pages, which give no formula):
+ *   score(t) = sum_h w_h * max(0, <q_h, kidx_t>)    (f32, tensor cores)
+ * topk [nq][k]: the k best visible entries under (score desc, id asc);
+ * pool [nq][p] (optional, p = 0 and pool = NULL to skip): the p best, the
+ * candidate pool a Reindex layer re-scores. Both lists are in ascending id
+ * order and padded with -1 when fewer entries are visible; topk is a subset
+ * of pool. Scores are exact (hence the ids bit-exact) whenever every
+ * partial sum is an integer below 2^24, as with small-integer E4M3 data.
+ * Requires 1 <= hi <= 16, di in {64, 128}, 1 <= k, 0 <= p, k <= p if p > 0.
+ * ws: at least csa2_index_full_workspace_size(nq, n_max) bytes.
+ */
+csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq,
+                            int32_t q_per_seq, int32_t hi, const int32_t *q_limit,
+                            int64_t n_max, const csa2_kv_desc *kv, int32_t k, int32_t p,
+                            int32_t *topk, int32_t *pool, void *ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+size_t csa2_index_full_workspace_size(int32_t nq, int64_t n_max);
+
+/*
+ * Reindex-mode indexer ([P3]: Reindex "takes the complete KV cache from
+ * Full mode and re-filters important items"; [P4]: "re-scores to pick new
+ * Top-K", later layers "search only within that pool").
+ * pool [nq][p]: ids from a Full layer (-1 entries are padding; any order;
+ * no duplicates). Scores the pool ids with this layer's qidx/w as in
+ * csa2_index_full and writes their Top-k under (score desc, id asc) to
+ * topk [nq][k], in pool order, padded with -1. p <= 16384.
+ * ws: at least csa2_index_reindex_workspace_size(nq, p) bytes.
+ */
+csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq,
+                               int32_t q_per_seq, int32_t hi, const int32_t *pool, int32_t p,
+                               const csa2_kv_desc *kv, int32_t k, int32_t *topk, void *ws,
+                               size_t ws_bytes, cudaStream_t stream);
+
+size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p);
+
+/*
+ * Sparse + sliding-window decode attention ([P3] modes and FP4 paragraphs:
+ * attention over the selected global entries, FP4 values restored for
+ * computation; SWA KV kept at FP8).
+ *   q_bf16 [nq][h][d] bf16, query i of sequence i / q_per_seq.
+ *   topk [nq][k]: global entry ids (-1 = empty); each row is dequantised
+ *   (E2M1 code x E4M3 scale, exact in f16) and used as key and value.
+ *   Window rows of query i: rows swa_begin[i] .. swa_end[i]-1 of the E4M3
+ *   buffer swa + (i / q_per_seq) * swa_seq_stride * d (raw E4M3, no scale),
+ *   also key and value; w_max >= every swa_end[i] - swa_begin[i].
+ * Per head, over the union S of selected rows and window rows:
+ *   o_h = sum_j softmax_j(softmax_scale * <q_h, v_j>) v_j
+ * written as bf16 o [nq][h][d]; lse [nq][h] (nullable) gets the natural-log
+ * sum of exp of the scaled scores. An empty S gives o = 0, lse = -inf.
+ * Arithmetic: q converted to f16 (|q| must be finite in f16), f16 tensor-core
+ * products with f32 accumulation, f32 online softmax, probabilities rounded
+ * to f16 for the P*V product. h in {16, 32, 64}.
+ * ws: at least csa2_sparse_attn_workspace_size(nq, h, k, w_max) bytes.
+ */
+csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_per_seq,
+                                    int32_t h, const csa2_kv_desc *kv, const int32_t *topk,
+                                    int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
+                                    const int32_t *swa_begin, const int32_t *swa_end,
+                                    int32_t w_max, float softmax_scale, void *o_bf16, float *lse,
+                                    void *ws, size_t ws_bytes, cudaStream_t stream);
+
+size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * *code receives 0 when no device-side condition was recorded since the
+ * last call, else a bit set of CSA2_DEVERR_* values. Returns CSA2_OK, or
+ * CSA2_ERR_DEVICE when *code != 0, or CSA2_ERR_CUDA. */
+#define CSA2_DEVERR_BAD_ROW 1u       /* id / page / position outside the cache */
+#define CSA2_DEVERR_WAIT_TIMEOUT 2u  /* a bounded barrier wait gave up         */
+#define CSA2_DEVERR_SELECT 4u        /* selection produced more ids than asked  */
+csa2_status csa2_device_status(cudaStream_t stream, uint32_t *code);
+
+const char *csa2_status_string(csa2_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t csa2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,79 @@
+// append.cuh -- FP4 E2M1 quantise + append of new latent KV rows.
+//
+// DeepSeek V4.1-Flash Cuts KV Cache by 437x (ainewsfeed.tech), paragraph
+// "V4.1-Flash also uses FP4 quantization": the long-term global KV is stored
+// in FP4; DeepSeek V4.1 Flash Architecture Breakdown (nashnova.com),
+// section "How are cache precision and storage arranged?": E2M1 scheme.
+// The pages give no scale rule; this kernel uses one E4M3 scale per block of
+// 16 values, s = E4M3_RNE_satfinite(amax / 6), codes E2M1_RNE_satfinite of
+// x / value(s), ties to the even mantissa, and all-zero codes when value(s)
+// is 0.
+//
+// Layout: one warp per 512-value row. Lane l owns block l (values 16l ..
+// 16l+15): it reads 32 contiguous bytes of bf16 input, writes 8 bytes of
+// codes and 1 scale byte, so a warp moves 1 KiB in and 288 B out with fully
+// coalesced 16-byte loads. HBM-bound: 1312 algorithmic bytes per row.
+//
+// The E2M1 rounding compares |x| against the seven decision points of the
+// grid scaled by value(s) instead of dividing. The products t * value(s)
+// are exact in binary32 (at most 3 + 4 significant bits), and for bf16 x
+// (8 significant bits) the quotient x / value(s) cannot land within half a
+// binary32 ulp of a decision point without being equal to it, so the
+// comparison gives the same code as rounding the binary32 quotient.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+constexpr int kAppendWarps = 8;
+
+__global__ void __launch_bounds__(kAppendWarps * 32)
+    k_append_fp4(const uint16_t *__restrict__ x, int32_t n, const int32_t *__restrict__ seq,
+                 const int64_t *__restrict__ pos, csa2_kv_desc kv) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+    if (r >= n) return;
+    const int32_t b = seq[r];
+    int64_t row = -1;
+    if (b >= 0 && b < kv.batch) row = physical_row(kv, b, pos[r]);
+    if (row < 0) {
+        if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
+        return;
+    }
+    // 16 bf16 values of this lane's block
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16);
+    uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(wds[i] << 16);
+        f[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));  // fmaxf drops NaN operands
+    const uint32_t s = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+    const float sv = __half2float(__ushort_as_half((uint16_t)(e4m3x2_to_f16x2((uint16_t)s) & 0xFFFFu)));
+    // decision points of the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}; at an
+    // exact midpoint the even-mantissa neighbour wins ('>' keeps the lower
+    // point, '>=' takes the upper one)
+    const float t1 = 0.25f * sv, t2 = 0.75f * sv, t3 = 1.25f * sv, t4 = 1.75f * sv;
+    const float t5 = 2.5f * sv, t6 = 3.5f * sv, t7 = 5.0f * sv;
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(f[i]);
+        uint32_t c = (uint32_t)(a > t1) + (uint32_t)(a >= t2) + (uint32_t)(a > t3) + (uint32_t)(a >= t4) +
+                     (uint32_t)(a > t5) + (uint32_t)(a >= t6) + (uint32_t)(a > t7);
+        c |= (__float_as_uint(f[i]) >> 31) << 3;
+        if (sv == 0.0f) c = 0u;
+        packed[i >> 3] |= c << (4 * (i & 7));
+    }
+    uint2 *dst = reinterpret_cast<uint2 *>(kv.codes + row * (CSA2_D / 2) + lane * 8);
+    *dst = make_uint2(packed[0], packed[1]);
+    kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
+}
+
+}  // namespace csa2

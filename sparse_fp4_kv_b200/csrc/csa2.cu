@@ -1,0 +1,413 @@
+// csa2.cu -- the C ABI of libcsa2.so (declared in include/csa2.h): host-side
+// argument checks, launch planning, tensor-map encoding and kernel launches.
+// All kernels live in this one translation unit (append.cuh, indexer.cuh,
+// attention.cuh) so the device error word is a single module variable.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "append.cuh"
+#include "attention.cuh"
+#include "indexer.cuh"
+
+using namespace csa2;
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+csa2_status check_launch() {
+    return cudaGetLastError() == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA;
+}
+
+csa2_status check_kv(const csa2_kv_desc *kv, bool need_kidx) {
+    if (!kv) return CSA2_ERR_INVALID_ARG;
+    if (kv->d != CSA2_D) return CSA2_ERR_UNSUPPORTED;
+    if (!kv->codes || !kv->scales || !kv->page_table || !kv->seq_len) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(kv->codes, 16) || !aligned(kv->scales, 16) || !aligned(kv->page_table, 4) ||
+        !aligned(kv->seq_len, 4))
+        return CSA2_ERR_INVALID_ARG;
+    if (kv->rows_cap <= 0 || kv->batch <= 0 || kv->max_pages <= 0 || kv->page_size <= 0) return CSA2_ERR_INVALID_ARG;
+    if (kv->page_size % 32 != 0) return CSA2_ERR_UNSUPPORTED;
+    if (kv->page_size < 128 && 128 % kv->page_size != 0) return CSA2_ERR_UNSUPPORTED;
+    if (kv->page_size > 128 && kv->page_size % 128 != 0) return CSA2_ERR_UNSUPPORTED;
+    if (kv->rows_cap > INT32_MAX) return CSA2_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+    if (need_kidx) {
+        if (!kv->kidx || !aligned(kv->kidx, 16)) return CSA2_ERR_INVALID_ARG;
+        if (kv->di != 64 && kv->di != 128) return CSA2_ERR_UNSUPPORTED;
+    }
+    return CSA2_OK;
+}
+
+// cuTensorMapEncodeTiled, fetched through the runtime so that the library
+// does not link the driver library directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_kidx_map(CUtensorMap *tm, const csa2_kv_desc *kv, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kv->di, (cuuint64_t)kv->rows_cap};
+    const cuuint64_t strides[1] = {(cuuint64_t)kv->di};
+    const cuuint32_t box[2] = {(cuuint32_t)kv->di, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = kv->di == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(kv->kidx), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- Full indexer workspace ------------------------------------------------
+struct FullLayout {
+    int64_t key_stride;
+    int32_t n_sel_chunks;
+    size_t off_keys, off_hist0, off_hist1, off_hist2, off_cnt, total;
+};
+
+FullLayout full_layout(int32_t nq, int64_t n_max) {
+    FullLayout L{};
+    L.key_stride = (int64_t)align_up((size_t)std::max<int64_t>(n_max, 1), 128);
+    L.n_sel_chunks = (int32_t)((std::max<int64_t>(n_max, 1) + kSelChunk - 1) / kSelChunk);
+    size_t off = 0;
+    L.off_keys = off;
+    off = align_up(off + (size_t)nq * L.key_stride * 4, 256);
+    L.off_hist0 = off;
+    off = align_up(off + (size_t)nq * kHist0Bins * 4, 256);
+    L.off_hist1 = off;
+    off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
+    L.off_hist2 = off;
+    off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
+    L.off_cnt = off;
+    off = align_up(off + (size_t)nq * 2 * L.n_sel_chunks * 2 * 4, 256);
+    L.total = off;
+    return L;
+}
+
+// ---- attention planning ------------------------------------------------------
+struct AttnPlan {
+    int32_t tiles, tiles_per_split, splits;
+};
+
+AttnPlan plan_attn(int32_t nq, int32_t k, int32_t w_max, int sms) {
+    AttnPlan P{};
+    const int64_t rows = (int64_t)k + std::max(0, w_max);
+    P.tiles = (int32_t)std::max<int64_t>(1, (rows + kAttnTile - 1) / kAttnTile);
+    double best = 1e30;
+    for (int32_t tps = 1; tps <= P.tiles; ++tps) {
+        const int32_t splits = (P.tiles + tps - 1) / tps;
+        const int64_t ctas = (int64_t)nq * splits;
+        const int64_t waves = (ctas + sms - 1) / sms;
+        // tile-times on the critical path, plus a small charge for the
+        // partial outputs and the combine pass when a query is split
+        const double cost = (double)waves * tps + (splits > 1 ? 0.35 + 0.02 * splits : 0.0);
+        if (cost < best - 1e-9) {
+            best = cost;
+            P.tiles_per_split = tps;
+            P.splits = splits;
+        }
+    }
+    return P;
+}
+
+struct AttnLayout {
+    size_t off_o, off_lse, total;
+};
+
+AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P) {
+    AttnLayout L{};
+    if (P.splits <= 1) return L;
+    L.off_o = 0;
+    L.off_lse = align_up((size_t)nq * P.splits * h * CSA2_D * 4, 256);
+    L.total = align_up(L.off_lse + (size_t)nq * P.splits * h * 4, 256);
+    return L;
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t csa2_version(void) { return kVersion; }
+
+const char *csa2_status_string(csa2_status s) {
+    switch (s) {
+        case CSA2_OK: return "ok";
+        case CSA2_ERR_INVALID_ARG: return "invalid argument";
+        case CSA2_ERR_UNSUPPORTED: return "unsupported configuration";
+        case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+        case CSA2_ERR_CUDA: return "CUDA error";
+        case CSA2_ERR_DEVICE: return "device-side error recorded";
+    }
+    return "unknown status";
+}
+
+csa2_status csa2_device_status(cudaStream_t stream, uint32_t *code) {
+    if (!code) return CSA2_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return CSA2_ERR_CUDA;
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof v) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_dev_error, &z, sizeof z) != cudaSuccess) return CSA2_ERR_CUDA;
+    *code = v;
+    return v ? CSA2_ERR_DEVICE : CSA2_OK;
+}
+
+csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
+                            const csa2_kv_desc *kv, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, false);
+    if (st != CSA2_OK) return st;
+    if (n < 0) return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
+        return CSA2_ERR_INVALID_ARG;
+    const unsigned grid = (unsigned)((n + kAppendWarps - 1) / kAppendWarps);
+    k_append_fp4<<<grid, kAppendWarps * 32, 0, stream>>>(static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
+    return check_launch();
+}
+
+size_t csa2_index_full_workspace_size(int32_t nq, int64_t n_max) {
+    if (nq <= 0 || n_max < 0) return 0;
+    return full_layout(nq, n_max).total;
+}
+
+csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq, int32_t hi,
+                            const int32_t *q_limit, int64_t n_max, const csa2_kv_desc *kv, int32_t k, int32_t p,
+                            int32_t *topk, int32_t *pool, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
+        return CSA2_ERR_INVALID_ARG;
+    if (hi < 1 || hi > kScanN) return CSA2_ERR_UNSUPPORTED;
+    if (k < 1 || p < 0 || (p > 0 && p < k) || n_max < 0) return CSA2_ERR_INVALID_ARG;
+    if (n_max > (int64_t)kv->max_pages * kv->page_size) return CSA2_ERR_INVALID_ARG;
+    if (!qidx || !w || !topk || !aligned(qidx, 16) || !aligned(w, 4) || !aligned(topk, 4))
+        return CSA2_ERR_INVALID_ARG;
+    if ((p > 0) != (pool != nullptr) || (pool && !aligned(pool, 4))) return CSA2_ERR_INVALID_ARG;
+    if (q_limit && !aligned(q_limit, 4)) return CSA2_ERR_INVALID_ARG;
+    const FullLayout L = full_layout(nq, n_max);
+    if (!ws || ws_bytes < L.total || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+
+    const int box_rows = std::min(128, (int)kv->page_size);
+    CUtensorMap tm;
+    if (!make_kidx_map(&tm, kv, box_rows)) return CSA2_ERR_CUDA;
+
+    if (cudaMemsetAsync(wsb + L.off_hist0, 0, L.off_cnt - L.off_hist0, stream) != cudaSuccess) return CSA2_ERR_CUDA;
+
+    ScanParams sp{};
+    sp.qidx = qidx;
+    sp.w = w;
+    sp.q_limit = q_limit;
+    sp.kv = *kv;
+    sp.keys = reinterpret_cast<uint32_t *>(wsb + L.off_keys);
+    sp.hist0 = reinterpret_cast<uint32_t *>(wsb + L.off_hist0);
+    sp.key_stride = L.key_stride;
+    sp.q_per_seq = q_per_seq;
+    sp.hi = hi;
+    sp.box_rows = box_rows;
+    const int64_t tiles_max = std::max<int64_t>(1, (n_max + kScanTile - 1) / kScanTile);
+    const int64_t target = (int64_t)num_sms() * 4;
+    int64_t chunk = std::max<int64_t>(4, ((int64_t)nq * tiles_max + target - 1) / target);
+    chunk = std::min<int64_t>(chunk, 256);
+    sp.chunk_tiles = (int32_t)chunk;
+    const dim3 sgrid((unsigned)((tiles_max + chunk - 1) / chunk), (unsigned)nq);
+    if (kv->di == 64) {
+        static bool ok = set_smem(k_index_scan<64>, ScanCfg<64>::kSmem);
+        if (!ok) return CSA2_ERR_CUDA;
+        k_index_scan<64><<<sgrid, kScanThreads, ScanCfg<64>::kSmem, stream>>>(tm, sp);
+    } else {
+        static bool ok = set_smem(k_index_scan<128>, ScanCfg<128>::kSmem);
+        if (!ok) return CSA2_ERR_CUDA;
+        k_index_scan<128><<<sgrid, kScanThreads, ScanCfg<128>::kSmem, stream>>>(tm, sp);
+    }
+    if ((st = check_launch()) != CSA2_OK) return st;
+
+    SelParams sel{};
+    sel.keys = sp.keys;
+    sel.q_limit = q_limit;
+    sel.kv = *kv;
+    sel.hist0 = sp.hist0;
+    sel.hist1 = reinterpret_cast<uint32_t *>(wsb + L.off_hist1);
+    sel.hist2 = reinterpret_cast<uint32_t *>(wsb + L.off_hist2);
+    sel.cnt = reinterpret_cast<uint32_t *>(wsb + L.off_cnt);
+    sel.out[0] = topk;
+    sel.out[1] = pool;
+    sel.rank[0] = k;
+    sel.rank[1] = p;
+    sel.key_stride = L.key_stride;
+    sel.q_per_seq = q_per_seq;
+    sel.n_chunks = L.n_sel_chunks;
+    const dim3 grid((unsigned)L.n_sel_chunks, (unsigned)nq);
+    k_sel_hist<1><<<grid, kSelThreads, 0, stream>>>(sel);
+    k_sel_hist<2><<<grid, kSelThreads, 0, stream>>>(sel);
+    k_sel_count<<<grid, kSelThreads, 0, stream>>>(sel);
+    k_sel_emit<<<grid, kSelThreads, 0, stream>>>(sel);
+    return check_launch();
+}
+
+size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p) {
+    if (nq <= 0 || p <= 0) return 0;
+    return align_up((size_t)nq * p * 4, 256) * 2;
+}
+
+csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq, int32_t hi,
+                               const int32_t *pool, int32_t p, const csa2_kv_desc *kv, int32_t k, int32_t *topk,
+                               void *ws, size_t ws_bytes, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
+        return CSA2_ERR_INVALID_ARG;
+    if (hi < 1 || hi > kScanN) return CSA2_ERR_UNSUPPORTED;
+    if (k < 1 || p < 1) return CSA2_ERR_INVALID_ARG;
+    if (p > kReindexMaxPool) return CSA2_ERR_UNSUPPORTED;
+    if (!qidx || !w || !pool || !topk || !aligned(qidx, 16) || !aligned(w, 4) || !aligned(pool, 4) ||
+        !aligned(topk, 4))
+        return CSA2_ERR_INVALID_ARG;
+    const size_t half = align_up((size_t)nq * p * 4, 256);
+    if (!ws || ws_bytes < 2 * half || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+    ReindexParams rp{};
+    rp.qidx = qidx;
+    rp.w = w;
+    rp.pool = pool;
+    rp.kv = *kv;
+    rp.keys = static_cast<uint32_t *>(ws);
+    rp.ids = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + half);
+    rp.topk = topk;
+    rp.p = p;
+    rp.k = k;
+    rp.hi = hi;
+    rp.q_per_seq = q_per_seq;
+    const dim3 grid((unsigned)((p + kReindexThreads - 1) / kReindexThreads), (unsigned)nq);
+    if (kv->di == 64)
+        k_reindex_score<64><<<grid, kReindexThreads, 0, stream>>>(rp);
+    else
+        k_reindex_score<128><<<grid, kReindexThreads, 0, stream>>>(rp);
+    if ((st = check_launch()) != CSA2_OK) return st;
+    const size_t smem = (size_t)p * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4;
+    static bool ok = set_smem(k_reindex_select, (size_t)kReindexMaxPool * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4);
+    if (!ok) return CSA2_ERR_CUDA;
+    k_reindex_select<<<nq, kReindexSelThreads, smem, stream>>>(rp);
+    return check_launch();
+}
+
+size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max) {
+    if (nq <= 0 || h <= 0 || k < 0) return 0;
+    const AttnPlan P = plan_attn(nq, k, w_max, num_sms());
+    return attn_layout(nq, h, P).total;
+}
+
+csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                    const csa2_kv_desc *kv, const int32_t *topk, int32_t k, const uint8_t *swa,
+                                    int64_t swa_seq_stride, const int32_t *swa_begin, const int32_t *swa_end,
+                                    int32_t w_max, float softmax_scale, void *o_bf16, float *lse, void *ws,
+                                    size_t ws_bytes, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, false);
+    if (st != CSA2_OK) return st;
+    if (h != 16 && h != 32 && h != 64) return CSA2_ERR_UNSUPPORTED;
+    if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
+        return CSA2_ERR_INVALID_ARG;
+    if (k < 0 || w_max < 0 || (k > 0 && !topk) || (topk && !aligned(topk, 4))) return CSA2_ERR_INVALID_ARG;
+    if (!q_bf16 || !o_bf16 || !aligned(q_bf16, 16) || !aligned(o_bf16, 16) || (lse && !aligned(lse, 4)))
+        return CSA2_ERR_INVALID_ARG;
+    const bool has_swa = swa_begin != nullptr;
+    if (has_swa && (!swa || !swa_end || !aligned(swa, 16) || !aligned(swa_begin, 4) || !aligned(swa_end, 4)))
+        return CSA2_ERR_INVALID_ARG;
+    if (!has_swa && w_max > 0) return CSA2_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return CSA2_ERR_INVALID_ARG;
+    const AttnPlan P = plan_attn(nq, k, has_swa ? w_max : 0, num_sms());
+    const AttnLayout L = attn_layout(nq, h, P);
+    if (L.total > 0 && (!ws || ws_bytes < L.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
+
+    AttnParams ap{};
+    ap.q = static_cast<const uint16_t *>(q_bf16);
+    ap.kv = *kv;
+    ap.topk = topk;
+    ap.swa = swa;
+    ap.swa_seq_stride = swa_seq_stride;
+    ap.swa_begin = has_swa ? swa_begin : nullptr;
+    ap.swa_end = has_swa ? swa_end : nullptr;
+    ap.o = static_cast<uint16_t *>(o_bf16);
+    ap.lse = lse;
+    ap.o_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_o) : nullptr;
+    ap.lse_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_lse) : nullptr;
+    ap.scale_log2 = softmax_scale * 1.4426950408889634f;
+    ap.k = k;
+    ap.q_per_seq = q_per_seq;
+    ap.n_splits = P.splits;
+    ap.tiles_per_split = P.tiles_per_split;
+    const dim3 grid((unsigned)P.splits, (unsigned)nq);
+    switch (h) {
+        case 64: {
+            static bool ok = set_smem(k_sparse_attn<64>, AttnCfg<64>::kSmem);
+            if (!ok) return CSA2_ERR_CUDA;
+            k_sparse_attn<64><<<grid, kAttnThreads, AttnCfg<64>::kSmem, stream>>>(ap);
+            break;
+        }
+        case 32: {
+            static bool ok = set_smem(k_sparse_attn<32>, AttnCfg<32>::kSmem);
+            if (!ok) return CSA2_ERR_CUDA;
+            k_sparse_attn<32><<<grid, kAttnThreads, AttnCfg<32>::kSmem, stream>>>(ap);
+            break;
+        }
+        default: {
+            static bool ok = set_smem(k_sparse_attn<16>, AttnCfg<16>::kSmem);
+            if (!ok) return CSA2_ERR_CUDA;
+            k_sparse_attn<16><<<grid, kAttnThreads, AttnCfg<16>::kSmem, stream>>>(ap);
+            break;
+        }
+    }
+    if ((st = check_launch()) != CSA2_OK) return st;
+    if (P.splits > 1) {
+        const dim3 cgrid((unsigned)(h / kCombineHeads), (unsigned)nq);
+        const size_t csmem = (size_t)kCombineHeads * (P.splits + 1) * 4;
+        switch (h) {
+            case 64:
+                k_attn_combine<64><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                                                                             P.splits);
+                break;
+            case 32:
+                k_attn_combine<32><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                                                                             P.splits);
+                break;
+            default:
+                k_attn_combine<16><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                                                                             P.splits);
+                break;
+        }
+        st = check_launch();
+    }
+    return st;
+}
+
+}  // extern "C"

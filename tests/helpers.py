@@ -1,0 +1,60 @@
+"""Shared helpers of the GPU parity tests: building small caches on both
+sides from the same seeded inputs and comparing id lists."""
+import numpy as np
+import torch
+
+import oracle
+from sparse_fp4_kv_b200 import synth
+
+ATTN_TOL = 2e-3  # max |o_gpu - o_oracle| (bf16 output), from the acceptance bar
+
+
+def bf16_bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def int_e4m3_np(rng, shape, lo=-8, hi=8):
+    v = rng.integers(lo, hi + 1, size=shape).astype(np.float32)
+    return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def paged_layout(rng, lens, ps, shuffle=True, spare_pages=3):
+    """Page table [batch, max_pages] over a pool of physical pages."""
+    npages = [max(1, (int(l) + ps - 1) // ps) for l in lens]
+    total = sum(npages) + spare_pages
+    perm = rng.permutation(total) if shuffle else np.arange(total)
+    pt = np.full((len(lens), max(npages)), -1, np.int32)
+    off = 0
+    for b, c in enumerate(npages):
+        pt[b, :c] = perm[off:off + c]
+        off += c
+    return pt, total * ps
+
+
+def compare_ids(gpu_row, oracle_row, what=""):
+    """GPU lists are in ascending id order then -1; oracle lists are in score
+    order then -1. Same multiset of ids and same padding length required."""
+    g = np.asarray(gpu_row)
+    o = np.asarray(oracle_row)
+    assert g.shape == o.shape, what
+    ng = int((g >= 0).sum())
+    no = int((o >= 0).sum())
+    assert ng == no, f"{what}: {ng} ids vs {no}"
+    assert np.all(g[ng:] == -1), f"{what}: padding"
+    np.testing.assert_array_equal(np.sort(g[:ng]), np.sort(o[:no]), err_msg=what)
+
+
+def kv_from_numpy(codes, scales, kidx, page_table, seq_len, ps, device):
+    from sparse_fp4_kv_b200 import binding as B
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    return B.KvCache(t(codes), t(scales), t(kidx) if kidx is not None else None, t(page_table),
+                     t(np.asarray(seq_len, np.int32)), ps)
+
+
+def device_status_clean():
+    from sparse_fp4_kv_b200 import binding as B
+    return B.csa2_device_status() == 0
+
+
+def normal_bf16_rows(seed, stream, n, d=512):
+    return synth.normal_bf16(seed, stream, 0, n * d).view(n, d)

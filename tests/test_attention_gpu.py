@@ -1,0 +1,110 @@
+"""Sparse + window attention kernel against the oracle (f64): outputs within
+2e-3 max-abs (bf16 out), log-sum-exp within 1e-3. Covers 16/32/64 heads,
+ragged tile counts, -1 ids, empty windows, paged caches, single-split and
+split-and-combine launches, and the degenerate empty set."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import ATTN_TOL, bf16_bits, device_status_clean, kv_from_numpy, paged_layout
+from sparse_fp4_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sparse_fp4_kv_b200 import build
+    build.build()
+    from sparse_fp4_kv_b200 import binding
+    return binding
+
+
+def _cache(rng, lens, ps, seed):
+    pt, cap = paged_layout(rng, lens, ps)
+    x = synth.normal_bf16(seed, 1, 0, cap * 512).view(cap, 512)
+    codes, scales = oracle.quantize_rows(bf16_bits(x))
+    return pt, cap, codes, scales
+
+
+def _run(B, dev, lens, ps, h, k, w, q_per_seq=1, seed=0, neg_frac=0.05, swa_rows=None, uniform=False):
+    rng = np.random.default_rng(seed)
+    pt, cap, codes, scales = _cache(rng, lens, ps, seed)
+    if uniform:
+        codes[:] = codes[0]
+        scales[:] = scales[0]
+    nb = len(lens)
+    nq = nb * q_per_seq
+    topk = np.full((nq, k), -1, np.int32)
+    for qi in range(nq):
+        n = lens[qi // q_per_seq]
+        m = min(k, n)
+        ids = rng.permutation(n)[:m].astype(np.int32)
+        ids[rng.random(m) < neg_frac] = -1
+        topk[qi, :m] = ids
+        topk[qi] = rng.permutation(topk[qi])
+    swa_rows = swa_rows or max(w, 1)
+    swa = synth.normal_e4m3(seed, 4, 0, nb * swa_rows * 512).view(nb, swa_rows, 512).numpy()
+    if uniform:
+        swa[:] = 0
+    begin = rng.integers(0, swa_rows - w + 1, nq).astype(np.int32)
+    end = (begin + w).astype(np.int32)
+    q = synth.normal_bf16(seed, 3, 0, nq * h * 512).view(nq, h, 512)
+    scale = 1.0 / math.sqrt(512)
+    kv = kv_from_numpy(codes, scales, None, pt, lens, ps, dev)
+    o = torch.full((nq, h, 512), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((nq, h), float("nan"), dtype=torch.float32, device=dev)
+    ws = B.workspace(B.csa2_sparse_attn_workspace_size(nq, h, k, w), dev)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    B.csa2_sparse_attn_decode(q.to(dev), q_per_seq, kv, d(topk) if k > 0 else None, d(swa), swa_rows, d(begin),
+                              d(end), w, scale, o, lse, ws)
+    torch.cuda.synchronize()
+    assert device_status_clean()
+    go = o.float().cpu().numpy()
+    gl = lse.cpu().numpy()
+    worst = 0.0
+    for qi in range(nq):
+        b = qi // q_per_seq
+        oo, ol = oracle.sparse_attn(bf16_bits(q[qi]), codes, scales, pt[b], ps, topk[qi],
+                                    swa[b][begin[qi]:end[qi]] if w > 0 else None, scale)
+        err = np.abs(go[qi] - oo).max()
+        worst = max(worst, err)
+        assert err <= ATTN_TOL, f"q{qi}: max |o - oracle| = {err}"
+        fin = np.isfinite(ol)
+        assert np.all(np.isfinite(gl[qi]) == fin)
+        np.testing.assert_allclose(gl[qi][fin], ol[fin], atol=1e-3, rtol=0)
+    return go, gl, worst
+
+
+@pytest.mark.parametrize("h", [16, 32, 64])
+def test_heads_ragged_tiles(B, cuda_device, h):
+    _run(B, cuda_device, [900, 1500], 64, h, 300, 77, seed=h)
+
+
+def test_single_query_many_tiles_split(B, cuda_device):
+    # one query, 20 tiles -> split across CTAs and merged
+    _run(B, cuda_device, [70000], 128, 64, 2048, 512, seed=1)
+
+
+def test_many_queries_single_split(B, cuda_device):
+    # enough queries that each one runs in a single CTA
+    _run(B, cuda_device, [600] * 4, 64, 32, 256, 33, q_per_seq=80, seed=2, swa_rows=160)
+
+
+def test_no_window_and_window_only(B, cuda_device):
+    _run(B, cuda_device, [500], 64, 64, 200, 0, seed=3)
+    _run(B, cuda_device, [500], 64, 64, 0, 130, seed=4)
+
+
+def test_empty_set_gives_zero(B, cuda_device):
+    go, gl, _ = _run(B, cuda_device, [300], 64, 16, 64, 0, seed=5, neg_frac=1.0)
+    assert np.all(go == 0) and np.all(np.isneginf(gl))
+
+
+def test_identical_rows_return_that_row(B, cuda_device):
+    go, _, _ = _run(B, cuda_device, [400], 64, 32, 256, 0, seed=6, uniform=True, neg_frac=0.0)
+    v = go[0]
+    assert np.allclose(v, v[0:1], atol=0)

@@ -1,0 +1,170 @@
+"""Full and Reindex indexer kernels against the oracle. Inputs are
+small-integer E4M3 values, so every score is an exact integer in binary32
+and the Top-k / pool id sets must match the oracle's exactly (ties broken
+toward the lower id). Covers contiguous and shuffled-paged caches, di 64 and
+128, 1..16 heads, ragged lengths, causal per-query limits, sequences shorter
+than k, all-equal scores and the largest per-head dot products."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import compare_ids, device_status_clean, int_e4m3_np, kv_from_numpy, paged_layout
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    from sparse_fp4_kv_b200 import build
+    build.build()
+    from sparse_fp4_kv_b200 import binding
+    return binding
+
+
+def _case(rng, lens, ps, di, hi, q_per_seq=1, kidx_fn=None, shuffle=True):
+    pt, cap = paged_layout(rng, lens, ps, shuffle=shuffle)
+    kidx = kidx_fn(cap, di) if kidx_fn else int_e4m3_np(rng, (cap, di))
+    nq = len(lens) * q_per_seq
+    qidx = int_e4m3_np(rng, (nq, hi, di))
+    w = rng.integers(1, 5, (nq, hi)).astype(np.float32)
+    codes = np.zeros((cap, 256), np.uint8)
+    scales = np.zeros((cap, 32), np.uint8)
+    return pt, cap, kidx, qidx, w, codes, scales
+
+
+def _run_full(B, dev, lens, ps, di, hi, k, p, q_per_seq=1, q_limit=None, kidx_fn=None, seed=0, shuffle=True):
+    rng = np.random.default_rng(seed)
+    pt, cap, kidx, qidx, w, codes, scales = _case(rng, lens, ps, di, hi, q_per_seq, kidx_fn, shuffle)
+    kv = kv_from_numpy(codes, scales, kidx, pt, lens, ps, dev)
+    nq = qidx.shape[0]
+    n_max = max(lens) if q_limit is None else int(max(q_limit))
+    topk = torch.full((nq, k), -7, dtype=torch.int32, device=dev)
+    pool = torch.full((nq, p), -7, dtype=torch.int32, device=dev) if p > 0 else None
+    ws = B.workspace(B.csa2_index_full_workspace_size(nq, n_max), dev)
+    ql = torch.from_numpy(np.asarray(q_limit, np.int32)).to(dev) if q_limit is not None else None
+    B.csa2_index_full(torch.from_numpy(qidx).to(dev), torch.from_numpy(w).to(dev), q_per_seq, ql, n_max, kv, k, p,
+                      topk, pool, ws)
+    torch.cuda.synchronize()
+    assert device_status_clean()
+    g_topk = topk.cpu().numpy()
+    g_pool = pool.cpu().numpy() if pool is not None else None
+    keys = ws[: nq * ((max(n_max, 1) + 127) // 128 * 128) * 4].view(torch.int32).cpu().numpy().view(np.uint32)
+    keys = keys.reshape(nq, -1)
+    for qi in range(nq):
+        b = qi // q_per_seq
+        lim = lens[b] if q_limit is None else int(q_limit[qi])
+        ot, op, osc = oracle.index_full(qidx[qi], w[qi], kidx, pt[b], ps, lim, k, p, want_scores=True)
+        # scores: the kernel's ordered keys decode to the oracle's exact scores
+        u = keys[qi, :lim]
+        f = np.where(u & 0x80000000, u & 0x7FFFFFFF, ~u).astype(np.uint32).view(np.float32)
+        np.testing.assert_array_equal(f.astype(np.float64), osc, err_msg=f"scores q{qi}")
+        compare_ids(g_topk[qi], ot, f"topk q{qi}")
+        assert np.all(np.diff(g_topk[qi][g_topk[qi] >= 0]) > 0), "ascending ids"
+        if p > 0:
+            compare_ids(g_pool[qi], op, f"pool q{qi}")
+            assert set(g_topk[qi][g_topk[qi] >= 0]) <= set(g_pool[qi][g_pool[qi] >= 0])
+    return g_topk, g_pool, (pt, kidx, qidx, w, kv)
+
+
+def test_full_contiguous_di64(B, cuda_device):
+    _run_full(B, cuda_device, [4096 + 37], 4224, 64, 4, 512, 1024, shuffle=False)
+
+
+def test_full_paged_ragged_batch(B, cuda_device):
+    _run_full(B, cuda_device, [1000, 130, 2047, 64], 64, 64, 4, 100, 300)
+
+
+def test_full_di128_eight_heads(B, cuda_device):
+    _run_full(B, cuda_device, [5000, 3333], 128, 128, 8, 256, 700, seed=1)
+
+
+def test_full_page32_and_head_extremes(B, cuda_device):
+    _run_full(B, cuda_device, [777], 32, 64, 1, 50, 0, seed=2)
+    _run_full(B, cuda_device, [900, 1200], 256, 128, 16, 64, 128, seed=3)
+
+
+def test_full_short_sequences_pad(B, cuda_device):
+    _run_full(B, cuda_device, [50, 1, 200], 64, 64, 4, 64, 128, seed=4)
+
+
+def test_full_causal_queries(B, cuda_device):
+    total = 3000
+    q_limit = [total - 40 + j + 1 for j in range(40)]
+    _run_full(B, cuda_device, [total], 3072, 64, 4, 200, 0, q_per_seq=40, q_limit=q_limit, seed=5,
+              shuffle=False)
+
+
+def test_full_all_ties_take_lowest_ids(B, cuda_device):
+    same = lambda cap, di: np.full((cap, di), 0x38, np.uint8)  # every key = 1.0
+    topk, pool, _ = _run_full(B, cuda_device, [2500], 64, 64, 4, 300, 900, kidx_fn=same, seed=6)
+    assert list(topk[0]) == list(range(300))
+    assert list(pool[0]) == list(range(900))
+
+
+def test_full_largest_dot_products_exact(B, cuda_device):
+    # |q_h . k| up to 64 * 64 (di 64) and 128 * 64 (di 128): accumulation must be exact
+    def extreme(cap, di):
+        rng = np.random.default_rng(7)
+        v = np.where(rng.random((cap, di)) < 0.97, 8.0, -8.0).astype(np.float32)
+        return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    _run_full(B, cuda_device, [3000], 64, 64, 4, 333, 1000, kidx_fn=extreme, seed=7)
+    _run_full(B, cuda_device, [3000], 64, 128, 8, 333, 1000, kidx_fn=extreme, seed=8)
+
+
+@pytest.mark.parametrize("di,hi", [(64, 4), (128, 8)])
+def test_reindex_matches_oracle(B, cuda_device, di, hi):
+    lens = [3000, 1800]
+    topk, pool, (pt, kidx, _, _, kv) = _run_full(B, cuda_device, lens, 64, di, hi, 200, 600, seed=9)
+    rng = np.random.default_rng(10)
+    nq = len(lens)
+    qidx = int_e4m3_np(rng, (nq, hi, di))
+    w = rng.integers(1, 5, (nq, hi)).astype(np.float32)
+    # the Full layer's pool, shuffled, with -1 padding spread through it
+    pools = np.full((nq, 700), -1, np.int32)
+    for qi in range(nq):
+        ids = pool[qi][pool[qi] >= 0]
+        pos = rng.permutation(700)[: ids.size]
+        pools[qi, pos] = rng.permutation(ids)
+    out = torch.full((nq, 200), -7, dtype=torch.int32, device=cuda_device)
+    ws = B.workspace(B.csa2_index_reindex_workspace_size(nq, 700), cuda_device)
+    B.csa2_index_reindex(torch.from_numpy(qidx).to(cuda_device), torch.from_numpy(w).to(cuda_device), 1,
+                         torch.from_numpy(pools).to(cuda_device), kv, 200, out, ws)
+    torch.cuda.synchronize()
+    assert device_status_clean()
+    g = out.cpu().numpy()
+    for qi in range(nq):
+        want = oracle.index_reindex(qidx[qi], w[qi], kidx, pt[qi], 64, pools[qi], 200)
+        compare_ids(g[qi], want, f"reindex q{qi}")
+
+
+def test_reindex_with_every_entry_equals_full(B, cuda_device):
+    n = 2000
+    topk, _, (pt, kidx, qidx, w, kv) = _run_full(B, cuda_device, [n], 64, 64, 4, 150, 0, seed=11)
+    rng = np.random.default_rng(12)
+    allp = rng.permutation(n).astype(np.int32)[None, :]
+    out = torch.empty((1, 150), dtype=torch.int32, device=cuda_device)
+    ws = B.workspace(B.csa2_index_reindex_workspace_size(1, n), cuda_device)
+    B.csa2_index_reindex(torch.from_numpy(qidx).to(cuda_device), torch.from_numpy(w).to(cuda_device), 1,
+                         torch.from_numpy(allp).to(cuda_device), kv, 150, out, ws)
+    torch.cuda.synchronize()
+    assert sorted(out.cpu().numpy()[0]) == sorted(topk[0])
+
+
+def test_reindex_ties_and_short_pool(B, cuda_device):
+    n = 600
+    same = lambda cap, di: np.full((cap, di), 0x38, np.uint8)
+    _, _, (pt, kidx, qidx, w, kv) = _run_full(B, cuda_device, [n], 64, 64, 4, 10, 0, kidx_fn=same, seed=13)
+    pool = np.array([[500, -1, 3, 77, 2, -1, 599, 4, 1, 0, 300]], np.int32)
+    out = torch.empty((1, 6), dtype=torch.int32, device=cuda_device)
+    ws = B.workspace(B.csa2_index_reindex_workspace_size(1, pool.shape[1]), cuda_device)
+    B.csa2_index_reindex(torch.from_numpy(qidx).to(cuda_device), torch.from_numpy(w).to(cuda_device), 1,
+                         torch.from_numpy(pool).to(cuda_device), kv, 6, out, ws)
+    torch.cuda.synchronize()
+    assert sorted(out.cpu().numpy()[0]) == [0, 1, 2, 3, 4, 77]
+    out2 = torch.empty((1, 12), dtype=torch.int32, device=cuda_device)
+    B.csa2_index_reindex(torch.from_numpy(qidx).to(cuda_device), torch.from_numpy(w).to(cuda_device), 1,
+                         torch.from_numpy(pool).to(cuda_device), kv, 12, out2, ws)
+    torch.cuda.synchronize()
+    g = out2.cpu().numpy()[0]
+    assert sorted(g[:9]) == sorted(pool[0][pool[0] >= 0]) and list(g[9:]) == [-1, -1, -1]
