@@ -106,9 +106,9 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq,
                             cudaStream_t stream);
 
 /*
- * Full-mode indexer ([P3] modes paragraph: Full "reads the entire context,
- * generates complete KV and index data, and selects Top-K"; [P4]: the first
- * Full layer builds the candidate pool of the hierarchical indexer).
+ * Full-mode indexer ([P3] modes paragraph: a Full layer scores the whole
+ * context and keeps its Top-K; [P4]: the first Full layer also builds the
+ * candidate pool of the hierarchical indexer).
  * nq queries; query i belongs to sequence i / q_per_seq.
  *   qidx [nq][hi][di] E4M3, w [nq][hi] f32.
  *   q_limit [nq]: number of entries query i may see (entries 0..q_limit-1);
@@ -133,9 +133,9 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq,
 size_t csa2_index_full_workspace_size(int32_t nq, int64_t n_max);
 
 /*
- * Reindex-mode indexer ([P3]: Reindex "takes the complete KV cache from
- * Full mode and re-filters important items"; [P4]: "re-scores to pick new
- * Top-K", later layers "search only within that pool").
+ * Reindex-mode indexer ([P3]: a Reindex layer keeps no cache of its own and
+ * filters again what a Full layer produced; [P4]: it scores anew to choose
+ * its own Top-K, and deeper layers look only inside the Full layer's pool).
  * pool [nq][p]: ids from a Full layer (-1 entries are padding; any order;
  * no duplicates). Scores the pool ids with this layer's qidx/w as in
  * csa2_index_full and writes their Top-k under (score desc, id asc) to

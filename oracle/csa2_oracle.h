@@ -36,7 +36,7 @@
 extern "C" {
 #endif
 
-/* ---- number formats ([P4] "E2M1 scheme"; [OCP-MX]; [OCP-FP8]) ---------- */
+/* ---- number formats ([P4]: E2M1 for the main KV; [OCP-MX]; [OCP-FP8]) --- */
 
 /* Value of a 4-bit E2M1 code (bit 3 sign, bits 2..1 exponent, bit 0 mantissa,
  * exponent bias 1, no infinities or NaN). */

@@ -11,7 +11,7 @@ assigns each layer one of three static operating modes"; DeepSeek V4.1 Flash
 Architecture Breakdown, section "How does the cache compress along three
 dimensions at once?"): a Reindex layer re-scores the pool of the most recent
 Full layer; a Reuse layer takes the Top-k of the most recent layer that
-produced one ("directly reuses prior KV and indices"), or, in the variant
+produced one (Reuse takes over earlier indices as they are), or, in the variant
 reuse_from='full', of the most recent Full layer.
 """
 import math

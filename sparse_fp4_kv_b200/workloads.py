@@ -181,9 +181,8 @@ RECIPES = {
 def resolve_schedule(modes, reuse_from="previous"):
     """[(mode, source_layer)] for a mode string. Reindex re-scores the pool of
     the most recent Full layer. Reuse takes the Top-k of the most recent layer
-    that produced one (reuse_from='previous', the reading that Reuse "directly
-    reuses prior KV and indices") or of the most recent Full layer
-    (reuse_from='full')."""
+    that produced one (reuse_from='previous': Reuse takes over the earlier
+    indices as they are) or of the most recent Full layer (reuse_from='full')."""
     out, last_full, last_idx = [], None, None
     for layer, m in enumerate(modes):
         if m == "F":
