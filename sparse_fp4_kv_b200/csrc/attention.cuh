@@ -13,17 +13,20 @@
 //
 // Work unit: one query and a split of its attended rows (selected global
 // entries followed by its window rows), 128 rows per tile. Per tile:
-//   1. all 8 warps gather the tile: a warp per row, 16 values per lane; FP4
-//      codes are widened with cvt.rn.f16x2.e2m1x2 and multiplied by the
-//      block scale (exact in f16), window bytes with cvt.rn.f16x2.e4m3x2;
-//      the f16 tile lands in shared memory in the 128B-swizzled K-major
-//      layout (rows = entries, 64-value column blocks 16 KiB apart).
+//   1. all 8 warps dequantise the tile's rows (fetched into registers while
+//      the previous tile was on the tensor cores): FP4 codes are widened
+//      with cvt.rn.f16x2.e2m1x2 and multiplied by the block scale (exact in
+//      f16), window bytes with cvt.rn.f16x2.e4m3x2; the f16 tile lands in
+//      shared memory in the 128B-swizzled K-major layout (rows = entries,
+//      64-value column blocks 16 KiB apart); then the loads of the next
+//      tile are issued.
 //   2. one thread issues S^T = KV * Q^T with tcgen05.mma kind::f16
 //      (M = 128 rows, N = H heads, K = 512) into TMEM.
 //   3. warps 0..3 (one TMEM lane quarter each, a thread per row) read S^T,
 //      reduce the per-head tile maximum across the 128 rows (transposed
-//      butterfly + shared memory), run the online softmax in base 2 and
-//      write P^T (f16) into a swizzled M/N-major tile.
+//      butterfly + shared memory), run the online softmax in base 2, write
+//      P^T (f16) into a swizzled M/N-major tile and reduce the per-head sum
+//      of the tile's probabilities the same way.
 //   4. one thread issues O^T += V^T * P^T (A = the same KV tile read
 //      M/N-major, d in four chunks of 128, B = P^T) into TMEM.
 // The running maximum is only raised when a tile's maximum exceeds it by
@@ -51,8 +54,8 @@ struct AttnCfg {
     static constexpr int kColS = 0;
     static constexpr int kColO = H;
     static constexpr uint32_t kTmemCols = H == 64 ? 512u : (H == 32 ? 256u : 128u);
-    static constexpr int kMisc = 128 * 4 /*valid*/ + 4 * H * 4 /*red*/ + 2 * H * 4 /*m, alpha*/ + H * 4 /*l*/ +
-                                 64 /*bars, slot, flags*/;
+    static constexpr int kMisc = 8 * 128 * 5 /*resolved rows*/ + 128 * 4 /*valid*/ + 4 * H * 4 /*red*/ +
+                                 3 * H * 4 /*m, alpha, l*/ + 64 /*bars, slot, flags*/;
     static constexpr size_t kSmem = 1024 + (size_t)kKvBytes + kQBytes + kPBytes + kMisc;
 };
 
@@ -121,80 +124,173 @@ __device__ __forceinline__ void warp_transpose_reduce(float (&v)[H]) {
     }
 }
 
-template <int H>
-__device__ __forceinline__ void store_warp_reduced(float *dst /*[H]*/, const float (&v)[H]) {
+// Write the warp-reduced values of N columns (layout of warp_transpose_reduce)
+// to dst[0..N).
+template <int N>
+__device__ __forceinline__ void store_warp_reduced(float *dst, const float (&v)[N]) {
     const int lane = threadIdx.x & 31;
-    if (H == 64) {
+    if (N == 64) {
         dst[2 * lane] = v[0];
         dst[2 * lane + 1] = v[1];
-    } else if (H == 32) {
-        dst[lane] = v[0];
     } else {
-        if ((lane & 1) == 0) dst[lane >> 1] = v[0];
+        constexpr int R = N >= 32 ? 1 : 32 / N;  // lanes holding the same column
+        if (lane % R == 0) dst[lane / R] = v[0];
     }
 }
 
-// Gather + dequantise one attended row into the f16 tile (whole warp).
-__device__ __forceinline__ bool gather_row(const AttnParams &p, int32_t u, int32_t b, int32_t nw, int32_t wb,
-                                           int64_t j, int e, uint8_t *kv_tile) {
-    const int lane = threadIdx.x & 31;
-    uint32_t h0[4] = {0u, 0u, 0u, 0u}, h1[4] = {0u, 0u, 0u, 0u};
-    bool valid = false;
-    if (j < p.k) {
-        const int32_t id = p.topk[(int64_t)u * p.k + j];
-        if (id >= 0) {
-            const int64_t row = physical_row(p.kv, b, id);
-            if (row >= 0) {
-                valid = true;
-                const uint2 cw = __ldg(reinterpret_cast<const uint2 *>(p.kv.codes + row * (CSA2_D / 2)) + lane);
-                const uint32_t s = __ldg(p.kv.scales + row * (CSA2_D / CSA2_BLOCK) + lane);
-                const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)(s | (s << 8)));
-                e2m1x8_to_f16x8(cw.x, h0);
-                e2m1x8_to_f16x8(cw.y, h1);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    h0[i] = hmul2_u32(h0[i], s2);
-                    h1[i] = hmul2_u32(h1[i], s2);
+// ---------------------------------------------------------------------------
+// Tile gather: each warp owns 16 rows of the 128-row tile. Lanes 0..15
+// resolve the rows' sources in parallel (id -> page table -> physical row,
+// or window row), then every lane issues its 16-value slice of all 16 rows
+// back to back, so 16 independent loads per lane are in flight. The raw
+// bytes stay in registers until the f16 tile buffer is free again, which
+// lets the loads of tile t+1 run under the tensor-core work of tile t.
+// ---------------------------------------------------------------------------
+constexpr int kRowsPerWarp = kAttnTile / (kAttnThreads / 32);  // 16
+constexpr int kResolveTiles = 8;  // rows resolved per batch: 8 tiles = 1024 rows
+
+struct TileRaw {
+    uint4 v[kRowsPerWarp];  // FP4 row: {codes lo, codes hi, scale byte, 0}; window row: 16 E4M3 bytes
+    uint32_t kinds;         // 2 bits per row: 0 empty, 1 FP4 global entry, 2 window row
+};
+
+// Resolve the sources of rows [j0, j0 + n) of the query's attended list into
+// shared memory: physical FP4 row (kind 1), window buffer row (kind 2) or
+// nothing (kind 0). All threads take part; two dependent loads per row, all
+// rows in flight together.
+__device__ __forceinline__ void resolve_rows(const AttnParams &p, int32_t u, int32_t b, int32_t nw, int32_t wb,
+                                             int64_t j0, int n, int32_t *rsrc, uint8_t *rkind) {
+    for (int i = threadIdx.x; i < n; i += kAttnThreads) {
+        const int64_t j = j0 + i;
+        int32_t src = 0;
+        uint8_t kind = 0;
+        if (j < p.k) {
+            const int32_t id = p.topk[(int64_t)u * p.k + j];
+            if (id >= 0) {
+                const int64_t row = physical_row(p.kv, b, id);
+                if (row >= 0) {
+                    src = (int32_t)row;
+                    kind = 1;
+                } else {
+                    set_error(CSA2_DEVERR_BAD_ROW);
                 }
-            } else if (lane == 0) {
-                set_error(CSA2_DEVERR_BAD_ROW);
             }
+        } else if (j < (int64_t)p.k + nw) {
+            src = (int32_t)(wb + (j - p.k));
+            kind = 2;
         }
-    } else if (j < (int64_t)p.k + nw) {
-        valid = true;
-        const int64_t r = (int64_t)b * p.swa_seq_stride + wb + (j - p.k);
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.swa + r * CSA2_D) + lane);
-        h0[0] = e4m3x2_to_f16x2((uint16_t)(v.x & 0xFFFFu));
-        h0[1] = e4m3x2_to_f16x2((uint16_t)(v.x >> 16));
-        h0[2] = e4m3x2_to_f16x2((uint16_t)(v.y & 0xFFFFu));
-        h0[3] = e4m3x2_to_f16x2((uint16_t)(v.y >> 16));
-        h1[0] = e4m3x2_to_f16x2((uint16_t)(v.z & 0xFFFFu));
-        h1[1] = e4m3x2_to_f16x2((uint16_t)(v.z >> 16));
-        h1[2] = e4m3x2_to_f16x2((uint16_t)(v.w & 0xFFFFu));
-        h1[3] = e4m3x2_to_f16x2((uint16_t)(v.w >> 16));
+        rsrc[i] = src;
+        rkind[i] = kind;
     }
-    *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane)) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
-    *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane + 1)) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
-    return valid;
+}
+
+// Issue the loads of one tile's rows (resolved sources at rsrc/rkind + off):
+// every lane loads its 16-value slice of the warp's 16 rows back to back.
+__device__ __forceinline__ void fetch_tile(const AttnParams &p, int32_t b, const int32_t *rsrc, const uint8_t *rkind,
+                                           int off, TileRaw &raw) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int base = off + warp * kRowsPerWarp;
+    const int32_t my_src = lane < kRowsPerWarp ? rsrc[base + lane] : 0;
+    const uint32_t my_kind = lane < kRowsPerWarp ? rkind[base + lane] : 0u;
+    const uint8_t *swa_seq = p.swa ? p.swa + (int64_t)b * p.swa_seq_stride * CSA2_D : nullptr;
+    raw.kinds = 0;
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+        const int64_t src = __shfl_sync(0xFFFFFFFFu, my_src, r);
+        const uint32_t kd = __shfl_sync(0xFFFFFFFFu, my_kind, r);
+        raw.kinds |= kd << (2 * r);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (kd == 1) {
+            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(p.kv.codes + src * (CSA2_D / 2)) + lane);
+            v = make_uint4(c.x, c.y, (uint32_t)__ldg(p.kv.scales + src * (CSA2_D / CSA2_BLOCK) + lane), 0u);
+        } else if (kd == 2) {
+            v = __ldg(reinterpret_cast<const uint4 *>(swa_seq + src * CSA2_D) + lane);
+        }
+        raw.v[r] = v;
+    }
+}
+
+// Dequantise the fetched rows into the f16 tile (128B-swizzled K-major) and
+// record which rows hold data.
+__device__ __forceinline__ void store_tile(const TileRaw &raw, uint8_t *kv_tile, int32_t *valid_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+        const uint32_t kd = (raw.kinds >> (2 * r)) & 3u;
+        const uint4 v = raw.v[r];
+        uint32_t h0[4] = {0u, 0u, 0u, 0u}, h1[4] = {0u, 0u, 0u, 0u};
+        if (kd == 1) {
+            const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)(v.z | (v.z << 8)));
+            e2m1x8_to_f16x8(v.x, h0);
+            e2m1x8_to_f16x8(v.y, h1);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                h0[i] = hmul2_u32(h0[i], s2);
+                h1[i] = hmul2_u32(h1[i], s2);
+            }
+        } else if (kd == 2) {
+            h0[0] = e4m3x2_to_f16x2((uint16_t)(v.x & 0xFFFFu));
+            h0[1] = e4m3x2_to_f16x2((uint16_t)(v.x >> 16));
+            h0[2] = e4m3x2_to_f16x2((uint16_t)(v.y & 0xFFFFu));
+            h0[3] = e4m3x2_to_f16x2((uint16_t)(v.y >> 16));
+            h1[0] = e4m3x2_to_f16x2((uint16_t)(v.z & 0xFFFFu));
+            h1[1] = e4m3x2_to_f16x2((uint16_t)(v.z >> 16));
+            h1[2] = e4m3x2_to_f16x2((uint16_t)(v.w & 0xFFFFu));
+            h1[3] = e4m3x2_to_f16x2((uint16_t)(v.w >> 16));
+        }
+        const int e = warp * kRowsPerWarp + r;
+        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane)) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane + 1)) =
+            make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        if (lane == 0) valid_s[e] = kd != 0u;
+    }
+}
+
+// NC consecutive S^T columns of this thread's row (TMEM lane), scaled to
+// base-2 logits (-inf for an empty row).
+template <int NC>
+__device__ __forceinline__ void load_scores(uint32_t taddr, float scale_log2, bool valid, float (&s)[NC]) {
+    if (NC == 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < NC; ++i) s[i] = valid ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+    } else if (NC == 16) {
+        uint32_t r[16];
+        tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < NC; ++i) s[i] = valid ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+    } else {
+        uint32_t r[8];
+        tmem_ld8(taddr, *reinterpret_cast<uint32_t(*)[8]>(r));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < NC; ++i) s[i] = valid ? __uint_as_float(r[i]) * scale_log2 : -INFINITY;
+    }
 }
 
 template <int H>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     using Cfg = AttnCfg<H>;
+    constexpr int HG = H / 2;  // heads per softmax warp group
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kv_tile = base;
     uint8_t *q_tile = kv_tile + Cfg::kKvBytes;
     uint8_t *p_tile = q_tile + Cfg::kQBytes;
-    int32_t *valid_s = reinterpret_cast<int32_t *>(p_tile + Cfg::kPBytes);
+    int32_t *rsrc = reinterpret_cast<int32_t *>(p_tile + Cfg::kPBytes);  // [kResolveTiles * 128]
+    uint8_t *rkind = reinterpret_cast<uint8_t *>(rsrc + kResolveTiles * kAttnTile);
+    int32_t *valid_s = reinterpret_cast<int32_t *>(rkind + kResolveTiles * kAttnTile);
     float *red = reinterpret_cast<float *>(valid_s + kAttnTile);  // [4][H]
     float *m_run = red + 4 * H;
     float *alpha = m_run + H;
-    float *l_fin = alpha + H;
-    uint64_t *bar_s = reinterpret_cast<uint64_t *>(l_fin + H);
+    float *l_run = alpha + H;
+    uint64_t *bar_s = reinterpret_cast<uint64_t *>(l_run + H);
     uint64_t *bar_o = bar_s + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_o + 1);
-    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);
+    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [2] (per head group)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t split = blockIdx.x, u = blockIdx.y;
@@ -206,7 +302,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     const int64_t t_begin = (int64_t)split * p.tiles_per_split;
     const int64_t t_end = min(tiles_total, t_begin + p.tiles_per_split);
 
-    // ---- set-up: TMEM, barriers, Q tile (bf16 -> f16, K-major SW128) ----
+    // ---- prologue: resolve the first rows, start their loads, stage Q ----------
+    if (t_begin < t_end)
+        resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile,
+                     (int)min((int64_t)kResolveTiles, t_end - t_begin) * kAttnTile, rsrc, rkind);
     if (warp == 0) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
@@ -214,46 +313,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     if (tid == 0) {
         mbar_init(bar_s, 1);
         mbar_init(bar_o, 1);
-        *rescale_tile = -1;
+        rescale_tile[0] = rescale_tile[1] = -1;
         fence_mbar_init();
     }
-    if (tid < H) m_run[tid] = -INFINITY;
+    if (tid < H) {
+        m_run[tid] = -INFINITY;
+        l_run[tid] = 0.0f;
+    }
+    __syncthreads();
+    TileRaw raw;
+    raw.kinds = 0;
+    if (t_begin < t_end) fetch_tile(p, b, rsrc, rkind, 0, raw);
     {
+        // Q: bf16 -> f16 into the K-major 128B-swizzled B tile; loads in
+        // batches of 8 per thread so they are in flight together
         const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (int64_t)u * H * CSA2_D);
-        for (int i = tid; i < H * (CSA2_D / 8); i += kAttnThreads) {
-            const int h = i / (CSA2_D / 8), c64 = i % (CSA2_D / 8);
-            const uint4 v = __ldg(qsrc + i);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
+        constexpr int kChunks = H * (CSA2_D / 8);
+        constexpr int kPer = kChunks / kAttnThreads;  // 16 / 8 / 4 for H = 64 / 32 / 16
+        constexpr int kBatch = kPer < 4 ? kPer : 4;
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const float lo = __uint_as_float(w4[t] << 16), hi = __uint_as_float(w4[t] & 0xFFFF0000u);
-                const __half2 hh = __floats2half2_rn(lo, hi);
-                o4[t] = *reinterpret_cast<const uint32_t *>(&hh);
+        for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+            uint4 v[kBatch];
+#pragma unroll
+            for (int t = 0; t < kBatch; ++t) v[t] = __ldg(qsrc + tid + (i0 + t) * kAttnThreads);
+#pragma unroll
+            for (int t = 0; t < kBatch; ++t) {
+                const int i = tid + (i0 + t) * kAttnThreads;
+                const int h = i / (CSA2_D / 8), c64 = i % (CSA2_D / 8);
+                const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const __half2 hh =
+                        __floats2half2_rn(__uint_as_float(w4[q] << 16), __uint_as_float(w4[q] & 0xFFFF0000u));
+                    o4[q] = *reinterpret_cast<const uint32_t *>(&hh);
+                }
+                *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
-            *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t kv_addr = smem_u32(kv_tile), q_addr = smem_u32(q_tile), p_addr = smem_u32(p_tile);
-
-    float l_part[H];  // per-row partial softmax denominators (warps 0..3)
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int quarter = warp & 3, grp = warp >> 2;  // TMEM lane quarter, head group
+    float l_part[HG];                                // this row's partial softmax denominators
 #pragma unroll
-    for (int h = 0; h < H; ++h) l_part[h] = 0.0f;
+    for (int i = 0; i < HG; ++i) l_part[i] = 0.0f;
 
     bool ok = true;
     int it = 0;
     for (int64_t tt = t_begin; tt < t_end && ok; ++tt, ++it) {
-        const int64_t j0 = tt * kAttnTile;
-        // 1. gather + dequantise the tile (16 rows per warp)
-        for (int r = 0; r < kAttnTile / 8; ++r) {
-            const int e = warp * (kAttnTile / 8) + r;
-            const bool v = gather_row(p, u, b, nw, wb, j0 + e, e, kv_tile);
-            if (lane == 0) valid_s[e] = v ? 1 : 0;
+        // 1. the f16 tile buffer is free (previous P*V done): dequantise this
+        //    tile, then put the next tile's loads in flight
+        store_tile(raw, kv_tile, valid_s);
+        if (tt + 1 < t_end) {
+            const int rel = (int)((tt + 1 - t_begin) % kResolveTiles);
+            if (rel == 0) {
+                // next batch of resolved rows (rare: splits of more than 8 tiles)
+                __syncthreads();
+                resolve_rows(p, u, b, nw, wb, (tt + 1) * kAttnTile,
+                             (int)min((int64_t)kResolveTiles, t_end - (tt + 1)) * kAttnTile, rsrc, rkind);
+                __syncthreads();
+            }
+            fetch_tile(p, b, rsrc, rkind, rel * kAttnTile, raw);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -273,122 +398,122 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
             }
             tc_commit(bar_s);
         }
-        if (warp < 4) {
-            // 3. online softmax, one row per thread
+        {
+            // 3. online softmax: thread = row (TMEM lane), warps 0..3 take heads
+            //    [0, H/2), warps 4..7 heads [H/2, H); each group of 4 warps
+            //    synchronises on its own named barrier
             const bool got = mbar_wait(bar_s, it & 1);
             tc_fence_after();
-            float s[H];
-#pragma unroll
-            for (int c = 0; c < H; c += (H >= 32 ? 32 : 16)) {
-                if (H >= 32) {
-                    uint32_t r32[32];
-                    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + Cfg::kColS + c, r32);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r32[i]);
-                } else {
-                    uint32_t r16[16];
-                    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + Cfg::kColS + c, r16);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) s[c + i] = __uint_as_float(r16[i]);
-                }
+            const int row = quarter * 32 + lane;
+            const bool row_valid = valid_s[row] != 0 && got;
+            const uint32_t s_addr = lane_addr + Cfg::kColS + grp * HG;
+            {
+                float v[HG];
+                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
+                warp_transpose_reduce<HG, true>(v);
+                store_warp_reduced<HG>(red + quarter * H + grp * HG, v);
             }
-            const bool row_valid = valid_s[tid] != 0 && got;
-#pragma unroll
-            for (int h = 0; h < H; ++h) s[h] = row_valid ? s[h] * p.scale_log2 : -INFINITY;
-            float mx[H];
-#pragma unroll
-            for (int h = 0; h < H; ++h) mx[h] = s[h];
-            warp_transpose_reduce<H, true>(mx);
-            store_warp_reduced<H>(red + warp * H, mx);
-            named_bar_sync(1, 128);
-            if (tid < H) {
-                const float mt = fmaxf(fmaxf(red[tid], red[H + tid]), fmaxf(red[2 * H + tid], red[3 * H + tid]));
-                const float mo = m_run[tid];
+            named_bar_sync(1 + grp, 128);
+            if (quarter == 0 && lane < HG) {
+                const int h = grp * HG + lane;
+                const float mt = fmaxf(fmaxf(red[h], red[H + h]), fmaxf(red[2 * H + h], red[3 * H + h]));
+                const float mo = m_run[h];
                 float a = 1.0f, mn = mo;
                 if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt > -INFINITY)) {
                     mn = mt;
                     a = (mo == -INFINITY) ? 0.0f : exp2f(mo - mt);
-                    if (mo != -INFINITY) *rescale_tile = (int32_t)it;
+                    if (mo != -INFINITY) rescale_tile[grp] = (int32_t)it;
                 }
-                m_run[tid] = mn;
-                alpha[tid] = a;
+                m_run[h] = mn;
+                alpha[h] = a;
             }
-            named_bar_sync(1, 128);
-            // probabilities -> P^T (f16), partial denominators
+            named_bar_sync(1 + grp, 128);
+            // probabilities -> P^T (f16), per-row partial denominators
+            {
+                float v[HG];
+                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
 #pragma unroll
-            for (int c = 0; c < H / 8; ++c) {
-                uint32_t pk[4];
+                for (int g = 0; g < HG / 8; ++g) {
+                    const float4 ma = *reinterpret_cast<const float4 *>(m_run + grp * HG + 8 * g);
+                    const float4 mb = *reinterpret_cast<const float4 *>(m_run + grp * HG + 8 * g + 4);
+                    const float4 aa = *reinterpret_cast<const float4 *>(alpha + grp * HG + 8 * g);
+                    const float4 ab = *reinterpret_cast<const float4 *>(alpha + grp * HG + 8 * g + 4);
+                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+                    const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
+                    uint32_t pk[4];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int h = 8 * c + 2 * t;
-                    const float m0 = m_run[h], m1 = m_run[h + 1];
-                    const float p0 = (m0 == -INFINITY) ? 0.0f : exp2f(s[h] - m0);
-                    const float p1 = (m1 == -INFINITY) ? 0.0f : exp2f(s[h + 1] - m1);
-                    l_part[h] = fmaf(l_part[h], alpha[h], p0);
-                    l_part[h + 1] = fmaf(l_part[h + 1], alpha[h + 1], p1);
-                    const __half2 hh = __floats2half2_rn(p0, p1);
-                    pk[t] = *reinterpret_cast<const uint32_t *>(&hh);
+                    for (int t = 0; t < 4; ++t) {
+                        const int i = 8 * g + 2 * t;
+                        const float p0 = (mm[2 * t] == -INFINITY) ? 0.0f : exp2f(v[i] - mm[2 * t]);
+                        const float p1 = (mm[2 * t + 1] == -INFINITY) ? 0.0f : exp2f(v[i + 1] - mm[2 * t + 1]);
+                        l_part[i] = fmaf(l_part[i], al[2 * t], p0);
+                        l_part[i + 1] = fmaf(l_part[i + 1], al[2 * t + 1], p1);
+                        const __half2 hh = __floats2half2_rn(p0, p1);
+                        pk[t] = *reinterpret_cast<const uint32_t *>(&hh);
+                    }
+                    *reinterpret_cast<uint4 *>(p_tile + p_chunk_off<H>(row, grp * (HG / 8) + g)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4 *>(p_tile + p_chunk_off<H>(tid, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            // rare: raise of the running maximum -> rescale O^T in TMEM
-            if (*rescale_tile == it) {
+            // rare: raise of the running maximum -> rescale this group's O^T columns
+            if (rescale_tile[grp] == it) {
 #pragma unroll 1
                 for (int dc = 0; dc < 4; ++dc) {
 #pragma unroll
-                    for (int c = 0; c < H; c += 16) {
-                        uint32_t r16[16];
-                        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + Cfg::kColO + dc * H + c;
-                        tmem_ld16(ta, r16);
+                    for (int c = 0; c < HG; c += 8) {
+                        uint32_t r8[8];
+                        const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
+                        tmem_ld8(ta, r8);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha[c + i]);
-                        tmem_st16(ta, r16);
+                        for (int i = 0; i < 8; ++i)
+                            r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha[grp * HG + c + i]);
+                        tmem_st8(ta, r8);
                     }
                 }
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar_sync(1, 128);
             if (!got) ok = false;
-            // 4. O^T += V^T * P^T
-            if (tid == 0 && ok) {
-                tc_fence_after();
-                const uint32_t idesc = idesc_f16_f32(128, H, 1, 1);
+        }
+        ok = __syncthreads_and(ok);
+        tc_fence_after();
+        // 4. O^T += V^T * P^T
+        if (tid == 0 && ok) {
+            const uint32_t idesc = idesc_f16_f32(128, H, 1, 1);
 #pragma unroll
-                for (int dc = 0; dc < 4; ++dc) {
+            for (int dc = 0; dc < 4; ++dc) {
 #pragma unroll
-                    for (int kk = 0; kk < kAttnTile / 16; ++kk) {
-                        const uint64_t ad = make_sdesc(kv_addr + dc * 32768 + kk * 2048, 16384, 1024, kSw128);
-                        const uint64_t bd = make_sdesc(p_addr + kk * 2 * Cfg::kPGroup, 16, Cfg::kPGroup, Cfg::kPSwizzle);
-                        mma_f16(tmem + Cfg::kColO + dc * H, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < kAttnTile / 16; ++kk) {
+                    const uint64_t ad = make_sdesc(kv_addr + dc * 32768 + kk * 2048, 16384, 1024, kSw128);
+                    const uint64_t bd = make_sdesc(p_addr + kk * 2 * Cfg::kPGroup, 16, Cfg::kPGroup, Cfg::kPSwizzle);
+                    mma_f16(tmem + Cfg::kColO + dc * H, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(bar_o);
             }
+            tc_commit(bar_o);
         }
         // the next tile overwrites KV / P: wait for this tile's P*V
         if (ok && !mbar_wait(bar_o, it & 1)) ok = false;
         tc_fence_after();
         ok = __syncthreads_and(ok);
     }
-
-    // ---- final denominators ----
-    if (warp < 4) {
-        warp_transpose_reduce<H, false>(l_part);
-        store_warp_reduced<H>(red + warp * H, l_part);
-    }
+    // ---- final denominators: reduce the per-row partials over the 128 rows ----
     __syncthreads();
-    if (tid < H) l_fin[tid] = (red[tid] + red[H + tid]) + (red[2 * H + tid] + red[3 * H + tid]);
+    warp_transpose_reduce<HG, false>(l_part);
+    store_warp_reduced<HG>(red + quarter * H + grp * HG, l_part);
+    __syncthreads();
+    if (tid < H) {
+        const float l = (red[tid] + red[H + tid]) + (red[2 * H + tid] + red[3 * H + tid]);
+        l_run[tid] = l;
+        alpha[tid] = l > 0.0f ? 1.0f / l : 0.0f;  // reused as 1 / l
+    }
     __syncthreads();
 
     // ---- epilogue: O^T (TMEM) -> o = O / l ----
     {
-        const int quarter = warp & 3, half = warp >> 2;
         constexpr int HC = H / 2;
+        const int half = grp;
         const bool single = p.n_splits == 1;
 #pragma unroll 1
         for (int dc = 0; dc < 4; ++dc) {
@@ -419,20 +544,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
 #pragma unroll
                 for (int i = 0; i < HC; ++i) vals[i] = 0.0f;
             }
+            if (single) {
+                uint16_t *dst = p.o + ((int64_t)u * H + half * HC) * CSA2_D + dd;
 #pragma unroll
-            for (int i = 0; i < HC; ++i) {
-                const int h = half * HC + i;
-                const float l = l_fin[h];
-                const float o = l > 0.0f ? vals[i] / l : 0.0f;
-                if (single) {
-                    p.o[((int64_t)u * H + h) * CSA2_D + dd] = f32_to_bf16_bits(o);
-                } else {
-                    p.o_part[(((int64_t)u * p.n_splits + split) * H + h) * CSA2_D + dd] = o;
-                }
+                for (int i = 0; i < HC; ++i) dst[(int64_t)i * CSA2_D] = f32_to_bf16_bits(vals[i] * alpha[half * HC + i]);
+            } else {
+                float *dst = p.o_part + (((int64_t)u * p.n_splits + split) * H + half * HC) * CSA2_D + dd;
+#pragma unroll
+                for (int i = 0; i < HC; ++i) dst[(int64_t)i * CSA2_D] = vals[i] * alpha[half * HC + i];
             }
         }
         if (tid < H) {
-            const float l = l_fin[tid];
+            const float l = l_run[tid];
             const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
             if (single) {
                 if (p.lse) p.lse[(int64_t)u * H + tid] = lse;
@@ -451,54 +574,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
 
 // Merge the splits of each query: o = sum_s exp(lse_s - M) o_s / L,
 // lse = M + log L with M = max_s lse_s, L = sum_s exp(lse_s - M).
-constexpr int kCombineThreads = 256;
-constexpr int kCombineHeads = 4;  // heads per CTA
+// One CTA per (query, 4 heads); each thread owns one float4 of a head and
+// loads that float4 of every split before combining, so the loads overlap.
+constexpr int kCombineThreads = 128;
+constexpr int kCombineHeads = 1;  // heads per CTA (128 float4 per head)
+constexpr int kCombineBatch = 8;  // split loads in flight per thread
 
 template <int H>
 __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *__restrict__ o_part,
                                                                   const float *__restrict__ lse_part,
                                                                   uint16_t *__restrict__ o, float *__restrict__ lse,
                                                                   int32_t n_splits) {
-    extern __shared__ float wsm[];  // [kCombineHeads][n_splits + 1]
+    extern __shared__ float wsm[];  // [n_splits + 1]
     const int32_t u = blockIdx.y;
-    const int h0 = blockIdx.x * kCombineHeads;
-    if (threadIdx.x < kCombineHeads) {
-        const int h = h0 + threadIdx.x;
+    const int h = blockIdx.x;
+    const int d4 = threadIdx.x;  // 128 threads x 4 values = 512
+    if (threadIdx.x < 32) {
         float M = -INFINITY;
-        for (int s = 0; s < n_splits; ++s) M = fmaxf(M, lse_part[((int64_t)u * n_splits + s) * H + h]);
+        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, lse_part[((int64_t)u * n_splits + s) * H + h]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
         float L = 0.0f;
-        float *w = wsm + threadIdx.x * (n_splits + 1);
-        for (int s = 0; s < n_splits; ++s) {
+        for (int s = threadIdx.x; s < n_splits; s += 32) {
             const float ls = lse_part[((int64_t)u * n_splits + s) * H + h];
-            w[s] = (M == -INFINITY) ? 0.0f : expf(ls - M);
-            L += w[s];
+            const float w = (M == -INFINITY) ? 0.0f : expf(ls - M);
+            wsm[s] = w;
+            L += w;
         }
-        w[n_splits] = L;
-        if (lse) lse[(int64_t)u * H + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+        if (threadIdx.x == 0) {
+            wsm[n_splits] = L;
+            if (lse) lse[(int64_t)u * H + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+        }
     }
     __syncthreads();
-    // kCombineHeads * 512 outputs, 4 consecutive per thread
-    for (int i = threadIdx.x; i < kCombineHeads * CSA2_D / 4; i += kCombineThreads) {
-        const int hl = i / (CSA2_D / 4), d4 = i % (CSA2_D / 4);
-        const int h = h0 + hl;
-        const float *w = wsm + hl * (n_splits + 1);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < n_splits; ++s) {
-            if (w[s] == 0.0f) continue;
-            const float4 v =
-                __ldg(reinterpret_cast<const float4 *>(o_part + (((int64_t)u * n_splits + s) * H + h) * CSA2_D) + d4);
-            acc.x = fmaf(w[s], v.x, acc.x);
-            acc.y = fmaf(w[s], v.y, acc.y);
-            acc.z = fmaf(w[s], v.z, acc.z);
-            acc.w = fmaf(w[s], v.w, acc.w);
+    const float *src = o_part + ((int64_t)u * n_splits * H + h) * CSA2_D;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n_splits; s0 += kCombineBatch) {
+        float4 v[kCombineBatch];
+#pragma unroll
+        for (int t = 0; t < kCombineBatch; ++t)
+            v[t] = (s0 + t < n_splits)
+                       ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(s0 + t) * H * CSA2_D) + d4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < kCombineBatch; ++t) {
+            if (s0 + t >= n_splits) break;
+            const float w = wsm[s0 + t];
+            acc.x = fmaf(w, v[t].x, acc.x);
+            acc.y = fmaf(w, v[t].y, acc.y);
+            acc.z = fmaf(w, v[t].z, acc.z);
+            acc.w = fmaf(w, v[t].w, acc.w);
         }
-        const float L = w[n_splits];
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        uint16_t *dst = o + ((int64_t)u * H + h) * CSA2_D + d4 * 4;
-        const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc.x * inv) | ((uint32_t)f32_to_bf16_bits(acc.y * inv) << 16);
-        const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc.z * inv) | ((uint32_t)f32_to_bf16_bits(acc.w * inv) << 16);
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
     }
+    const float L = wsm[n_splits];
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    uint16_t *dst = o + ((int64_t)u * H + h) * CSA2_D + d4 * 4;
+    const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc.x * inv) | ((uint32_t)f32_to_bf16_bits(acc.y * inv) << 16);
+    const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc.z * inv) | ((uint32_t)f32_to_bf16_bits(acc.w * inv) << 16);
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
 }
 
 }  // namespace csa2

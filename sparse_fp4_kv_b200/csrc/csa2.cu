@@ -390,7 +390,7 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
     if ((st = check_launch()) != CSA2_OK) return st;
     if (P.splits > 1) {
         const dim3 cgrid((unsigned)(h / kCombineHeads), (unsigned)nq);
-        const size_t csmem = (size_t)kCombineHeads * (P.splits + 1) * 4;
+        const size_t csmem = (size_t)(P.splits + 1) * 4;
         switch (h) {
             case 64:
                 k_attn_combine<64><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle.stack as ostack
-from helpers import ATTN_TOL, compare_ids, device_status_clean
+from helpers import attn_excess, compare_ids, device_status_clean
 from sparse_fp4_kv_b200.workloads import RECIPES
 
 pytestmark = pytest.mark.gpu
@@ -39,7 +39,7 @@ def _compare(dec, ref, recipe):
             if mode == "full" and recipe.p > 0:
                 compare_ids(dec.pool[l].cpu().numpy()[qi], ref["pool"][l][qi], f"pool layer {l} q{qi}")
             err = np.abs(g_o[qi] - ref["o"][l][qi]).max()
-            assert err <= ATTN_TOL, f"layer {l} q{qi}: {err}"
+            assert attn_excess(g_o[qi], ref["o"][l][qi]) <= 1.0, f"layer {l} q{qi}: {err}"
             fin = np.isfinite(ref["lse"][l][qi])
             np.testing.assert_allclose(g_lse[qi][fin], ref["lse"][l][qi][fin], atol=1e-3, rtol=0)
 
@@ -78,8 +78,7 @@ def test_reuse_source_full_variant(built, cuda_device):
         assert dec.schedule[l] == ("reuse", 0 if l < 10 else 10)
         for qi, want in ref["topk"][l].items():
             compare_ids(dec.topk_of(l).cpu().numpy()[qi], want, f"layer {l}")
-            err = np.abs(dec.o[l].float().cpu().numpy()[qi] - ref["o"][l][qi]).max()
-            assert err <= ATTN_TOL
+            assert attn_excess(dec.o[l].float().cpu().numpy()[qi], ref["o"][l][qi]) <= 1.0
 
 
 def test_reuse_layer_reproduces_source_output(built, cuda_device):
