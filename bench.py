@@ -266,30 +266,42 @@ def run_ours(args):
         assert err == cu.CUresult.CUDA_SUCCESS
         return ev
 
-    attn_layers = list(range(recipe.layers))
-    ev_pairs = [(new_event(), new_event()) for _ in attn_layers]
+    # external timing events around every C-ABI call inside the graph: the
+    # attention call of every layer (the roofline kernel) and the others
+    # for the per-call breakdown
+    calls = [("append", None)]
+    for l, (mode, _) in enumerate(dec.schedule):
+        if mode in ("full", "reindex"):
+            calls.append((mode, l))
+        calls.append(("attention", l))
+    ev_pairs = [(new_event(), new_event()) for _ in calls]
     ext = cu.CUevent_record_flags.CU_EVENT_RECORD_EXTERNAL
 
     def step_with_events(s):
-        dec.append(s)
         h = cu.CUstream(s.cuda_stream)
-        for i, l in enumerate(attn_layers):
-            mode, src = dec.schedule[l]
-            # the indexer call of the layer, then the timed attention launch
-            r = dec.r
-            if mode == "full":
+        r = dec.r
+        for (kind, l), (e0, e1) in zip(calls, ev_pairs):
+            cu.cuEventRecordWithFlags(e0, h, ext)
+            if kind == "append":
+                dec.append(s)
+            elif kind == "full":
                 B.csa2_index_full(dec.qidx[l], dec.w[l], r.q_per_seq, dec.q_limit, dec.n_max, dec.kv, r.k,
                                   r.p if dec.pool[l] is not None else 0, dec.topk[l], dec.pool[l], dec.ws_full, s)
-            elif mode == "reindex":
+            elif kind == "reindex":
+                src = dec.schedule[l][1]
                 B.csa2_index_reindex(dec.qidx[l], dec.w[l], r.q_per_seq, dec.pool[src], dec.kv, r.k, dec.topk[l],
                                      dec.ws_reindex, s)
-            cu.cuEventRecordWithFlags(ev_pairs[i][0], h, ext)
-            B.csa2_sparse_attn_decode(dec.q[l], r.q_per_seq, dec.kv, dec.topk_of(l), dec.swa[l], dec.swa[l].shape[1],
-                                      dec.swa_begin, dec.swa_end, r.w, dec.scale, dec.o[l], dec.lse[l], dec.ws_attn,
-                                      s)
-            cu.cuEventRecordWithFlags(ev_pairs[i][1], h, ext)
+            else:
+                B.csa2_sparse_attn_decode(dec.q[l], r.q_per_seq, dec.kv, dec.topk_of(l), dec.swa[l],
+                                          dec.swa[l].shape[1], dec.swa_begin, dec.swa_end, r.w, dec.scale, dec.o[l],
+                                          dec.lse[l], dec.ws_attn, s)
+            cu.cuEventRecordWithFlags(e1, h, ext)
 
-    # eager warm-up (first calls set kernel attributes), then capture
+    # eager warm-up (first calls set kernel attributes), then capture two
+    # graphs of the step: the plain one that is timed, and one with external
+    # timing events around every call (event nodes sit between the kernels
+    # and stop programmatic launch overlap, so it only feeds the per-call
+    # breakdown and the roofline kernel's duration)
     with torch.cuda.stream(stream):
         step_with_events(stream)
     stream.synchronize()
@@ -297,13 +309,17 @@ def run_ours(args):
         raise RuntimeError("device error during warm-up")
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
+        dec.step(stream)
+    stream.synchronize()
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
         step_with_events(stream)
     stream.synchronize()
 
     def timed_steps(g, n, record):
         st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        per_step, attn = [], []
+        per_step, attn = [], {}
         for i in range(n):
             with torch.cuda.stream(stream):
                 flush.fill_(i & 0xFF)
@@ -313,9 +329,9 @@ def run_ours(args):
             en[i].synchronize()
             per_step.append(st[i].elapsed_time(en[i]))
             if record:
-                for a, b in ev_pairs:
+                for (kind, _), (a, b) in zip(calls, ev_pairs):
                     err, ms = cu.cuEventElapsedTime(a, b)
-                    attn.append(ms)
+                    attn.setdefault(kind, []).append(ms)
         return per_step, attn
 
     launches_per_step = count_launches(dec, recipe)
@@ -327,11 +343,13 @@ def run_ours(args):
     clocks = Clocks(local)
     clocks.start()
     time.sleep(0.3)
-    per_step, attn = timed_steps(graph, args.steps, True)
+    per_step, _ = timed_steps(graph, args.steps, False)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
+    # instrumented replays right after the timed loop: per-call durations
+    _, attn = timed_steps(graph_ev, args.steps, True)
     if B.csa2_device_status(stream) != 0:
         raise RuntimeError("device error during the timed steps")
     total_ms = sum(per_step)
@@ -349,7 +367,8 @@ def run_ours(args):
         e2e = run_e2e(args, dec, stream, flush, graph_fn=step_with_events, world=world, dev=dev)
 
     hbm_gbs, bf16_burst, bf16_sust, peak_kind = peaks()
-    attn_ms = statistics.mean(attn) if attn else float("nan")
+    breakdown = {k: 1e3 * statistics.mean(v) for k, v in attn.items()}
+    attn_ms = statistics.mean(attn["attention"]) if attn else float("nan")
     achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
     kernel = f"k_sparse_attn<{recipe.h}>"
     line = {
@@ -366,9 +385,14 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": bf16_sust,
                      "unit": "TFLOP/s", "frac": achieved_tf / bf16_sust,
                      "peak_source": f"{peak_kind} bf16 dense sustained (f16 runs at the bf16 rate)",
-                     "launch_us": attn_ms * 1e3, "flops_per_launch": attn_fl, "bytes_per_launch": attn_by,
+                     "launch_us": attn_ms * 1e3, "launch_note": "event-timed attention call (attention kernel + "
+                     "split combine) in the instrumented replay", "flops_per_launch": attn_fl, "bytes_per_launch": attn_by,
                      "hbm_frac": attn_by / (attn_ms * 1e-3) / (hbm_gbs * 1e9),
                      "traffic": recorded_traffic(kernel, recipe.name)},
+        "breakdown_us_per_call": breakdown,
+        "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented replay "
+                          "of the same step (event nodes between calls prevent launch overlap)",
+        "breakdown_calls_per_step": {k: len(v) // args.steps for k, v in attn.items()},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
@@ -383,7 +407,7 @@ def run_ours(args):
                       f"({dt:.1f} s)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
+    del graph, graph_ev
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

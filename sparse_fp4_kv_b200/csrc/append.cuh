@@ -31,6 +31,8 @@ constexpr int kAppendWarps = 8;
 __global__ void __launch_bounds__(kAppendWarps * 32)
     k_append_fp4(const uint16_t *__restrict__ x, int32_t n, const int32_t *__restrict__ seq,
                  const int64_t *__restrict__ pos, csa2_kv_desc kv) {
+    pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
     if (r >= n) return;

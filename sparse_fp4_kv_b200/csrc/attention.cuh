@@ -295,17 +295,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t split = blockIdx.x, u = blockIdx.y;
     const int32_t b = u / p.q_per_seq;
-    const int32_t wb = p.swa_begin ? p.swa_begin[u] : 0;
-    const int32_t nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
-    const int64_t n_total = (int64_t)p.k + nw;
-    const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
-    const int64_t t_begin = (int64_t)split * p.tiles_per_split;
-    const int64_t t_end = min(tiles_total, t_begin + p.tiles_per_split);
 
-    // ---- prologue: resolve the first rows, start their loads, stage Q ----------
-    if (t_begin < t_end)
-        resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile,
-                     (int)min((int64_t)kResolveTiles, t_end - t_begin) * kAttnTile, rsrc, rkind);
+    // ---- set-up that reads no global memory, then wait for the previous kernel ----
+    pdl_trigger();
     if (warp == 0) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
@@ -320,6 +312,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         m_run[tid] = -INFINITY;
         l_run[tid] = 0.0f;
     }
+    pdl_wait();
+    const int32_t wb = p.swa_begin ? p.swa_begin[u] : 0;
+    const int32_t nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
+    const int64_t n_total = (int64_t)p.k + nw;
+    const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
+    const int64_t t_begin = (int64_t)split * p.tiles_per_split;
+    const int64_t t_end = min(tiles_total, t_begin + p.tiles_per_split);
+
+    // ---- prologue: resolve the first rows, start their loads, stage Q ----------
+    if (t_begin < t_end)
+        resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile,
+                     (int)min((int64_t)kResolveTiles, t_end - t_begin) * kAttnTile, rsrc, rkind);
     __syncthreads();
     TileRaw raw;
     raw.kinds = 0;
@@ -510,11 +514,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     }
     __syncthreads();
 
-    // ---- epilogue: O^T (TMEM) -> o = O / l ----
+    // ---- epilogue: O^T (TMEM) -> o = O / l, staged through the free KV tile
+    //      buffer as [h][512] f32 so the global writes are coalesced 16 B ----
     {
         constexpr int HC = H / 2;
         const int half = grp;
-        const bool single = p.n_splits == 1;
+        float *stage = reinterpret_cast<float *>(kv_tile);  // [H][512] f32 = H * 2 KiB <= 128 KiB
 #pragma unroll 1
         for (int dc = 0; dc < 4; ++dc) {
             const int dd = dc * 128 + quarter * 32 + lane;
@@ -544,20 +549,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
 #pragma unroll
                 for (int i = 0; i < HC; ++i) vals[i] = 0.0f;
             }
-            if (single) {
-                uint16_t *dst = p.o + ((int64_t)u * H + half * HC) * CSA2_D + dd;
 #pragma unroll
-                for (int i = 0; i < HC; ++i) dst[(int64_t)i * CSA2_D] = f32_to_bf16_bits(vals[i] * alpha[half * HC + i]);
-            } else {
-                float *dst = p.o_part + (((int64_t)u * p.n_splits + split) * H + half * HC) * CSA2_D + dd;
-#pragma unroll
-                for (int i = 0; i < HC; ++i) dst[(int64_t)i * CSA2_D] = vals[i] * alpha[half * HC + i];
+            for (int i = 0; i < HC; ++i) stage[(half * HC + i) * CSA2_D + dd] = vals[i] * alpha[half * HC + i];
+        }
+        __syncthreads();
+        if (p.n_splits == 1) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (int64_t)u * H * CSA2_D);
+            for (int i = tid; i < H * CSA2_D / 8; i += kAttnThreads) {
+                const float4 x0 = reinterpret_cast<const float4 *>(stage)[2 * i];
+                const float4 x1 = reinterpret_cast<const float4 *>(stage)[2 * i + 1];
+                dst[i] = make_uint4((uint32_t)f32_to_bf16_bits(x0.x) | ((uint32_t)f32_to_bf16_bits(x0.y) << 16),
+                                    (uint32_t)f32_to_bf16_bits(x0.z) | ((uint32_t)f32_to_bf16_bits(x0.w) << 16),
+                                    (uint32_t)f32_to_bf16_bits(x1.x) | ((uint32_t)f32_to_bf16_bits(x1.y) << 16),
+                                    (uint32_t)f32_to_bf16_bits(x1.z) | ((uint32_t)f32_to_bf16_bits(x1.w) << 16));
             }
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D);
+            for (int i = tid; i < H * CSA2_D / 4; i += kAttnThreads) dst[i] = reinterpret_cast<const float4 *>(stage)[i];
         }
         if (tid < H) {
             const float l = l_run[tid];
             const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-            if (single) {
+            if (p.n_splits == 1) {
                 if (p.lse) p.lse[(int64_t)u * H + tid] = lse;
             } else {
                 p.lse_part[((int64_t)u * p.n_splits + split) * H + tid] = lse;
@@ -586,6 +599,8 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
                                                                   uint16_t *__restrict__ o, float *__restrict__ lse,
                                                                   int32_t n_splits) {
     extern __shared__ float wsm[];  // [n_splits + 1]
+    pdl_trigger();
+    pdl_wait();
     const int32_t u = blockIdx.y;
     const int h = blockIdx.x;
     const int d4 = threadIdx.x;  // 128 threads x 4 values = 512

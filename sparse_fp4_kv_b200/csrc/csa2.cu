@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "append.cuh"
 #include "attention.cuh"
@@ -89,7 +90,7 @@ bool make_kidx_map(CUtensorMap *tm, const csa2_kv_desc *kv, int box_rows) {
 struct FullLayout {
     int64_t key_stride;
     int32_t n_sel_chunks;
-    size_t off_keys, off_hist0, off_hist1, off_hist2, off_cnt, total;
+    size_t off_keys, off_hist0, off_hist1, off_hist2, off_state, off_cnt, total;
 };
 
 FullLayout full_layout(int32_t nq, int64_t n_max) {
@@ -105,6 +106,8 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
     off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
     L.off_hist2 = off;
     off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
+    L.off_state = off;
+    off = align_up(off + (size_t)nq * kStateWords * 4, 256);
     L.off_cnt = off;
     off = align_up(off + (size_t)nq * 2 * L.n_sel_chunks * 2 * 4, 256);
     L.total = off;
@@ -150,9 +153,50 @@ AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P) {
     return L;
 }
 
+// Dynamic shared memory limit of a kernel, and the maximal shared-memory
+// carveout, which every kernel of the library requests so that consecutive
+// launches do not change the L1 / shared split of the SMs.
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess &&
+           cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel on the stream is still running; every kernel of
+// the library waits (griddepcontrol.wait) for its predecessor's completion
+// before it reads global memory, and lets its own dependents start early.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args &&...args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename K>
+bool prefer_shared(K kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+
+// One-time attribute set-up of the kernels without large dynamic shared memory.
+bool init_small_kernels() {
+    static const bool ok = prefer_shared(k_append_fp4) && prefer_shared(k_sel_hist<1>) &&
+                           prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
+                           prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
+                           prefer_shared(k_attn_combine<16>) && prefer_shared(k_attn_combine<32>) &&
+                           prefer_shared(k_attn_combine<64>);
+    return ok;
 }
 
 }  // namespace
@@ -191,8 +235,9 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
     if (n == 0) return CSA2_OK;
     if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
         return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
     const unsigned grid = (unsigned)((n + kAppendWarps - 1) / kAppendWarps);
-    k_append_fp4<<<grid, kAppendWarps * 32, 0, stream>>>(static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
+    launch(k_append_fp4, dim3(grid), dim3(kAppendWarps * 32), 0, stream, static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
     return check_launch();
 }
 
@@ -217,6 +262,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     if (q_limit && !aligned(q_limit, 4)) return CSA2_ERR_INVALID_ARG;
     const FullLayout L = full_layout(nq, n_max);
     if (!ws || ws_bytes < L.total || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
 
     const int box_rows = std::min(128, (int)kv->page_size);
@@ -232,12 +278,15 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sp.kv = *kv;
     sp.keys = reinterpret_cast<uint32_t *>(wsb + L.off_keys);
     sp.hist0 = reinterpret_cast<uint32_t *>(wsb + L.off_hist0);
+    sp.state = reinterpret_cast<uint32_t *>(wsb + L.off_state);
+    sp.rank[0] = k;
+    sp.rank[1] = p;
     sp.key_stride = L.key_stride;
     sp.q_per_seq = q_per_seq;
     sp.hi = hi;
     sp.box_rows = box_rows;
     const int64_t tiles_max = std::max<int64_t>(1, (n_max + kScanTile - 1) / kScanTile);
-    const int64_t target = (int64_t)num_sms() * 4;
+    const int64_t target = (int64_t)num_sms() * 2;  // about two resident CTAs per SM, one wave
     int64_t chunk = std::max<int64_t>(4, ((int64_t)nq * tiles_max + target - 1) / target);
     chunk = std::min<int64_t>(chunk, 256);
     sp.chunk_tiles = (int32_t)chunk;
@@ -245,11 +294,11 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     if (kv->di == 64) {
         static bool ok = set_smem(k_index_scan<64>, ScanCfg<64>::kSmem);
         if (!ok) return CSA2_ERR_CUDA;
-        k_index_scan<64><<<sgrid, kScanThreads, ScanCfg<64>::kSmem, stream>>>(tm, sp);
+        launch(k_index_scan<64>, sgrid, dim3(kScanThreads), ScanCfg<64>::kSmem, stream, tm, sp);
     } else {
         static bool ok = set_smem(k_index_scan<128>, ScanCfg<128>::kSmem);
         if (!ok) return CSA2_ERR_CUDA;
-        k_index_scan<128><<<sgrid, kScanThreads, ScanCfg<128>::kSmem, stream>>>(tm, sp);
+        launch(k_index_scan<128>, sgrid, dim3(kScanThreads), ScanCfg<128>::kSmem, stream, tm, sp);
     }
     if ((st = check_launch()) != CSA2_OK) return st;
 
@@ -257,7 +306,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sel.keys = sp.keys;
     sel.q_limit = q_limit;
     sel.kv = *kv;
-    sel.hist0 = sp.hist0;
+    sel.state = sp.state;
     sel.hist1 = reinterpret_cast<uint32_t *>(wsb + L.off_hist1);
     sel.hist2 = reinterpret_cast<uint32_t *>(wsb + L.off_hist2);
     sel.cnt = reinterpret_cast<uint32_t *>(wsb + L.off_cnt);
@@ -269,10 +318,10 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sel.q_per_seq = q_per_seq;
     sel.n_chunks = L.n_sel_chunks;
     const dim3 grid((unsigned)L.n_sel_chunks, (unsigned)nq);
-    k_sel_hist<1><<<grid, kSelThreads, 0, stream>>>(sel);
-    k_sel_hist<2><<<grid, kSelThreads, 0, stream>>>(sel);
-    k_sel_count<<<grid, kSelThreads, 0, stream>>>(sel);
-    k_sel_emit<<<grid, kSelThreads, 0, stream>>>(sel);
+    launch(k_sel_hist<1>, dim3(grid), dim3(kSelThreads), 0, stream, sel);
+    launch(k_sel_hist<2>, dim3(grid), dim3(kSelThreads), 0, stream, sel);
+    launch(k_sel_count, dim3(grid), dim3(kSelThreads), 0, stream, sel);
+    launch(k_sel_emit, dim3(grid), dim3(kSelThreads), 0, stream, sel);
     return check_launch();
 }
 
@@ -296,6 +345,7 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
         return CSA2_ERR_INVALID_ARG;
     const size_t half = align_up((size_t)nq * p * 4, 256);
     if (!ws || ws_bytes < 2 * half || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
     ReindexParams rp{};
     rp.qidx = qidx;
     rp.w = w;
@@ -310,14 +360,14 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     rp.q_per_seq = q_per_seq;
     const dim3 grid((unsigned)((p + kReindexThreads - 1) / kReindexThreads), (unsigned)nq);
     if (kv->di == 64)
-        k_reindex_score<64><<<grid, kReindexThreads, 0, stream>>>(rp);
+        launch(k_reindex_score<64>, dim3(grid), dim3(kReindexThreads), 0, stream, rp);
     else
-        k_reindex_score<128><<<grid, kReindexThreads, 0, stream>>>(rp);
+        launch(k_reindex_score<128>, dim3(grid), dim3(kReindexThreads), 0, stream, rp);
     if ((st = check_launch()) != CSA2_OK) return st;
     const size_t smem = (size_t)p * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4;
     static bool ok = set_smem(k_reindex_select, (size_t)kReindexMaxPool * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4);
     if (!ok) return CSA2_ERR_CUDA;
-    k_reindex_select<<<nq, kReindexSelThreads, smem, stream>>>(rp);
+    launch(k_reindex_select, dim3(nq), dim3(kReindexSelThreads), smem, stream, rp);
     return check_launch();
 }
 
@@ -348,6 +398,7 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
     const AttnPlan P = plan_attn(nq, k, has_swa ? w_max : 0, num_sms());
     const AttnLayout L = attn_layout(nq, h, P);
     if (L.total > 0 && (!ws || ws_bytes < L.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
 
     AttnParams ap{};
     ap.q = static_cast<const uint16_t *>(q_bf16);
@@ -371,19 +422,19 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
         case 64: {
             static bool ok = set_smem(k_sparse_attn<64>, AttnCfg<64>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            k_sparse_attn<64><<<grid, kAttnThreads, AttnCfg<64>::kSmem, stream>>>(ap);
+            launch(k_sparse_attn<64>, grid, dim3(kAttnThreads), AttnCfg<64>::kSmem, stream, ap);
             break;
         }
         case 32: {
             static bool ok = set_smem(k_sparse_attn<32>, AttnCfg<32>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            k_sparse_attn<32><<<grid, kAttnThreads, AttnCfg<32>::kSmem, stream>>>(ap);
+            launch(k_sparse_attn<32>, grid, dim3(kAttnThreads), AttnCfg<32>::kSmem, stream, ap);
             break;
         }
         default: {
             static bool ok = set_smem(k_sparse_attn<16>, AttnCfg<16>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            k_sparse_attn<16><<<grid, kAttnThreads, AttnCfg<16>::kSmem, stream>>>(ap);
+            launch(k_sparse_attn<16>, grid, dim3(kAttnThreads), AttnCfg<16>::kSmem, stream, ap);
             break;
         }
     }
@@ -393,15 +444,15 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
         const size_t csmem = (size_t)(P.splits + 1) * 4;
         switch (h) {
             case 64:
-                k_attn_combine<64><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                launch(k_attn_combine<64>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
                                                                              P.splits);
                 break;
             case 32:
-                k_attn_combine<32><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                launch(k_attn_combine<32>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
                                                                              P.splits);
                 break;
             default:
-                k_attn_combine<16><<<cgrid, kCombineThreads, csmem, stream>>>(ap.o_part, ap.lse_part, ap.o, lse,
+                launch(k_attn_combine<16>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
                                                                              P.splits);
                 break;
         }

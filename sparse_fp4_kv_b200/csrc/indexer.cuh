@@ -59,12 +59,21 @@ struct ScanParams {
     csa2_kv_desc kv;
     uint32_t *keys;    // [nq][key_stride]
     uint32_t *hist0;   // [nq][4096]
+    uint32_t *state;   // [nq][kStateWords]
     int64_t key_stride;
     int32_t q_per_seq;
     int32_t hi;
     int32_t chunk_tiles;
     int32_t box_rows;
+    int32_t rank[2];   // k, p (0 = no pool)
 };
+
+// Per-query selection state, per target tau (0 = Top-k, 1 = pool):
+//   [8 tau + 0] digit-0 bin, [+1] rank left inside it, [+2] digit-1 bin,
+//   [+3] rank left, [+4] digit-2 bin, [+5] equal keys to take, [+6] key T
+// and counters of finished CTAs: [16] scan, [17] pass 1, [18] pass 2.
+constexpr int kStateWords = 32;
+constexpr int kCtrScan = 16;
 
 __device__ __forceinline__ int64_t query_limit(const int32_t *q_limit, const csa2_kv_desc &kv, int32_t qi,
                                                int32_t q_per_seq) {
@@ -88,6 +97,91 @@ __device__ __forceinline__ void hist_add_warp(uint32_t *hist, uint32_t bin) {
     if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
+// ---------------------------------------------------------------------------
+// Block-wide helpers for the selection kernels
+// ---------------------------------------------------------------------------
+// Exclusive prefix sum over the block (NT threads); scratch holds NT/32 + 1
+// words. Returns the exclusive prefix, *total gets the block sum.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratch, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < NT / 32 ? scratch[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < NT / 32) scratch[lane] = s;  // inclusive warp prefix
+        if (lane == NT / 32 - 1) scratch[NT / 32] = s;
+    }
+    __syncthreads();
+    const uint32_t warp_excl = warp ? scratch[warp - 1] : 0u;
+    const uint32_t res = warp_excl + x - v;
+    if (total) *total = scratch[NT / 32];
+    __syncthreads();
+    return res;
+}
+
+// Bins are ordered by key; the r-th largest key (r >= 1, r <= sum of the
+// histogram) lies in the bin b with above(b) < r <= above(b) + h[b], where
+// above(b) counts keys in bins > b. Returns b and r - above(b).
+// Thread i owns PER consecutive bins from the top (nbins <= NT * PER); its
+// loads are all issued before any is used. kGlobal: the histogram lives in
+// global memory (filled by other CTAs' atomics, read through L2) rather than
+// in this CTA's shared memory.
+template <int NT, int PER, bool kGlobal>
+__device__ __forceinline__ void find_rank_bin(const uint32_t *h, int nbins, uint32_t r, uint32_t *scratch,
+                                              uint32_t &bin, uint32_t &rank_in_bin) {
+    const int top = nbins - 1 - (int)threadIdx.x * PER;
+    uint32_t v[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const int b = top - j;
+        v[j] = b >= 0 ? (kGlobal ? __ldcg(h + b) : h[b]) : 0u;
+    }
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) sum += v[j];
+    const uint32_t excl = block_excl_scan<NT>(sum, scratch, nullptr);
+    if (excl < r && r <= excl + sum) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            if (acc < r && acc + v[j] >= r) {
+                scratch[NT / 32 + 1] = (uint32_t)(top - j);
+                scratch[NT / 32 + 2] = r - acc;
+            }
+            acc += v[j];
+        }
+    }
+    __syncthreads();
+    bin = scratch[NT / 32 + 1];
+    rank_in_bin = scratch[NT / 32 + 2];
+    __syncthreads();
+}
+
+// True in every thread of the CTA that is the last of n CTAs to arrive on
+// *counter; the global writes of all n CTAs are then visible to it. No CTA
+// waits for another.
+__device__ __forceinline__ bool last_block(uint32_t *counter, uint32_t n, uint32_t *flag_smem) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *flag_smem = (atomicAdd(counter, 1u) == n - 1) ? 1u : 0u;
+    __syncthreads();
+    const bool last = *flag_smem != 0u;
+    if (last) __threadfence();
+    return last;
+}
+
 template <int DI>
 __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
     using Cfg = ScanCfg<DI>;
@@ -105,6 +199,8 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t qi = blockIdx.y;
     const int32_t b = qi / p.q_per_seq;
+    pdl_trigger();
+    pdl_wait();
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
     const int64_t start = (int64_t)blockIdx.x * p.chunk_tiles * kScanTile;
     if (start >= limit) return;
@@ -219,115 +315,71 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
         tc_fence_after();
         tmem_dealloc(tmem, 32);
     }
-}
-
-// ---------------------------------------------------------------------------
-// Block-wide helpers for the selection kernels
-// ---------------------------------------------------------------------------
-// Exclusive prefix sum over the block (NT threads); scratch holds NT/32 + 1
-// words. Returns the exclusive prefix, *total gets the block sum.
-template <int NT>
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratch, uint32_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t s = lane < NT / 32 ? scratch[lane] : 0u;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, s, o);
-            if (lane >= o) s += y;
-        }
-        if (lane < NT / 32) scratch[lane] = s;  // inclusive warp prefix
-        if (lane == NT / 32 - 1) scratch[NT / 32] = s;
-    }
-    __syncthreads();
-    const uint32_t warp_excl = warp ? scratch[warp - 1] : 0u;
-    const uint32_t res = warp_excl + x - v;
-    if (total) *total = scratch[NT / 32];
-    __syncthreads();
-    return res;
-}
-
-// Bins are ordered by key; the r-th largest key (r >= 1, r <= sum of the
-// histogram) lies in the bin b with above(b) < r <= above(b) + h[b], where
-// above(b) counts keys in bins > b. Returns b and r - above(b).
-template <int NT>
-__device__ __forceinline__ void find_rank_bin(const uint32_t *h, int nbins, uint32_t r, uint32_t *scratch,
-                                              uint32_t &bin, uint32_t &rank_in_bin) {
-    const int per = nbins / NT;
-    const int top = nbins - 1 - (int)threadIdx.x * per;  // this thread: bins top, top-1, ...
-    uint32_t sum = 0;
-    for (int j = 0; j < per; ++j) sum += h[top - j];
-    const uint32_t excl = block_excl_scan<NT>(sum, scratch, nullptr);
-    if (excl < r && r <= excl + sum) {
-        uint32_t acc = excl;
-        for (int j = 0; j < per; ++j) {
-            const uint32_t c = h[top - j];
-            if (acc + c >= r) {
-                scratch[NT / 32 + 1] = (uint32_t)(top - j);
-                scratch[NT / 32 + 2] = r - acc;
-                break;
+    // the last CTA of this query locates the digit-0 bin of each target rank
+    const int64_t chunk = (int64_t)p.chunk_tiles * kScanTile;
+    uint32_t *scratch = hist;  // the shared histogram is no longer needed
+    if (last_block(&p.state[(int64_t)qi * kStateWords + kCtrScan], (uint32_t)((limit + chunk - 1) / chunk),
+                   scratch + 64)) {
+        for (int tau = 0; tau < 2; ++tau) {
+            const int64_t r = p.rank[tau];
+            if (r <= 0 || r >= limit) continue;
+            uint32_t bin, rem;
+            find_rank_bin<kScanThreads, (kHist0Bins + kScanThreads - 1) / kScanThreads, true>(p.hist0 + (int64_t)qi * kHist0Bins, kHist0Bins, (uint32_t)r, scratch, bin,
+                                        rem);
+            if (tid == 0) {
+                p.state[(int64_t)qi * kStateWords + 8 * tau + 0] = bin;
+                p.state[(int64_t)qi * kStateWords + 8 * tau + 1] = rem;
             }
-            acc += c;
         }
     }
-    __syncthreads();
-    bin = scratch[NT / 32 + 1];
-    rank_in_bin = scratch[NT / 32 + 2];
-    __syncthreads();
 }
 
 struct SelParams {
     const uint32_t *keys;
     const int32_t *q_limit;
     csa2_kv_desc kv;
-    const uint32_t *hist0;  // [nq][4096]
-    uint32_t *hist1;        // [nq][2][1024]
-    uint32_t *hist2;        // [nq][2][1024]
-    uint32_t *cnt;          // [nq][2][n_chunks][2]
-    int32_t *out[2];        // topk [nq][k], pool [nq][p]
-    int32_t rank[2];        // k, p (0 = no pool)
+    uint32_t *hist1;  // [nq][2][1024]
+    uint32_t *hist2;  // [nq][2][1024]
+    uint32_t *cnt;    // [nq][2][n_chunks][2]
+    uint32_t *state;  // [nq][kStateWords]
+    int32_t *out[2];  // topk [nq][k], pool [nq][p]
+    int32_t rank[2];  // k, p (0 = no pool)
     int64_t key_stride;
     int32_t q_per_seq;
     int32_t n_chunks;
 };
 
-// Threshold state of one target (rank r) of one query after `digits` digits.
-struct SelTarget {
-    bool active;      // r < number of visible entries (else everything is taken)
-    uint32_t b0, b1, b2, need;  // digit bins and the rank left inside the last bin
-};
-
-template <int DIGITS>
-__device__ __forceinline__ SelTarget sel_target(const SelParams &p, int32_t qi, int tau, int64_t limit,
-                                                uint32_t *scratch) {
-    SelTarget st{};
-    const int64_t r = p.rank[tau];
-    st.active = r > 0 && r < limit;
-    if (!st.active) return st;
-    uint32_t rem = (uint32_t)r;
-    find_rank_bin<kSelThreads>(p.hist0 + (int64_t)qi * kHist0Bins, kHist0Bins, rem, scratch, st.b0, rem);
-    if (DIGITS >= 2)
-        find_rank_bin<kSelThreads>(p.hist1 + ((int64_t)qi * 2 + tau) * kHistBins, kHistBins, rem, scratch, st.b1,
-                                   rem);
-    if (DIGITS >= 3)
-        find_rank_bin<kSelThreads>(p.hist2 + ((int64_t)qi * 2 + tau) * kHistBins, kHistBins, rem, scratch, st.b2,
-                                   rem);
-    st.need = rem;
-    return st;
+// A target needs a threshold only when fewer than all visible entries are
+// asked for; otherwise every visible entry is taken.
+__device__ __forceinline__ bool sel_active(const SelParams &p, int tau, int64_t limit) {
+    return p.rank[tau] > 0 && (int64_t)p.rank[tau] < limit;
 }
 
-// PASS 1: histogram of digit 1 (bits 19..10) among keys whose digit 0
-// matches; PASS 2: digit 2 (bits 9..0) among keys matching digits 0 and 1.
+// The kSelPer consecutive keys t0 .. t0+kSelPer-1 of this thread (64-byte
+// aligned; keys at or beyond `end` read as 0 and must be masked by the
+// caller), loaded with four 16-byte loads in flight together.
+__device__ __forceinline__ void load_key_slice(const uint32_t *keys, int64_t t0, int64_t end,
+                                               uint32_t (&k)[kSelPer]) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(keys + t0);
+    uint4 v[kSelPer / 4];
+#pragma unroll
+    for (int i = 0; i < kSelPer / 4; ++i) v[i] = t0 + 4 * i < end ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int i = 0; i < kSelPer / 4; ++i) {
+        k[4 * i + 0] = v[i].x;
+        k[4 * i + 1] = v[i].y;
+        k[4 * i + 2] = v[i].z;
+        k[4 * i + 3] = v[i].w;
+    }
+}
+
+// PASS 1: histogram of digit 1 (bits 19..10) among keys whose digit 0 is the
+// threshold bin; PASS 2: digit 2 (bits 9..0) among keys matching digits 0
+// and 1. The last CTA of each query then locates the next threshold digit.
 template <int PASS>
 __global__ void __launch_bounds__(kSelThreads) k_sel_hist(SelParams p) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ uint32_t nh[2][kHistBins];
     __shared__ uint32_t scratch[kSelThreads / 32 + 4];
     const int32_t qi = blockIdx.y;
@@ -335,50 +387,83 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_hist(SelParams p) {
     const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
     if (c0 >= limit) return;
     const int64_t c1 = min(limit, c0 + kSelChunk);
-    SelTarget st[2];
-    for (int tau = 0; tau < 2; ++tau) st[tau] = sel_target<PASS>(p, qi, tau, limit, scratch);
-    if (!st[0].active && !st[1].active) return;
+    const uint32_t *st = p.state + (int64_t)qi * kStateWords;
+    bool act[2];
+    uint32_t b0[2], b1[2];
+    for (int tau = 0; tau < 2; ++tau) {
+        act[tau] = sel_active(p, tau, limit);
+        b0[tau] = act[tau] ? __ldcg(st + 8 * tau + 0) : 0u;
+        b1[tau] = act[tau] ? __ldcg(st + 8 * tau + 2) : 0u;
+    }
+    if (!act[0] && !act[1]) return;
     for (int i = threadIdx.x; i < 2 * kHistBins; i += kSelThreads) (&nh[0][0])[i] = 0u;
     __syncthreads();
     const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
-    for (int64_t t = c0 + threadIdx.x; t < c1; t += kSelThreads) {
-        const uint32_t key = keys[t];
+    const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
+    uint32_t kreg[kSelPer];
+    load_key_slice(keys, s0, c1, kreg);
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+        const uint32_t key = kreg[j];
+        const bool in = s0 + j < c1;
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
-            if (!st[tau].active || (key >> 20) != st[tau].b0) continue;
-            if (PASS == 1) {
-                atomicAdd(&nh[tau][(key >> 10) & 1023u], 1u);
-            } else if (((key >> 10) & 1023u) == st[tau].b1) {
-                atomicAdd(&nh[tau][key & 1023u], 1u);
-            }
+            if (!act[tau]) continue;
+            bool match = in && (key >> 20) == b0[tau];
+            if (PASS == 2) match = match && ((key >> 10) & 1023u) == b1[tau];
+            hist_add_warp(nh[tau], match ? (PASS == 1 ? (key >> 10) & 1023u : key & 1023u) : 0xFFFFFFFFu);
         }
     }
     __syncthreads();
-    uint32_t *dst = PASS == 1 ? p.hist1 : p.hist2;
+    uint32_t *dst = (PASS == 1 ? p.hist1 : p.hist2) + (int64_t)qi * 2 * kHistBins;
     for (int i = threadIdx.x; i < 2 * kHistBins; i += kSelThreads) {
         const uint32_t v = (&nh[0][0])[i];
-        if (v) atomicAdd(&dst[(int64_t)qi * 2 * kHistBins + i], v);
+        if (v) atomicAdd(&dst[i], v);
+    }
+    const uint32_t n_part = (uint32_t)((limit + kSelChunk - 1) / kSelChunk);
+    if (last_block(p.state + (int64_t)qi * kStateWords + kCtrScan + PASS, n_part, scratch + kSelThreads / 32 + 3)) {
+        uint32_t *stw = p.state + (int64_t)qi * kStateWords;
+        for (int tau = 0; tau < 2; ++tau) {
+            if (!act[tau]) continue;
+            const uint32_t r = __ldcg(stw + 8 * tau + (PASS == 1 ? 1 : 3));
+            uint32_t bin, rem;
+            find_rank_bin<kSelThreads, kHistBins / kSelThreads, true>(dst + tau * kHistBins, kHistBins, r, scratch, bin, rem);
+            if (threadIdx.x == 0) {
+                if (PASS == 1) {
+                    stw[8 * tau + 2] = bin;
+                    stw[8 * tau + 3] = rem;
+                } else {
+                    stw[8 * tau + 4] = bin;
+                    stw[8 * tau + 5] = rem;
+                    stw[8 * tau + 6] = (b0[tau] << 20) | (b1[tau] << 10) | bin;
+                }
+            }
+        }
     }
 }
 
 // Counts, per chunk, the keys above and equal to each target's threshold.
 __global__ void __launch_bounds__(kSelThreads) k_sel_count(SelParams p) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ uint32_t scratch[kSelThreads / 32 + 4];
     const int32_t qi = blockIdx.y;
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
     const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
     const int64_t c1 = min(limit, c0 + kSelChunk);
-    SelTarget st[2];
-    for (int tau = 0; tau < 2; ++tau) st[tau] = sel_target<3>(p, qi, tau, limit, scratch);
     const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
+    const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
+    uint32_t kreg[kSelPer];
+    if (sel_active(p, 0, limit) || sel_active(p, 1, limit)) load_key_slice(keys, s0, c1, kreg);
     for (int tau = 0; tau < 2; ++tau) {
-        if (!st[tau].active) continue;
-        const uint32_t T = (st[tau].b0 << 20) | (st[tau].b1 << 10) | st[tau].b2;
+        if (!sel_active(p, tau, limit)) continue;
+        const uint32_t T = __ldcg(p.state + (int64_t)qi * kStateWords + 8 * tau + 6);
         uint32_t gt = 0, eq = 0;
-        for (int64_t t = c0 + threadIdx.x; t < c1; t += kSelThreads) {
-            const uint32_t key = keys[t];
-            gt += key > T;
-            eq += key == T;
+#pragma unroll
+        for (int j = 0; j < kSelPer; ++j) {
+            const bool in = s0 + j < c1;
+            gt += in && kreg[j] > T;
+            eq += in && kreg[j] == T;
         }
         uint32_t tgt, teq;
         block_excl_scan<kSelThreads>(gt, scratch, &tgt);
@@ -393,19 +478,18 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_count(SelParams p) {
 
 // Writes the selected ids of each target in ascending id order.
 __global__ void __launch_bounds__(kSelThreads) k_sel_emit(SelParams p) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ uint32_t scratch[kSelThreads / 32 + 4];
     const int32_t qi = blockIdx.y;
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
     const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
     const int64_t c1 = min(limit, c0 + kSelChunk);
-    SelTarget st[2];
-    for (int tau = 0; tau < 2; ++tau) st[tau] = sel_target<3>(p, qi, tau, limit, scratch);
     const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
     // this thread's contiguous slice of the chunk
     const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
     uint32_t kreg[kSelPer];
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j) kreg[j] = (s0 + j < c1) ? keys[s0 + j] : 0u;
+    load_key_slice(keys, s0, c1, kreg);
     for (int tau = 0; tau < 2; ++tau) {
         const int32_t r_out = p.rank[tau];
         if (r_out <= 0 || p.out[tau] == nullptr) continue;
@@ -414,20 +498,21 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_emit(SelParams p) {
             const int64_t nsel = min((int64_t)r_out, limit);
             for (int64_t j = nsel + threadIdx.x; j < r_out; j += kSelThreads) out[j] = -1;
         }
-        if (!st[tau].active) {
-            // fewer visible entries than requested: take every visible entry
+        if (!sel_active(p, tau, limit)) {
+            // no more visible entries than requested: take every visible entry
             for (int j = 0; j < kSelPer; ++j)
                 if (s0 + j < c1) out[s0 + j] = (int32_t)(s0 + j);
             continue;
         }
-        const uint32_t T = (st[tau].b0 << 20) | (st[tau].b1 << 10) | st[tau].b2;
-        const uint32_t need = st[tau].need;
+        const uint32_t *st = p.state + (int64_t)qi * kStateWords + 8 * tau;
+        const uint32_t T = __ldcg(st + 6);
+        const uint32_t need = __ldcg(st + 5);
         // counts of the chunks before this one
         const uint32_t *cnt = p.cnt + ((int64_t)qi * 2 + tau) * p.n_chunks * 2;
         uint32_t bgt = 0, beq = 0;
         for (int c = threadIdx.x; c < (int)blockIdx.x; c += kSelThreads) {
-            bgt += cnt[2 * c];
-            beq += cnt[2 * c + 1];
+            bgt += __ldcg(cnt + 2 * c);
+            beq += __ldcg(cnt + 2 * c + 1);
         }
         uint32_t base_gt, base_eq;
         block_excl_scan<kSelThreads>(bgt, scratch, &base_gt);
@@ -481,6 +566,8 @@ struct ReindexParams {
 
 template <int DI>
 __global__ void __launch_bounds__(kReindexThreads) k_reindex_score(ReindexParams p) {
+    pdl_trigger();
+    pdl_wait();
     __shared__ float qf[kScanN][DI];
     __shared__ float wf[kScanN];
     const int32_t qi = blockIdx.y;
@@ -534,6 +621,8 @@ __global__ void __launch_bounds__(kReindexThreads) k_reindex_score(ReindexParams
 // (score key << 32 | ~id) among the valid pool entries, emitted in pool
 // order.
 __global__ void __launch_bounds__(kReindexSelThreads) k_reindex_select(ReindexParams p) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ uint8_t smem_raw[];
     uint64_t *k64 = reinterpret_cast<uint64_t *>(smem_raw);   // [p]
     uint32_t *hist = reinterpret_cast<uint32_t *>(k64 + p.p); // [2048]
@@ -557,27 +646,48 @@ __global__ void __launch_bounds__(kReindexSelThreads) k_reindex_select(ReindexPa
     const uint32_t r = min((uint32_t)p.k, nvalid);
     uint64_t T = 0;  // select valid keys >= T
     if (nvalid > (uint32_t)p.k) {
-        uint64_t prefix = 0, pmask = 0;
+        // bits every valid key shares need no radix pass: start at the highest
+        // bit in which two keys differ
+        __shared__ unsigned long long and_acc, or_acc;
+        if (threadIdx.x == 0) {
+            and_acc = ~0ull;
+            or_acc = 0ull;
+        }
+        __syncthreads();
+        unsigned long long a = ~0ull, o = 0ull;
+        for (int j = threadIdx.x; j < p.p; j += NT)
+            if (ids[j] >= 0) {
+                a &= k64[j];
+                o |= k64[j];
+            }
+        atomicAnd(&and_acc, a);
+        atomicOr(&or_acc, o);
+        __syncthreads();
+        const unsigned long long diff = and_acc ^ or_acc;  // nonzero: keys are unique
+        const int hb = 63 - __clzll((long long)diff);
+        uint64_t prefix = hb == 63 ? 0ull : (and_acc & ~((1ull << (hb + 1)) - 1ull));
+        uint64_t pmask = hb == 63 ? 0ull : ~((1ull << (hb + 1)) - 1ull);
         uint32_t rem = r;
-        const int shifts[6] = {53, 42, 31, 20, 10, 0};
-        const int bits[6] = {11, 11, 11, 11, 10, 10};
-        for (int ps = 0; ps < 6; ++ps) {
-            const int nb = 1 << bits[ps];
+        for (int top = hb; top >= 0; top -= 11) {
+            const int nbits = top + 1 < 11 ? top + 1 : 11;
+            const int shift = top + 1 - nbits;
+            const int nb = 1 << nbits;
             for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
             __syncthreads();
             for (int j = threadIdx.x; j < p.p; j += NT) {
                 const uint64_t v = k64[j];
                 if (ids[j] >= 0 && (v & pmask) == prefix)
-                    atomicAdd(&hist[(uint32_t)(v >> shifts[ps]) & (uint32_t)(nb - 1)], 1u);
+                    atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
             }
             __syncthreads();
             uint32_t bin, inbin;
-            find_rank_bin<NT>(hist, nb, rem, scratch, bin, inbin);
-            prefix |= (uint64_t)bin << shifts[ps];
-            pmask |= (uint64_t)(nb - 1) << shifts[ps];
+            find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
+            prefix |= (uint64_t)bin << shift;
+            pmask |= (uint64_t)(nb - 1) << shift;
             rem = inbin;
-            if (hist[bin] == rem) break;  // every key of this bin is taken
+            const bool all_taken = hist[bin] == rem;  // every key of this bin is taken
             __syncthreads();
+            if (all_taken) break;
         }
         T = prefix;
         __syncthreads();
