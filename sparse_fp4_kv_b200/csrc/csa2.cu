@@ -6,7 +6,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <numeric>
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 #include <cstdint>
 #include <mutex>
 #include <utility>
@@ -14,6 +17,7 @@
 #include "append.cuh"
 #include "attention.cuh"
 #include "indexer.cuh"
+#include "indexer_fused.cuh"
 
 using namespace csa2;
 
@@ -24,6 +28,23 @@ constexpr int32_t kVersion = 100;  // 0.1.0
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int max_smem_optin() {
+    int dev = 0, n = 232448;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    return n;
+}
+
+// CSA2_FULL_PATH=multipass forces the multi-launch Full indexer even where the
+// single-launch cluster path applies (both are complete implementations; the
+// switch lets tests exercise both at small sizes).
+bool force_multipass() {
+    static const bool v = [] {
+        const char *e = std::getenv("CSA2_FULL_PATH");
+        return e != nullptr && std::strcmp(e, "multipass") == 0;
+    }();
+    return v;
+}
 
 int num_sms() {
     int dev = 0, n = 148;
@@ -50,6 +71,7 @@ csa2_status check_kv(const csa2_kv_desc *kv, bool need_kidx) {
     if (need_kidx) {
         if (!kv->kidx || !aligned(kv->kidx, 16)) return CSA2_ERR_INVALID_ARG;
         if (kv->di != 64 && kv->di != 128) return CSA2_ERR_UNSUPPORTED;
+        if ((kv->rows_cap * kv->di) % 128 != 0) return CSA2_ERR_UNSUPPORTED;  // keys are read as 128-byte rows
     }
     return CSA2_OK;
 }
@@ -73,14 +95,16 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// The indexer keys viewed as 128-byte rows (two entries per row when di is 64),
+// loaded as boxes of box_rows rows with the 128B swizzle.
 bool make_kidx_map(CUtensorMap *tm, const csa2_kv_desc *kv, int box_rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kv->di, (cuuint64_t)kv->rows_cap};
-    const cuuint64_t strides[1] = {(cuuint64_t)kv->di};
-    const cuuint32_t box[2] = {(cuuint32_t)kv->di, (cuuint32_t)box_rows};
+    const cuuint64_t dims[2] = {128, (cuuint64_t)(kv->rows_cap * kv->di / 128)};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapSwizzle sw = kv->di == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(kv->kidx), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -156,11 +180,23 @@ AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P) {
 // Dynamic shared memory limit of a kernel, and the maximal shared-memory
 // carveout, which every kernel of the library requests so that consecutive
 // launches do not change the L1 / shared split of the SMs.
+// `bytes` is capped at the opt-in maximum minus the kernel's static shared
+// memory. A failed attribute call is cleared from the runtime's last error.
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess &&
-           cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    const size_t cap = (size_t)max_smem_optin() - fa.sharedSizeBytes;
+    const bool ok =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)std::min(bytes, cap)) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    return ok;
 }
 
 // Launch with programmatic dependent launch allowed: the kernel may start
@@ -180,6 +216,27 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Same, as a thread-block cluster of `cluster` CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                           unsigned cluster, Args &&...args) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -265,9 +322,55 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
 
-    const int box_rows = std::min(128, (int)kv->page_size);
+    const int epr = 128 / kv->di;                                  // entries per 128-byte row
+    // rows per TMA box: a box holds gcd(page_size, tile) entries, so it never crosses a page
+    const int box_rows = std::gcd((int)kv->page_size, 128 * epr) / epr;
+    const int tile_entries = 128 * epr;
     CUtensorMap tm;
     if (!make_kidx_map(&tm, kv, box_rows)) return CSA2_ERR_CUDA;
+
+    // Single launch: one cluster of kFusedCluster CTAs per query, every score
+    // kept in shared memory, when a query's entries fit.
+    {
+        const int64_t slice = (int64_t)align_up(
+            (size_t)((std::max<int64_t>(n_max, 1) + kFusedCluster - 1) / kFusedCluster), (size_t)tile_entries);
+        const size_t stage_bytes = 128 * 128;
+        const size_t fixed = (kv->di == 64 ? FusedCfg<64>::kFixed : FusedCfg<128>::kFixed) + 64 * 8 + 16;
+        const size_t budget = (size_t)max_smem_optin();
+        int stages = 0;
+        if (fixed + (size_t)slice * 4 < budget) stages = (int)std::min<size_t>(16, (budget - fixed - slice * 4) / stage_bytes);
+        const bool pages_fit = slice / kv->page_size + 2 <= kMaxScanPages;
+        if (stages >= 3 && pages_fit && !force_multipass()) {
+            FusedParams fp{};
+            fp.qidx = qidx;
+            fp.w = w;
+            fp.q_limit = q_limit;
+            fp.kv = *kv;
+            fp.out[0] = topk;
+            fp.out[1] = pool;
+            fp.rank[0] = k;
+            fp.rank[1] = p;
+            fp.q_per_seq = q_per_seq;
+            fp.hi = hi;
+            fp.box_rows = box_rows;
+            fp.slice = (int32_t)slice;
+            fp.stages = stages;
+            const dim3 fgrid(kFusedCluster, (unsigned)nq);
+            if (kv->di == 64) {
+                const size_t smem = FusedCfg<64>::smem((int)slice, stages);
+                static bool ok = set_smem(k_index_full_fused<64>, (size_t)max_smem_optin());
+                if (!ok) return CSA2_ERR_CUDA;
+                launch_cluster(k_index_full_fused<64>, fgrid, dim3(kFusedThreads), smem, stream, kFusedCluster, tm, fp);
+            } else {
+                const size_t smem = FusedCfg<128>::smem((int)slice, stages);
+                static bool ok = set_smem(k_index_full_fused<128>, (size_t)max_smem_optin());
+                if (!ok) return CSA2_ERR_CUDA;
+                launch_cluster(k_index_full_fused<128>, fgrid, dim3(kFusedThreads), smem, stream, kFusedCluster, tm,
+                               fp);
+            }
+            return check_launch();
+        }
+    }
 
     if (cudaMemsetAsync(wsb + L.off_hist0, 0, L.off_cnt - L.off_hist0, stream) != cudaSuccess) return CSA2_ERR_CUDA;
 
@@ -285,10 +388,11 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sp.q_per_seq = q_per_seq;
     sp.hi = hi;
     sp.box_rows = box_rows;
-    const int64_t tiles_max = std::max<int64_t>(1, (n_max + kScanTile - 1) / kScanTile);
+    const int64_t tiles_max = std::max<int64_t>(1, (n_max + tile_entries - 1) / tile_entries);
     const int64_t target = (int64_t)num_sms() * 2;  // about two resident CTAs per SM, one wave
     int64_t chunk = std::max<int64_t>(4, ((int64_t)nq * tiles_max + target - 1) / target);
     chunk = std::min<int64_t>(chunk, 256);
+    chunk = std::min<int64_t>(chunk, std::max<int64_t>(1, ((int64_t)(kMaxScanPages - 2) * kv->page_size) / tile_entries));
     sp.chunk_tiles = (int32_t)chunk;
     const dim3 sgrid((unsigned)((tiles_max + chunk - 1) / chunk), (unsigned)nq);
     if (kv->di == 64) {
@@ -327,7 +431,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
 
 size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p) {
     if (nq <= 0 || p <= 0) return 0;
-    return align_up((size_t)nq * p * 4, 256) * 2;
+    return align_up((size_t)nq * p * 8, 256);
 }
 
 csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq, int32_t hi,
@@ -343,31 +447,29 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     if (!qidx || !w || !pool || !topk || !aligned(qidx, 16) || !aligned(w, 4) || !aligned(pool, 4) ||
         !aligned(topk, 4))
         return CSA2_ERR_INVALID_ARG;
-    const size_t half = align_up((size_t)nq * p * 4, 256);
-    if (!ws || ws_bytes < 2 * half || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+    if (!ws || ws_bytes < csa2_index_reindex_workspace_size(nq, p) || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
     ReindexParams rp{};
     rp.qidx = qidx;
     rp.w = w;
     rp.pool = pool;
     rp.kv = *kv;
-    rp.keys = static_cast<uint32_t *>(ws);
-    rp.ids = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + half);
+    rp.k64 = static_cast<unsigned long long *>(ws);
     rp.topk = topk;
     rp.p = p;
     rp.k = k;
     rp.hi = hi;
     rp.q_per_seq = q_per_seq;
-    const dim3 grid((unsigned)((p + kReindexThreads - 1) / kReindexThreads), (unsigned)nq);
+    const dim3 grid((unsigned)((p + kReindexScoreThreads - 1) / kReindexScoreThreads), (unsigned)nq);
     if (kv->di == 64)
-        launch(k_reindex_score<64>, dim3(grid), dim3(kReindexThreads), 0, stream, rp);
+        launch(k_reindex_score<64>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
     else
-        launch(k_reindex_score<128>, dim3(grid), dim3(kReindexThreads), 0, stream, rp);
+        launch(k_reindex_score<128>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
     if ((st = check_launch()) != CSA2_OK) return st;
-    const size_t smem = (size_t)p * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4;
-    static bool ok = set_smem(k_reindex_select, (size_t)kReindexMaxPool * 8 + 2048 * 4 + (kReindexSelThreads / 32 + 4) * 4);
+    const size_t smem = 2048 * 4 + (kReindexSelectThreads / 32 + 8) * 4 + (size_t)p * 8;
+    static bool ok = set_smem(k_reindex_select, (size_t)max_smem_optin());
     if (!ok) return CSA2_ERR_CUDA;
-    launch(k_reindex_select, dim3(nq), dim3(kReindexSelThreads), smem, stream, rp);
+    launch(k_reindex_select, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
     return check_launch();
 }
 

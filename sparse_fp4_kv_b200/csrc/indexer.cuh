@@ -25,8 +25,8 @@
 // Selection: exact radix select on the 32-bit key in three digits
 // (12 + 10 + 10 bits) with global histograms, then an ordered emission in
 // which equal keys are taken in ascending id order, so the output lists are
-// sorted by id. Reindex keeps (key, id) pairs of one pool in shared memory
-// and selects on the 64-bit key (score key, ~id), which is unique.
+// sorted by id. Reindex (indexer_fused.cuh) keeps the pool's 64-bit keys
+// (score key, ~id), which are unique, in shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -42,14 +42,28 @@ constexpr int kSelThreads = 512;
 constexpr int kSelChunk = 8192;  // entries per selection CTA
 constexpr int kSelPer = kSelChunk / kSelThreads;
 
+// Scan geometry. The indexer keys reach the tensor cores as 128-byte
+// shared-memory rows (128B swizzle). With di = 64 a row holds two
+// consecutive entries (kEpr = 2): the B operand carries two copies of the
+// query heads, [q_h | 0] in rows 0..15 and [0 | q_h] in rows 16..31, so
+// output column h scores a row's first entry and column 16 + h its second.
+// TMA then moves 128-byte rows, which it does at full speed. With di = 128
+// a row is one entry (kEpr = 1). A tile is 128 rows (256 or 128 entries).
+template <int DI>
+struct ScanGeom {
+    static constexpr int kEpr = 128 / DI;
+    static constexpr int kTile = 128 * kEpr;     // entries per tile
+    static constexpr int kN = kScanN * kEpr;     // MMA N
+    static constexpr int kStageBytes = 128 * 128;
+    static constexpr int kQBytes = kN * 128;     // B operand tile
+};
+
 template <int DI>
 struct ScanCfg {
-    static constexpr int kStages = DI == 64 ? 6 : 4;
-    static constexpr int kStageBytes = kScanTile * DI;
-    static constexpr uint32_t kSwizzle = DI == 64 ? kSw64 : kSw128;
-    static constexpr int kQBytes = kScanN * DI;
-    static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStageBytes + 2048 /*q tile*/ +
-                                    kHist0Bins * 4 + 256 /*barriers + tmem slot*/;
+    static constexpr int kStages = 4;
+    static constexpr int kStageBytes = ScanGeom<DI>::kStageBytes;
+    static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStageBytes + 4096 /*q tile*/ +
+                                    kHist0Bins * 4 + 256 /*barriers + tmem slot*/ + 4 * 2048 /*page table*/;
 };
 
 struct ScanParams {
@@ -81,13 +95,24 @@ __device__ __forceinline__ int64_t query_limit(const int32_t *q_limit, const csa
     return lim < 0 ? 0 : lim;
 }
 
-// Byte offset of 16-byte chunk c of row r inside a K-major swizzled tile
-// whose rows are DI bytes (DI = 64: 64B swizzle, DI = 128: 128B swizzle).
+// Build the B operand (query heads, K-major, 128B swizzle) of one query:
+// kN rows of 128 bytes (see ScanGeom), zero where no head.
 template <int DI>
-__device__ __forceinline__ uint32_t kmajor_chunk_offset(int r, int c) {
-    const int rr = r & 7;
-    const int sw = DI == 128 ? rr : ((rr >> 1) & 3);
-    return (uint32_t)((r >> 3) * (8 * DI) + rr * DI + ((c ^ sw) << 4));
+__device__ __forceinline__ void build_q_tile(uint8_t *qt, const uint8_t *q /*[hi][DI]*/, int hi, int nthreads) {
+    using G = ScanGeom<DI>;
+    for (int i = threadIdx.x; i < G::kN * 8; i += nthreads) {
+        const int r = i / 8, c = i % 8;
+        const int h = r % kScanN, half = r / kScanN;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (h < hi) {
+            if (DI == 128) {
+                v = *reinterpret_cast<const uint4 *>(q + h * DI + c * 16);
+            } else if (c / 4 == half) {
+                v = *reinterpret_cast<const uint4 *>(q + h * DI + (c % 4) * 16);
+            }
+        }
+        *reinterpret_cast<uint4 *>(qt + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
 }
 
 // Warp-aggregated shared-memory histogram increment (bin 0xFFFFFFFF = skip).
@@ -182,6 +207,141 @@ __device__ __forceinline__ bool last_block(uint32_t *counter, uint32_t n, uint32
     return last;
 }
 
+// ---------------------------------------------------------------------------
+// Scan pipeline pieces shared by the multi-launch and the cluster Full paths.
+// The MMA thread commits kScanBatch tiles at a time into one of two
+// kScanBatch*16-column TMEM buffers, so the epilogue pays one barrier
+// round trip per kScanBatch tiles.
+// ---------------------------------------------------------------------------
+constexpr int kScanBatch = 4;
+
+// Page-table entries of the pages that hold entries [start, start + n) of
+// sequence b, staged in shared memory by the whole CTA so that the TMA
+// producer never waits on a global load (entries outside the table read -1).
+constexpr int kMaxScanPages = 2048;
+__device__ __forceinline__ int stage_pages(const csa2_kv_desc &kv, int32_t b, int64_t start, int64_t n,
+                                           int32_t *ptab, int nthreads) {
+    if (n <= 0) return 0;
+    const int64_t pg0 = start / kv.page_size;
+    const int npg = (int)((start + n - 1) / kv.page_size - pg0 + 1);
+    for (int i = threadIdx.x; i < npg && i < kMaxScanPages; i += nthreads) {
+        const int64_t pg = pg0 + i;
+        ptab[i] = pg < kv.max_pages ? kv.page_table[(int64_t)b * kv.max_pages + pg] : -1;
+    }
+    return npg;
+}
+
+// TMA producer: tile i = 128 smem rows = kTile entries, loaded as boxes of
+// box_rows rows (a box never crosses a page). Boxes whose first entry is past
+// the limit are skipped (their rows are not read). Physical rows come from
+// the staged page-table entries.
+template <int DI>
+__device__ __forceinline__ void scan_tma_loop(const csa2_kv_desc &kv, const int32_t *ptab, int64_t start,
+                                              int64_t limit, int ntiles, int nstages, int box_rows,
+                                              uint8_t *stage_base, const CUtensorMap *tm, uint64_t *full_b,
+                                              uint64_t *empty_b) {
+    using G = ScanGeom<DI>;
+    const int nbox = 128 / box_rows;
+    const int64_t ps = kv.page_size;
+    const int64_t pg0 = start / ps;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % nstages;
+        if (!mbar_wait(&empty_b[s], ((i / nstages) & 1) ^ 1)) return;
+        const int64_t t0 = start + (int64_t)i * G::kTile;
+        int nvalid = 0;
+        for (int j = 0; j < nbox; ++j) nvalid += (t0 + (int64_t)j * box_rows * G::kEpr < limit);
+        mbar_arrive_expect_tx(&full_b[s], (uint32_t)(nvalid * box_rows * 128));
+        for (int j = 0; j < nvalid; ++j) {
+            const int64_t t = t0 + (int64_t)j * box_rows * G::kEpr;
+            const int64_t pi = t / ps - pg0;
+            const int64_t phys = pi < kMaxScanPages ? ptab[pi] : -1;
+            int64_t row = phys * ps + (t % ps);
+            if (phys < 0 || row + (int64_t)box_rows * G::kEpr > kv.rows_cap) {
+                set_error(CSA2_DEVERR_BAD_ROW);
+                row = 0;
+            }
+            tma_load_2d(stage_base + (size_t)s * G::kStageBytes + j * box_rows * 128, tm, &full_b[s], 0,
+                        (int32_t)(row / G::kEpr));
+        }
+    }
+}
+
+template <int DI>
+__device__ __forceinline__ void scan_mma_loop(int ntiles, int nstages, const uint8_t *stage_base, uint32_t qaddr,
+                                              uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
+                                              uint64_t *tempty, uint32_t tmem) {
+    using G = ScanGeom<DI>;
+    const uint32_t idesc = idesc_e4m3_f32(128, G::kN);
+    const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
+    for (int g = 0; g < nbatch; ++g) {
+        const int a = g & 1;
+        if (!mbar_wait(&tempty[a], ((g >> 1) & 1) ^ 1)) return;
+        for (int j = 0; j < kScanBatch; ++j) {
+            const int i = g * kScanBatch + j;
+            if (i >= ntiles) break;
+            const int s = i % nstages;
+            if (!mbar_wait(&full_b[s], (i / nstages) & 1)) return;
+            tc_fence_after();
+            const uint32_t aaddr = smem_u32(stage_base + (size_t)s * G::kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = make_sdesc(aaddr + kk * 32, 16, 1024, kSw128);
+                const uint64_t bd = make_sdesc(qaddr + kk * 32, 16, 1024, kSw128);
+                mma_e4m3(tmem + a * (kScanBatch * G::kN) + j * G::kN, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&empty_b[s]);
+        }
+        tc_commit(&tfull[a]);
+    }
+}
+
+// Epilogue of one TMEM lane quarter (a whole warp): for every entry of every
+// tile it computes the score and calls consume(tile, entry_in_tile, key) with
+// all 32 lanes (kEpr calls per tile).
+template <int DI, typename Consume>
+__device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)[kScanN], int hi, uint64_t *tfull,
+                                                   uint64_t *tempty, uint32_t tmem, int quarter, Consume consume) {
+    using G = ScanGeom<DI>;
+    const int lane = threadIdx.x & 31;
+    const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
+    for (int g = 0; g < nbatch; ++g) {
+        const int a = g & 1;
+        const bool ok = mbar_wait(&tfull[a], (g >> 1) & 1);
+        if (!__all_sync(0xFFFFFFFFu, ok)) break;
+        tc_fence_after();
+        float sc[kScanBatch][G::kEpr];
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            uint32_t r[G::kN];
+            const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + a * (kScanBatch * G::kN) + j * G::kN;
+            if (G::kN == 32) {
+                tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(r));
+            } else {
+                tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(r));
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < G::kEpr; ++u) {
+                float v = 0.0f;
+#pragma unroll
+                for (int h = 0; h < kScanN; ++h)
+                    if (h < hi) v = fmaf(wv[h], fmaxf(__uint_as_float(r[u * kScanN + h]), 0.0f), v);
+                sc[j][u] = v + 0.0f;
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[a]);
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            const int i = g * kScanBatch + j;
+            if (i >= ntiles) break;
+#pragma unroll
+            for (int u = 0; u < G::kEpr; ++u) consume(i, G::kEpr * (quarter * 32 + lane) + u, score_key(sc[j][u]));
+        }
+    }
+}
+
 template <int DI>
 __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
     using Cfg = ScanCfg<DI>;
@@ -189,12 +349,13 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
     uint8_t *qt = stages + Cfg::kStages * Cfg::kStageBytes;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(qt + 2048);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(qt + 4096);
     uint64_t *full = reinterpret_cast<uint64_t *>(hist + kHist0Bins);
     uint64_t *empty = full + Cfg::kStages;
     uint64_t *tfull = empty + Cfg::kStages;
     uint64_t *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    int32_t *ptab = reinterpret_cast<int32_t *>(tmem_slot + 2);  // [kMaxScanPages]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t qi = blockIdx.y;
@@ -202,19 +363,15 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
     pdl_trigger();
     pdl_wait();
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
-    const int64_t start = (int64_t)blockIdx.x * p.chunk_tiles * kScanTile;
+    using G = ScanGeom<DI>;
+    const int64_t start = (int64_t)blockIdx.x * p.chunk_tiles * G::kTile;
     if (start >= limit) return;
     const int64_t rem = limit - start;
-    const int ntiles = (int)min((int64_t)p.chunk_tiles, (rem + kScanTile - 1) / kScanTile);
+    const int ntiles = (int)min((int64_t)p.chunk_tiles, (rem + G::kTile - 1) / G::kTile);
 
     for (int i = tid; i < kHist0Bins; i += kScanThreads) hist[i] = 0u;
-    // B operand: query heads as rows 0..hi-1 of a [16][DI] K-major tile
-    for (int i = tid; i < Cfg::kQBytes / 16; i += kScanThreads) {
-        const int r = i / (DI / 16), c = i % (DI / 16);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < p.hi) v = *reinterpret_cast<const uint4 *>(p.qidx + ((int64_t)qi * p.hi + r) * DI + c * 16);
-        *reinterpret_cast<uint4 *>(qt + kmajor_chunk_offset<DI>(r, c)) = v;
-    }
+    build_q_tile<DI>(qt, p.qidx + (int64_t)qi * p.hi * DI, p.hi, kScanThreads);
+    stage_pages(p.kv, b, start, min(rem, (int64_t)ntiles * G::kTile), ptab, kScanThreads);
     if (tid == 0) {
         for (int s = 0; s < Cfg::kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -227,7 +384,7 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 32);
+        tmem_alloc(tmem_slot, 2 * kScanBatch * G::kN);
         tmem_relinquish();
     }
     fence_proxy_async_smem();
@@ -237,75 +394,23 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // TMA producer
-            const int nbox = kScanTile / p.box_rows;
-            for (int i = 0; i < ntiles; ++i) {
-                const int s = i % Cfg::kStages;
-                if (!mbar_wait(&empty[s], ((i / Cfg::kStages) & 1) ^ 1)) break;
-                const int64_t t0 = start + (int64_t)i * kScanTile;
-                int nvalid = 0;
-                for (int j = 0; j < nbox; ++j) nvalid += (t0 + (int64_t)j * p.box_rows < limit);
-                mbar_arrive_expect_tx(&full[s], (uint32_t)(nvalid * p.box_rows * DI));
-                for (int j = 0; j < nvalid; ++j) {
-                    int64_t row = physical_row(p.kv, b, t0 + (int64_t)j * p.box_rows);
-                    if (row < 0) {
-                        set_error(CSA2_DEVERR_BAD_ROW);
-                        row = 0;
-                    }
-                    tma_load_2d(stages + s * Cfg::kStageBytes + j * p.box_rows * DI, &tm, &full[s], 0, (int32_t)row);
-                }
-            }
-        }
+        if (lane == 0)
+            scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, Cfg::kStages, p.box_rows, stages, &tm, full, empty);
     } else if (warp == 1) {
-        if (lane == 0) {
-            // MMA issuer
-            const uint32_t idesc = idesc_e4m3_f32(128, kScanN);
-            const uint32_t qaddr = smem_u32(qt);
-            for (int i = 0; i < ntiles; ++i) {
-                const int s = i % Cfg::kStages, a = i & 1;
-                if (!mbar_wait(&full[s], (i / Cfg::kStages) & 1)) break;
-                if (!mbar_wait(&tempty[a], ((i >> 1) & 1) ^ 1)) break;
-                tc_fence_after();
-                const uint32_t aaddr = smem_u32(stages + s * Cfg::kStageBytes);
-#pragma unroll
-                for (int kk = 0; kk < DI / 32; ++kk) {
-                    const uint64_t ad = make_sdesc(aaddr + kk * 32, 16, 8 * DI, Cfg::kSwizzle);
-                    const uint64_t bd = make_sdesc(qaddr + kk * 32, 16, 8 * DI, Cfg::kSwizzle);
-                    mma_e4m3(tmem + a * kScanN, ad, bd, idesc, kk > 0 ? 1u : 0u);
-                }
-                tc_commit(&empty[s]);
-                tc_commit(&tfull[a]);
-            }
-        }
+        if (lane == 0)
+            scan_mma_loop<DI>(ntiles, Cfg::kStages, stages, smem_u32(qt), full, empty, tfull, tempty, tmem);
     } else {
         // epilogue: warps 2..5 cover TMEM lane quarters 2, 3, 0, 1
-        const int quarter = warp & 3;
         float wv[kScanN];
 #pragma unroll
         for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
-        for (int i = 0; i < ntiles; ++i) {
-            const int a = i & 1;
-            const bool ok = mbar_wait(&tfull[a], (i >> 1) & 1);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
-            tc_fence_after();
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + a * kScanN, r);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[a]);
-            float sc = 0.0f;
-#pragma unroll
-            for (int h = 0; h < kScanN; ++h)
-                if (h < p.hi) sc = fmaf(wv[h], fmaxf(__uint_as_float(r[h]), 0.0f), sc);
-            sc += 0.0f;
-            const int64_t t = start + (int64_t)i * kScanTile + quarter * 32 + lane;
+        uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
+        scan_epilogue_loop<DI>(ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3, [&](int i, int e, uint32_t key) {
+            const int64_t t = start + (int64_t)i * G::kTile + e;
             const bool valid = t < limit;
-            const uint32_t key = score_key(sc);
-            if (valid) p.keys[(int64_t)qi * p.key_stride + t] = key;
+            if (valid) keys[t] = key;
             hist_add_warp(hist, valid ? (key >> 20) : 0xFFFFFFFFu);
-        }
+        });
     }
     tc_fence_before();
     __syncthreads();
@@ -313,10 +418,10 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
         if (hist[i]) atomicAdd(&p.hist0[(int64_t)qi * kHist0Bins + i], hist[i]);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 32);
+        tmem_dealloc(tmem, 2 * kScanBatch * G::kN);
     }
     // the last CTA of this query locates the digit-0 bin of each target rank
-    const int64_t chunk = (int64_t)p.chunk_tiles * kScanTile;
+    const int64_t chunk = (int64_t)p.chunk_tiles * G::kTile;
     uint32_t *scratch = hist;  // the shared histogram is no longer needed
     if (last_block(&p.state[(int64_t)qi * kStateWords + kCtrScan], (uint32_t)((limit + chunk - 1) / chunk),
                    scratch + 64)) {
@@ -547,10 +652,8 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_emit(SelParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Reindex: score the pool ids of a Full layer, then exact Top-k of the pool
+// Reindex parameters (kernel in indexer_fused.cuh)
 // ---------------------------------------------------------------------------
-constexpr int kReindexThreads = 128;
-constexpr int kReindexSelThreads = 1024;
 constexpr int kReindexMaxPool = 16384;
 
 struct ReindexParams {
@@ -558,157 +661,9 @@ struct ReindexParams {
     const float *w;
     const int32_t *pool;
     csa2_kv_desc kv;
-    uint32_t *keys;  // [nq][p]
-    int32_t *ids;    // [nq][p]
+    unsigned long long *k64;  // [nq][p] workspace: (score key << 32 | ~id), 0 = empty
     int32_t *topk;   // [nq][k]
     int32_t p, k, hi, q_per_seq;
 };
-
-template <int DI>
-__global__ void __launch_bounds__(kReindexThreads) k_reindex_score(ReindexParams p) {
-    pdl_trigger();
-    pdl_wait();
-    __shared__ float qf[kScanN][DI];
-    __shared__ float wf[kScanN];
-    const int32_t qi = blockIdx.y;
-    for (int i = threadIdx.x; i < p.hi * DI; i += kReindexThreads) {
-        const uint8_t v = p.qidx[(int64_t)qi * p.hi * DI + i];
-        qf[i / DI][i % DI] = e4m3x2_to_float2((uint16_t)v).x;
-    }
-    if (threadIdx.x < p.hi) wf[threadIdx.x] = p.w[(int64_t)qi * p.hi + threadIdx.x];
-    __syncthreads();
-    const int32_t j = blockIdx.x * kReindexThreads + threadIdx.x;
-    if (j >= p.p) return;
-    int32_t id = p.pool[(int64_t)qi * p.p + j];
-    uint32_t key = 0u;
-    if (id >= 0) {
-        const int64_t row = physical_row(p.kv, qi / p.q_per_seq, id);
-        if (row < 0) {
-            set_error(CSA2_DEVERR_BAD_ROW);
-            id = -1;
-        } else {
-            float kf[DI];
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.kv.kidx + row * DI);
-#pragma unroll
-            for (int c = 0; c < DI / 16; ++c) {
-                const uint4 v = __ldg(src + c);
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 lo = e4m3x2_to_float2((uint16_t)(wv[u] & 0xFFFFu));
-                    const float2 hi2 = e4m3x2_to_float2((uint16_t)(wv[u] >> 16));
-                    kf[c * 16 + u * 4 + 0] = lo.x;
-                    kf[c * 16 + u * 4 + 1] = lo.y;
-                    kf[c * 16 + u * 4 + 2] = hi2.x;
-                    kf[c * 16 + u * 4 + 3] = hi2.y;
-                }
-            }
-            float sc = 0.0f;
-            for (int h = 0; h < p.hi; ++h) {
-                float dot = 0.0f;
-#pragma unroll
-                for (int i = 0; i < DI; ++i) dot = fmaf(qf[h][i], kf[i], dot);
-                sc = fmaf(wf[h], fmaxf(dot, 0.0f), sc);
-            }
-            key = score_key(sc + 0.0f);
-        }
-    }
-    p.keys[(int64_t)qi * p.p + j] = key;
-    p.ids[(int64_t)qi * p.p + j] = id;
-}
-
-// One CTA per query: radix select of the k largest 64-bit keys
-// (score key << 32 | ~id) among the valid pool entries, emitted in pool
-// order.
-__global__ void __launch_bounds__(kReindexSelThreads) k_reindex_select(ReindexParams p) {
-    pdl_trigger();
-    pdl_wait();
-    extern __shared__ uint8_t smem_raw[];
-    uint64_t *k64 = reinterpret_cast<uint64_t *>(smem_raw);   // [p]
-    uint32_t *hist = reinterpret_cast<uint32_t *>(k64 + p.p); // [2048]
-    uint32_t *scratch = hist + 2048;                          // [NT/32 + 4]
-    const int32_t qi = blockIdx.x;
-    const int NT = kReindexSelThreads;
-    const uint32_t *keys = p.keys + (int64_t)qi * p.p;
-    const int32_t *ids = p.ids + (int64_t)qi * p.p;
-    uint32_t nvalid_t = 0;
-    for (int j = threadIdx.x; j < p.p; j += NT) {
-        const int32_t id = ids[j];
-        uint64_t v = 0;
-        if (id >= 0) {
-            v = ((uint64_t)keys[j] << 32) | (uint64_t)(~(uint32_t)id);
-            ++nvalid_t;
-        }
-        k64[j] = v;
-    }
-    uint32_t nvalid;
-    block_excl_scan<NT>(nvalid_t, scratch, &nvalid);
-    const uint32_t r = min((uint32_t)p.k, nvalid);
-    uint64_t T = 0;  // select valid keys >= T
-    if (nvalid > (uint32_t)p.k) {
-        // bits every valid key shares need no radix pass: start at the highest
-        // bit in which two keys differ
-        __shared__ unsigned long long and_acc, or_acc;
-        if (threadIdx.x == 0) {
-            and_acc = ~0ull;
-            or_acc = 0ull;
-        }
-        __syncthreads();
-        unsigned long long a = ~0ull, o = 0ull;
-        for (int j = threadIdx.x; j < p.p; j += NT)
-            if (ids[j] >= 0) {
-                a &= k64[j];
-                o |= k64[j];
-            }
-        atomicAnd(&and_acc, a);
-        atomicOr(&or_acc, o);
-        __syncthreads();
-        const unsigned long long diff = and_acc ^ or_acc;  // nonzero: keys are unique
-        const int hb = 63 - __clzll((long long)diff);
-        uint64_t prefix = hb == 63 ? 0ull : (and_acc & ~((1ull << (hb + 1)) - 1ull));
-        uint64_t pmask = hb == 63 ? 0ull : ~((1ull << (hb + 1)) - 1ull);
-        uint32_t rem = r;
-        for (int top = hb; top >= 0; top -= 11) {
-            const int nbits = top + 1 < 11 ? top + 1 : 11;
-            const int shift = top + 1 - nbits;
-            const int nb = 1 << nbits;
-            for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
-            __syncthreads();
-            for (int j = threadIdx.x; j < p.p; j += NT) {
-                const uint64_t v = k64[j];
-                if (ids[j] >= 0 && (v & pmask) == prefix)
-                    atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
-            }
-            __syncthreads();
-            uint32_t bin, inbin;
-            find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
-            prefix |= (uint64_t)bin << shift;
-            pmask |= (uint64_t)(nb - 1) << shift;
-            rem = inbin;
-            const bool all_taken = hist[bin] == rem;  // every key of this bin is taken
-            __syncthreads();
-            if (all_taken) break;
-        }
-        T = prefix;
-        __syncthreads();
-    }
-    // ordered emission (pool order)
-    const int per = (p.p + NT - 1) / NT;
-    const int j0 = threadIdx.x * per;
-    uint32_t mine = 0;
-    for (int j = j0; j < min(p.p, j0 + per); ++j) mine += (ids[j] >= 0 && k64[j] >= T);
-    uint32_t pos = block_excl_scan<NT>(mine, scratch, nullptr);
-    int32_t *out = p.topk + (int64_t)qi * p.k;
-    for (int j = j0; j < min(p.p, j0 + per); ++j) {
-        if (!(ids[j] >= 0 && k64[j] >= T)) continue;
-        if (pos < (uint32_t)p.k) {
-            out[pos] = ids[j];
-        } else {
-            set_error(CSA2_DEVERR_SELECT);
-        }
-        ++pos;
-    }
-    for (int j = (int)r + threadIdx.x; j < p.k; j += NT) out[j] = -1;
-}
 
 }  // namespace csa2

@@ -1,0 +1,489 @@
+// indexer_fused.cuh -- Full-mode indexer in one launch: score scan and exact
+// Top-k / pool selection of a query by one thread-block cluster.
+//
+// Same method as indexer.cuh (DeepSeek V4.1-Flash Cuts KV Cache by 437x,
+// paragraph "CSA2 assigns each layer one of three static operating modes":
+// Full mode scores the whole context and keeps its Top-K; the first Full
+// layer also builds the pool of the hierarchical indexer), for sequences of
+// up to kFusedCluster * slice entries.
+//
+// CTA r of a query's cluster owns entries [r*S, (r+1)*S). It streams their
+// indexer keys by TMA through a deep shared-memory ring into tcgen05 FP8
+// MMAs (as k_index_scan) and keeps every 32-bit score key in shared memory
+// together with a 4096-bin histogram of the keys' top 12 bits. The radix
+// select (digits 12/10/10) then runs on shared memory: each digit's
+// histograms are summed across the cluster over distributed shared memory
+// (CTA r sums one slice of the bins, then every CTA gathers all slices),
+// with hardware cluster barriers between steps. The emission is ordered by
+// CTA rank and, inside a CTA, by entry, so the output ids are ascending and
+// ties at the threshold go to the lowest ids. No global scratch, no memset,
+// no second launch.
+#pragma once
+
+#include "indexer.cuh"
+
+namespace csa2 {
+
+constexpr int kFusedCluster = 8;
+constexpr int kFusedThreads = 256;
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+template <typename T>
+__device__ __forceinline__ T *cluster_peer(T *p, uint32_t rank) {
+    return static_cast<T *>(__cluster_map_shared_rank(static_cast<void *>(p), rank));
+}
+
+// Sum the local histograms h[0..nbins) (same shared-memory offset in every
+// CTA of the cluster) over the cluster into full[0..nbins). CTA r first
+// sums bins [r*nbins/C, (r+1)*nbins/C) from every CTA into slice[], then
+// every CTA gathers all slices.
+__device__ __forceinline__ void cluster_hist_sum(uint32_t *h, uint32_t *slice, uint32_t *full, int nbins,
+                                                 uint32_t rank) {
+    const int per = nbins / kFusedCluster;
+    cluster_sync_all();  // every CTA's local histogram is complete
+    for (int i = threadIdx.x; i < per; i += kFusedThreads) {
+        uint32_t s = 0;
+#pragma unroll
+        for (int r = 0; r < kFusedCluster; ++r) s += cluster_peer(h, (uint32_t)r)[rank * per + i];
+        slice[i] = s;
+    }
+    cluster_sync_all();
+    for (int i = threadIdx.x; i < nbins; i += kFusedThreads) {
+        const int owner = i / per;
+        full[i] = cluster_peer(slice, (uint32_t)owner)[i - owner * per];
+    }
+    cluster_sync_all();  // peers may reuse h / slice after this
+}
+
+struct FusedParams {
+    const uint8_t *qidx;
+    const float *w;
+    const int32_t *q_limit;
+    csa2_kv_desc kv;
+    int32_t *out[2];  // topk [nq][k], pool [nq][p]
+    int32_t rank[2];  // k, p (0 = no pool)
+    int32_t q_per_seq;
+    int32_t hi;
+    int32_t box_rows;
+    int32_t slice;    // entries per CTA (multiple of 128)
+    int32_t stages;   // TMA ring depth
+};
+
+template <int DI>
+struct FusedCfg {
+    static constexpr int kStageBytes = ScanGeom<DI>::kStageBytes;
+    // fixed part: q tile, hist0, full, slice, local digit hists, small words
+    static constexpr size_t kFixed = 1024 + 4096 + 4096 * 4 + 4096 * 4 + 512 * 4 + 2048 * 4 + 512 + 4 * kMaxScanPages;
+    static size_t smem(int slice, int stages) {
+        return kFixed + (size_t)stages * kStageBytes + (size_t)slice * 4 + 64 * 8 + 16;
+    }
+};
+
+template <int DI>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    k_index_full_fused(const __grid_constant__ CUtensorMap tm, FusedParams p) {
+    using Cfg = FusedCfg<DI>;
+    using G = ScanGeom<DI>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = base;
+    uint8_t *qt = stages + (size_t)p.stages * Cfg::kStageBytes;
+    uint32_t *hist0 = reinterpret_cast<uint32_t *>(qt + 4096);
+    uint32_t *full = hist0 + 4096;
+    uint32_t *slice = full + 4096;
+    uint32_t *nh = slice + 512;            // [2][1024] local digit-1/2 histograms
+    uint32_t *words = nh + 2048;           // 128 words: scratch + counts
+    uint32_t *scratch = words;             // block-scan scratch (kFusedThreads/32 + 4)
+    uint32_t *cnt = words + 32;            // [2 targets][gt, eq] of this CTA
+    uint32_t *keys = words + 128;          // [slice]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(keys + p.slice);
+    uint64_t *full_b = bars;
+    uint64_t *empty_b = bars + p.stages;
+    uint64_t *tfull = empty_b + p.stages;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    int32_t *ptab = reinterpret_cast<int32_t *>(tmem_slot + 2);  // [kMaxScanPages]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_rank();
+    const int32_t qi = blockIdx.y;
+    const int32_t b = qi / p.q_per_seq;
+
+    // ---- set-up that reads no global memory ----
+    pdl_trigger();
+    for (int i = tid; i < 4096; i += kFusedThreads) hist0[i] = 0u;
+    if (tid == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 2 * kScanBatch * G::kN);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+    const int64_t start = (int64_t)crank * p.slice;
+    const int64_t n_loc = max((int64_t)0, min(limit, start + p.slice) - start);
+    const int ntiles = (int)((n_loc + G::kTile - 1) / G::kTile);
+    build_q_tile<DI>(qt, p.qidx + (int64_t)qi * p.hi * DI, p.hi, kFusedThreads);
+    stage_pages(p.kv, b, start, n_loc, ptab, kFusedThreads);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- scan: TMA -> tcgen05 FP8 MMA -> scores into shared memory ----
+    if (warp == 0) {
+        if (lane == 0)
+            scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, p.stages, p.box_rows, stages, &tm, full_b, empty_b);
+    } else if (warp == 1) {
+        if (lane == 0)
+            scan_mma_loop<DI>(ntiles, p.stages, stages, smem_u32(qt), full_b, empty_b, tfull, tempty, tmem);
+    } else if (warp < 6) {
+        float wv[kScanN];
+#pragma unroll
+        for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
+        scan_epilogue_loop<DI>(ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3, [&](int i, int e_in, uint32_t key) {
+            const int e = i * G::kTile + e_in;
+            const bool valid = e < n_loc;
+            if (valid) keys[e] = key;
+            hist_add_warp(hist0, valid ? (key >> 20) : 0xFFFFFFFFu);
+        });
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * kScanBatch * G::kN);
+    }
+
+    // ---- cluster-wide radix select on the shared-memory keys ----
+    bool act[2];
+    uint32_t rem[2] = {0u, 0u}, b0[2] = {0u, 0u}, b1[2] = {0u, 0u}, T[2] = {0u, 0u};
+    for (int tau = 0; tau < 2; ++tau) {
+        act[tau] = p.rank[tau] > 0 && (int64_t)p.rank[tau] < limit;
+        rem[tau] = (uint32_t)max(p.rank[tau], 0);
+    }
+    // digit 0 (bits 31..20): the histogram built during the scan
+    cluster_hist_sum(hist0, slice, full, 4096, crank);
+    for (int tau = 0; tau < 2; ++tau)
+        if (act[tau]) find_rank_bin<kFusedThreads, 4096 / kFusedThreads, false>(full, 4096, rem[tau], scratch,
+                                                                                b0[tau], rem[tau]);
+    // digits 1 (bits 19..10) and 2 (bits 9..0)
+    for (int digit = 1; digit <= 2; ++digit) {
+        for (int i = tid; i < 2048; i += kFusedThreads) nh[i] = 0u;
+        __syncthreads();
+        for (int64_t i0 = 0; i0 < n_loc; i0 += kFusedThreads) {
+            const int64_t i = i0 + tid;
+            const uint32_t key = i < n_loc ? keys[i] : 0u;
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau) {
+                if (!act[tau]) continue;
+                bool m = i < n_loc && (key >> 20) == b0[tau];
+                if (digit == 2) m = m && ((key >> 10) & 1023u) == b1[tau];
+                if (__ballot_sync(0xFFFFFFFFu, m))  // most chunks hold no key of the threshold bin
+                    hist_add_warp(nh + tau * 1024,
+                                  m ? (digit == 1 ? (key >> 10) & 1023u : key & 1023u) : 0xFFFFFFFFu);
+            }
+        }
+        __syncthreads();
+        cluster_hist_sum(nh, slice, full, 2048, crank);
+        for (int tau = 0; tau < 2; ++tau) {
+            if (!act[tau]) continue;
+            uint32_t bin;
+            find_rank_bin<kFusedThreads, 1024 / kFusedThreads, false>(full + tau * 1024, 1024, rem[tau], scratch,
+                                                                      bin, rem[tau]);
+            if (digit == 1) {
+                b1[tau] = bin;
+            } else {
+                T[tau] = (b0[tau] << 20) | (b1[tau] << 10) | bin;
+            }
+        }
+    }
+
+    // ---- ordered emission: counts of every CTA, then this CTA's ids ----
+    // Warp w owns the key range [w*R, (w+1)*R) (R a multiple of 32) and walks
+    // it 32 consecutive keys at a time, lane = key, so shared-memory reads are
+    // conflict-free; ranks inside a chunk come from ballots.
+    constexpr int kWarps = kFusedThreads / 32;
+    const int64_t R = ((n_loc + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int64_t w0 = (int64_t)warp * R, w1 = min(n_loc, w0 + R);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t *wcnt = words + 64;  // [kWarps] per-warp counts
+    uint32_t *wcnt2 = words + 72; // [kWarps]
+    for (int tau = 0; tau < 2; ++tau) {
+        uint32_t gt = 0, eq = 0;
+        if (act[tau]) {
+            for (int64_t c = w0; c < w1; c += 32) {
+                const int64_t i = c + lane;
+                const uint32_t key = i < w1 ? keys[i] : 0u;
+                gt += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key > T[tau]));
+                eq += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]));
+            }
+        }
+        if (lane == 0) {
+            wcnt[warp] = gt;
+            wcnt2[warp] = eq;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t tg = 0, te = 0;
+            for (int ww = 0; ww < kWarps; ++ww) {
+                tg += wcnt[ww];
+                te += wcnt2[ww];
+            }
+            cnt[2 * tau] = tg;
+            cnt[2 * tau + 1] = te;
+        }
+        __syncthreads();
+    }
+    cluster_sync_all();
+    for (int tau = 0; tau < 2; ++tau) {
+        const int32_t r_out = p.rank[tau];
+        if (r_out <= 0 || p.out[tau] == nullptr) continue;
+        int32_t *out = p.out[tau] + (int64_t)qi * r_out;
+        if (crank == 0) {
+            const int64_t nsel = min((int64_t)r_out, limit);
+            for (int64_t j = nsel + tid; j < r_out; j += kFusedThreads) out[j] = -1;
+        }
+        if (!act[tau]) {
+            for (int64_t i = tid; i < n_loc; i += kFusedThreads) out[start + i] = (int32_t)(start + i);
+            continue;
+        }
+        uint32_t base_gt = 0, base_eq = 0;
+        for (uint32_t r = 0; r < crank; ++r) {
+            const uint32_t *pc = cluster_peer(cnt, r);
+            base_gt += pc[2 * tau];
+            base_eq += pc[2 * tau + 1];
+        }
+        const uint32_t need = rem[tau];
+        // per-warp counts of this target, then exclusive prefixes over warps
+        uint32_t wg = 0, we = 0;
+        for (int64_t c = w0; c < w1; c += 32) {
+            const int64_t i = c + lane;
+            const uint32_t key = i < w1 ? keys[i] : 0u;
+            we += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]));
+        }
+        if (lane == 0) wcnt[warp] = we;
+        __syncthreads();
+        uint32_t eq_base = base_eq;
+        for (int ww = 0; ww < warp; ++ww) eq_base += wcnt[ww];
+        __syncthreads();
+        // selected counts per warp (ties decided by their global rank among equal keys)
+        {
+            uint32_t er = eq_base, sel = 0;
+            for (int64_t c = w0; c < w1; c += 32) {
+                const int64_t i = c + lane;
+                const uint32_t key = i < w1 ? keys[i] : 0u;
+                const uint32_t em = __ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]);
+                const bool s_ = i < w1 && (key > T[tau] || (key == T[tau] && er + __popc(em & lt_mask) < need));
+                sel += __popc(__ballot_sync(0xFFFFFFFFu, s_));
+                er += __popc(em);
+            }
+            wg = sel;
+        }
+        if (lane == 0) wcnt[warp] = wg;
+        __syncthreads();
+        uint32_t pos = base_gt + min(base_eq, need);
+        for (int ww = 0; ww < warp; ++ww) pos += wcnt[ww];
+        __syncthreads();
+        {
+            uint32_t er = eq_base;
+            for (int64_t c = w0; c < w1; c += 32) {
+                const int64_t i = c + lane;
+                const uint32_t key = i < w1 ? keys[i] : 0u;
+                const uint32_t em = __ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]);
+                const bool s_ = i < w1 && (key > T[tau] || (key == T[tau] && er + __popc(em & lt_mask) < need));
+                const uint32_t sm = __ballot_sync(0xFFFFFFFFu, s_);
+                if (s_) {
+                    const uint32_t at = pos + __popc(sm & lt_mask);
+                    if (at < (uint32_t)r_out) {
+                        out[at] = (int32_t)(start + i);
+                    } else {
+                        set_error(CSA2_DEVERR_SELECT);
+                    }
+                }
+                pos += __popc(sm);
+                er += __popc(em);
+            }
+        }
+    }
+    cluster_sync_all();  // peers read cnt[] above; keep this CTA's shared memory alive until they are done
+}
+
+// ---------------------------------------------------------------------------
+// Reindex: (1) k_reindex_score, many CTAs: gather the indexer keys of the
+// pool ids (a row per thread, all its loads in flight), score them on the
+// CUDA cores (exact for small-integer E4M3 data, like the tensor-core
+// path) and write the unique 64-bit keys (score key << 32 | ~id; 0 for an
+// empty slot) to the workspace; (2) k_reindex_select, one CTA per query:
+// load the pool's keys into shared memory and select the k largest with a
+// radix select that starts at the highest bit in which two keys differ;
+// output in pool order.
+// ---------------------------------------------------------------------------
+constexpr int kReindexScoreThreads = 128;
+constexpr int kReindexSelectThreads = 1024;
+
+template <int DI>
+__global__ void __launch_bounds__(kReindexScoreThreads) k_reindex_score(ReindexParams p) {
+    __shared__ __align__(16) float qf[kScanN * DI];
+    __shared__ float wf[kScanN];
+    const int32_t qi = blockIdx.y;
+    const int32_t b = qi / p.q_per_seq;
+    pdl_trigger();
+    pdl_wait();
+    const int32_t j = blockIdx.x * kReindexScoreThreads + threadIdx.x;
+    // this thread's row goes out before the query is staged
+    int32_t id = (j < p.p) ? p.pool[(int64_t)qi * p.p + j] : -1;
+    int64_t row = id >= 0 ? physical_row(p.kv, b, id) : -1;
+    if (id >= 0 && row < 0) {
+        set_error(CSA2_DEVERR_BAD_ROW);
+        id = -1;
+    }
+    uint4 kv[DI / 16];
+#pragma unroll
+    for (int c = 0; c < DI / 16; ++c)
+        kv[c] = row >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.kv.kidx + row * DI) + c) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < p.hi * DI; i += kReindexScoreThreads)
+        qf[i] = e4m3x2_to_float2((uint16_t)p.qidx[(int64_t)qi * p.hi * DI + i]).x;
+    if (threadIdx.x < p.hi) wf[threadIdx.x] = p.w[(int64_t)qi * p.hi + threadIdx.x];
+    __syncthreads();
+    if (j >= p.p) return;
+    unsigned long long v = 0ull;  // 0 marks an empty slot (a valid key has ~id >= 2^31)
+    if (id >= 0) {
+        float dot[kScanN];
+#pragma unroll
+        for (int h = 0; h < kScanN; ++h) dot[h] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < DI / 16; ++c) {
+            const uint32_t wv[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
+            float kf[16];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 lo = e4m3x2_to_float2((uint16_t)(wv[t] & 0xFFFFu));
+                const float2 hi2 = e4m3x2_to_float2((uint16_t)(wv[t] >> 16));
+                kf[t * 4 + 0] = lo.x;
+                kf[t * 4 + 1] = lo.y;
+                kf[t * 4 + 2] = hi2.x;
+                kf[t * 4 + 3] = hi2.y;
+            }
+#pragma unroll
+            for (int h = 0; h < kScanN; ++h) {
+                if (h >= p.hi) break;
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4 *>(&qf[h * DI + c * 16 + i]);
+                    dot[h] = fmaf(q4.x, kf[i], dot[h]);
+                    dot[h] = fmaf(q4.y, kf[i + 1], dot[h]);
+                    dot[h] = fmaf(q4.z, kf[i + 2], dot[h]);
+                    dot[h] = fmaf(q4.w, kf[i + 3], dot[h]);
+                }
+            }
+        }
+        float sc = 0.0f;
+#pragma unroll
+        for (int h = 0; h < kScanN; ++h)
+            if (h < p.hi) sc = fmaf(wf[h], fmaxf(dot[h], 0.0f), sc);
+        v = ((unsigned long long)score_key(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)id);
+    }
+    p.k64[(int64_t)qi * p.p + j] = v;
+}
+
+__global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(ReindexParams p) {
+    constexpr int NT = kReindexSelectThreads;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                                 // [2048]
+    uint32_t *scratch = hist + 2048;                                                         // [NT/32 + 8]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p]
+    __shared__ unsigned long long and_acc, or_acc;
+    const int32_t qi = blockIdx.x;
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        and_acc = ~0ull;
+        or_acc = 0ull;
+    }
+    pdl_wait();
+    __syncthreads();
+    uint32_t nvalid_t = 0;
+    unsigned long long a_loc = ~0ull, o_loc = 0ull;
+    const unsigned long long *src = p.k64 + (int64_t)qi * p.p;
+    for (int j = threadIdx.x; j < p.p; j += NT) {
+        const unsigned long long v = __ldcg(src + j);
+        k64[j] = v;
+        if ((uint32_t)v >= 0x80000000u) {
+            ++nvalid_t;
+            a_loc &= v;
+            o_loc |= v;
+        }
+    }
+    atomicAnd(&and_acc, a_loc);
+    atomicOr(&or_acc, o_loc);
+    uint32_t nvalid;
+    block_excl_scan<NT>(nvalid_t, scratch, &nvalid);  // its barriers also publish k64 and the reductions
+    const uint32_t r = min((uint32_t)p.k, nvalid);
+    uint64_t T = 1ull;  // select keys >= T (every valid key is >= 2^31)
+    if (nvalid > (uint32_t)p.k) {
+        const unsigned long long diff = and_acc ^ or_acc;
+        const int hb = 63 - __clzll((long long)diff);
+        uint64_t prefix = hb == 63 ? 0ull : (and_acc & ~((1ull << (hb + 1)) - 1ull));
+        uint64_t pmask = hb == 63 ? 0ull : ~((1ull << (hb + 1)) - 1ull);
+        uint32_t rem = r;
+        for (int top = hb; top >= 0; top -= 11) {
+            const int nbits = top + 1 < 11 ? top + 1 : 11;
+            const int shift = top + 1 - nbits;
+            const int nb = 1 << nbits;
+            for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
+            __syncthreads();
+            for (int j = threadIdx.x; j < p.p; j += NT) {
+                const uint64_t v = k64[j];
+                if ((uint32_t)v >= 0x80000000u && (v & pmask) == prefix)
+                    atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
+            }
+            __syncthreads();
+            uint32_t bin, inbin;
+            find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
+            prefix |= (uint64_t)bin << shift;
+            pmask |= (uint64_t)(nb - 1) << shift;
+            rem = inbin;
+            const bool all_taken = hist[bin] == rem;
+            __syncthreads();
+            if (all_taken) break;
+        }
+        T = prefix;
+    }
+    // ordered emission (pool order)
+    const int per = (p.p + NT - 1) / NT;
+    const int j0 = threadIdx.x * per;
+    uint32_t mine = 0;
+    for (int j = j0; j < min(p.p, j0 + per); ++j) mine += (uint32_t)k64[j] >= 0x80000000u && k64[j] >= T;
+    uint32_t pos = block_excl_scan<NT>(mine, scratch, nullptr);
+    int32_t *out = p.topk + (int64_t)qi * p.k;
+    for (int j = j0; j < min(p.p, j0 + per); ++j) {
+        const uint64_t v = k64[j];
+        if (!((uint32_t)v >= 0x80000000u && v >= T)) continue;
+        if (pos < (uint32_t)p.k) {
+            out[pos] = (int32_t)(~(uint32_t)v);
+        } else {
+            set_error(CSA2_DEVERR_SELECT);
+        }
+        ++pos;
+    }
+    for (int j = (int)r + threadIdx.x; j < p.k; j += NT) out[j] = -1;
+}
+
+}  // namespace csa2
