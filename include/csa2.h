@@ -177,6 +177,36 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
 
 size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max);
 
+/*
+ * The same decode attention for callers that cannot allocate device memory
+ * (for example code running where cudaMalloc is not permitted, or a caller
+ * that owns no allocator). The paper has no counterpart: it is a library
+ * convenience. Arguments, results and errors are those of
+ * csa2_sparse_attn_decode, without ws / ws_bytes: the split partials live in
+ * a fixed array of CSA2_ATTN_STATIC_SCRATCH_BYTES bytes that the library
+ * holds in device global memory (one copy per device), and nothing is
+ * allocated by the call.
+ * Limit: when csa2_sparse_attn_workspace_size(nq, h, k, w_max) (w_max taken
+ * as 0 without a window) exceeds CSA2_ATTN_STATIC_SCRATCH_BYTES the call
+ * returns CSA2_ERR_WORKSPACE and launches nothing; use
+ * csa2_sparse_attn_decode with a caller-owned workspace instead.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress with that device current); make that first call
+ * before any stream capture begins. No part of the array has to start at
+ * zero: each call writes every partial it reads back.
+ * Concurrency: all calls on one device share the one array, so two calls
+ * whose kernels can overlap (different streams, or different host threads,
+ * without ordering between them) race on it and give wrong results. Order
+ * such calls on one stream, or use csa2_sparse_attn_decode.
+ */
+#define CSA2_ATTN_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+csa2_status csa2_sparse_attn_decode_static(const void *q_bf16, int32_t nq, int32_t q_per_seq,
+                                           int32_t h, const csa2_kv_desc *kv, const int32_t *topk,
+                                           int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
+                                           const int32_t *swa_begin, const int32_t *swa_end,
+                                           int32_t w_max, float softmax_scale, void *o_bf16,
+                                           float *lse, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * *code receives 0 when no device-side condition was recorded since the
  * last call, else a bit set of CSA2_DEVERR_* values. Returns CSA2_OK, or

@@ -20,6 +20,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 CSA2_D = 512
+CSA2_ATTN_STATIC_SCRATCH_BYTES = 16 << 20
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration",
           3: "workspace missing or too small", 4: "CUDA error", 5: "device-side error recorded"}
 
@@ -59,6 +60,8 @@ _SIGS = {
     "csa2_sparse_attn_decode": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
                                        _f32, _vp, _vp, _vp, _sz, _vp]),
     "csa2_sparse_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "csa2_sparse_attn_decode_static": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
+                                              _f32, _vp, _vp, _vp]),
     "csa2_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "csa2_status_string": (ctypes.c_char_p, [_i32]),
     "csa2_version": (_i32, []),
@@ -162,6 +165,20 @@ def csa2_sparse_attn_decode(q_bf16, q_per_seq, kv: KvCache, topk, swa, swa_seq_s
         _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
         _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_bf16), _ptr(lse),
         _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def csa2_sparse_attn_decode_static(q_bf16, q_per_seq, kv: KvCache, topk, swa, swa_seq_stride, swa_begin, swa_end,
+                                   w_max, softmax_scale, o_bf16, lse, stream=None):
+    """csa2_sparse_attn_decode with the library's fixed device scratch
+    (CSA2_ATTN_STATIC_SCRATCH_BYTES) in place of a caller workspace, for
+    callers that cannot allocate device memory. Calls whose kernels can
+    overlap on one device share that scratch and race."""
+    nq, h = q_bf16.shape[0], q_bf16.shape[1]
+    k = topk.shape[1] if topk is not None else 0
+    _check("csa2_sparse_attn_decode_static", _lib.csa2_sparse_attn_decode_static(
+        _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
+        _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_bf16), _ptr(lse),
+        _stream(stream)))
 
 
 def csa2_device_status(stream=None):

@@ -564,3 +564,58 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without a caller workspace, for callers that cannot
+// allocate device memory. The split partials go to a fixed array in device
+// global memory, one copy per device (the module is loaded per device). Its
+// address is looked up once per device, with that device current, and then
+// handed to the regular attention path as its workspace, so the kernels and
+// their arithmetic are exactly those of csa2_sparse_attn_decode. Each call
+// writes every partial before the combine reads it, so the array needs no
+// clearing. Calls on one device share the array: overlapping calls race.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) uint8_t g_attn_scratch[CSA2_ATTN_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_attn_scratch_mu;
+void *g_attn_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of this device's copy of g_attn_scratch, or null on error.
+void *attn_scratch_of_current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_attn_scratch_mu);
+    if (!g_attn_scratch_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_attn_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_attn_scratch_ptr[dev] = ptr;
+    }
+    return g_attn_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" csa2_status csa2_sparse_attn_decode_static(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                                      const csa2_kv_desc *kv, const int32_t *topk, int32_t k,
+                                                      const uint8_t *swa, int64_t swa_seq_stride,
+                                                      const int32_t *swa_begin, const int32_t *swa_end, int32_t w_max,
+                                                      float softmax_scale, void *o_bf16, float *lse,
+                                                      cudaStream_t stream) {
+    // the same workspace the regular path would ask for (no window: w_max 0)
+    const size_t need = csa2_sparse_attn_workspace_size(nq, h, k, swa_begin ? w_max : 0);
+    if (need > CSA2_ATTN_STATIC_SCRATCH_BYTES) return CSA2_ERR_WORKSPACE;
+    void *scratch = attn_scratch_of_current_device();
+    if (!scratch) return CSA2_ERR_CUDA;
+    return csa2_sparse_attn_decode(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end,
+                                   w_max, softmax_scale, o_bf16, lse, scratch, CSA2_ATTN_STATIC_SCRATCH_BYTES,
+                                   stream);
+}
