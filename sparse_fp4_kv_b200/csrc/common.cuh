@@ -83,14 +83,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete. Gives up after a
-// bounded number of polls (well over a second), records the timeout in the
-// device error word and returns false so the caller can unwind.
-constexpr uint32_t kWaitPolls = 1u << 24;
+// Waits for the phase with the given parity to complete. Gives up after
+// about one second of global-timer time (a few hundred fast polls first,
+// then polls spaced by short sleeps), records the timeout in the device
+// error word and returns false so the caller can unwind.
+constexpr uint64_t kWaitNs = 1000000000ull;
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
         if (mbar_try_wait(bar, parity)) return true;
-        if (i > 256) __nanosleep(64);
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < kWaitNs) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(64);
     }
     set_error(CSA2_DEVERR_WAIT_TIMEOUT);
     return false;

@@ -240,6 +240,53 @@ cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Attributes of the single-launch Full kernels (maximal dynamic shared
+// memory; 16-CTA clusters need the non-portable size), set once, and how many
+// 16-CTA clusters of the kernel the device holds at once (0 if none, or if a
+// call failed).
+template <int DI>
+bool fused_attrs() {
+    static const bool ok = [] {
+        bool good = set_smem(k_index_full_fused<DI, kFusedClusterSmall>, (size_t)max_smem_optin()) &&
+                    set_smem(k_index_full_fused<DI, kFusedClusterLarge>, (size_t)max_smem_optin());
+        if (cudaFuncSetAttribute(k_index_full_fused<DI, kFusedClusterLarge>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            good = false;
+        }
+        return good;
+    }();
+    return ok;
+}
+
+int fused_clusters_of_16(bool di64) {
+    static int n[2] = {-1, -1};
+    int &v = n[di64 ? 1 : 0];
+    if (v >= 0) return v;
+    v = 0;
+    if (!(di64 ? fused_attrs<64>() : fused_attrs<128>())) return v;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kFusedClusterLarge;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kFusedClusterLarge, 1);
+    cfg.blockDim = dim3(kFusedThreads);
+    cfg.dynamicSmemBytes = (size_t)max_smem_optin() - 1024;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    const cudaError_t e = di64 ? cudaOccupancyMaxActiveClusters(&c, k_index_full_fused<64, kFusedClusterLarge>, &cfg)
+                               : cudaOccupancyMaxActiveClusters(&c, k_index_full_fused<128, kFusedClusterLarge>, &cfg);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        c = 0;
+    }
+    v = c;
+    return v;
+}
+
 template <typename K>
 bool prefer_shared(K kernel) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -329,18 +376,25 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     CUtensorMap tm;
     if (!make_kidx_map(&tm, kv, box_rows)) return CSA2_ERR_CUDA;
 
-    // Single launch: one cluster of kFusedCluster CTAs per query, every score
-    // kept in shared memory, when a query's entries fit.
+    // Single launch: one cluster per query, every score kept in shared
+    // memory, when a query's entries fit. Clusters of 16 CTAs when the device
+    // holds one for every query at once, else 8.
     {
-        const int64_t slice = (int64_t)align_up(
-            (size_t)((std::max<int64_t>(n_max, 1) + kFusedCluster - 1) / kFusedCluster), (size_t)tile_entries);
+        const bool di64 = kv->di == 64;
+        const int cl = (fused_clusters_of_16(di64) >= nq && n_max >= (int64_t)kFusedClusterLarge * 2 * tile_entries)
+                           ? kFusedClusterLarge
+                           : kFusedClusterSmall;
+        const int64_t slice = (int64_t)align_up((size_t)((std::max<int64_t>(n_max, 1) + cl - 1) / cl),
+                                                (size_t)tile_entries);
         const size_t stage_bytes = 128 * 128;
-        const size_t fixed = (kv->di == 64 ? FusedCfg<64>::kFixed : FusedCfg<128>::kFixed) + 64 * 8 + 16;
+        const size_t fixed = (di64 ? FusedCfg<64>::kFixed : FusedCfg<128>::kFixed) + 64 * 8 + 16;
         const size_t budget = (size_t)max_smem_optin();
         int stages = 0;
         if (fixed + (size_t)slice * 4 < budget) stages = (int)std::min<size_t>(16, (budget - fixed - slice * 4) / stage_bytes);
         const bool pages_fit = slice / kv->page_size + 2 <= kMaxScanPages;
-        if (stages >= 3 && pages_fit && !force_multipass()) {
+        // the emission's chunk masks (16 B per 32 keys and warp) reuse the TMA ring
+        const bool masks_fit = (size_t)slice / 2 + 128 <= (size_t)stages * stage_bytes;
+        if (stages >= 3 && pages_fit && masks_fit && !force_multipass()) {
             FusedParams fp{};
             fp.qidx = qidx;
             fp.w = w;
@@ -355,18 +409,17 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
             fp.box_rows = box_rows;
             fp.slice = (int32_t)slice;
             fp.stages = stages;
-            const dim3 fgrid(kFusedCluster, (unsigned)nq);
-            if (kv->di == 64) {
-                const size_t smem = FusedCfg<64>::smem((int)slice, stages);
-                static bool ok = set_smem(k_index_full_fused<64>, (size_t)max_smem_optin());
-                if (!ok) return CSA2_ERR_CUDA;
-                launch_cluster(k_index_full_fused<64>, fgrid, dim3(kFusedThreads), smem, stream, kFusedCluster, tm, fp);
+            const dim3 fgrid((unsigned)cl, (unsigned)nq);
+            const size_t smem = di64 ? FusedCfg<64>::smem((int)slice, stages) : FusedCfg<128>::smem((int)slice, stages);
+            auto go = [&](auto kernel) {
+                launch_cluster(kernel, fgrid, dim3(kFusedThreads), smem, stream, (unsigned)cl, tm, fp);
+            };
+            if (di64) {
+                if (cl == kFusedClusterLarge) go(k_index_full_fused<64, kFusedClusterLarge>);
+                else go(k_index_full_fused<64, kFusedClusterSmall>);
             } else {
-                const size_t smem = FusedCfg<128>::smem((int)slice, stages);
-                static bool ok = set_smem(k_index_full_fused<128>, (size_t)max_smem_optin());
-                if (!ok) return CSA2_ERR_CUDA;
-                launch_cluster(k_index_full_fused<128>, fgrid, dim3(kFusedThreads), smem, stream, kFusedCluster, tm,
-                               fp);
+                if (cl == kFusedClusterLarge) go(k_index_full_fused<128, kFusedClusterLarge>);
+                else go(k_index_full_fused<128, kFusedClusterSmall>);
             }
             return check_launch();
         }

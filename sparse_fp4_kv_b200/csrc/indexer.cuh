@@ -231,37 +231,75 @@ __device__ __forceinline__ int stage_pages(const csa2_kv_desc &kv, int32_t b, in
     return npg;
 }
 
-// TMA producer: tile i = 128 smem rows = kTile entries, loaded as boxes of
-// box_rows rows (a box never crosses a page). Boxes whose first entry is past
-// the limit are skipped (their rows are not read). Physical rows come from
-// the staged page-table entries.
+// TMA producer, run by a whole warp (lane 0 issues): tile i = 128 smem rows =
+// kTile entries, loaded as boxes of box_rows rows. A box never crosses a
+// page (box_rows * kEpr divides the page size), so the page index and the
+// offset inside the page advance by whole boxes without any division. Boxes
+// whose first entry is past the limit are skipped (their rows are not read).
+// Physical rows come from the staged page-table entries.
 template <int DI>
 __device__ __forceinline__ void scan_tma_loop(const csa2_kv_desc &kv, const int32_t *ptab, int64_t start,
                                               int64_t limit, int ntiles, int nstages, int box_rows,
                                               uint8_t *stage_base, const CUtensorMap *tm, uint64_t *full_b,
                                               uint64_t *empty_b) {
     using G = ScanGeom<DI>;
+    const bool leader = (threadIdx.x & 31) == 0;
     const int nbox = 128 / box_rows;
-    const int64_t ps = kv.page_size;
-    const int64_t pg0 = start / ps;
-    for (int i = 0; i < ntiles; ++i) {
-        const int s = i % nstages;
-        if (!mbar_wait(&empty_b[s], ((i / nstages) & 1) ^ 1)) return;
-        const int64_t t0 = start + (int64_t)i * G::kTile;
-        int nvalid = 0;
-        for (int j = 0; j < nbox; ++j) nvalid += (t0 + (int64_t)j * box_rows * G::kEpr < limit);
-        mbar_arrive_expect_tx(&full_b[s], (uint32_t)(nvalid * box_rows * 128));
-        for (int j = 0; j < nvalid; ++j) {
-            const int64_t t = t0 + (int64_t)j * box_rows * G::kEpr;
-            const int64_t pi = t / ps - pg0;
-            const int64_t phys = pi < kMaxScanPages ? ptab[pi] : -1;
-            int64_t row = phys * ps + (t % ps);
-            if (phys < 0 || row + (int64_t)box_rows * G::kEpr > kv.rows_cap) {
-                set_error(CSA2_DEVERR_BAD_ROW);
-                row = 0;
+    const int32_t step = box_rows * G::kEpr;  // entries per box
+    const int32_t ps = kv.page_size;
+    // entry positions fit in 32 bits (sequence lengths are int32)
+    int32_t pi = 0, off = (int32_t)(start % ps);
+    int32_t t = (int32_t)start;
+    const int32_t lim = (int32_t)min(limit, (int64_t)INT32_MAX);
+    // ring slot and phase advance without divisions (this loop is latency-bound)
+    int s = 0;
+    uint32_t phase = 0;
+    // Fast path: one box per tile and the whole range inside one page (every
+    // contiguous cache): consecutive tiles are consecutive rows.
+    const int64_t span = (int64_t)ntiles * G::kTile;
+    if (nbox == 1 && ntiles > 0 && off + span <= ps && ptab[0] >= 0 &&
+        (int64_t)ptab[0] * ps + off + span <= kv.rows_cap) {
+        int32_t y = (int32_t)(((int64_t)ptab[0] * ps + off) / G::kEpr);
+        for (int i = 0; i < ntiles; ++i) {
+            if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
+            if (leader) {
+                mbar_arrive_expect_tx(&full_b[s], (uint32_t)G::kStageBytes);
+                tma_load_2d(stage_base + (size_t)s * G::kStageBytes, tm, &full_b[s], 0, y);
             }
-            tma_load_2d(stage_base + (size_t)s * G::kStageBytes + j * box_rows * 128, tm, &full_b[s], 0,
-                        (int32_t)(row / G::kEpr));
+            y += 128;
+            if (++s == nstages) {
+                s = 0;
+                phase ^= 1u;
+            }
+        }
+        return;
+    }
+    for (int i = 0; i < ntiles; ++i) {
+        if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
+        int nvalid = 0;
+        for (int j = 0; j < nbox; ++j) nvalid += (t + j * step < lim);
+        if (leader) mbar_arrive_expect_tx(&full_b[s], (uint32_t)(nvalid * box_rows * 128));
+        for (int j = 0; j < nbox; ++j) {
+            if (j < nvalid && leader) {
+                const int64_t phys = pi < kMaxScanPages ? ptab[pi] : -1;
+                int64_t row = phys * ps + off;
+                if (phys < 0 || row + step > kv.rows_cap) {
+                    set_error(CSA2_DEVERR_BAD_ROW);
+                    row = 0;
+                }
+                tma_load_2d(stage_base + (size_t)s * G::kStageBytes + j * box_rows * 128, tm, &full_b[s], 0,
+                            (int32_t)(row / G::kEpr));
+            }
+            t += step;
+            off += step;
+            if (off == ps) {
+                off = 0;
+                ++pi;
+            }
+        }
+        if (++s == nstages) {
+            s = 0;
+            phase ^= 1u;
         }
     }
 }
@@ -273,14 +311,15 @@ __device__ __forceinline__ void scan_mma_loop(int ntiles, int nstages, const uin
     using G = ScanGeom<DI>;
     const uint32_t idesc = idesc_e4m3_f32(128, G::kN);
     const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
+    int s = 0;
+    uint32_t phase = 0;
     for (int g = 0; g < nbatch; ++g) {
         const int a = g & 1;
         if (!mbar_wait(&tempty[a], ((g >> 1) & 1) ^ 1)) return;
         for (int j = 0; j < kScanBatch; ++j) {
             const int i = g * kScanBatch + j;
             if (i >= ntiles) break;
-            const int s = i % nstages;
-            if (!mbar_wait(&full_b[s], (i / nstages) & 1)) return;
+            if (!mbar_wait(&full_b[s], phase)) return;
             tc_fence_after();
             const uint32_t aaddr = smem_u32(stage_base + (size_t)s * G::kStageBytes);
 #pragma unroll
@@ -290,6 +329,10 @@ __device__ __forceinline__ void scan_mma_loop(int ntiles, int nstages, const uin
                 mma_e4m3(tmem + a * (kScanBatch * G::kN) + j * G::kN, ad, bd, idesc, kk > 0 ? 1u : 0u);
             }
             tc_commit(&empty_b[s]);
+            if (++s == nstages) {
+                s = 0;
+                phase ^= 1u;
+            }
         }
         tc_commit(&tfull[a]);
     }
@@ -394,8 +437,7 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0)
-            scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, Cfg::kStages, p.box_rows, stages, &tm, full, empty);
+        scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, Cfg::kStages, p.box_rows, stages, &tm, full, empty);
     } else if (warp == 1) {
         if (lane == 0)
             scan_mma_loop<DI>(ntiles, Cfg::kStages, stages, smem_u32(qt), full, empty, tfull, tempty, tmem);

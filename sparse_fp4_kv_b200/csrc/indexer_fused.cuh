@@ -5,7 +5,7 @@
 // paragraph "CSA2 assigns each layer one of three static operating modes":
 // Full mode scores the whole context and keeps its Top-K; the first Full
 // layer also builds the pool of the hierarchical indexer), for sequences of
-// up to kFusedCluster * slice entries.
+// up to (cluster size) * slice entries.
 //
 // CTA r of a query's cluster owns entries [r*S, (r+1)*S). It streams their
 // indexer keys by TMA through a deep shared-memory ring into tcgen05 FP8
@@ -24,7 +24,10 @@
 
 namespace csa2 {
 
-constexpr int kFusedCluster = 8;
+// CTAs per query: 8 (portable), or 16 when the device can hold a cluster of
+// 16 such CTAs for every query at once.
+constexpr int kFusedClusterSmall = 8;
+constexpr int kFusedClusterLarge = 16;
 constexpr int kFusedThreads = 256;
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -44,14 +47,15 @@ __device__ __forceinline__ T *cluster_peer(T *p, uint32_t rank) {
 // CTA of the cluster) over the cluster into full[0..nbins). CTA r first
 // sums bins [r*nbins/C, (r+1)*nbins/C) from every CTA into slice[], then
 // every CTA gathers all slices.
+template <int CL>
 __device__ __forceinline__ void cluster_hist_sum(uint32_t *h, uint32_t *slice, uint32_t *full, int nbins,
                                                  uint32_t rank) {
-    const int per = nbins / kFusedCluster;
+    const int per = nbins / CL;
     cluster_sync_all();  // every CTA's local histogram is complete
     for (int i = threadIdx.x; i < per; i += kFusedThreads) {
         uint32_t s = 0;
 #pragma unroll
-        for (int r = 0; r < kFusedCluster; ++r) s += cluster_peer(h, (uint32_t)r)[rank * per + i];
+        for (int r = 0; r < CL; ++r) s += cluster_peer(h, (uint32_t)r)[rank * per + i];
         slice[i] = s;
     }
     cluster_sync_all();
@@ -59,7 +63,10 @@ __device__ __forceinline__ void cluster_hist_sum(uint32_t *h, uint32_t *slice, u
         const int owner = i / per;
         full[i] = cluster_peer(slice, (uint32_t)owner)[i - owner * per];
     }
-    cluster_sync_all();  // peers may reuse h / slice after this
+    __syncthreads();
+    // No closing cluster barrier: peers read h only before the second barrier
+    // above, and read slice only before they reach the first barrier of the
+    // next call (or the kernel's final barrier), so both may be rewritten now.
 }
 
 struct FusedParams {
@@ -86,7 +93,7 @@ struct FusedCfg {
     }
 };
 
-template <int DI>
+template <int DI, int CL>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_index_full_fused(const __grid_constant__ CUtensorMap tm, FusedParams p) {
     using Cfg = FusedCfg<DI>;
@@ -149,8 +156,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---- scan: TMA -> tcgen05 FP8 MMA -> scores into shared memory ----
     if (warp == 0) {
-        if (lane == 0)
-            scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, p.stages, p.box_rows, stages, &tm, full_b, empty_b);
+        scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, p.stages, p.box_rows, stages, &tm, full_b, empty_b);
     } else if (warp == 1) {
         if (lane == 0)
             scan_mma_loop<DI>(ntiles, p.stages, stages, smem_u32(qt), full_b, empty_b, tfull, tempty, tmem);
@@ -175,34 +181,54 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     // ---- cluster-wide radix select on the shared-memory keys ----
     bool act[2];
     uint32_t rem[2] = {0u, 0u}, b0[2] = {0u, 0u}, b1[2] = {0u, 0u}, T[2] = {0u, 0u};
+    #pragma unroll
     for (int tau = 0; tau < 2; ++tau) {
         act[tau] = p.rank[tau] > 0 && (int64_t)p.rank[tau] < limit;
         rem[tau] = (uint32_t)max(p.rank[tau], 0);
     }
     // digit 0 (bits 31..20): the histogram built during the scan
-    cluster_hist_sum(hist0, slice, full, 4096, crank);
+    cluster_hist_sum<CL>(hist0, slice, full, 4096, crank);
+    #pragma unroll
     for (int tau = 0; tau < 2; ++tau)
         if (act[tau]) find_rank_bin<kFusedThreads, 4096 / kFusedThreads, false>(full, 4096, rem[tau], scratch,
                                                                                 b0[tau], rem[tau]);
-    // digits 1 (bits 19..10) and 2 (bits 9..0)
+    // digits 1 (bits 19..10) and 2 (bits 9..0): each thread takes 4 keys per
+    // step (one 16-byte load); most steps hold no key of the threshold bin
+    // and cost one ballot
+    const int nl = (int)n_loc;
     for (int digit = 1; digit <= 2; ++digit) {
         for (int i = tid; i < 2048; i += kFusedThreads) nh[i] = 0u;
         __syncthreads();
-        for (int64_t i0 = 0; i0 < n_loc; i0 += kFusedThreads) {
-            const int64_t i = i0 + tid;
-            const uint32_t key = i < n_loc ? keys[i] : 0u;
+        const int shift = digit == 1 ? 20 : 10;
+        uint32_t pre[2];
 #pragma unroll
-            for (int tau = 0; tau < 2; ++tau) {
-                if (!act[tau]) continue;
-                bool m = i < n_loc && (key >> 20) == b0[tau];
-                if (digit == 2) m = m && ((key >> 10) & 1023u) == b1[tau];
-                if (__ballot_sync(0xFFFFFFFFu, m))  // most chunks hold no key of the threshold bin
-                    hist_add_warp(nh + tau * 1024,
-                                  m ? (digit == 1 ? (key >> 10) & 1023u : key & 1023u) : 0xFFFFFFFFu);
-            }
+        for (int tau = 0; tau < 2; ++tau) pre[tau] = digit == 1 ? b0[tau] : ((b0[tau] << 10) | b1[tau]);
+        // the trip count is the same for every thread (warp-wide ballots inside)
+        for (int base4 = 0; base4 < nl; base4 += 4 * kFusedThreads) {
+            const int i0 = base4 + 4 * tid;
+            // keys has room up to the slice end, a multiple of 4 entries
+            const uint4 k4 = i0 < nl ? *reinterpret_cast<const uint4 *>(keys + i0) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+            bool m[2][4];
+            bool any = false;
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    m[tau][j] = act[tau] && i0 + j < nl && (kk[j] >> shift) == pre[tau];
+                    any |= m[tau][j];
+                }
+            if (__ballot_sync(0xFFFFFFFFu, any) == 0u) continue;
+#pragma unroll
+            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (__ballot_sync(0xFFFFFFFFu, m[tau][j]))
+                        hist_add_warp(nh + tau * 1024, m[tau][j] ? (kk[j] >> (shift - 10)) & 1023u : 0xFFFFFFFFu);
         }
         __syncthreads();
-        cluster_hist_sum(nh, slice, full, 2048, crank);
+        cluster_hist_sum<CL>(nh, slice, full, 2048, crank);
+        #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
             if (!act[tau]) continue;
             uint32_t bin;
@@ -218,41 +244,53 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---- ordered emission: counts of every CTA, then this CTA's ids ----
     // Warp w owns the key range [w*R, (w+1)*R) (R a multiple of 32) and walks
-    // it 32 consecutive keys at a time, lane = key, so shared-memory reads are
-    // conflict-free; ranks inside a chunk come from ballots.
+    // it 32 consecutive keys at a time (lane = key, conflict-free reads). One
+    // pass records, per chunk of 32 keys and per target, the ballot masks of
+    // keys above and equal to the threshold (in the TMA ring, free after the
+    // scan) and the per-warp counts; the output position of every warp then
+    // follows from the counts alone: keys above the threshold are all taken,
+    // keys equal to it are taken in entry order up to the remaining rank.
     constexpr int kWarps = kFusedThreads / 32;
-    const int64_t R = ((n_loc + kWarps - 1) / kWarps + 31) / 32 * 32;
-    const int64_t w0 = (int64_t)warp * R, w1 = min(n_loc, w0 + R);
+    const int R = ((nl + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int cpw = R / 32;
+    const int w0 = warp * R, w1 = min(nl, w0 + R);
     const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t *wcnt = words + 64;  // [kWarps] per-warp counts
-    uint32_t *wcnt2 = words + 72; // [kWarps]
-    for (int tau = 0; tau < 2; ++tau) {
-        uint32_t gt = 0, eq = 0;
-        if (act[tau]) {
-            for (int64_t c = w0; c < w1; c += 32) {
-                const int64_t i = c + lane;
-                const uint32_t key = i < w1 ? keys[i] : 0u;
-                gt += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key > T[tau]));
-                eq += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]));
-            }
+    uint32_t *wgt = words + 64;  // [2 targets][kWarps] keys above the threshold
+    uint32_t *weq = words + 80;  // [2 targets][kWarps] keys equal to it
+    uint4 *masks = reinterpret_cast<uint4 *>(stages) + (int64_t)warp * cpw;  // [cpw]: gt0, eq0, gt1, eq1
+    {
+        uint32_t gt0 = 0, eq0 = 0, gt1 = 0, eq1 = 0;
+#pragma unroll 4
+        for (int c = 0; c < cpw; ++c) {
+            const int i = w0 + c * 32 + lane;
+            const bool in = i < w1;
+            const uint32_t key = in ? keys[i] : 0u;
+            const uint32_t mg0 = __ballot_sync(0xFFFFFFFFu, in && act[0] && key > T[0]);
+            const uint32_t me0 = __ballot_sync(0xFFFFFFFFu, in && act[0] && key == T[0]);
+            const uint32_t mg1 = __ballot_sync(0xFFFFFFFFu, in && act[1] && key > T[1]);
+            const uint32_t me1 = __ballot_sync(0xFFFFFFFFu, in && act[1] && key == T[1]);
+            if (lane == 0) masks[c] = make_uint4(mg0, me0, mg1, me1);
+            gt0 += __popc(mg0);
+            eq0 += __popc(me0);
+            gt1 += __popc(mg1);
+            eq1 += __popc(me1);
         }
         if (lane == 0) {
-            wcnt[warp] = gt;
-            wcnt2[warp] = eq;
+            wgt[warp] = gt0;
+            weq[warp] = eq0;
+            wgt[kWarps + warp] = gt1;
+            weq[kWarps + warp] = eq1;
         }
-        __syncthreads();
-        if (tid == 0) {
-            uint32_t tg = 0, te = 0;
-            for (int ww = 0; ww < kWarps; ++ww) {
-                tg += wcnt[ww];
-                te += wcnt2[ww];
-            }
-            cnt[2 * tau] = tg;
-            cnt[2 * tau + 1] = te;
-        }
-        __syncthreads();
+    }
+    __syncthreads();
+    if (tid < 4) {
+        const uint32_t *src = (tid & 1) ? weq : wgt;
+        uint32_t t = 0;
+        for (int ww = 0; ww < kWarps; ++ww) t += src[(tid >> 1) * kWarps + ww];
+        cnt[tid] = t;  // [tau][gt, eq]
     }
     cluster_sync_all();
+    #pragma unroll
     for (int tau = 0; tau < 2; ++tau) {
         const int32_t r_out = p.rank[tau];
         if (r_out <= 0 || p.out[tau] == nullptr) continue;
@@ -272,55 +310,33 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             base_eq += pc[2 * tau + 1];
         }
         const uint32_t need = rem[tau];
-        // per-warp counts of this target, then exclusive prefixes over warps
-        uint32_t wg = 0, we = 0;
-        for (int64_t c = w0; c < w1; c += 32) {
-            const int64_t i = c + lane;
-            const uint32_t key = i < w1 ? keys[i] : 0u;
-            we += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]));
+        // equal keys before this warp, and the output position of its first id
+        uint32_t er = base_eq, pos = base_gt + min(base_eq, need);
+        for (int ww = 0; ww < warp; ++ww) {
+            const uint32_t e = weq[tau * kWarps + ww];
+            pos += wgt[tau * kWarps + ww] + (need > er ? min(need - er, e) : 0u);
+            er += e;
         }
-        if (lane == 0) wcnt[warp] = we;
-        __syncthreads();
-        uint32_t eq_base = base_eq;
-        for (int ww = 0; ww < warp; ++ww) eq_base += wcnt[ww];
-        __syncthreads();
-        // selected counts per warp (ties decided by their global rank among equal keys)
-        {
-            uint32_t er = eq_base, sel = 0;
-            for (int64_t c = w0; c < w1; c += 32) {
-                const int64_t i = c + lane;
-                const uint32_t key = i < w1 ? keys[i] : 0u;
-                const uint32_t em = __ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]);
-                const bool s_ = i < w1 && (key > T[tau] || (key == T[tau] && er + __popc(em & lt_mask) < need));
-                sel += __popc(__ballot_sync(0xFFFFFFFFu, s_));
-                er += __popc(em);
+#pragma unroll 4
+        for (int c = 0; c < cpw; ++c) {
+            const uint4 m4 = masks[c];
+            const uint32_t g = tau ? m4.z : m4.x, e = tau ? m4.w : m4.y;
+            if ((g | e) == 0u) continue;
+            uint32_t sm = g;
+            if (e != 0u && er < need) {
+                const bool take = ((e >> lane) & 1u) && er + __popc(e & lt_mask) < need;
+                sm |= __ballot_sync(0xFFFFFFFFu, take);
             }
-            wg = sel;
-        }
-        if (lane == 0) wcnt[warp] = wg;
-        __syncthreads();
-        uint32_t pos = base_gt + min(base_eq, need);
-        for (int ww = 0; ww < warp; ++ww) pos += wcnt[ww];
-        __syncthreads();
-        {
-            uint32_t er = eq_base;
-            for (int64_t c = w0; c < w1; c += 32) {
-                const int64_t i = c + lane;
-                const uint32_t key = i < w1 ? keys[i] : 0u;
-                const uint32_t em = __ballot_sync(0xFFFFFFFFu, i < w1 && key == T[tau]);
-                const bool s_ = i < w1 && (key > T[tau] || (key == T[tau] && er + __popc(em & lt_mask) < need));
-                const uint32_t sm = __ballot_sync(0xFFFFFFFFu, s_);
-                if (s_) {
-                    const uint32_t at = pos + __popc(sm & lt_mask);
-                    if (at < (uint32_t)r_out) {
-                        out[at] = (int32_t)(start + i);
-                    } else {
-                        set_error(CSA2_DEVERR_SELECT);
-                    }
+            if ((sm >> lane) & 1u) {
+                const uint32_t at = pos + __popc(sm & lt_mask);
+                if (at < (uint32_t)r_out) {
+                    out[at] = (int32_t)start + w0 + c * 32 + lane;
+                } else {
+                    set_error(CSA2_DEVERR_SELECT);
                 }
-                pos += __popc(sm);
-                er += __popc(em);
             }
+            pos += __popc(sm);
+            er += __popc(e);
         }
     }
     cluster_sync_all();  // peers read cnt[] above; keep this CTA's shared memory alive until they are done

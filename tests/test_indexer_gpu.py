@@ -101,6 +101,13 @@ def test_full_causal_queries(B, cuda_device):
               shuffle=False)
 
 
+def test_full_long_sequences_ragged(B, cuda_device):
+    # long enough that a query's entries are spread over 16 CTAs (when the
+    # device holds 16-CTA clusters for every query), with ragged tails
+    _run_full(B, cuda_device, [40000 + 17, 33333], 40064, 64, 4, 2048, 4096, shuffle=False, seed=14)
+    _run_full(B, cuda_device, [36000 + 5], 36096, 128, 8, 1000, 3000, shuffle=False, seed=15)
+
+
 def test_full_all_ties_take_lowest_ids(B, cuda_device):
     same = lambda cap, di: np.full((cap, di), 0x38, np.uint8)  # every key = 1.0
     topk, pool, _ = _run_full(B, cuda_device, [2500], 64, 64, 4, 300, 900, kidx_fn=same, seed=6)
