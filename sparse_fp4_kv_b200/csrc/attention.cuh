@@ -12,26 +12,27 @@
 //     o_h = sum_j softmax_j(scale * <q_h, v_j>) v_j.
 //
 // Work unit: one query and a split of its attended rows (selected global
-// entries followed by its window rows), 128 rows per tile. Per tile:
-//   1. all 8 warps dequantise the tile's rows (fetched into registers while
-//      the previous tile was on the tensor cores): FP4 codes are widened
-//      with cvt.rn.f16x2.e2m1x2 and multiplied by the block scale (exact in
-//      f16), window bytes with cvt.rn.f16x2.e4m3x2; the f16 tile lands in
-//      shared memory in the 128B-swizzled K-major layout (rows = entries,
-//      64-value column blocks 16 KiB apart); then the loads of the next
-//      tile are issued.
-//   2. one thread issues S^T = KV * Q^T with tcgen05.mma kind::f16
-//      (M = 128 rows, N = H heads, K = 512) into TMEM.
-//   3. warps 0..3 (one TMEM lane quarter each, a thread per row) read S^T,
-//      reduce the per-head tile maximum across the 128 rows (transposed
-//      butterfly + shared memory), run the online softmax in base 2, write
-//      P^T (f16) into a swizzled M/N-major tile and reduce the per-head sum
-//      of the tile's probabilities the same way.
-//   4. one thread issues O^T += V^T * P^T (A = the same KV tile read
-//      M/N-major, d in four chunks of 128, B = P^T) into TMEM.
-// The running maximum is only raised when a tile's maximum exceeds it by
-// more than 2^8, so O^T (in TMEM) is rescaled rarely; probabilities stay
-// below 2^8 and are exact in range for f16.
+// entries followed by its window rows), 128 rows per tile. The f16 tile is
+// handled in four chunks of 128 latent columns (32 KiB each), so the work
+// overlaps across chunks and tiles:
+//   1. sixteen warps dequantise chunk c of tile t (raw bytes fetched into
+//      registers one tile ahead) as soon as the P*V products of tile t-1 on
+//      that chunk are done: FP4 codes widened with cvt.rn.f16x2.e2m1x2 and
+//      multiplied by the block scale (exact in f16), window bytes widened with
+//      cvt.rn.f16x2.e4m3x2, stored in the 128B-swizzled K-major layout;
+//   2. one elected thread of a seventeenth warp issues S^T += KV_c * Q_c^T
+//      (tcgen05.mma kind::f16, M = 128 rows, N = H heads) for each chunk as
+//      soon as every thread has stored it, then commits S; meanwhile the
+//      sixteen warps put the loads of tile t+1 in flight;
+//   3. the warps (a thread per row, up to four head groups) run the online
+//      softmax in base 2 on S^T from TMEM and write P^T (f16). The running
+//      maximum is only raised when some score exceeds it by more than 2^8, so
+//      the common case needs no tile maximum: one vote per head group decides;
+//      a raise takes the full path (tile maximum, rescale of O^T in TMEM);
+//   4. the same thread issues O^T += V^T * P^T chunk by chunk (A = the same KV
+//      chunk read M/N-major, B = P^T), committing each chunk separately so
+//      step 1 of the next tile can reuse it at once.
+// Probabilities stay below 2^8 and are exact in range for f16.
 // Splits of one query are merged by k_attn_combine with their
 // log-sum-exp values.
 #pragma once
@@ -40,7 +41,11 @@
 
 namespace csa2 {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnWorkWarps = 16;                     // dequantise, softmax, epilogue
+constexpr int kAttnWorkThreads = kAttnWorkWarps * 32;
+constexpr int kAttnThreads = kAttnWorkThreads + 32;  // + the warp that issues the tensor-core products
+constexpr int kMmaWarp = kAttnWorkWarps;
+constexpr uint32_t kBarWork = 5;                      // named barrier of the work warps (1..4: head groups)
 constexpr int kAttnTile = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -55,7 +60,7 @@ struct AttnCfg {
     static constexpr int kColO = H;
     static constexpr uint32_t kTmemCols = H == 64 ? 512u : (H == 32 ? 256u : 128u);
     static constexpr int kMisc = 8 * 128 * 5 /*resolved rows*/ + 128 * 4 /*valid*/ + 4 * H * 4 /*red*/ +
-                                 3 * H * 4 /*m, alpha, l*/ + 64 /*bars, slot, flags*/;
+                                 3 * H * 4 /*m, alpha, l*/ + 128 /*bars, slot, flags*/;
     static constexpr size_t kSmem = 1024 + (size_t)kKvBytes + kQBytes + kPBytes + kMisc;
 };
 
@@ -139,28 +144,30 @@ __device__ __forceinline__ void store_warp_reduced(float *dst, const float (&v)[
 }
 
 // ---------------------------------------------------------------------------
-// Tile gather: each warp owns 16 rows of the 128-row tile. Lanes 0..15
-// resolve the rows' sources in parallel (id -> page table -> physical row,
-// or window row), then every lane issues its 16-value slice of all 16 rows
-// back to back, so 16 independent loads per lane are in flight. The raw
-// bytes stay in registers until the f16 tile buffer is free again, which
+// Tile gather: each work warp owns 8 rows of the 128-row tile. For latent
+// chunk c (128 columns) lane l holds columns 128c + 16(l%8) .. +15 of rows
+// 4j + l/8 (j = 0, 1), so every lane takes part in every chunk's
+// dequantisation. All 8 loads of a lane are issued back to back; the raw
+// bytes stay in registers until the chunk's f16 slot is free again, which
 // lets the loads of tile t+1 run under the tensor-core work of tile t.
 // ---------------------------------------------------------------------------
-constexpr int kRowsPerWarp = kAttnTile / (kAttnThreads / 32);  // 16
+constexpr int kRowsPerWarp = kAttnTile / kAttnWorkWarps;  // 8
+constexpr int kRowGroups = kRowsPerWarp / 4;                // rows of a lane per chunk
 constexpr int kResolveTiles = 8;  // rows resolved per batch: 8 tiles = 1024 rows
 
 struct TileRaw {
-    uint4 v[kRowsPerWarp];  // FP4 row: {codes lo, codes hi, scale byte, 0}; window row: 16 E4M3 bytes
-    uint32_t kinds;         // 2 bits per row: 0 empty, 1 FP4 global entry, 2 window row
+    uint4 v[4 * kRowGroups];  // [chunk * kRowGroups + j]: FP4 piece {codes lo, codes hi, scale byte, 0};
+                              // window piece: 16 E4M3 bytes
+    uint32_t kinds;  // 2 bits per j: 0 empty, 1 FP4 global entry, 2 window row
 };
 
 // Resolve the sources of rows [j0, j0 + n) of the query's attended list into
 // shared memory: physical FP4 row (kind 1), window buffer row (kind 2) or
-// nothing (kind 0). All threads take part; two dependent loads per row, all
-// rows in flight together.
+// nothing (kind 0). The work warps take part; two dependent loads per row,
+// all rows in flight together.
 __device__ __forceinline__ void resolve_rows(const AttnParams &p, int32_t u, int32_t b, int32_t nw, int32_t wb,
                                              int64_t j0, int n, int32_t *rsrc, uint8_t *rkind) {
-    for (int i = threadIdx.x; i < n; i += kAttnThreads) {
+    for (int i = threadIdx.x; i < n; i += kAttnWorkThreads) {
         const int64_t j = j0 + i;
         int32_t src = 0;
         uint8_t kind = 0;
@@ -184,40 +191,48 @@ __device__ __forceinline__ void resolve_rows(const AttnParams &p, int32_t u, int
     }
 }
 
-// Issue the loads of one tile's rows (resolved sources at rsrc/rkind + off):
-// every lane loads its 16-value slice of the warp's 16 rows back to back.
+// Issue the loads of latent chunks [C0, C1) of one tile's rows (resolved
+// sources at rsrc/rkind + off).
+template <int C0, int C1>
 __device__ __forceinline__ void fetch_tile(const AttnParams &p, int32_t b, const int32_t *rsrc, const uint8_t *rkind,
                                            int off, TileRaw &raw) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int base = off + warp * kRowsPerWarp;
-    const int32_t my_src = lane < kRowsPerWarp ? rsrc[base + lane] : 0;
-    const uint32_t my_kind = lane < kRowsPerWarp ? rkind[base + lane] : 0u;
+    const int piece = lane & 7;
     const uint8_t *swa_seq = p.swa ? p.swa + (int64_t)b * p.swa_seq_stride * CSA2_D : nullptr;
     raw.kinds = 0;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const int64_t src = __shfl_sync(0xFFFFFFFFu, my_src, r);
-        const uint32_t kd = __shfl_sync(0xFFFFFFFFu, my_kind, r);
-        raw.kinds |= kd << (2 * r);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (kd == 1) {
-            const uint2 c = __ldg(reinterpret_cast<const uint2 *>(p.kv.codes + src * (CSA2_D / 2)) + lane);
-            v = make_uint4(c.x, c.y, (uint32_t)__ldg(p.kv.scales + src * (CSA2_D / CSA2_BLOCK) + lane), 0u);
-        } else if (kd == 2) {
-            v = __ldg(reinterpret_cast<const uint4 *>(swa_seq + src * CSA2_D) + lane);
+    for (int j = 0; j < kRowGroups; ++j) {
+        const int r = off + warp * kRowsPerWarp + 4 * j + (lane >> 3);
+        const int64_t src = rsrc[r];
+        const uint32_t kd = rkind[r];
+        raw.kinds |= kd << (2 * j);
+#pragma unroll
+        for (int c = C0; c < C1; ++c) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (kd == 1) {
+                const uint2 cc =
+                    __ldg(reinterpret_cast<const uint2 *>(p.kv.codes + src * (CSA2_D / 2) + c * 64 + piece * 8));
+                v = make_uint4(cc.x, cc.y, (uint32_t)__ldg(p.kv.scales + src * (CSA2_D / CSA2_BLOCK) + c * 8 + piece),
+                               0u);
+            } else if (kd == 2) {
+                v = __ldg(reinterpret_cast<const uint4 *>(swa_seq + src * CSA2_D + c * 128 + piece * 16));
+            }
+            raw.v[c * kRowGroups + j] = v;
         }
-        raw.v[r] = v;
     }
 }
 
-// Dequantise the fetched rows into the f16 tile (128B-swizzled K-major) and
-// record which rows hold data.
-__device__ __forceinline__ void store_tile(const TileRaw &raw, uint8_t *kv_tile, int32_t *valid_s) {
+// Dequantise latent chunk c of the fetched rows into the f16 tile
+// (128B-swizzled K-major); chunk 0 also records which rows hold data. Lanes
+// of pieces 4..7 store their second 16-byte half first, so the eight lanes
+// of each store phase hit eight different bank groups.
+__device__ __forceinline__ void store_chunk(const TileRaw &raw, int c, uint8_t *kv_tile, int32_t *valid_s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int piece = lane & 7;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const uint32_t kd = (raw.kinds >> (2 * r)) & 3u;
-        const uint4 v = raw.v[r];
+    for (int j = 0; j < kRowGroups; ++j) {
+        const uint32_t kd = (raw.kinds >> (2 * j)) & 3u;
+        const uint4 v = raw.v[c * kRowGroups + j];
         uint32_t h0[4] = {0u, 0u, 0u, 0u}, h1[4] = {0u, 0u, 0u, 0u};
         if (kd == 1) {
             const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)(v.z | (v.z << 8)));
@@ -238,12 +253,26 @@ __device__ __forceinline__ void store_tile(const TileRaw &raw, uint8_t *kv_tile,
             h1[2] = e4m3x2_to_f16x2((uint16_t)(v.w & 0xFFFFu));
             h1[3] = e4m3x2_to_f16x2((uint16_t)(v.w >> 16));
         }
-        const int e = warp * kRowsPerWarp + r;
-        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane)) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
-        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 2 * lane + 1)) =
-            make_uint4(h1[0], h1[1], h1[2], h1[3]);
-        if (lane == 0) valid_s[e] = kd != 0u;
+        const int e = warp * kRowsPerWarp + 4 * j + (lane >> 3);
+        const int c64 = 16 * c + 2 * piece;
+        const bool swap = piece >= 4;
+        const uint4 first = swap ? make_uint4(h1[0], h1[1], h1[2], h1[3]) : make_uint4(h0[0], h0[1], h0[2], h0[3]);
+        const uint4 second = swap ? make_uint4(h0[0], h0[1], h0[2], h0[3]) : make_uint4(h1[0], h1[1], h1[2], h1[3]);
+        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, c64 + (swap ? 1 : 0))) = first;
+        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, c64 + (swap ? 0 : 1))) = second;
+        if (c == 0 && piece == 0) valid_s[e] = kd != 0u;
     }
+}
+
+// OR of `pred` over the `n` threads of named barrier `id`.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0u;
 }
 
 // NC consecutive S^T columns of this thread's row (TMEM lane), scaled to
@@ -274,7 +303,8 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float scale_log2, bo
 template <int H>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     using Cfg = AttnCfg<H>;
-    constexpr int HG = H / 2;  // heads per softmax warp group
+    constexpr int G = H >= 32 ? 4 : 2;  // softmax head groups (4 warps each, a warp per TMEM lane quarter)
+    constexpr int HG = H / G;            // heads per group
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kv_tile = base;
@@ -287,10 +317,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     float *m_run = red + 4 * H;
     float *alpha = m_run + H;
     float *l_run = alpha + H;
-    uint64_t *bar_s = reinterpret_cast<uint64_t *>(l_run + H);
-    uint64_t *bar_o = bar_s + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_o + 1);
-    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [2] (per head group)
+    uint64_t *bar_kv = reinterpret_cast<uint64_t *>(l_run + H);  // [4] chunk c of the tile stored
+    uint64_t *bar_pv = bar_kv + 4;                               // [4] P*V of chunk c done
+    uint64_t *bar_s = bar_pv + 4;                                // S^T of the tile ready
+    uint64_t *bar_p = bar_s + 1;                                 // P^T of the tile written
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_p + 1);
+    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [4] (per head group)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t split = blockIdx.x, u = blockIdx.y;
@@ -303,9 +335,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         tmem_relinquish();
     }
     if (tid == 0) {
+        for (int c = 0; c < 4; ++c) {
+            mbar_init(&bar_kv[c], kAttnWorkThreads);
+            mbar_init(&bar_pv[c], 1);
+        }
         mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
-        rescale_tile[0] = rescale_tile[1] = -1;
+        mbar_init(bar_p, kAttnWorkThreads);
+        rescale_tile[0] = rescale_tile[1] = rescale_tile[2] = rescale_tile[3] = -1;
         fence_mbar_init();
     }
     if (tid < H) {
@@ -319,262 +355,314 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
     const int64_t t_begin = (int64_t)split * p.tiles_per_split;
     const int64_t t_end = min(tiles_total, t_begin + p.tiles_per_split);
+    const int ntiles = (int)max((int64_t)0, t_end - t_begin);
 
-    // ---- prologue: resolve the first rows, start their loads, stage Q ----------
-    if (t_begin < t_end)
-        resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile,
-                     (int)min((int64_t)kResolveTiles, t_end - t_begin) * kAttnTile, rsrc, rkind);
-    __syncthreads();
+    // ---- prologue: Q loads in flight first, then resolve the first rows and
+    //      start their loads, then Q (bf16 -> f16) into the K-major
+    //      128B-swizzled B tile ----
     TileRaw raw;
     raw.kinds = 0;
-    if (t_begin < t_end) fetch_tile(p, b, rsrc, rkind, 0, raw);
-    {
-        // Q: bf16 -> f16 into the K-major 128B-swizzled B tile; loads in
-        // batches of 8 per thread so they are in flight together
+    const bool mma_warp = warp == kMmaWarp;
+    if (!mma_warp) {
         const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (int64_t)u * H * CSA2_D);
         constexpr int kChunks = H * (CSA2_D / 8);
-        constexpr int kPer = kChunks / kAttnThreads;  // 16 / 8 / 4 for H = 64 / 32 / 16
-        constexpr int kBatch = kPer < 4 ? kPer : 4;
+        constexpr int kPer = kChunks / kAttnWorkThreads;  // 8 / 4 / 2 for H = 64 / 32 / 16
+        uint4 qv[kPer];
 #pragma unroll
-        for (int i0 = 0; i0 < kPer; i0 += kBatch) {
-            uint4 v[kBatch];
+        for (int t = 0; t < kPer; ++t) qv[t] = __ldg(qsrc + tid + t * kAttnWorkThreads);
+        if (ntiles > 0)
+            resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile, min(kResolveTiles, ntiles) * kAttnTile, rsrc, rkind);
+        named_bar_sync(kBarWork, kAttnWorkThreads);
+        if (ntiles > 0) fetch_tile<0, 4>(p, b, rsrc, rkind, 0, raw);
 #pragma unroll
-            for (int t = 0; t < kBatch; ++t) v[t] = __ldg(qsrc + tid + (i0 + t) * kAttnThreads);
+        for (int t = 0; t < kPer; ++t) {
+            const int i = tid + t * kAttnWorkThreads;
+            const int h = i / (CSA2_D / 8), c64 = i % (CSA2_D / 8);
+            const uint32_t w4[4] = {qv[t].x, qv[t].y, qv[t].z, qv[t].w};
+            uint32_t o4[4];
 #pragma unroll
-            for (int t = 0; t < kBatch; ++t) {
-                const int i = tid + (i0 + t) * kAttnThreads;
-                const int h = i / (CSA2_D / 8), c64 = i % (CSA2_D / 8);
-                const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
-                uint32_t o4[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const __half2 hh =
-                        __floats2half2_rn(__uint_as_float(w4[q] << 16), __uint_as_float(w4[q] & 0xFFFF0000u));
-                    o4[q] = *reinterpret_cast<const uint32_t *>(&hh);
-                }
-                *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            for (int q = 0; q < 4; ++q) {
+                const __half2 hh =
+                    __floats2half2_rn(__uint_as_float(w4[q] << 16), __uint_as_float(w4[q] & 0xFFFF0000u));
+                o4[q] = *reinterpret_cast<const uint32_t *>(&hh);
             }
+            *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t kv_addr = smem_u32(kv_tile), q_addr = smem_u32(q_tile), p_addr = smem_u32(p_tile);
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int quarter = warp & 3, grp = warp >> 2;  // TMEM lane quarter, head group
-    float l_part[HG];                                // this row's partial softmax denominators
-#pragma unroll
-    for (int i = 0; i < HG; ++i) l_part[i] = 0.0f;
 
-    bool ok = true;
-    int it = 0;
-    for (int64_t tt = t_begin; tt < t_end && ok; ++tt, ++it) {
-        // 1. the f16 tile buffer is free (previous P*V done): dequantise this
-        //    tile, then put the next tile's loads in flight
-        store_tile(raw, kv_tile, valid_s);
-        if (tt + 1 < t_end) {
-            const int rel = (int)((tt + 1 - t_begin) % kResolveTiles);
-            if (rel == 0) {
-                // next batch of resolved rows (rare: splits of more than 8 tiles)
-                __syncthreads();
-                resolve_rows(p, u, b, nw, wb, (tt + 1) * kAttnTile,
-                             (int)min((int64_t)kResolveTiles, t_end - (tt + 1)) * kAttnTile, rsrc, rkind);
-                __syncthreads();
-            }
-            fetch_tile(p, b, rsrc, rkind, rel * kAttnTile, raw);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // 2. S^T = KV * Q^T
-        if (tid == 0) {
-            const uint32_t idesc = idesc_f16_f32(128, H, 0, 0);
-#pragma unroll
-            for (int kb = 0; kb < CSA2_D / 64; ++kb) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = make_sdesc(kv_addr + kb * 16384 + kk * 32, 16, 1024, kSw128);
-                    const uint64_t bd = make_sdesc(q_addr + kb * (H * 128) + kk * 32, 16, 1024, kSw128);
-                    mma_f16(tmem + Cfg::kColS, ad, bd, idesc, (kb | kk) ? 1u : 0u);
-                }
-            }
-            tc_commit(bar_s);
-        }
-        {
-            // 3. online softmax: thread = row (TMEM lane), warps 0..3 take heads
-            //    [0, H/2), warps 4..7 heads [H/2, H); each group of 4 warps
-            //    synchronises on its own named barrier
-            const bool got = mbar_wait(bar_s, it & 1);
-            tc_fence_after();
-            const int row = quarter * 32 + lane;
-            const bool row_valid = valid_s[row] != 0 && got;
-            const uint32_t s_addr = lane_addr + Cfg::kColS + grp * HG;
-            {
-                float v[HG];
-                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
-                warp_transpose_reduce<HG, true>(v);
-                store_warp_reduced<HG>(red + quarter * H + grp * HG, v);
-            }
-            named_bar_sync(1 + grp, 128);
-            if (quarter == 0 && lane < HG) {
-                const int h = grp * HG + lane;
-                const float mt = fmaxf(fmaxf(red[h], red[H + h]), fmaxf(red[2 * H + h], red[3 * H + h]));
-                const float mo = m_run[h];
-                float a = 1.0f, mn = mo;
-                if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt > -INFINITY)) {
-                    mn = mt;
-                    a = (mo == -INFINITY) ? 0.0f : exp2f(mo - mt);
-                    if (mo != -INFINITY) rescale_tile[grp] = (int32_t)it;
-                }
-                m_run[h] = mn;
-                alpha[h] = a;
-            }
-            named_bar_sync(1 + grp, 128);
-            // probabilities -> P^T (f16), per-row partial denominators
-            {
-                float v[HG];
-                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
-#pragma unroll
-                for (int g = 0; g < HG / 8; ++g) {
-                    const float4 ma = *reinterpret_cast<const float4 *>(m_run + grp * HG + 8 * g);
-                    const float4 mb = *reinterpret_cast<const float4 *>(m_run + grp * HG + 8 * g + 4);
-                    const float4 aa = *reinterpret_cast<const float4 *>(alpha + grp * HG + 8 * g);
-                    const float4 ab = *reinterpret_cast<const float4 *>(alpha + grp * HG + 8 * g + 4);
-                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-                    const float al[8] = {aa.x, aa.y, aa.z, aa.w, ab.x, ab.y, ab.z, ab.w};
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const int i = 8 * g + 2 * t;
-                        const float p0 = (mm[2 * t] == -INFINITY) ? 0.0f : exp2f(v[i] - mm[2 * t]);
-                        const float p1 = (mm[2 * t + 1] == -INFINITY) ? 0.0f : exp2f(v[i + 1] - mm[2 * t + 1]);
-                        l_part[i] = fmaf(l_part[i], al[2 * t], p0);
-                        l_part[i + 1] = fmaf(l_part[i + 1], al[2 * t + 1], p1);
-                        const __half2 hh = __floats2half2_rn(p0, p1);
-                        pk[t] = *reinterpret_cast<const uint32_t *>(&hh);
-                    }
-                    *reinterpret_cast<uint4 *>(p_tile + p_chunk_off<H>(row, grp * (HG / 8) + g)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
-            // rare: raise of the running maximum -> rescale this group's O^T columns
-            if (rescale_tile[grp] == it) {
+    {
+        const uint32_t idesc_s = idesc_f16_f32(128, H, 0, 0);
+        const uint32_t idesc_o = idesc_f16_f32(128, H, 1, 1);
+        // base descriptors; an operand offset is added to the start-address
+        // field (address / 16, shared memory stays below 2^18 bytes)
+        const uint64_t a_s = make_sdesc(kv_addr, 16, 1024, kSw128);
+        const uint64_t b_s = make_sdesc(q_addr, 16, 1024, kSw128);
+        const uint64_t a_o = make_sdesc(kv_addr, 16384, 1024, kSw128);
+        const uint64_t b_o = make_sdesc(p_addr, 16, Cfg::kPGroup, Cfg::kPSwizzle);
+        if (mma_warp) {
+            // ---- one elected thread issues every tensor-core product ----
+            if (lane == 0) {
+                bool ok = true;
+                for (int it = 0; it < ntiles && ok; ++it) {
+                    const uint32_t ph = (uint32_t)it & 1u;
+                    // S^T += KV_c * Q_c^T, chunk by chunk as the work warps store them
 #pragma unroll 1
-                for (int dc = 0; dc < 4; ++dc) {
+                    for (int c = 0; c < 4 && ok; ++c) {
+                        if (!mbar_wait(&bar_kv[c], ph)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < HG; c += 8) {
+                        for (int kb = 2 * c; kb < 2 * c + 2; ++kb) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_f16(tmem + Cfg::kColS, a_s + (uint64_t)((kb * 16384 + kk * 32) >> 4),
+                                        b_s + (uint64_t)((kb * (H * 128) + kk * 32) >> 4), idesc_s,
+                                        (kb | kk) ? 1u : 0u);
+                        }
+                    }
+                    if (!ok) break;
+                    tc_commit(bar_s);
+                    // O^T += V^T * P^T once the softmax has written P^T, chunk by chunk
+                    if (!mbar_wait(bar_p, ph)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int dc = 0; dc < 4; ++dc) {
+#pragma unroll
+                        for (int kk = 0; kk < kAttnTile / 16; ++kk)
+                            mma_f16(tmem + Cfg::kColO + dc * H, a_o + (uint64_t)((dc * 32768 + kk * 2048) >> 4),
+                                    b_o + (uint64_t)((kk * 2 * Cfg::kPGroup) >> 4), idesc_o,
+                                    (it > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(&bar_pv[dc]);
+                    }
+                }
+            }
+            __syncwarp();
+        } else {
+        // ---- work warps: dequantise, fetch ahead, online softmax, epilogue ----
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int quarter = warp & 3, grp = warp >> 2;  // TMEM lane quarter, head group
+        const bool soft = grp < G;                       // this warp runs the softmax of group grp
+        float l_part[HG];                                // this row's partial softmax denominators
+#pragma unroll
+        for (int i = 0; i < HG; ++i) l_part[i] = 0.0f;
+        bool ok = true;
+        for (int it = 0; it < ntiles; ++it) {
+            const int64_t tt = t_begin + it;
+            // 1. dequantise chunk c as soon as the previous tile's P*V on it is done
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (it > 0 && ok && !mbar_wait(&bar_pv[c], (uint32_t)(it - 1) & 1u)) ok = false;
+                store_chunk(raw, c, kv_tile, valid_s);
+                fence_proxy_async_smem();
+                mbar_arrive(&bar_kv[c]);
+            }
+            // 2. the next tile's loads go in flight under this tile's products
+            const int rel = (it + 1) % kResolveTiles;
+            if (tt + 1 < t_end) {
+                if (rel == 0) {
+                    // next batch of resolved rows (rare: splits of more than 8 tiles)
+                    named_bar_sync(kBarWork, kAttnWorkThreads);
+                    resolve_rows(p, u, b, nw, wb, (tt + 1) * kAttnTile,
+                                 (int)min((int64_t)kResolveTiles, t_end - (tt + 1)) * kAttnTile, rsrc, rkind);
+                    named_bar_sync(kBarWork, kAttnWorkThreads);
+                }
+                fetch_tile<0, 4>(p, b, rsrc, rkind, rel * kAttnTile, raw);
+            }
+            // 3. online softmax: thread = row (TMEM lane), warps 4g..4g+3 take
+            //    the heads [g*HG, (g+1)*HG) of group g
+            if (soft) {
+                const bool got = ok && mbar_wait(bar_s, (uint32_t)it & 1u);
+                if (!got) ok = false;
+                tc_fence_after();
+                const int row = quarter * 32 + lane;
+                const bool row_valid = valid_s[row] != 0 && got;
+                const uint32_t s_addr = lane_addr + Cfg::kColS + grp * HG;
+                float v[HG];
+                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
+                // does any score exceed its head's running maximum by more than 2^8?
+                bool raise = false;
+                {
+#pragma unroll
+                    for (int g = 0; g < HG / 4; ++g) {
+                        const float4 mm = *reinterpret_cast<const float4 *>(m_run + grp * HG + 4 * g);
+                        raise |= v[4 * g] > mm.x + kRescaleThreshold;
+                        raise |= v[4 * g + 1] > mm.y + kRescaleThreshold;
+                        raise |= v[4 * g + 2] > mm.z + kRescaleThreshold;
+                        raise |= v[4 * g + 3] > mm.w + kRescaleThreshold;
+                    }
+                    raise = named_bar_or(1 + grp, 128, raise);
+                    if (raise) {
+                        // full path: tile maximum per head, new running maximum
+                        float mx[HG];
+#pragma unroll
+                        for (int i = 0; i < HG; ++i) mx[i] = v[i];
+                        warp_transpose_reduce<HG, true>(mx);
+                        store_warp_reduced<HG>(red + quarter * H + grp * HG, mx);
+                        named_bar_sync(1 + grp, 128);
+                        if (quarter == 0 && lane < HG) {
+                            const int h = grp * HG + lane;
+                            const float mt = fmaxf(fmaxf(red[h], red[H + h]), fmaxf(red[2 * H + h], red[3 * H + h]));
+                            const float mo = m_run[h];
+                            float a = 1.0f, mn = mo;
+                            if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt > -INFINITY)) {
+                                mn = mt;
+                                a = (mo == -INFINITY) ? 0.0f : exp2f(mo - mt);
+                                if (mo != -INFINITY) rescale_tile[grp] = it;
+                            }
+                            m_run[h] = mn;
+                            alpha[h] = a;
+                        }
+                        named_bar_sync(1 + grp, 128);
+                    }
+                }
+                // probabilities -> P^T (f16), per-row partial denominators
+                {
+#pragma unroll
+                    for (int g = 0; g < HG / 8; ++g) {
+                        const int h0 = grp * HG + 8 * g;  // first head of these 8
+                        const float4 ma = *reinterpret_cast<const float4 *>(m_run + h0);
+                        const float4 mb = *reinterpret_cast<const float4 *>(m_run + h0 + 4);
+                        const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+                        float al[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                        if (raise) {
+                            const float4 aa = *reinterpret_cast<const float4 *>(alpha + h0);
+                            const float4 ab = *reinterpret_cast<const float4 *>(alpha + h0 + 4);
+                            al[0] = aa.x, al[1] = aa.y, al[2] = aa.z, al[3] = aa.w;
+                            al[4] = ab.x, al[5] = ab.y, al[6] = ab.z, al[7] = ab.w;
+                        }
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const int i = 8 * g + 2 * t;
+                            const float p0 = (mm[2 * t] == -INFINITY) ? 0.0f : exp2f(v[i] - mm[2 * t]);
+                            const float p1 = (mm[2 * t + 1] == -INFINITY) ? 0.0f : exp2f(v[i + 1] - mm[2 * t + 1]);
+                            l_part[i] = fmaf(l_part[i], al[2 * t], p0);
+                            l_part[i + 1] = fmaf(l_part[i + 1], al[2 * t + 1], p1);
+                            const __half2 h2 = __floats2half2_rn(p0, p1);
+                            pk[t] = *reinterpret_cast<const uint32_t *>(&h2);
+                        }
+                        *reinterpret_cast<uint4 *>(p_tile + p_chunk_off<H>(row, h0 >> 3)) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+                // rare: a raise of the running maximum -> rescale this group's
+                // O^T columns (every earlier P*V is complete: the S^T commit of
+                // this tile came after them)
+                if (raise && rescale_tile[grp] == it) {
+#pragma unroll 1
+                    for (int dc = 0; dc < 4; ++dc) {
+#pragma unroll
+                        for (int c = 0; c < HG; c += 8) {
+                            uint32_t r8[8];
+                            const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
+                            tmem_ld8(ta, r8);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha[grp * HG + c + i]);
+                            tmem_st8(ta, r8);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+            }
+            mbar_arrive(bar_p);
+        }
+        // the last tile's P*V
+        if (ntiles > 0 && ok && !mbar_wait(&bar_pv[3], (uint32_t)(ntiles - 1) & 1u)) ok = false;
+        tc_fence_after();
+
+        // ---- final denominators: reduce the per-row partials over the 128 rows ----
+        named_bar_sync(kBarWork, kAttnWorkThreads);
+        if (soft) {
+            warp_transpose_reduce<HG, false>(l_part);
+            store_warp_reduced<HG>(red + quarter * H + grp * HG, l_part);
+        }
+        named_bar_sync(kBarWork, kAttnWorkThreads);
+        if (tid < H) {
+            const float l = (red[tid] + red[H + tid]) + (red[2 * H + tid] + red[3 * H + tid]);
+            l_run[tid] = l;
+            alpha[tid] = l > 0.0f ? 1.0f / l : 0.0f;  // reused as 1 / l
+        }
+        named_bar_sync(kBarWork, kAttnWorkThreads);
+
+        // ---- epilogue: O^T (TMEM) -> o = O / l, staged through the free KV tile
+        //      buffer as [h][512] f32 so the global writes are coalesced 16 B ----
+        {
+            constexpr int HC = HG;
+            const int half = grp;
+            float *stage = reinterpret_cast<float *>(kv_tile);  // [H][512] f32 = H * 2 KiB <= 128 KiB
+#pragma unroll 1
+            for (int dc = 0; dc < 4 && soft; ++dc) {
+                const int dd = dc * 128 + quarter * 32 + lane;
+                float vals[HC];
+                if (ntiles > 0) {
+                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + half * HC;
+                    if (HC == 32) {
+                        uint32_t r32[32];
+                        tmem_ld32(ta, r32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r32[i % 32]);
+                    } else if (HC == 16) {
+                        uint32_t r16[16];
+                        tmem_ld16(ta, r16);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r16[i % 16]);
+                    } else {
                         uint32_t r8[8];
-                        const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
                         tmem_ld8(ta, r8);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha[grp * HG + c + i]);
-                        tmem_st8(ta, r8);
+                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r8[i % 8]);
                     }
-                }
-                tmem_wait_st();
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            if (!got) ok = false;
-        }
-        ok = __syncthreads_and(ok);
-        tc_fence_after();
-        // 4. O^T += V^T * P^T
-        if (tid == 0 && ok) {
-            const uint32_t idesc = idesc_f16_f32(128, H, 1, 1);
-#pragma unroll
-            for (int dc = 0; dc < 4; ++dc) {
-#pragma unroll
-                for (int kk = 0; kk < kAttnTile / 16; ++kk) {
-                    const uint64_t ad = make_sdesc(kv_addr + dc * 32768 + kk * 2048, 16384, 1024, kSw128);
-                    const uint64_t bd = make_sdesc(p_addr + kk * 2 * Cfg::kPGroup, 16, Cfg::kPGroup, Cfg::kPSwizzle);
-                    mma_f16(tmem + Cfg::kColO + dc * H, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-            }
-            tc_commit(bar_o);
-        }
-        // the next tile overwrites KV / P: wait for this tile's P*V
-        if (ok && !mbar_wait(bar_o, it & 1)) ok = false;
-        tc_fence_after();
-        ok = __syncthreads_and(ok);
-    }
-    // ---- final denominators: reduce the per-row partials over the 128 rows ----
-    __syncthreads();
-    warp_transpose_reduce<HG, false>(l_part);
-    store_warp_reduced<HG>(red + quarter * H + grp * HG, l_part);
-    __syncthreads();
-    if (tid < H) {
-        const float l = (red[tid] + red[H + tid]) + (red[2 * H + tid] + red[3 * H + tid]);
-        l_run[tid] = l;
-        alpha[tid] = l > 0.0f ? 1.0f / l : 0.0f;  // reused as 1 / l
-    }
-    __syncthreads();
-
-    // ---- epilogue: O^T (TMEM) -> o = O / l, staged through the free KV tile
-    //      buffer as [h][512] f32 so the global writes are coalesced 16 B ----
-    {
-        constexpr int HC = H / 2;
-        const int half = grp;
-        float *stage = reinterpret_cast<float *>(kv_tile);  // [H][512] f32 = H * 2 KiB <= 128 KiB
-#pragma unroll 1
-        for (int dc = 0; dc < 4; ++dc) {
-            const int dd = dc * 128 + quarter * 32 + lane;
-            float vals[HC];
-            if (it > 0) {
-                const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + half * HC;
-                if (HC == 32) {
-                    uint32_t r32[32];
-                    tmem_ld32(ta, r32);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r32[i % 32]);
-                } else if (HC == 16) {
-                    uint32_t r16[16];
-                    tmem_ld16(ta, r16);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r16[i % 16]);
                 } else {
-                    uint32_t r8[8];
-                    tmem_ld8(ta, r8);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r8[i % 8]);
+                    for (int i = 0; i < HC; ++i) vals[i] = 0.0f;
+                }
+#pragma unroll
+                for (int i = 0; i < HC; ++i) stage[(half * HC + i) * CSA2_D + dd] = vals[i] * alpha[half * HC + i];
+            }
+            named_bar_sync(kBarWork, kAttnWorkThreads);
+            if (p.n_splits == 1) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.o + (int64_t)u * H * CSA2_D);
+                for (int i = tid; i < H * CSA2_D / 8; i += kAttnWorkThreads) {
+                    const float4 x0 = reinterpret_cast<const float4 *>(stage)[2 * i];
+                    const float4 x1 = reinterpret_cast<const float4 *>(stage)[2 * i + 1];
+                    dst[i] = make_uint4((uint32_t)f32_to_bf16_bits(x0.x) | ((uint32_t)f32_to_bf16_bits(x0.y) << 16),
+                                        (uint32_t)f32_to_bf16_bits(x0.z) | ((uint32_t)f32_to_bf16_bits(x0.w) << 16),
+                                        (uint32_t)f32_to_bf16_bits(x1.x) | ((uint32_t)f32_to_bf16_bits(x1.y) << 16),
+                                        (uint32_t)f32_to_bf16_bits(x1.z) | ((uint32_t)f32_to_bf16_bits(x1.w) << 16));
                 }
             } else {
-#pragma unroll
-                for (int i = 0; i < HC; ++i) vals[i] = 0.0f;
+                float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D);
+                for (int i = tid; i < H * CSA2_D / 4; i += kAttnWorkThreads)
+                    dst[i] = reinterpret_cast<const float4 *>(stage)[i];
             }
-#pragma unroll
-            for (int i = 0; i < HC; ++i) stage[(half * HC + i) * CSA2_D + dd] = vals[i] * alpha[half * HC + i];
+            if (tid < H) {
+                const float l = l_run[tid];
+                const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                if (p.n_splits == 1) {
+                    if (p.lse) p.lse[(int64_t)u * H + tid] = lse;
+                } else {
+                    p.lse_part[((int64_t)u * p.n_splits + split) * H + tid] = lse;
+                }
+            }
         }
-        __syncthreads();
-        if (p.n_splits == 1) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.o + (int64_t)u * H * CSA2_D);
-            for (int i = tid; i < H * CSA2_D / 8; i += kAttnThreads) {
-                const float4 x0 = reinterpret_cast<const float4 *>(stage)[2 * i];
-                const float4 x1 = reinterpret_cast<const float4 *>(stage)[2 * i + 1];
-                dst[i] = make_uint4((uint32_t)f32_to_bf16_bits(x0.x) | ((uint32_t)f32_to_bf16_bits(x0.y) << 16),
-                                    (uint32_t)f32_to_bf16_bits(x0.z) | ((uint32_t)f32_to_bf16_bits(x0.w) << 16),
-                                    (uint32_t)f32_to_bf16_bits(x1.x) | ((uint32_t)f32_to_bf16_bits(x1.y) << 16),
-                                    (uint32_t)f32_to_bf16_bits(x1.z) | ((uint32_t)f32_to_bf16_bits(x1.w) << 16));
-            }
-        } else {
-            float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D);
-            for (int i = tid; i < H * CSA2_D / 4; i += kAttnThreads) dst[i] = reinterpret_cast<const float4 *>(stage)[i];
-        }
-        if (tid < H) {
-            const float l = l_run[tid];
-            const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-            if (p.n_splits == 1) {
-                if (p.lse) p.lse[(int64_t)u * H + tid] = lse;
-            } else {
-                p.lse_part[((int64_t)u * p.n_splits + split) * H + tid] = lse;
-            }
         }
     }
     tc_fence_before();

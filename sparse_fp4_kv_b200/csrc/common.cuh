@@ -107,6 +107,45 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
+// Thread-block clusters: a full barrier of every thread of every CTA of the
+// cluster (release / acquire), the CTA's rank, and the address of the same
+// shared-memory object in another CTA of the cluster.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+template <typename T>
+__device__ __forceinline__ T *cluster_peer(T *p, uint32_t rank) {
+    return static_cast<T *>(__cluster_map_shared_rank(const_cast<void *>(static_cast<const void *>(p)), rank));
+}
+
+// Shared-memory address (shared::cluster window) of the same object in CTA
+// `rank` of the cluster, and 16-byte / 4-byte loads through it.
+__device__ __forceinline__ uint32_t cluster_smem_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------------------
 // TMA (non-multicast tile loads only)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *tm, uint64_t *bar, int32_t x,

@@ -139,6 +139,11 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
 }
 
 // ---- attention planning ------------------------------------------------------
+// A query's attended rows are cut into `splits` runs of `tiles_per_split`
+// tiles, one CTA each; split runs are merged through f32 partials in the
+// workspace by a second kernel. Cost in tile-times: waves of CTAs times the
+// tiles of a CTA plus a fixed charge for its prologue and epilogue, plus a
+// charge per split for writing and merging the partials.
 struct AttnPlan {
     int32_t tiles, tiles_per_split, splits;
 };
@@ -147,14 +152,19 @@ AttnPlan plan_attn(int32_t nq, int32_t k, int32_t w_max, int sms) {
     AttnPlan P{};
     const int64_t rows = (int64_t)k + std::max(0, w_max);
     P.tiles = (int32_t)std::max<int64_t>(1, (rows + kAttnTile - 1) / kAttnTile);
+    // a fixed split count (tuning and tests), else the cost model
+    if (const char *e = std::getenv("CSA2_ATTN_SPLITS")) {
+        const int32_t want = std::max(1, std::min(P.tiles, (int32_t)std::atoi(e)));
+        P.tiles_per_split = (P.tiles + want - 1) / want;
+        P.splits = (P.tiles + P.tiles_per_split - 1) / P.tiles_per_split;
+        return P;
+    }
+    constexpr double kFixed = 1.2, kMergePerSplit = 0.1;
     double best = 1e30;
     for (int32_t tps = 1; tps <= P.tiles; ++tps) {
         const int32_t splits = (P.tiles + tps - 1) / tps;
-        const int64_t ctas = (int64_t)nq * splits;
-        const int64_t waves = (ctas + sms - 1) / sms;
-        // tile-times on the critical path, plus a small charge for the
-        // partial outputs and the combine pass when a query is split
-        const double cost = (double)waves * tps + (splits > 1 ? 0.35 + 0.02 * splits : 0.0);
+        const double waves = (double)(((int64_t)nq * splits + sms - 1) / sms);
+        const double cost = waves * (tps + kFixed) + (splits > 1 ? kMergePerSplit * splits : 0.0);
         if (cost < best - 1e-9) {
             best = cost;
             P.tiles_per_split = tps;
@@ -168,6 +178,7 @@ struct AttnLayout {
     size_t off_o, off_lse, total;
 };
 
+// Split partials: f32 [nq][S][H][512], then the log-sum-exp values [nq][S][H].
 AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P) {
     AttnLayout L{};
     if (P.splits <= 1) return L;
@@ -528,6 +539,7 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
 
 size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max) {
     if (nq <= 0 || h <= 0 || k < 0) return 0;
+    if (h != 16 && h != 32 && h != 64) return 0;
     const AttnPlan P = plan_attn(nq, k, w_max, num_sms());
     return attn_layout(nq, h, P).total;
 }
@@ -573,23 +585,24 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
     ap.n_splits = P.splits;
     ap.tiles_per_split = P.tiles_per_split;
     const dim3 grid((unsigned)P.splits, (unsigned)nq);
+    auto go = [&](auto kernel, size_t smem) { launch(kernel, grid, dim3(kAttnThreads), smem, stream, ap); };
     switch (h) {
         case 64: {
             static bool ok = set_smem(k_sparse_attn<64>, AttnCfg<64>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            launch(k_sparse_attn<64>, grid, dim3(kAttnThreads), AttnCfg<64>::kSmem, stream, ap);
+            go(k_sparse_attn<64>, AttnCfg<64>::kSmem);
             break;
         }
         case 32: {
             static bool ok = set_smem(k_sparse_attn<32>, AttnCfg<32>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            launch(k_sparse_attn<32>, grid, dim3(kAttnThreads), AttnCfg<32>::kSmem, stream, ap);
+            go(k_sparse_attn<32>, AttnCfg<32>::kSmem);
             break;
         }
         default: {
             static bool ok = set_smem(k_sparse_attn<16>, AttnCfg<16>::kSmem);
             if (!ok) return CSA2_ERR_CUDA;
-            launch(k_sparse_attn<16>, grid, dim3(kAttnThreads), AttnCfg<16>::kSmem, stream, ap);
+            go(k_sparse_attn<16>, AttnCfg<16>::kSmem);
             break;
         }
     }

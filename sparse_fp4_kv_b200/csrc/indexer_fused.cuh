@@ -30,18 +30,6 @@ constexpr int kFusedClusterSmall = 8;
 constexpr int kFusedClusterLarge = 16;
 constexpr int kFusedThreads = 256;
 
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-template <typename T>
-__device__ __forceinline__ T *cluster_peer(T *p, uint32_t rank) {
-    return static_cast<T *>(__cluster_map_shared_rank(static_cast<void *>(p), rank));
-}
 
 // Sum the local histograms h[0..nbins) (same shared-memory offset in every
 // CTA of the cluster) over the cluster into full[0..nbins). CTA r first

@@ -89,6 +89,16 @@ def test_single_query_many_tiles_split(B, cuda_device):
     _run(B, cuda_device, [70000], 128, 64, 2048, 512, seed=1)
 
 
+@pytest.mark.parametrize("splits", ["1", "3", "7", "auto"])
+def test_several_queries_split_ragged(B, cuda_device, monkeypatch, splits):
+    # several queries with ragged row counts, 32 and 16 heads, the split
+    # count fixed (1: no merge; 3, 7: ragged last split) or chosen by the plan
+    if splits != "auto":
+        monkeypatch.setenv("CSA2_ATTN_SPLITS", splits)
+    _run(B, cuda_device, [9000, 5000, 3000], 64, 32, 1300, 200, seed=21)
+    _run(B, cuda_device, [9000, 7000], 64, 16, 1800, 300, seed=22)
+
+
 def test_many_queries_single_split(B, cuda_device):
     # enough queries that each one runs in a single CTA
     _run(B, cuda_device, [600] * 4, 64, 32, 256, 33, q_per_seq=80, seed=2, swa_rows=160)
