@@ -20,6 +20,7 @@ its own independent batch of sequences (weak scaling, no collective on the
 data path).
 """
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -39,7 +40,7 @@ UNIT = "query-steps/s/layer"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="stack20")
@@ -113,43 +114,53 @@ def recorded_traffic(kernel, workload):
 # clocks sampler
 # ---------------------------------------------------------------------------
 class Clocks:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 50 ms; only the samples taken between mark()
+    calls (the timed region) are summarised."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.window = [None, None]
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+
+    def mark(self, which):
+        self.window[which] = datetime.datetime.now()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[2]), float(parts[3]),
+                             [n for n, v in zip(names, parts[6:10]) if v.lower() == "active"]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        t0, t1 = self.window
+        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        use = inside if inside else rows
+        reasons = sorted({n for r in use for n in r[3]})
+        return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
+                "sm_max_mhz": max(r[2] for r in use) if use else None, "reasons": reasons,
+                "samples": len(use), "samples_in_timed_region": len(inside),
+                "power_w_note": "50 ms nvidia-smi sampling"}
 
 
 # ---------------------------------------------------------------------------
@@ -252,8 +263,9 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
+    from sparse_fp4_kv_b200.ranks import job_throughput, max_over_ranks, rank_recipe
     base = RECIPES[args.workload]
-    recipe = base.scaled(seed=base.seed + 1000 * rank) if world > 1 else base
+    recipe = rank_recipe(base, rank, world)
     dec = Csa2Decoder(recipe, dev)
     by, fl, attn_by, attn_fl = algorithmic(recipe, dec.lens, dec.schedule)
 
@@ -342,9 +354,11 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     clocks = Clocks(local)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.2)  # the sampler is running
+    clocks.mark(0)
     per_step, _ = timed_steps(graph, args.steps, False)
     torch.cuda.synchronize(dev)
+    clocks.mark(1)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -352,14 +366,8 @@ def run_ours(args):
     _, attn = timed_steps(graph_ev, args.steps, True)
     if B.csa2_device_status(stream) != 0:
         raise RuntimeError("device error during the timed steps")
-    total_ms = sum(per_step)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    ms = total_ms / args.steps
-    units = recipe.nq * recipe.layers * world
-    value = units / (ms * 1e-3)
+    total_ms = max_over_ranks(sum(per_step), dev)
+    value, ms = job_throughput(recipe.nq * recipe.layers, world, total_ms, args.steps)
 
     # e2e: host buffers in pinned memory, copies inside the timed region
     e2e = None
