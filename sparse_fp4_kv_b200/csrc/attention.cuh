@@ -599,59 +599,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         }
         named_bar_sync(kBarWork, kAttnWorkThreads);
 
-        // ---- epilogue: O^T (TMEM) -> o = O / l, staged through the free KV tile
-        //      buffer as [h][512] f32 so the global writes are coalesced 16 B ----
+        // ---- epilogue: O^T (TMEM) -> o = O / l written straight from registers:
+        //      a thread owns latent column d = 128*dc + 32*quarter + lane of its
+        //      group's heads, so each store instruction of a warp covers 32
+        //      consecutive columns of one head (coalesced); the four TMEM loads
+        //      of a thread are in flight together ----
         {
-            constexpr int HC = HG;
-            const int half = grp;
-            float *stage = reinterpret_cast<float *>(kv_tile);  // [H][512] f32 = H * 2 KiB <= 128 KiB
-#pragma unroll 1
-            for (int dc = 0; dc < 4 && soft; ++dc) {
-                const int dd = dc * 128 + quarter * 32 + lane;
-                float vals[HC];
+            if (soft) {
+                uint32_t vals[4][HG];  // raw f32 bits
                 if (ntiles > 0) {
-                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + half * HC;
-                    if (HC == 32) {
-                        uint32_t r32[32];
-                        tmem_ld32(ta, r32);
-                        tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r32[i % 32]);
-                    } else if (HC == 16) {
-                        uint32_t r16[16];
-                        tmem_ld16(ta, r16);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r16[i % 16]);
-                    } else {
-                        uint32_t r8[8];
-                        tmem_ld8(ta, r8);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < HC; ++i) vals[i] = __uint_as_float(r8[i % 8]);
+                    for (int dc = 0; dc < 4; ++dc) {
+                        const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + grp * HG;
+                        if (HG == 16) {
+                            tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&vals[dc][0]));
+                        } else {
+                            tmem_ld8(ta, *reinterpret_cast<uint32_t(*)[8]>(&vals[dc][0]));
+                        }
                     }
+                    tmem_wait_ld();
                 } else {
 #pragma unroll
-                    for (int i = 0; i < HC; ++i) vals[i] = 0.0f;
-                }
+                    for (int dc = 0; dc < 4; ++dc)
 #pragma unroll
-                for (int i = 0; i < HC; ++i) stage[(half * HC + i) * CSA2_D + dd] = vals[i] * alpha[half * HC + i];
-            }
-            named_bar_sync(kBarWork, kAttnWorkThreads);
-            if (p.n_splits == 1) {
-                uint4 *dst = reinterpret_cast<uint4 *>(p.o + (int64_t)u * H * CSA2_D);
-                for (int i = tid; i < H * CSA2_D / 8; i += kAttnWorkThreads) {
-                    const float4 x0 = reinterpret_cast<const float4 *>(stage)[2 * i];
-                    const float4 x1 = reinterpret_cast<const float4 *>(stage)[2 * i + 1];
-                    dst[i] = make_uint4((uint32_t)f32_to_bf16_bits(x0.x) | ((uint32_t)f32_to_bf16_bits(x0.y) << 16),
-                                        (uint32_t)f32_to_bf16_bits(x0.z) | ((uint32_t)f32_to_bf16_bits(x0.w) << 16),
-                                        (uint32_t)f32_to_bf16_bits(x1.x) | ((uint32_t)f32_to_bf16_bits(x1.y) << 16),
-                                        (uint32_t)f32_to_bf16_bits(x1.z) | ((uint32_t)f32_to_bf16_bits(x1.w) << 16));
+                        for (int i = 0; i < HG; ++i) vals[dc][i] = 0u;
                 }
-            } else {
-                float4 *dst = reinterpret_cast<float4 *>(p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D);
-                for (int i = tid; i < H * CSA2_D / 4; i += kAttnWorkThreads)
-                    dst[i] = reinterpret_cast<const float4 *>(stage)[i];
+                const int d0 = quarter * 32 + lane;
+                if (p.n_splits == 1) {
+                    uint16_t *dst = p.o + (int64_t)u * H * CSA2_D;
+#pragma unroll
+                    for (int i = 0; i < HG; ++i) {
+                        const int h = grp * HG + i;
+                        const float inv = alpha[h];
+#pragma unroll
+                        for (int dc = 0; dc < 4; ++dc)
+                            dst[(int64_t)h * CSA2_D + dc * 128 + d0] = f32_to_bf16_bits(__uint_as_float(vals[dc][i]) * inv);
+                    }
+                } else {
+                    float *dst = p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D;
+#pragma unroll
+                    for (int i = 0; i < HG; ++i) {
+                        const int h = grp * HG + i;
+                        const float inv = alpha[h];
+#pragma unroll
+                        for (int dc = 0; dc < 4; ++dc)
+                            dst[(int64_t)h * CSA2_D + dc * 128 + d0] = __uint_as_float(vals[dc][i]) * inv;
+                    }
+                }
             }
             if (tid < H) {
                 const float l = l_run[tid];
