@@ -78,6 +78,72 @@ def algorithmic(recipe, lens, schedule):
     return by, fl, attn_by, attn_fl
 
 
+def step_roofline_us(recipe, lens, schedule, hbm_gbs, tc_tflops):
+    """t_roof of one step in microseconds: the sum over the step's kernels of
+    max(algorithmic bytes / HBM peak, flops / tensor peak); the indexer's
+    FP8 products are counted at twice the bf16 peak."""
+    nq, h, d = recipe.nq, recipe.h, 512
+    n_vis = [int(l) for l in lens.tolist()]
+    bw, tc = hbm_gbs * 1e9, tc_tflops * 1e12
+    rows_app = recipe.append if recipe.chunked else recipe.batch
+    t = rows_app * (d * 2 + d // 2 + d // 16) / bw
+    parts = {"append": t}
+    for mode, src in schedule:
+        if mode == "full":
+            b = f = 0.0
+            for qi in range(nq):
+                n = n_vis[qi // recipe.q_per_seq]
+                b += n * recipe.di
+                f += 2.0 * recipe.hi * recipe.di * n
+            parts["full"] = parts.get("full", 0.0) + max(b / bw, f / (2 * tc))
+        elif mode == "reindex":
+            b = nq * recipe.p * (recipe.di + 4)
+            f = 2.0 * nq * recipe.hi * recipe.di * recipe.p
+            parts["reindex"] = parts.get("reindex", 0.0) + max(b / bw, f / (2 * tc))
+        a_by = nq * (recipe.k * (d // 2 + d // 16 + 4) + recipe.w * d + 2 * 2 * h * d)
+        a_fl = 4.0 * nq * h * (recipe.k + recipe.w) * d
+        parts["attention"] = parts.get("attention", 0.0) + max(a_by / bw, a_fl / tc)
+    return sum(parts.values()) * 1e6, {k: v * 1e6 for k, v in parts.items()}
+
+
+def time_append_chunk512(B, dev, hbm_gbs, reps=20):
+    """The 32,768-row FP4 append of the chunked-prefill workload (a 256K-entry
+    cache), timed on its own: CUDA events around each call, L2 flushed before
+    each."""
+    import torch
+    from sparse_fp4_kv_b200.workloads import RECIPES
+    r = RECIPES["chunk512"]
+    cap, n = r.cap, r.append
+    codes = torch.zeros((cap, 256), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((cap, 32), dtype=torch.uint8, device=dev)
+    kidx = torch.zeros((cap, r.di), dtype=torch.uint8, device=dev)
+    pt = torch.zeros((1, 1), dtype=torch.int32, device=dev)
+    sl = torch.full((1,), cap, dtype=torch.int32, device=dev)
+    kv = B.KvCache(codes, scales, kidx, pt, sl, cap)
+    x = r.latent_rows(0, r.prefill, r.prefill + n, dev).contiguous()
+    seq = torch.zeros(n, dtype=torch.int32, device=dev)
+    pos = torch.arange(r.prefill, r.prefill + n, dtype=torch.int64, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        B.csa2_append_fp4(x, seq, pos, kv)
+    ts = []
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.csa2_append_fp4(x, seq, pos, kv)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    us = ts[len(ts) // 2]
+    by = n * (512 * 2 + 256 + 32)
+    return {"rows": n, "us_median": us, "algorithmic_bytes": by, "achieved_gbs": by / (us * 1e-6) / 1e9,
+            "peak_gbs": hbm_gbs, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+            "note": "bf16 rows in, FP4 codes + E4M3 scales out, 256K-entry cache; CUDA events around the call "
+                    "(launch included), median of %d after an L2 flush" % reps}
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -210,6 +276,37 @@ def reference_layers(recipe):
     end = modes.find("R")
     end = len(modes) if end < 0 else end + 1
     return list(range(min(end, 6)))
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def _oracle_worker(job):
+    recipe, seq, layers = job
+    return oracle_sample(recipe, layers, seq)
+
+
+def oracle_all_cores(recipe, layers):
+    """The oracle on independent sequences at once, one process each (spawned,
+    no GPU), up to one per core: units of all processes over the longest
+    process's compute time."""
+    import multiprocessing as mp
+    procs = max(1, min(os.cpu_count() or 1, recipe.batch))
+    with mp.get_context("spawn").Pool(procs) as pool:
+        res = pool.map(_oracle_worker, [(recipe, s, layers) for s in range(procs)])
+    dt = max(r[0] for r in res)
+    n = sum(r[1] for r in res)
+    return {"value": n / dt, "unit": UNIT, "cores": procs,
+            "sample": f"sequences 0..{procs - 1}, layers {layers[0]}..{layers[-1]}, one process per sequence "
+                      f"({dt:.1f} s)"}
 
 
 def run_reference(args):
@@ -375,6 +472,10 @@ def run_ours(args):
         e2e = run_e2e(args, dec, stream, flush, graph_fn=step_with_events, world=world, dev=dev)
 
     hbm_gbs, bf16_burst, bf16_sust, peak_kind = peaks()
+    t_roof, t_parts = step_roofline_us(recipe, dec.lens, dec.schedule, hbm_gbs, bf16_sust)
+    step_rl = {"t_roof_us": t_roof, "parts_us": t_parts, "step_us": ms * 1e3, "frac": t_roof / (ms * 1e3),
+               "peaks": f"{peak_kind}: {hbm_gbs} GB/s HBM, {bf16_sust} TF/s bf16 sustained (FP8 at 2x)"}
+    append_c4 = time_append_chunk512(B, dev, hbm_gbs) if world == 1 else None
     breakdown = {k: 1e3 * statistics.mean(v) for k, v in attn.items()}
     attn_ms = statistics.mean(attn["attention"]) if attn else float("nan")
     achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
@@ -397,6 +498,8 @@ def run_ours(args):
                      "split combine) in the instrumented replay", "flops_per_launch": attn_fl, "bytes_per_launch": attn_by,
                      "hbm_frac": attn_by / (attn_ms * 1e-3) / (hbm_gbs * 1e9),
                      "traffic": recorded_traffic(kernel, recipe.name)},
+        "step_roofline": step_rl,
+        "append_chunk512": append_c4,
         "breakdown_us_per_call": breakdown,
         "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented replay "
                           "of the same step (event nodes between calls prevent launch overlap)",
@@ -412,7 +515,8 @@ def run_ours(args):
         line["cpu_baseline"] = {
             "value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"sequence 0, layers {layers[0]}..{layers[-1]} of {recipe.name}, single-threaded C oracle "
-                      f"({dt:.1f} s)"}
+                      f"({dt:.1f} s)", "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "all_cores": oracle_all_cores(recipe, layers)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, graph_ev
