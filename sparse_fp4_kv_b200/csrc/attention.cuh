@@ -669,11 +669,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
 
 // Merge the splits of each query: o = sum_s exp(lse_s - M) o_s / L,
 // lse = M + log L with M = max_s lse_s, L = sum_s exp(lse_s - M).
-// One CTA per (query, 4 heads); each thread owns one float4 of a head and
-// loads that float4 of every split before combining, so the loads overlap.
+// One CTA per (query, head); each thread owns one float4 of the head and
+// puts the loads of that float4 of the first 16 splits in flight before the
+// weights are computed, so the two memory latencies overlap.
 constexpr int kCombineThreads = 128;
-constexpr int kCombineHeads = 1;  // heads per CTA (128 float4 per head)
-constexpr int kCombineBatch = 8;  // split loads in flight per thread
+constexpr int kCombineHeads = 1;   // heads per CTA (128 float4 per head)
+constexpr int kCombineBatch = 16;  // split loads in flight per thread
 
 template <int H>
 __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *__restrict__ o_part,
@@ -686,6 +687,12 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
     const int32_t u = blockIdx.y;
     const int h = blockIdx.x;
     const int d4 = threadIdx.x;  // 128 threads x 4 values = 512
+    const float *src = o_part + ((int64_t)u * n_splits * H + h) * CSA2_D;
+    float4 v[kCombineBatch];
+#pragma unroll
+    for (int t = 0; t < kCombineBatch; ++t)
+        v[t] = t < n_splits ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)t * H * CSA2_D) + d4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
     if (threadIdx.x < 32) {
         float M = -INFINITY;
         for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, lse_part[((int64_t)u * n_splits + s) * H + h]);
@@ -706,15 +713,15 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
         }
     }
     __syncthreads();
-    const float *src = o_part + ((int64_t)u * n_splits * H + h) * CSA2_D;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < n_splits; s0 += kCombineBatch) {
-        float4 v[kCombineBatch];
+        if (s0 > 0) {
 #pragma unroll
-        for (int t = 0; t < kCombineBatch; ++t)
-            v[t] = (s0 + t < n_splits)
-                       ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(s0 + t) * H * CSA2_D) + d4)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int t = 0; t < kCombineBatch; ++t)
+                v[t] = (s0 + t < n_splits)
+                           ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(s0 + t) * H * CSA2_D) + d4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int t = 0; t < kCombineBatch; ++t) {
             if (s0 + t >= n_splits) break;
