@@ -36,6 +36,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
     if (r >= n) return;
+    // the row's values are loaded first, in flight while its destination is
+    // looked up (sequence, position, page table)
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
     const int32_t b = seq[r];
     int64_t row = -1;
     if (b >= 0 && b < kv.batch) row = physical_row(kv, b, pos[r]);
@@ -43,10 +47,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
         if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
         return;
     }
-    // 16 bf16 values of this lane's block
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16);
-    uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float f[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {

@@ -251,51 +251,54 @@ cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Attributes of the single-launch Full kernels (maximal dynamic shared
-// memory; 16-CTA clusters need the non-portable size), set once, and how many
-// 16-CTA clusters of the kernel the device holds at once (0 if none, or if a
-// call failed).
+// Attributes of the single-launch Full kernel (maximal dynamic shared
+// memory; clusters above 8 CTAs need the non-portable size), set once, and
+// how many clusters of each size the device holds at once (0: not possible).
 template <int DI>
-bool fused_attrs() {
-    static const bool ok = [] {
-        bool good = set_smem(k_index_full_fused<DI, kFusedClusterSmall>, (size_t)max_smem_optin()) &&
-                    set_smem(k_index_full_fused<DI, kFusedClusterLarge>, (size_t)max_smem_optin());
-        if (cudaFuncSetAttribute(k_index_full_fused<DI, kFusedClusterLarge>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+const int *fused_cluster_caps() {
+    static int caps[kFusedClusterMax + 1];
+    static std::once_flag once;
+    std::call_once(once, [] {
+        for (int c = 0; c <= kFusedClusterMax; ++c) caps[c] = 0;
+        if (!set_smem(k_index_full_fused<DI>, (size_t)max_smem_optin())) return;
+        if (cudaFuncSetAttribute(k_index_full_fused<DI>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
             cudaGetLastError();
-            good = false;
+        for (int c = kFusedClusterMin; c <= kFusedClusterMax; ++c) {
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)c;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)c, 1);
+            cfg.blockDim = dim3(kFusedThreads);
+            cfg.dynamicSmemBytes = (size_t)max_smem_optin() - 1024;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, k_index_full_fused<DI>, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                n = 0;
+            }
+            caps[c] = n;
         }
-        return good;
-    }();
-    return ok;
+    });
+    return caps;
 }
 
-int fused_clusters_of_16(bool di64) {
-    static int n[2] = {-1, -1};
-    int &v = n[di64 ? 1 : 0];
-    if (v >= 0) return v;
-    v = 0;
-    if (!(di64 ? fused_attrs<64>() : fused_attrs<128>())) return v;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kFusedClusterLarge;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kFusedClusterLarge, 1);
-    cfg.blockDim = dim3(kFusedThreads);
-    cfg.dynamicSmemBytes = (size_t)max_smem_optin() - 1024;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int c = 0;
-    const cudaError_t e = di64 ? cudaOccupancyMaxActiveClusters(&c, k_index_full_fused<64, kFusedClusterLarge>, &cfg)
-                               : cudaOccupancyMaxActiveClusters(&c, k_index_full_fused<128, kFusedClusterLarge>, &cfg);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        c = 0;
+// CTAs per query for the single-launch Full kernel: the largest size whose
+// clusters the device holds for all queries at once, as long as every CTA
+// keeps at least two tiles of entries; the portable 8 otherwise.
+int fused_cluster_size(bool di64, int32_t nq, int64_t n_max, int tile_entries) {
+    const int *caps = di64 ? fused_cluster_caps<64>() : fused_cluster_caps<128>();
+    if (const char *e = std::getenv("CSA2_FULL_CLUSTER")) {
+        const int c = std::atoi(e);
+        if (c >= kFusedClusterMin && c <= kFusedClusterMax && caps[c] > 0) return c;
     }
-    v = c;
-    return v;
+    for (int c = kFusedClusterMax; c > kFusedClusterMin; --c)
+        if (caps[c] >= nq && n_max >= (int64_t)c * 2 * tile_entries) return c;
+    return kFusedClusterMin;
 }
 
 template <typename K>
@@ -392,9 +395,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     // holds one for every query at once, else 8.
     {
         const bool di64 = kv->di == 64;
-        const int cl = (fused_clusters_of_16(di64) >= nq && n_max >= (int64_t)kFusedClusterLarge * 2 * tile_entries)
-                           ? kFusedClusterLarge
-                           : kFusedClusterSmall;
+        const int cl = fused_cluster_size(di64, nq, n_max, tile_entries);
         const int64_t slice = (int64_t)align_up((size_t)((std::max<int64_t>(n_max, 1) + cl - 1) / cl),
                                                 (size_t)tile_entries);
         const size_t stage_bytes = 128 * 128;
@@ -422,16 +423,12 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
             fp.stages = stages;
             const dim3 fgrid((unsigned)cl, (unsigned)nq);
             const size_t smem = di64 ? FusedCfg<64>::smem((int)slice, stages) : FusedCfg<128>::smem((int)slice, stages);
-            auto go = [&](auto kernel) {
-                launch_cluster(kernel, fgrid, dim3(kFusedThreads), smem, stream, (unsigned)cl, tm, fp);
-            };
-            if (di64) {
-                if (cl == kFusedClusterLarge) go(k_index_full_fused<64, kFusedClusterLarge>);
-                else go(k_index_full_fused<64, kFusedClusterSmall>);
-            } else {
-                if (cl == kFusedClusterLarge) go(k_index_full_fused<128, kFusedClusterLarge>);
-                else go(k_index_full_fused<128, kFusedClusterSmall>);
-            }
+            fp.csize = cl;
+            if (di64)
+                launch_cluster(k_index_full_fused<64>, fgrid, dim3(kFusedThreads), smem, stream, (unsigned)cl, tm, fp);
+            else
+                launch_cluster(k_index_full_fused<128>, fgrid, dim3(kFusedThreads), smem, stream, (unsigned)cl, tm,
+                               fp);
             return check_launch();
         }
     }

@@ -24,10 +24,10 @@
 
 namespace csa2 {
 
-// CTAs per query: 8 (portable), or 16 when the device can hold a cluster of
-// 16 such CTAs for every query at once.
-constexpr int kFusedClusterSmall = 8;
-constexpr int kFusedClusterLarge = 16;
+// CTAs per query: the largest cluster size up to kFusedClusterMax that the
+// device holds for every query at once (8, the portable size, otherwise).
+constexpr int kFusedClusterMin = 8;
+constexpr int kFusedClusterMax = 16;
 constexpr int kFusedThreads = 256;
 
 
@@ -35,21 +35,34 @@ constexpr int kFusedThreads = 256;
 // CTA of the cluster) over the cluster into full[0..nbins). CTA r first
 // sums bins [r*nbins/C, (r+1)*nbins/C) from every CTA into slice[], then
 // every CTA gathers all slices.
-template <int CL>
 __device__ __forceinline__ void cluster_hist_sum(uint32_t *h, uint32_t *slice, uint32_t *full, int nbins,
-                                                 uint32_t rank) {
-    const int per = nbins / CL;
+                                                 uint32_t rank, int CL) {
+    const int per = (nbins + CL - 1) / CL;  // bins summed by each CTA (the last one may sum fewer)
+    const int base = (int)rank * per;
     cluster_sync_all();  // every CTA's local histogram is complete
-    for (int i = threadIdx.x; i < per; i += kFusedThreads) {
+    // distributed shared memory loads have a long latency: each thread puts
+    // the loads of all CTAs (reduce) or of four bins (gather) in flight at once
+    for (int i = threadIdx.x; i < per && base + i < nbins; i += kFusedThreads) {
+        uint32_t v[kFusedClusterMax];
+#pragma unroll
+        for (int r = 0; r < kFusedClusterMax; ++r) v[r] = r < CL ? cluster_peer(h, (uint32_t)r)[base + i] : 0u;
         uint32_t s = 0;
 #pragma unroll
-        for (int r = 0; r < CL; ++r) s += cluster_peer(h, (uint32_t)r)[rank * per + i];
+        for (int r = 0; r < kFusedClusterMax; ++r) s += v[r];
         slice[i] = s;
     }
     cluster_sync_all();
-    for (int i = threadIdx.x; i < nbins; i += kFusedThreads) {
-        const int owner = i / per;
-        full[i] = cluster_peer(slice, (uint32_t)owner)[i - owner * per];
+    for (int i0 = threadIdx.x; i0 < nbins; i0 += 4 * kFusedThreads) {
+        uint32_t v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * kFusedThreads;
+            const int owner = i / per;
+            v[j] = i < nbins ? cluster_peer(slice, (uint32_t)owner)[i - owner * per] : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i0 + j * kFusedThreads < nbins) full[i0 + j * kFusedThreads] = v[j];
     }
     __syncthreads();
     // No closing cluster barrier: peers read h only before the second barrier
@@ -69,6 +82,7 @@ struct FusedParams {
     int32_t box_rows;
     int32_t slice;    // entries per CTA (multiple of 128)
     int32_t stages;   // TMA ring depth
+    int32_t csize;    // CTAs per query (cluster size)
 };
 
 template <int DI>
@@ -81,7 +95,7 @@ struct FusedCfg {
     }
 };
 
-template <int DI, int CL>
+template <int DI>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     k_index_full_fused(const __grid_constant__ CUtensorMap tm, FusedParams p) {
     using Cfg = FusedCfg<DI>;
@@ -175,7 +189,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         rem[tau] = (uint32_t)max(p.rank[tau], 0);
     }
     // digit 0 (bits 31..20): the histogram built during the scan
-    cluster_hist_sum<CL>(hist0, slice, full, 4096, crank);
+    cluster_hist_sum(hist0, slice, full, 4096, crank, p.csize);
     #pragma unroll
     for (int tau = 0; tau < 2; ++tau)
         if (act[tau]) find_rank_bin<kFusedThreads, 4096 / kFusedThreads, false>(full, 4096, rem[tau], scratch,
@@ -215,7 +229,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         hist_add_warp(nh + tau * 1024, m[tau][j] ? (kk[j] >> (shift - 10)) & 1023u : 0xFFFFFFFFu);
         }
         __syncthreads();
-        cluster_hist_sum<CL>(nh, slice, full, 2048, crank);
+        cluster_hist_sum(nh, slice, full, 2048, crank, p.csize);
         #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
             if (!act[tau]) continue;
@@ -292,10 +306,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             continue;
         }
         uint32_t base_gt = 0, base_eq = 0;
-        for (uint32_t r = 0; r < crank; ++r) {
-            const uint32_t *pc = cluster_peer(cnt, r);
-            base_gt += pc[2 * tau];
-            base_eq += pc[2 * tau + 1];
+        {
+            uint32_t g[kFusedClusterMax], e[kFusedClusterMax];  // all remote loads in flight at once
+#pragma unroll
+            for (int r = 0; r < kFusedClusterMax; ++r) {
+                const bool before = (uint32_t)r < crank;
+                const uint32_t *pc = cluster_peer(cnt, before ? (uint32_t)r : crank);
+                g[r] = before ? pc[2 * tau] : 0u;
+                e[r] = before ? pc[2 * tau + 1] : 0u;
+            }
+#pragma unroll
+            for (int r = 0; r < kFusedClusterMax; ++r) {
+                base_gt += g[r];
+                base_eq += e[r];
+            }
         }
         const uint32_t need = rem[tau];
         // equal keys before this warp, and the output position of its first id

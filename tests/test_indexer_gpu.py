@@ -101,9 +101,12 @@ def test_full_causal_queries(B, cuda_device):
               shuffle=False)
 
 
-def test_full_long_sequences_ragged(B, cuda_device):
-    # long enough that a query's entries are spread over 16 CTAs (when the
-    # device holds 16-CTA clusters for every query), with ragged tails
+@pytest.mark.parametrize("csize", ["auto", "10", "12", "16"])
+def test_full_long_sequences_ragged(B, cuda_device, monkeypatch, csize):
+    # long enough that a query's entries are spread over 8 to 16 CTAs (the
+    # cluster size chosen by the library, or fixed), with ragged tails
+    if csize != "auto":
+        monkeypatch.setenv("CSA2_FULL_CLUSTER", csize)
     _run_full(B, cuda_device, [40000 + 17, 33333], 40064, 64, 4, 2048, 4096, shuffle=False, seed=14)
     _run_full(B, cuda_device, [36000 + 5], 36096, 128, 8, 1000, 3000, shuffle=False, seed=15)
 
