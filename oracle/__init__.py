@@ -50,6 +50,9 @@ def lib():
             "orc_sparse_attn": (None, [c_u16p, i32, i32, c_u8p, c_u8p, c_i32p, i32, c_i32p, i32,
                                        c_u8p, i32, ctypes.c_double, c_f64p, c_f64p]),
             "orc_dequant_row": (None, [c_u8p, c_u8p, i32, c_f64p]),
+            "orc_e4m3_row": (None, [c_u16p, i32, c_u8p]),
+            "orc_append_swa_e4m3": (None, [c_u16p, i32, c_i32p, c_i64p, i64, c_u8p]),
+            "orc_append_kidx_e4m3": (None, [c_u16p, i32, i32, c_i32p, c_i64p, c_i32p, i32, i32, c_u8p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -121,6 +124,37 @@ def append_fp4(x_bf16_bits, seq, pos, page_table, page_size, codes, scales):
     lib().orc_append_fp4(_p(x, ctypes.c_uint16), n, d, _p(seq, ctypes.c_int32),
                          _p(pos, ctypes.c_int64), _p(pt, ctypes.c_int32), pt.shape[1],
                          int(page_size), _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8))
+
+
+def e4m3_row(x_bf16_bits):
+    """bf16 bits [width] -> E4M3 codes [width] (RNE, saturating, no scale)."""
+    x = _c(x_bf16_bits, np.uint16).reshape(-1)
+    out = np.zeros(x.shape[0], np.uint8)
+    lib().orc_e4m3_row(_p(x, ctypes.c_uint16), x.shape[0], _p(out, ctypes.c_uint8))
+    return out
+
+
+def append_swa_e4m3(x_bf16_bits, seq, pos, swa):
+    """Window rows into the ring buffer swa [batch][ring_rows][512] in place."""
+    x = _c(x_bf16_bits, np.uint16)
+    n = x.shape[0]
+    seq = _c(seq, np.int32)
+    pos = _c(pos, np.int64)
+    assert swa.dtype == np.uint8 and swa.flags["C_CONTIGUOUS"] and swa.shape[2] == 512
+    lib().orc_append_swa_e4m3(_p(x, ctypes.c_uint16), n, _p(seq, ctypes.c_int32), _p(pos, ctypes.c_int64),
+                              swa.shape[1], _p(swa, ctypes.c_uint8))
+
+
+def append_kidx_e4m3(x_bf16_bits, seq, pos, page_table, page_size, kidx):
+    """Indexer keys into the (paged) key array kidx [rows][di] in place."""
+    x = _c(x_bf16_bits, np.uint16)
+    n, di = x.shape
+    seq = _c(seq, np.int32)
+    pos = _c(pos, np.int64)
+    pt = _c(page_table, np.int32)
+    assert kidx.dtype == np.uint8 and kidx.flags["C_CONTIGUOUS"] and kidx.shape[1] == di
+    lib().orc_append_kidx_e4m3(_p(x, ctypes.c_uint16), n, di, _p(seq, ctypes.c_int32), _p(pos, ctypes.c_int64),
+                               _p(pt, ctypes.c_int32), pt.shape[1], int(page_size), _p(kidx, ctypes.c_uint8))
 
 
 def dequant_row(codes_row, scales_row):

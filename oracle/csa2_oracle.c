@@ -141,6 +141,27 @@ void orc_append_fp4(const uint16_t *x_bf16, int32_t n, int32_t d,
     }
 }
 
+void orc_e4m3_row(const uint16_t *x_bf16, int32_t width, uint8_t *out) {
+    for (int32_t i = 0; i < width; ++i) out[i] = (uint8_t)orc_e4m3_rne_sat(bf16_to_float(x_bf16[i]));
+}
+
+void orc_append_swa_e4m3(const uint16_t *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
+                         int64_t ring_rows, uint8_t *swa) {
+    for (int32_t i = 0; i < n; ++i) {
+        int64_t slot = pos[i] % ring_rows;
+        orc_e4m3_row(x_bf16 + (int64_t)i * 512, 512, swa + ((int64_t)seq[i] * ring_rows + slot) * 512);
+    }
+}
+
+void orc_append_kidx_e4m3(const uint16_t *x_bf16, int32_t n, int32_t di, const int32_t *seq,
+                          const int64_t *pos, const int32_t *page_table, int32_t max_pages,
+                          int32_t page_size, uint8_t *kidx) {
+    for (int32_t i = 0; i < n; ++i) {
+        int64_t row = orc_physical_row(page_table + (int64_t)seq[i] * max_pages, page_size, pos[i]);
+        orc_e4m3_row(x_bf16 + (int64_t)i * di, di, kidx + row * di);
+    }
+}
+
 void orc_dequant_row(const uint8_t *codes, const uint8_t *scales, int32_t d, double *out) {
     for (int32_t i = 0; i < d; ++i) {
         uint32_t c = (codes[i / 2] >> (4 * (i % 2))) & 15u;

@@ -77,6 +77,24 @@ void orc_append_fp4(const uint16_t *x_bf16, int32_t n, int32_t d,
                     const int32_t *page_table, int32_t max_pages, int32_t page_size,
                     uint8_t *codes, uint8_t *scales);
 
+/* ---- FP8 appends: the write side of the window KV and the indexer keys --
+ * [P3] "V4.1-Flash also uses FP4 quantization" (the short-window SWA KV is
+ * kept at FP8) and [P4] "How are cache precision and storage arranged?".
+ * Each bf16 value becomes E4M3_RNE_sat(value) (no scale); NaN keeps its sign
+ * and becomes the E4M3 NaN code 0x7F. */
+void orc_e4m3_row(const uint16_t *x_bf16, int32_t width, uint8_t *out);
+
+/* Window rows: row i (512 values) goes to ring slot pos[i] % ring_rows of
+ * sequence seq[i] in swa [batch][ring_rows][512]. */
+void orc_append_swa_e4m3(const uint16_t *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
+                         int64_t ring_rows, uint8_t *swa);
+
+/* Indexer keys: row i (di values) goes to the physical row of logical entry
+ * pos[i] of sequence seq[i] in kidx [rows][di]. */
+void orc_append_kidx_e4m3(const uint16_t *x_bf16, int32_t n, int32_t di, const int32_t *seq,
+                          const int64_t *pos, const int32_t *page_table, int32_t max_pages,
+                          int32_t page_size, uint8_t *kidx);
+
 /* ---- indexer ([P3] modes paragraph; [P4] three-dimension section) -------
  * score = sum_h w_h * max(0, sum_i q_{h,i} k_i), q and k E4M3, exact in double
  * for the integer-valued data the tests use; -0 is returned as +0. */

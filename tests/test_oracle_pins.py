@@ -429,3 +429,65 @@ def test_attention_padding_and_order_do_not_matter():
     o2, l2 = oracle.sparse_attn(q, codes, scales, pt, 8, perm, swa, 0.2)
     np.testing.assert_allclose(o1, o2, atol=1e-13)
     np.testing.assert_allclose(l1, l2, atol=1e-13)
+
+
+# ---- FP8 appends (window rows, indexer keys) --------------------------------
+
+def _all_bf16():
+    return np.arange(65536, dtype=np.uint32).astype(np.uint16)
+
+
+def test_e4m3_row_matches_torch_cast_in_range_and_saturates():
+    bits = _all_bf16()
+    got = oracle.e4m3_row(bits)
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float()
+    a = x.abs()
+    finite = torch.isfinite(x)
+    # inside the representable range torch's (non-saturating) cast is the RNE reference
+    inside = finite & (a < 464.0)
+    ref = x[inside].to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(got[inside.numpy()], ref)
+    # saturation: |x| >= 464 (incl. infinities) -> +-448
+    sat = (~torch.isnan(x)) & (a >= 464.0)
+    sign = (bits >> 15).astype(np.uint8)
+    np.testing.assert_array_equal(got[sat.numpy()], (0x7E | (sign << 7))[sat.numpy()])
+    # NaN keeps its sign and becomes 0x7F
+    nan = torch.isnan(x).numpy()
+    np.testing.assert_array_equal(got[nan], (0x7F | (sign << 7))[nan])
+
+
+def test_e4m3_row_worked_example():
+    x = np.array([1.0, -2.5, 448.0, 500.0, 0.0, 0.001953125, 3.3, -0.0], np.float32)
+    got = oracle.e4m3_row(_bf16_bits(x[None, :])[0])
+    # 1 = 0x38; -2.5 = 1|1000|010; 448 = 0x7E; 500 saturates; 0; 2^-9 = smallest subnormal;
+    # bf16(3.3) = 3.296875 -> 3.25 = 0|1000|101; -0 keeps its sign
+    assert [int(v) for v in got] == [0x38, 0xC2, 0x7E, 0x7E, 0x00, 0x01, 0x45, 0x80]
+
+
+def test_append_swa_ring_slots():
+    rng = np.random.default_rng(31)
+    ring, b = 7, 3
+    swa = np.full((b, ring, 512), 0xAA, np.uint8)
+    seq = np.array([0, 2, 2, 1], np.int32)
+    pos = np.array([3, 6, 7, 15], np.int64)         # 7 wraps to slot 0, 15 to slot 1
+    x = _bf16_bits(rng.standard_normal((4, 512)).astype(np.float32))
+    oracle.append_swa_e4m3(x, seq, pos, swa)
+    want = np.full_like(swa, 0xAA)
+    for i in range(4):
+        want[seq[i], pos[i] % ring] = oracle.e4m3_row(x[i])
+    np.testing.assert_array_equal(swa, want)
+
+
+def test_append_kidx_paged():
+    rng = np.random.default_rng(32)
+    ps, di = 4, 64
+    pt = np.array([[5, 2, 7], [0, 3, 6]], np.int32)
+    kidx = np.zeros((8 * ps, di), np.uint8)
+    seq = np.array([0, 1, 0], np.int32)
+    pos = np.array([5, 9, 11], np.int64)             # rows 2*4+1, 6*4+1, 7*4+3
+    x = _bf16_bits(rng.standard_normal((3, di)).astype(np.float32))
+    oracle.append_kidx_e4m3(x, seq, pos, pt, ps, kidx)
+    want = np.zeros_like(kidx)
+    for i, row in enumerate([9, 25, 31]):
+        want[row] = oracle.e4m3_row(x[i])
+    np.testing.assert_array_equal(kidx, want)
