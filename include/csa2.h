@@ -77,7 +77,7 @@ typedef enum {
 typedef struct {
     uint8_t *codes;
     uint8_t *scales;
-    const uint8_t *kidx;
+    uint8_t *kidx;
     const int32_t *page_table;
     const int32_t *seq_len;
     int64_t rows_cap;
@@ -104,6 +104,32 @@ typedef struct {
 csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq,
                             const int64_t *pos, const csa2_kv_desc *kv,
                             cudaStream_t stream);
+
+/*
+ * FP8 appends, the write side of the short-window KV and of the indexer keys
+ * ([P3] "V4.1-Flash also uses FP4 quantization": the short-window SWA KV is
+ * kept at FP8; [P4] "How are cache precision and storage arranged?").
+ * Every bf16 value is converted on its own to E4M3: round to nearest, ties to
+ * the even mantissa, saturating to +-448, no scale; a NaN keeps its sign and
+ * becomes the E4M3 NaN code 0x7F.
+ *
+ * csa2_append_swa_e4m3: x_bf16 [n][512] window rows; row i goes to ring slot
+ *   pos[i] % ring_rows of sequence seq[i] in swa [batch][ring_rows][512]
+ *   (the buffer csa2_sparse_attn_decode reads with swa_seq_stride =
+ *   ring_rows). pos >= 0.
+ * csa2_append_kidx_e4m3: x_bf16 [n][kv->di] indexer keys; row i goes to the
+ *   physical row of logical entry pos[i] of sequence seq[i] in kv->kidx.
+ * seq, pos: device arrays. Rows whose destination falls outside the buffer
+ * (bad sequence, negative position, outside the page table or the cache) are
+ * skipped and set the device error word. n = 0 is a no-op. x_bf16 16-byte
+ * aligned; swa 8-byte aligned.
+ */
+csa2_status csa2_append_swa_e4m3(const void *x_bf16, int32_t n, const int32_t *seq,
+                                 const int64_t *pos, uint8_t *swa, int32_t batch,
+                                 int64_t ring_rows, cudaStream_t stream);
+csa2_status csa2_append_kidx_e4m3(const void *x_bf16, int32_t n, const int32_t *seq,
+                                  const int64_t *pos, const csa2_kv_desc *kv,
+                                  cudaStream_t stream);
 
 /*
  * Full-mode indexer ([P3] modes paragraph: a Full layer scores the whole
@@ -156,9 +182,13 @@ size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p);
  *   q_bf16 [nq][h][d] bf16, query i of sequence i / q_per_seq.
  *   topk [nq][k]: global entry ids (-1 = empty); each row is dequantised
  *   (E2M1 code x E4M3 scale, exact in f16) and used as key and value.
- *   Window rows of query i: rows swa_begin[i] .. swa_end[i]-1 of the E4M3
- *   buffer swa + (i / q_per_seq) * swa_seq_stride * d (raw E4M3, no scale),
- *   also key and value; w_max >= every swa_end[i] - swa_begin[i].
+ *   Window rows of query i: the swa_end[i] - swa_begin[i] rows
+ *   (swa_begin[i] + j) mod swa_seq_stride of the E4M3 buffer
+ *   swa + (i / q_per_seq) * swa_seq_stride * d (raw E4M3, no scale; a ring of
+ *   swa_seq_stride rows per sequence, as csa2_append_swa_e4m3 writes it),
+ *   also key and value. A non-empty window needs 0 <= swa_begin[i] <
+ *   swa_seq_stride and swa_end[i] - swa_begin[i] <= min(w_max,
+ *   swa_seq_stride); otherwise it is dropped and the device error word set.
  * Per head, over the union S of selected rows and window rows:
  *   o_h = sum_j softmax_j(softmax_scale * <q_h, v_j>) v_j
  * written as bf16 o [nq][h][d]; lse [nq][h] (nullable) gets the natural-log

@@ -54,6 +54,8 @@ _SIGS = {
     "csa2_append_fp4": (_i32, [_vp, _i32, _vp, _vp, _kvp, _vp]),
     "csa2_index_full": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _i64, _kvp, _i32, _i32, _vp, _vp, _vp, _sz,
                                _vp]),
+    "csa2_append_swa_e4m3": (_i32, [_vp, _i32, _vp, _vp, _vp, _i32, _i64, _vp]),
+    "csa2_append_kidx_e4m3": (_i32, [_vp, _i32, _vp, _vp, _kvp, _vp]),
     "csa2_index_full_workspace_size": (_sz, [_i32, _i64]),
     "csa2_index_reindex": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _i32, _kvp, _i32, _vp, _vp, _sz, _vp]),
     "csa2_index_reindex_workspace_size": (_sz, [_i32, _i32]),
@@ -179,6 +181,19 @@ def csa2_sparse_attn_decode_static(q_bf16, q_per_seq, kv: KvCache, topk, swa, sw
         _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
         _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_bf16), _ptr(lse),
         _stream(stream)))
+
+
+def csa2_append_swa_e4m3(x_bf16, seq, pos, swa, stream=None):
+    """Window rows x [n][512] into ring slots pos % ring_rows of swa [batch][ring_rows][512]."""
+    _check("csa2_append_swa_e4m3", _lib.csa2_append_swa_e4m3(
+        _ptr(x_bf16), x_bf16.shape[0], _ptr(seq), _ptr(pos), _ptr(swa), swa.shape[0], swa.shape[1],
+        _stream(stream)))
+
+
+def csa2_append_kidx_e4m3(x_bf16, seq, pos, kv: KvCache, stream=None):
+    """Indexer keys x [n][di] into the physical rows of (seq, pos) of the key array."""
+    _check("csa2_append_kidx_e4m3", _lib.csa2_append_kidx_e4m3(
+        _ptr(x_bf16), x_bf16.shape[0], _ptr(seq), _ptr(pos), kv.desc, _stream(stream)))
 
 
 def csa2_device_status(stream=None):

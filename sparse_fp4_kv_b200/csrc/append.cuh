@@ -79,4 +79,62 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
     kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
 }
 
+// ---------------------------------------------------------------------------
+// FP8 appends: the write side of the short-window KV and of the indexer keys
+// (DeepSeek V4.1-Flash Cuts KV Cache by 437x, paragraph "V4.1-Flash also uses
+// FP4 quantization": the short-window SWA KV is kept at FP8; DeepSeek V4.1
+// Flash Architecture Breakdown, section "How are cache precision and storage
+// arranged?"). Each bf16 value is converted on its own to E4M3, round to
+// nearest even, saturating to +-448, no scale; NaN keeps its sign and becomes
+// the E4M3 NaN code 0x7F.
+//
+// A thread converts 8 consecutive values of a row: one 16-byte load, one
+// 8-byte store. Window rows go to ring slot pos % ring_rows of their
+// sequence; indexer keys go to the physical row of (seq, pos).
+// ---------------------------------------------------------------------------
+constexpr int kE4m3Threads = 256;
+
+// Two bf16 values (low half first) -> two E4M3 bytes (low byte first).
+__device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+    uint32_t r = out;
+    if ((w & 0x7FFFu) > 0x7F80u) r = (r & 0xFF00u) | ((w >> 8) & 0x80u) | 0x7Fu;                     // low NaN
+    if (((w >> 16) & 0x7FFFu) > 0x7F80u) r = (r & 0x00FFu) | (((w >> 24) & 0x80u) | 0x7Fu) << 8;  // high NaN
+    return r;
+}
+
+// mode 0: window rows (width 512) into swa [batch][ring_rows][512];
+// mode 1: indexer keys (width kv.di) into kv.kidx at the physical row.
+__global__ void __launch_bounds__(kE4m3Threads)
+    k_append_e4m3(const uint16_t *__restrict__ x, int32_t n, int32_t width, const int32_t *__restrict__ seq,
+                  const int64_t *__restrict__ pos, int32_t mode, uint8_t *__restrict__ swa, int32_t batch,
+                  int64_t ring_rows, csa2_kv_desc kv) {
+    pdl_trigger();
+    pdl_wait();
+    const int per_row = width / 8;
+    const int64_t t = (int64_t)blockIdx.x * kE4m3Threads + threadIdx.x;
+    if (t >= (int64_t)n * per_row) return;
+    const int64_t r = t / per_row;
+    const int c = (int)(t - r * per_row);
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * width) + c);
+    const int32_t b = seq[r];
+    const int64_t ps = pos[r];
+    uint8_t *row = nullptr;
+    if (mode == 0) {
+        if (b >= 0 && b < batch && ps >= 0) row = swa + ((int64_t)b * ring_rows + ps % ring_rows) * 512;
+    } else {
+        const int64_t pr = (b >= 0 && b < kv.batch) ? physical_row(kv, b, ps) : -1;
+        if (pr >= 0) row = kv.kidx + pr * kv.di;
+    }
+    if (row == nullptr) {
+        if (c == 0) set_error(CSA2_DEVERR_BAD_ROW);
+        return;
+    }
+    const uint32_t lo = e4m3x2_of_bf16x2(v.x) | (e4m3x2_of_bf16x2(v.y) << 16);
+    const uint32_t hi = e4m3x2_of_bf16x2(v.z) | (e4m3x2_of_bf16x2(v.w) << 16);
+    *reinterpret_cast<uint2 *>(row + c * 8) = make_uint2(lo, hi);
+}
+
 }  // namespace csa2

@@ -183,7 +183,9 @@ __device__ __forceinline__ void resolve_rows(const AttnParams &p, int32_t u, int
                 }
             }
         } else if (j < (int64_t)p.k + nw) {
-            src = (int32_t)(wb + (j - p.k));
+            int64_t slot = wb + (j - p.k);  // < 2 * stride
+            if (slot >= p.swa_seq_stride) slot -= p.swa_seq_stride;
+            src = (int32_t)slot;
             kind = 2;
         }
         rsrc[i] = src;
@@ -350,7 +352,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     }
     pdl_wait();
     const int32_t wb = p.swa_begin ? p.swa_begin[u] : 0;
-    const int32_t nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
+    int32_t nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
+    // the window is a run of ring slots: begin in [0, stride), at most stride rows
+    if (nw > 0 && (wb < 0 || wb >= p.swa_seq_stride || nw > p.swa_seq_stride)) {
+        if (tid == 0) set_error(CSA2_DEVERR_BAD_ROW);
+        nw = 0;
+    }
     const int64_t n_total = (int64_t)p.k + nw;
     const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
     const int64_t t_begin = (int64_t)split * p.tiles_per_split;

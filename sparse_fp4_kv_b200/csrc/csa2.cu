@@ -309,7 +309,7 @@ bool prefer_shared(K kernel) {
 
 // One-time attribute set-up of the kernels without large dynamic shared memory.
 bool init_small_kernels() {
-    static const bool ok = prefer_shared(k_append_fp4) && prefer_shared(k_sel_hist<1>) &&
+    static const bool ok = prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_hist<1>) &&
                            prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
                            prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
                            prefer_shared(k_attn_combine<16>) && prefer_shared(k_attn_combine<32>) &&
@@ -356,6 +356,37 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
     const unsigned grid = (unsigned)((n + kAppendWarps - 1) / kAppendWarps);
     launch(k_append_fp4, dim3(grid), dim3(kAppendWarps * 32), 0, stream, static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
+    return check_launch();
+}
+
+csa2_status csa2_append_swa_e4m3(const void *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
+                                 uint8_t *swa, int32_t batch, int64_t ring_rows, cudaStream_t stream) {
+    if (n < 0 || batch <= 0 || ring_rows <= 0) return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    if (!x_bf16 || !seq || !pos || !swa || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8) ||
+        !aligned(swa, 8))
+        return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    const int64_t threads = (int64_t)n * (CSA2_D / 8);
+    const unsigned grid = (unsigned)((threads + kE4m3Threads - 1) / kE4m3Threads);
+    launch(k_append_e4m3, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
+           (int32_t)CSA2_D, seq, pos, (int32_t)0, swa, batch, ring_rows, csa2_kv_desc{});
+    return check_launch();
+}
+
+csa2_status csa2_append_kidx_e4m3(const void *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
+                                  const csa2_kv_desc *kv, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (n < 0) return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
+        return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    const int64_t threads = (int64_t)n * (kv->di / 8);
+    const unsigned grid = (unsigned)((threads + kE4m3Threads - 1) / kE4m3Threads);
+    launch(k_append_e4m3, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
+           kv->di, seq, pos, (int32_t)1, static_cast<uint8_t *>(nullptr), (int32_t)0, (int64_t)1, *kv);
     return check_launch();
 }
 
