@@ -12,7 +12,10 @@ Architecture Breakdown, section "How does the cache compress along three
 dimensions at once?"): a Reindex layer re-scores the pool of the most recent
 Full layer; a Reuse layer takes the Top-k of the most recent layer that
 produced one (Reuse takes over earlier indices as they are), or, in the variant
-reuse_from='full', of the most recent Full layer.
+reuse_from='full', of the most recent Full layer. With one global cache per
+Full layer (the reading in which a Full layer generates its own global KV), a
+Full layer scores and attends over its own cache, a Reindex layer over its
+source Full layer's, a Reuse layer over its source layer's.
 """
 import math
 
@@ -44,24 +47,25 @@ def bf16_bits(t):
 
 
 class SeqCache:
-    """One sequence's logical cache (identity page table) built by the oracle."""
+    """One sequence's logical cache (identity page table) built by the oracle;
+    `cache` selects the cache of the per-Full-layer variant (0: shared)."""
 
-    def __init__(self, recipe, b):
+    def __init__(self, recipe, b, cache=0):
         lens = recipe.seq_lens()
         self.n = int(lens[b])
         rows = []
         if recipe.chunked:
-            rows.append(recipe.latent_rows(b, 0, recipe.prefill))
-            rows.append(recipe.latent_rows(b, recipe.prefill, self.n))
+            rows.append(recipe.latent_rows(b, 0, recipe.prefill, cache=cache))
+            rows.append(recipe.latent_rows(b, recipe.prefill, self.n, cache=cache))
         else:
-            rows.append(recipe.latent_rows(b, 0, self.n))
+            rows.append(recipe.latent_rows(b, 0, self.n, cache=cache))
         x = bf16_bits(torch.cat(rows))
         cap = max(self.n, 1)
         self.codes = np.zeros((cap, 256), np.uint8)
         self.scales = np.zeros((cap, 32), np.uint8)
         append_fp4(x, np.zeros(self.n, np.int32), np.arange(self.n, dtype=np.int64),
                    np.zeros((1, 1), np.int32), cap, self.codes, self.scales)
-        self.kidx = recipe.kidx_rows(b, 0, self.n).numpy()
+        self.kidx = recipe.kidx_rows(b, 0, self.n, cache=cache).numpy()
         self.page_table = np.zeros(1, np.int32)
         self.page_size = cap
 
@@ -76,13 +80,27 @@ def run(recipe, seqs, reuse_from="previous", layers=None, queries=None, attentio
     ql = recipe.q_limit()
     wb, we = recipe.swa_window()
     scale = 1.0 / math.sqrt(512.0)
+    # which cache every layer reads: one shared, or one per Full layer (a Full
+    # layer reads its own, Reindex its source Full layer's, Reuse its source's)
+    cache_of, fulls = [], 0
+    for layer, (mode, src) in enumerate(sched):
+        if not recipe.cache_per_full:
+            cache_of.append(0)
+        elif mode == "full":
+            cache_of.append(fulls)
+            fulls += 1
+        else:
+            cache_of.append(cache_of[src])
     for b in seqs:
-        c = SeqCache(recipe, b)
+        caches = {}
         qis = [b * recipe.q_per_seq + j for j in range(recipe.q_per_seq)]
         if queries is not None:
             qis = [qi for qi in qis if qi in queries]
         for layer in range(last + 1):
             mode, src = sched[layer]
+            if cache_of[layer] not in caches:
+                caches[cache_of[layer]] = SeqCache(recipe, b, cache_of[layer])
+            c = caches[cache_of[layer]]
             qidx = recipe.qidx(layer).numpy()
             w = recipe.weights(layer).numpy()
             need_attn = attention and layer in layers

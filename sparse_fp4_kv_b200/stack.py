@@ -15,7 +15,7 @@ import math
 import torch
 
 from . import binding as B
-from .workloads import Recipe, resolve_schedule
+from .workloads import Recipe, cache_of_layers, resolve_schedule
 
 
 class Csa2Decoder:
@@ -25,42 +25,55 @@ class Csa2Decoder:
         self.r = r = recipe
         self.device = device = torch.device(device)
         self.schedule = resolve_schedule(r.modes, reuse_from)
+        # global KV caches: one shared by all layers, or one per Full layer
+        self.cache_of = cache_of_layers(r.modes, self.schedule, r.cache_per_full)
         ps, pt, rows_cap = r.layout()
         self.page_size = ps
         lens = r.seq_lens()
         self.lens = lens
         self.n_max = int(lens.max())
-        self.codes = torch.zeros((rows_cap, 256), dtype=torch.uint8, device=device)
-        self.scales = torch.zeros((rows_cap, 32), dtype=torch.uint8, device=device)
-        self.kidx = torch.zeros((rows_cap, r.di), dtype=torch.uint8, device=device)
         self.page_table = pt.to(device)
         self.seq_len = lens.to(torch.int32).to(device)
-        self.kv = B.KvCache(self.codes, self.scales, self.kidx, self.page_table, self.seq_len, ps)
+        self.kvs = []
+        for c in range(r.caches()):
+            self.kvs.append(B.KvCache(torch.zeros((rows_cap, 256), dtype=torch.uint8, device=device),
+                                      torch.zeros((rows_cap, 32), dtype=torch.uint8, device=device),
+                                      torch.zeros((rows_cap, r.di), dtype=torch.uint8, device=device),
+                                      self.page_table, self.seq_len, ps))
+        # cache 0 (the shared cache, or the first Full layer's)
+        self.kv = self.kvs[0]
+        self.codes, self.scales, self.kidx = self.kv.codes, self.kv.scales, self.kv.kidx
 
         # ---- cache contents present before the step --------------------------------
         present = [r.prefill if r.chunked else int(l) for l in lens.tolist()]
-        for b in range(r.batch):
-            for t0 in range(0, present[b], build_chunk):
-                t1 = min(present[b], t0 + build_chunk)
-                self._write_rows(b, t0, t1, r.latent_rows(b, t0, t1, device))
-        if r.chunked:
-            # indexer keys of the rows the step appends (the key append itself is
-            # not part of this path; the keys are inputs of the Full layer)
-            for t0 in range(r.prefill, r.prefill + r.append, build_chunk):
-                t1 = min(r.prefill + r.append, t0 + build_chunk)
-                pos = torch.arange(t0, t1, dtype=torch.int64, device=device)
-                self.kidx[self.physical_rows(0, pos)] = r.kidx_rows(0, t0, t1, device)
+        for c, kv in enumerate(self.kvs):
+            for b in range(r.batch):
+                for t0 in range(0, present[b], build_chunk):
+                    t1 = min(present[b], t0 + build_chunk)
+                    self._write_rows(kv, c, b, t0, t1, r.latent_rows(b, t0, t1, device, cache=c))
+            if r.chunked:
+                # indexer keys of the rows the step appends (the key append itself
+                # is not part of this path; the keys are inputs of the Full layer)
+                for t0 in range(r.prefill, r.prefill + r.append, build_chunk):
+                    t1 = min(r.prefill + r.append, t0 + build_chunk)
+                    pos = torch.arange(t0, t1, dtype=torch.int64, device=device)
+                    kv.kidx[self.physical_rows(0, pos)] = r.kidx_rows(0, t0, t1, device, cache=c)
 
         # ---- step inputs -----------------------------------------------------------
+        self.x_news = []
+        for c in range(len(self.kvs)):
+            if r.chunked:
+                total = r.prefill + r.append
+                self.x_news.append(r.latent_rows(0, r.prefill, total, device, cache=c).contiguous())
+            else:
+                # the decoded token of each sequence: its last position
+                rows = [r.latent_rows(b, int(lens[b]) - 1, int(lens[b]), device, cache=c) for b in range(r.batch)]
+                self.x_news.append(torch.cat(rows).contiguous())
+        self.x_new = self.x_news[0]
         if r.chunked:
-            total = r.prefill + r.append
-            self.x_new = r.latent_rows(0, r.prefill, total, device).contiguous()
             self.x_seq = torch.zeros(r.append, dtype=torch.int32, device=device)
-            self.x_pos = torch.arange(r.prefill, total, dtype=torch.int64, device=device)
+            self.x_pos = torch.arange(r.prefill, r.prefill + r.append, dtype=torch.int64, device=device)
         else:
-            # the decoded token of each sequence: its last position
-            rows = [r.latent_rows(b, int(lens[b]) - 1, int(lens[b]), device) for b in range(r.batch)]
-            self.x_new = torch.cat(rows).contiguous()
             self.x_seq = torch.arange(r.batch, dtype=torch.int32, device=device)
             self.x_pos = (lens - 1).to(torch.int64).to(device)
         ql = r.q_limit()
@@ -89,14 +102,14 @@ class Csa2Decoder:
         self.ws_attn = B.workspace(B.csa2_sparse_attn_workspace_size(nq, r.h, r.k, r.w), device)
         torch.cuda.synchronize(device)
 
-    def _write_rows(self, b, t0, t1, x):
+    def _write_rows(self, kv, c, b, t0, t1, x):
         """Quantise + append latent rows (kernel) and store their indexer keys."""
         n = t1 - t0
         seq = torch.full((n,), b, dtype=torch.int32, device=self.device)
         pos = torch.arange(t0, t1, dtype=torch.int64, device=self.device)
-        B.csa2_append_fp4(x.contiguous(), seq, pos, self.kv)
+        B.csa2_append_fp4(x.contiguous(), seq, pos, kv)
         rows = self.physical_rows(b, pos)
-        self.kidx[rows] = self.r.kidx_rows(b, t0, t1, self.device)
+        kv.kidx[rows] = self.r.kidx_rows(b, t0, t1, self.device, cache=c)
 
     def physical_rows(self, b, pos):
         ps = self.page_size
@@ -108,19 +121,21 @@ class Csa2Decoder:
 
     # ---- one step -------------------------------------------------------------------
     def append(self, stream=None):
-        B.csa2_append_fp4(self.x_new, self.x_seq, self.x_pos, self.kv, stream)
+        for x, kv in zip(self.x_news, self.kvs):
+            B.csa2_append_fp4(x, self.x_seq, self.x_pos, kv, stream)
 
     def layer(self, l, stream=None):
         r = self.r
         mode, src = self.schedule[l]
+        kv = self.kvs[self.cache_of[l]]
         if mode == "full":
-            B.csa2_index_full(self.qidx[l], self.w[l], r.q_per_seq, self.q_limit, self.n_max, self.kv, r.k,
+            B.csa2_index_full(self.qidx[l], self.w[l], r.q_per_seq, self.q_limit, self.n_max, kv, r.k,
                               r.p if self.pool[l] is not None else 0, self.topk[l], self.pool[l], self.ws_full,
                               stream)
         elif mode == "reindex":
-            B.csa2_index_reindex(self.qidx[l], self.w[l], r.q_per_seq, self.pool[src], self.kv, r.k, self.topk[l],
+            B.csa2_index_reindex(self.qidx[l], self.w[l], r.q_per_seq, self.pool[src], kv, r.k, self.topk[l],
                                  self.ws_reindex, stream)
-        B.csa2_sparse_attn_decode(self.q[l], r.q_per_seq, self.kv, self.topk_of(l), self.swa[l],
+        B.csa2_sparse_attn_decode(self.q[l], r.q_per_seq, kv, self.topk_of(l), self.swa[l],
                                   self.swa[l].shape[1], self.swa_begin, self.swa_end, r.w, self.scale, self.o[l],
                                   self.lse[l], self.ws_attn, stream)
 

@@ -36,6 +36,7 @@ from . import synth
 S_LATENT, S_KIDX, S_LEN, S_PERM, S_APPEND, S_OUTLIER = 1, 2, 3, 4, 5, 6
 S_QIDX, S_W, S_Q, S_SWA = 100, 200, 300, 400
 T_STRIDE = 1 << 22  # counter stride between sequences (max entries per sequence)
+S_CACHE = 1000       # stream offset between the caches of the per-Full-layer variant
 
 
 @dataclass(frozen=True)
@@ -61,6 +62,7 @@ class Recipe:
     outlier_mul: float = 1.0
     swa_rows: int = 0        # window buffer rows per sequence (0 = w)
     chunked: bool = False    # queries at the last q_per_seq positions, causal
+    cache_per_full: bool = False  # every Full layer has its own global KV (cache c = c-th Full layer)
     extra: dict = field(default_factory=dict)
 
     # ---- sizes ----------------------------------------------------------------
@@ -102,21 +104,29 @@ class Recipe:
         return self.swa_rows or self.w
 
     # ---- values ---------------------------------------------------------------
-    def latent_rows(self, b, t0, t1, device="cpu"):
+    def latent_rows(self, b, t0, t1, device="cpu", cache=0):
         """bf16 [t1 - t0, 512]: latent rows of sequence b at positions t0..t1-1
-        (appended rows of the chunked workload carry the outliers)."""
+        of cache `cache` (appended rows of the chunked workload carry the
+        outliers). Cache 0 is the shared cache; with cache_per_full, cache c
+        belongs to the c-th Full layer and draws from its own streams."""
+        off = S_CACHE * cache
         if self.chunked and t1 > self.prefill:
             assert t0 >= self.prefill, "split prefill/append ranges"
             c0 = ((b * T_STRIDE) + (t0 - self.prefill)) * 512
-            return synth.normal_bf16(self.seed, S_APPEND, c0, (t1 - t0) * 512, device,
+            return synth.normal_bf16(self.seed, S_APPEND + off, c0, (t1 - t0) * 512, device,
                                      outlier_p=self.outlier_p, outlier_mul=self.outlier_mul,
-                                     outlier_stream=S_OUTLIER).view(t1 - t0, 512)
+                                     outlier_stream=S_OUTLIER + off).view(t1 - t0, 512)
         c0 = (b * T_STRIDE + t0) * 512
-        return synth.normal_bf16(self.seed, S_LATENT, c0, (t1 - t0) * 512, device).view(t1 - t0, 512)
+        return synth.normal_bf16(self.seed, S_LATENT + off, c0, (t1 - t0) * 512, device).view(t1 - t0, 512)
 
-    def kidx_rows(self, b, t0, t1, device="cpu"):
+    def kidx_rows(self, b, t0, t1, device="cpu", cache=0):
         c0 = (b * T_STRIDE + t0) * self.di
-        return synth.int_e4m3(self.seed, S_KIDX, c0, (t1 - t0) * self.di, device=device).view(t1 - t0, self.di)
+        return synth.int_e4m3(self.seed, S_KIDX + S_CACHE * cache, c0, (t1 - t0) * self.di,
+                              device=device).view(t1 - t0, self.di)
+
+    def caches(self):
+        """Number of global KV caches: 1 (shared by all layers) or one per Full layer."""
+        return max(1, self.modes.count("F")) if self.cache_per_full else 1
 
     def qidx(self, layer, device="cpu"):
         n = self.nq * self.hi * self.di
@@ -176,6 +186,22 @@ RECIPES = {
                        w=256, cap=262144, prefill=229376, append=32768, outlier_p=0.01, outlier_mul=20.0,
                        swa_rows=767, chunked=True),
 }
+
+
+def cache_of_layers(modes, schedule, per_full):
+    """Cache index read by every layer: 0 for all layers with one shared cache;
+    with one cache per Full layer, a Full layer reads its own, a Reindex layer
+    its source Full layer's, a Reuse layer its source layer's."""
+    if not per_full:
+        return [0] * len(modes)
+    out, fulls = [], 0
+    for layer, (mode, src) in enumerate(schedule):
+        if mode == "full":
+            out.append(fulls)
+            fulls += 1
+        else:
+            out.append(out[src])
+    return out
 
 
 def resolve_schedule(modes, reuse_from="previous"):

@@ -92,3 +92,21 @@ def test_reuse_layer_reproduces_source_output(built, cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(dec.o[3], dec.o[0])
     assert torch.equal(dec.lse[3], dec.lse[0])
+
+
+@pytest.mark.parametrize("reuse_from", ["previous", "full"])
+def test_one_cache_per_full_layer(built, cuda_device, reuse_from):
+    # the reading in which every Full layer generates its own global KV: two
+    # caches for stack20's two Full layers; Reindex and Reuse layers read their
+    # source's cache
+    from sparse_fp4_kv_b200.stack import Csa2Decoder
+    recipe = SMALL["stack20"].scaled(cache_per_full=True)
+    dec = Csa2Decoder(recipe, cuda_device, reuse_from=reuse_from)
+    assert len(dec.kvs) == 2 and dec.cache_of[:10] == [0] * 10 and dec.cache_of[10:] == [1] * 10
+    dec.step()
+    torch.cuda.synchronize()
+    assert device_status_clean()
+    ref = ostack.run(recipe, [0, 1], reuse_from=reuse_from)
+    _compare(dec, ref, recipe)
+    # the two caches really differ (different rows drawn for each)
+    assert not torch.equal(dec.kvs[0].codes, dec.kvs[1].codes)
