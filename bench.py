@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--workload", default="stack20")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sharded", action="store_true", help="skip the entry-range sharded side measurement")
     return ap.parse_args()
 
 
@@ -182,6 +183,40 @@ def time_append_e4m3(B, dev, hbm_gbs, reps=20):
                      "achieved_gbs": by / (us * 1e-6) / 1e9, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs}
     out["note"] = "bf16 in, E4M3 out; events around the call (launch included), median of %d after an L2 flush" % reps
     return out
+
+
+def time_sharded_hier1m(dev, world=2, reps=5):
+    """The 1M-entry sequence split by entry range into `world` shards, all on
+    this GPU one after another (local Full, key exchange, select, Reindex,
+    attention partials, merge); CUDA events around each step, L2 flushed
+    before each. One rank of a real split runs one shard's share of the
+    kernels plus the all-gathers whose sizes are given."""
+    import torch
+    from sparse_fp4_kv_b200.sharded import EntryShard, LocalGroup, ShardedDecoder, shard_ranges
+    from sparse_fp4_kv_b200.workloads import RECIPES
+    r = RECIPES["hier1m"]
+    shards = [EntryShard(r, off, n, dev) for off, n in shard_ranges(r.n, world)]
+    dec = ShardedDecoder(r, shards, LocalGroup(world))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dec.step()
+    ts = []
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dec.step()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    ms = ts[len(ts) // 2]
+    keys = sum((r.p if r.p else r.k) * 8 for m, _ in dec.schedule if m in ("full", "reindex")) * r.nq
+    parts = r.layers * r.nq * r.h * (512 + 1) * 4
+    del dec, shards
+    return {"workload": "hier1m", "shards": world, "ms_per_step_all_shards_one_gpu": ms,
+            "bytes_sent_per_rank_per_step": keys + parts,
+            "note": f"shards run sequentially on one GPU; median of {reps} steps (no append in the step)"}
 
 
 def peaks():
@@ -517,6 +552,7 @@ def run_ours(args):
                "peaks": f"{peak_kind}: {hbm_gbs} GB/s HBM, {bf16_sust} TF/s bf16 sustained (FP8 at 2x)"}
     append_c4 = time_append_chunk512(B, dev, hbm_gbs) if world == 1 else None
     append_f8 = time_append_e4m3(B, dev, hbm_gbs) if world == 1 else None
+    sharded = time_sharded_hier1m(dev) if world == 1 and not args.no_sharded else None
     breakdown = {k: 1e3 * statistics.mean(v) for k, v in attn.items()}
     attn_ms = statistics.mean(attn["attention"]) if attn else float("nan")
     achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
@@ -542,6 +578,7 @@ def run_ours(args):
         "step_roofline": step_rl,
         "append_chunk512": append_c4,
         "append_e4m3": append_f8,
+        "sharded_hier1m": sharded,
         "breakdown_us_per_call": breakdown,
         "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented replay "
                           "of the same step (event nodes between calls prevent launch overlap)",

@@ -196,7 +196,10 @@ size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p);
  * Arithmetic: q converted to f16 (|q| must be finite in f16), f16 tensor-core
  * products with f32 accumulation, f32 online softmax, probabilities rounded
  * to f16 for the P*V product. h in {16, 32, 64}.
- * ws: at least csa2_sparse_attn_workspace_size(nq, h, k, w_max) bytes.
+ * ws: at least csa2_sparse_attn_workspace_size(nq, h, k, w) bytes, with
+ * w = w_max when a window is given and w = 0 when swa_begin is NULL (the
+ * split plan follows the rows the call really has; the size is not monotone
+ * in w, so size a workspace shared by both kinds of call for both).
  */
 csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_per_seq,
                                     int32_t h, const csa2_kv_desc *kv, const int32_t *topk,
@@ -236,6 +239,44 @@ csa2_status csa2_sparse_attn_decode_static(const void *q_bf16, int32_t nq, int32
                                            const int32_t *swa_begin, const int32_t *swa_end,
                                            int32_t w_max, float softmax_scale, void *o_bf16,
                                            float *lse, cudaStream_t stream);
+
+/*
+ * Building blocks of a long sequence decoded with its entries split across
+ * GPUs by entry range (one exchange step per layer; the pages put 1M-token
+ * contexts on one sequence: [P3] "CSA2 tackles storage", [P4] "How does the
+ * cache compress along three dimensions at once?"). Each rank holds the
+ * entries [offset, offset + n_r) of the sequence in its own cache.
+ *
+ * csa2_score_ids: score the given entry ids (local to kv, -1 = empty) as the
+ *   indexer does, into unique 64-bit keys (ordered score key << 32 |
+ *   ~(id + id_offset)); empty ids give key 0. ids [nq][m], keys [nq][m].
+ *   id + id_offset must stay below 2^31.
+ * csa2_select_keys: the k largest keys of each query's m keys, written as
+ *   the ids they carry (~ of the low 32 bits), in key-array order, padded
+ *   with -1; key 0 is empty. Because the id is part of the key, equal scores
+ *   are taken in ascending id order. m <= 2^20 (up to about 28000 keys are
+ *   staged in shared memory, larger sets are re-read from L2 in every radix
+ *   pass). keys [nq][m], ids [nq][k].
+ * csa2_sparse_attn_partial: csa2_sparse_attn_decode over this rank's rows,
+ *   writing the normalised f32 o [nq][h][512] and lse [nq][h] (required)
+ *   instead of bf16 o; the same workspace.
+ * csa2_attn_merge: merge g such partials o_parts [g][nq][h][512],
+ *   lse_parts [g][nq][h] into bf16 o [nq][h][512] and lse [nq][h]
+ *   (nullable): o = sum_r exp(lse_r - M) o_r / sum_r exp(lse_r - M).
+ */
+csa2_status csa2_score_ids(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq,
+                           int32_t hi, const int32_t *ids, int32_t m, const csa2_kv_desc *kv,
+                           int32_t id_offset, unsigned long long *keys, cudaStream_t stream);
+csa2_status csa2_select_keys(const unsigned long long *keys, int32_t nq, int32_t m, int32_t k,
+                             int32_t *ids, cudaStream_t stream);
+csa2_status csa2_sparse_attn_partial(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                     const csa2_kv_desc *kv, const int32_t *topk, int32_t k,
+                                     const uint8_t *swa, int64_t swa_seq_stride,
+                                     const int32_t *swa_begin, const int32_t *swa_end,
+                                     int32_t w_max, float softmax_scale, float *o_f32, float *lse,
+                                     void *ws, size_t ws_bytes, cudaStream_t stream);
+csa2_status csa2_attn_merge(const float *o_parts, const float *lse_parts, int32_t g, int32_t nq,
+                            int32_t h, void *o_bf16, float *lse, cudaStream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word.
  * *code receives 0 when no device-side condition was recorded since the

@@ -64,6 +64,11 @@ _SIGS = {
     "csa2_sparse_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "csa2_sparse_attn_decode_static": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
                                               _f32, _vp, _vp, _vp]),
+    "csa2_score_ids": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _i32, _kvp, _i32, _vp, _vp]),
+    "csa2_select_keys": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "csa2_sparse_attn_partial": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
+                                        _f32, _vp, _vp, _vp, _sz, _vp]),
+    "csa2_attn_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "csa2_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "csa2_status_string": (ctypes.c_char_p, [_i32]),
     "csa2_version": (_i32, []),
@@ -194,6 +199,36 @@ def csa2_append_kidx_e4m3(x_bf16, seq, pos, kv: KvCache, stream=None):
     """Indexer keys x [n][di] into the physical rows of (seq, pos) of the key array."""
     _check("csa2_append_kidx_e4m3", _lib.csa2_append_kidx_e4m3(
         _ptr(x_bf16), x_bf16.shape[0], _ptr(seq), _ptr(pos), kv.desc, _stream(stream)))
+
+
+def csa2_score_ids(qidx, w, q_per_seq, ids, kv: KvCache, id_offset, keys, stream=None):
+    """Unique 64-bit keys (score key << 32 | ~(id + id_offset)) of ids [nq][m] (local to kv)."""
+    nq, hi = qidx.shape[0], qidx.shape[1]
+    _check("csa2_score_ids", _lib.csa2_score_ids(_ptr(qidx), _ptr(w), nq, q_per_seq, hi, _ptr(ids), ids.shape[1],
+                                                 kv.desc, int(id_offset), _ptr(keys), _stream(stream)))
+
+
+def csa2_select_keys(keys, k, ids, stream=None):
+    """The ids carried by the k largest of each query's keys [nq][m] (padded with -1)."""
+    _check("csa2_select_keys", _lib.csa2_select_keys(_ptr(keys), keys.shape[0], keys.shape[1], int(k), _ptr(ids),
+                                                     _stream(stream)))
+
+
+def csa2_sparse_attn_partial(q_bf16, q_per_seq, kv: KvCache, topk, swa, swa_seq_stride, swa_begin, swa_end,
+                             w_max, softmax_scale, o_f32, lse, ws, stream=None):
+    nq, h = q_bf16.shape[0], q_bf16.shape[1]
+    k = topk.shape[1] if topk is not None else 0
+    _check("csa2_sparse_attn_partial", _lib.csa2_sparse_attn_partial(
+        _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
+        _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_f32), _ptr(lse),
+        _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def csa2_attn_merge(o_parts, lse_parts, o_bf16, lse, stream=None):
+    """Merge g partials o_parts [g][nq][h][512] f32, lse_parts [g][nq][h] into bf16 o and lse."""
+    g, nq, h = o_parts.shape[0], o_parts.shape[1], o_parts.shape[2]
+    _check("csa2_attn_merge", _lib.csa2_attn_merge(_ptr(o_parts), _ptr(lse_parts), g, nq, h, _ptr(o_bf16), _ptr(lse),
+                                                   _stream(stream)))
 
 
 def csa2_device_status(stream=None):

@@ -81,6 +81,7 @@ struct AttnParams {
     int32_t q_per_seq;
     int32_t n_splits;
     int32_t tiles_per_split;
+    int32_t out_f32;   // write normalised f32 o (o_part, S = 1) instead of bf16 o
 };
 
 __device__ __forceinline__ uint32_t kv_chunk_off(int e, int c64) {
@@ -632,7 +633,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
                         for (int i = 0; i < HG; ++i) vals[dc][i] = 0u;
                 }
                 const int d0 = quarter * 32 + lane;
-                if (p.n_splits == 1) {
+                if (p.n_splits == 1 && !p.out_f32) {
                     uint16_t *dst = p.o + (int64_t)u * H * CSA2_D;
 #pragma unroll
                     for (int i = 0; i < HG; ++i) {
@@ -657,7 +658,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
             if (tid < H) {
                 const float l = l_run[tid];
                 const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                if (p.n_splits == 1) {
+                if (p.n_splits == 1 && !p.out_f32) {
                     if (p.lse) p.lse[(int64_t)u * H + tid] = lse;
                 } else {
                     p.lse_part[((int64_t)u * p.n_splits + split) * H + tid] = lse;
@@ -683,31 +684,42 @@ constexpr int kCombineThreads = 128;
 constexpr int kCombineHeads = 1;   // heads per CTA (128 float4 per head)
 constexpr int kCombineBatch = 16;  // split loads in flight per thread
 
-template <int H>
-__global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *__restrict__ o_part,
-                                                                  const float *__restrict__ lse_part,
-                                                                  uint16_t *__restrict__ o, float *__restrict__ lse,
-                                                                  int32_t n_splits) {
+// Partials of query u, part s: o at o_part + u * q_stride + s * s_stride
+// (+ h * 512), lse at lse_part + u * lq_stride + s * ls_stride (+ h). Output:
+// bf16 o [u][h][512] (F32 = false) or f32 (F32 = true).
+struct CombineArgs {
+    const float *o_part;
+    const float *lse_part;
+    int64_t q_stride, s_stride, lq_stride, ls_stride;
+    void *o;
+    float *lse;
+    int32_t n_splits;
+};
+
+template <int H, bool F32>
+__global__ void __launch_bounds__(kCombineThreads) k_attn_combine(CombineArgs a) {
     extern __shared__ float wsm[];  // [n_splits + 1]
     pdl_trigger();
     pdl_wait();
     const int32_t u = blockIdx.y;
     const int h = blockIdx.x;
     const int d4 = threadIdx.x;  // 128 threads x 4 values = 512
-    const float *src = o_part + ((int64_t)u * n_splits * H + h) * CSA2_D;
+    const int32_t n_splits = a.n_splits;
+    const float *src = a.o_part + (int64_t)u * a.q_stride + h * CSA2_D;
+    const float *lsrc = a.lse_part + (int64_t)u * a.lq_stride + h;
     float4 v[kCombineBatch];
 #pragma unroll
     for (int t = 0; t < kCombineBatch; ++t)
-        v[t] = t < n_splits ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)t * H * CSA2_D) + d4)
+        v[t] = t < n_splits ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)t * a.s_stride) + d4)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
     if (threadIdx.x < 32) {
         float M = -INFINITY;
-        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, lse_part[((int64_t)u * n_splits + s) * H + h]);
+        for (int s = threadIdx.x; s < n_splits; s += 32) M = fmaxf(M, lsrc[(int64_t)s * a.ls_stride]);
 #pragma unroll
         for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
         float L = 0.0f;
         for (int s = threadIdx.x; s < n_splits; s += 32) {
-            const float ls = lse_part[((int64_t)u * n_splits + s) * H + h];
+            const float ls = lsrc[(int64_t)s * a.ls_stride];
             const float w = (M == -INFINITY) ? 0.0f : expf(ls - M);
             wsm[s] = w;
             L += w;
@@ -716,7 +728,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
         for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
         if (threadIdx.x == 0) {
             wsm[n_splits] = L;
-            if (lse) lse[(int64_t)u * H + h] = L > 0.0f ? M + logf(L) : -INFINITY;
+            if (a.lse) a.lse[(int64_t)u * H + h] = L > 0.0f ? M + logf(L) : -INFINITY;
         }
     }
     __syncthreads();
@@ -726,7 +738,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
 #pragma unroll
             for (int t = 0; t < kCombineBatch; ++t)
                 v[t] = (s0 + t < n_splits)
-                           ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(s0 + t) * H * CSA2_D) + d4)
+                           ? __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(s0 + t) * a.s_stride) + d4)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -741,10 +753,15 @@ __global__ void __launch_bounds__(kCombineThreads) k_attn_combine(const float *_
     }
     const float L = wsm[n_splits];
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    uint16_t *dst = o + ((int64_t)u * H + h) * CSA2_D + d4 * 4;
-    const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc.x * inv) | ((uint32_t)f32_to_bf16_bits(acc.y * inv) << 16);
-    const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc.z * inv) | ((uint32_t)f32_to_bf16_bits(acc.w * inv) << 16);
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+    if (F32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + ((int64_t)u * H + h) * CSA2_D) + d4;
+        *dst = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    } else {
+        uint16_t *dst = static_cast<uint16_t *>(a.o) + ((int64_t)u * H + h) * CSA2_D + d4 * 4;
+        const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc.x * inv) | ((uint32_t)f32_to_bf16_bits(acc.y * inv) << 16);
+        const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc.z * inv) | ((uint32_t)f32_to_bf16_bits(acc.w * inv) << 16);
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+    }
 }
 
 }  // namespace csa2

@@ -312,8 +312,9 @@ bool init_small_kernels() {
     static const bool ok = prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_hist<1>) &&
                            prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
                            prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
-                           prefer_shared(k_attn_combine<16>) && prefer_shared(k_attn_combine<32>) &&
-                           prefer_shared(k_attn_combine<64>);
+                           prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
+                           prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
+                           prefer_shared(k_attn_combine<32, true>) && prefer_shared(k_attn_combine<64, true>);
     return ok;
 }
 
@@ -559,9 +560,9 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
         launch(k_reindex_score<128>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
     if ((st = check_launch()) != CSA2_OK) return st;
     const size_t smem = 2048 * 4 + (kReindexSelectThreads / 32 + 8) * 4 + (size_t)p * 8;
-    static bool ok = set_smem(k_reindex_select, (size_t)max_smem_optin());
+    static bool ok = set_smem(k_reindex_select<false>, (size_t)max_smem_optin());
     if (!ok) return CSA2_ERR_CUDA;
-    launch(k_reindex_select, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
+    launch(k_reindex_select<false>, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
     return check_launch();
 }
 
@@ -572,19 +573,36 @@ size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t
     return attn_layout(nq, h, P).total;
 }
 
-csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
-                                    const csa2_kv_desc *kv, const int32_t *topk, int32_t k, const uint8_t *swa,
-                                    int64_t swa_seq_stride, const int32_t *swa_begin, const int32_t *swa_end,
-                                    int32_t w_max, float softmax_scale, void *o_bf16, float *lse, void *ws,
-                                    size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+template <bool F32>
+void launch_combine(int32_t h, int32_t nq, const CombineArgs &ca, cudaStream_t stream) {
+    const dim3 cgrid((unsigned)(h / kCombineHeads), (unsigned)nq);
+    const size_t csmem = (size_t)(ca.n_splits + 1) * 4;
+    switch (h) {
+        case 64: launch(k_attn_combine<64, F32>, cgrid, dim3(kCombineThreads), csmem, stream, ca); break;
+        case 32: launch(k_attn_combine<32, F32>, cgrid, dim3(kCombineThreads), csmem, stream, ca); break;
+        default: launch(k_attn_combine<16, F32>, cgrid, dim3(kCombineThreads), csmem, stream, ca); break;
+    }
+}
+
+// Shared body of the decode entry points: o is bf16 (out_f32 false) or the
+// normalised f32 o of this call's rows (out_f32 true, lse required).
+csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h, const csa2_kv_desc *kv,
+                      const int32_t *topk, int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
+                      const int32_t *swa_begin, const int32_t *swa_end, int32_t w_max, float softmax_scale, void *o,
+                      bool out_f32, float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
     csa2_status st = check_kv(kv, false);
     if (st != CSA2_OK) return st;
     if (h != 16 && h != 32 && h != 64) return CSA2_ERR_UNSUPPORTED;
     if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
         return CSA2_ERR_INVALID_ARG;
     if (k < 0 || w_max < 0 || (k > 0 && !topk) || (topk && !aligned(topk, 4))) return CSA2_ERR_INVALID_ARG;
-    if (!q_bf16 || !o_bf16 || !aligned(q_bf16, 16) || !aligned(o_bf16, 16) || (lse && !aligned(lse, 4)))
+    if (!q_bf16 || !o || !aligned(q_bf16, 16) || !aligned(o, 16) || (lse && !aligned(lse, 4)))
         return CSA2_ERR_INVALID_ARG;
+    if (out_f32 && !lse) return CSA2_ERR_INVALID_ARG;
     const bool has_swa = swa_begin != nullptr;
     if (has_swa && (!swa || !swa_end || !aligned(swa, 16) || !aligned(swa_begin, 4) || !aligned(swa_end, 4)))
         return CSA2_ERR_INVALID_ARG;
@@ -603,10 +621,16 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
     ap.swa_seq_stride = swa_seq_stride;
     ap.swa_begin = has_swa ? swa_begin : nullptr;
     ap.swa_end = has_swa ? swa_end : nullptr;
-    ap.o = static_cast<uint16_t *>(o_bf16);
+    ap.o = out_f32 ? nullptr : static_cast<uint16_t *>(o);
     ap.lse = lse;
     ap.o_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_o) : nullptr;
     ap.lse_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_lse) : nullptr;
+    ap.out_f32 = out_f32 ? 1 : 0;
+    if (out_f32 && P.splits == 1) {
+        // one split: the kernel's f32 partial is the result
+        ap.o_part = static_cast<float *>(o);
+        ap.lse_part = lse;
+    }
     ap.scale_log2 = softmax_scale * 1.4426950408889634f;
     ap.k = k;
     ap.q_per_seq = q_per_seq;
@@ -636,25 +660,120 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_pe
     }
     if ((st = check_launch()) != CSA2_OK) return st;
     if (P.splits > 1) {
-        const dim3 cgrid((unsigned)(h / kCombineHeads), (unsigned)nq);
-        const size_t csmem = (size_t)(P.splits + 1) * 4;
-        switch (h) {
-            case 64:
-                launch(k_attn_combine<64>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
-                                                                             P.splits);
-                break;
-            case 32:
-                launch(k_attn_combine<32>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
-                                                                             P.splits);
-                break;
-            default:
-                launch(k_attn_combine<16>, dim3(cgrid), dim3(kCombineThreads), csmem, stream, ap.o_part, ap.lse_part, ap.o, lse,
-                                                                             P.splits);
-                break;
-        }
+        CombineArgs ca{};
+        ca.o_part = ap.o_part;
+        ca.lse_part = ap.lse_part;
+        ca.q_stride = (int64_t)P.splits * h * CSA2_D;
+        ca.s_stride = (int64_t)h * CSA2_D;
+        ca.lq_stride = (int64_t)P.splits * h;
+        ca.ls_stride = h;
+        ca.o = o;
+        ca.lse = lse;
+        ca.n_splits = P.splits;
+        if (out_f32)
+            launch_combine<true>(h, nq, ca, stream);
+        else
+            launch_combine<false>(h, nq, ca, stream);
         st = check_launch();
     }
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+csa2_status csa2_sparse_attn_decode(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                    const csa2_kv_desc *kv, const int32_t *topk, int32_t k, const uint8_t *swa,
+                                    int64_t swa_seq_stride, const int32_t *swa_begin, const int32_t *swa_end,
+                                    int32_t w_max, float softmax_scale, void *o_bf16, float *lse, void *ws,
+                                    size_t ws_bytes, cudaStream_t stream) {
+    return attn_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end, w_max,
+                     softmax_scale, o_bf16, false, lse, ws, ws_bytes, stream);
+}
+
+csa2_status csa2_sparse_attn_partial(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                     const csa2_kv_desc *kv, const int32_t *topk, int32_t k, const uint8_t *swa,
+                                     int64_t swa_seq_stride, const int32_t *swa_begin, const int32_t *swa_end,
+                                     int32_t w_max, float softmax_scale, float *o_f32, float *lse, void *ws,
+                                     size_t ws_bytes, cudaStream_t stream) {
+    return attn_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end, w_max,
+                     softmax_scale, o_f32, true, lse, ws, ws_bytes, stream);
+}
+
+csa2_status csa2_attn_merge(const float *o_parts, const float *lse_parts, int32_t g, int32_t nq, int32_t h,
+                            void *o_bf16, float *lse, cudaStream_t stream) {
+    if (h != 16 && h != 32 && h != 64) return CSA2_ERR_UNSUPPORTED;
+    if (g < 1 || nq <= 0 || nq > 65535) return CSA2_ERR_INVALID_ARG;
+    if (!o_parts || !lse_parts || !o_bf16 || !aligned(o_parts, 16) || !aligned(lse_parts, 4) ||
+        !aligned(o_bf16, 16) || (lse && !aligned(lse, 4)))
+        return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    CombineArgs ca{};
+    ca.o_part = o_parts;
+    ca.lse_part = lse_parts;
+    ca.q_stride = (int64_t)h * CSA2_D;
+    ca.s_stride = (int64_t)nq * h * CSA2_D;
+    ca.lq_stride = h;
+    ca.ls_stride = (int64_t)nq * h;
+    ca.o = o_bf16;
+    ca.lse = lse;
+    ca.n_splits = g;
+    launch_combine<false>(h, nq, ca, stream);
+    return check_launch();
+}
+
+csa2_status csa2_score_ids(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq, int32_t hi,
+                           const int32_t *ids, int32_t m, const csa2_kv_desc *kv, int32_t id_offset,
+                           unsigned long long *keys, cudaStream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
+        return CSA2_ERR_INVALID_ARG;
+    if (hi < 1 || hi > kScanN) return CSA2_ERR_UNSUPPORTED;
+    if (m < 1 || id_offset < 0) return CSA2_ERR_INVALID_ARG;
+    if (!qidx || !w || !ids || !keys || !aligned(qidx, 16) || !aligned(w, 4) || !aligned(ids, 4) ||
+        !aligned(keys, 8))
+        return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    ReindexParams rp{};
+    rp.qidx = qidx;
+    rp.w = w;
+    rp.pool = ids;
+    rp.kv = *kv;
+    rp.k64 = keys;
+    rp.p = m;
+    rp.hi = hi;
+    rp.q_per_seq = q_per_seq;
+    rp.id_offset = id_offset;
+    const dim3 grid((unsigned)((m + kReindexScoreThreads - 1) / kReindexScoreThreads), (unsigned)nq);
+    if (kv->di == 64)
+        launch(k_reindex_score<64>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
+    else
+        launch(k_reindex_score<128>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
+    return check_launch();
+}
+
+csa2_status csa2_select_keys(const unsigned long long *keys, int32_t nq, int32_t m, int32_t k, int32_t *ids,
+                             cudaStream_t stream) {
+    if (nq <= 0 || nq > 65535 || m < 1 || k < 1) return CSA2_ERR_INVALID_ARG;
+    if (m > kSelectKeysMax) return CSA2_ERR_UNSUPPORTED;
+    if (!keys || !ids || !aligned(keys, 8) || !aligned(ids, 4)) return CSA2_ERR_INVALID_ARG;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    ReindexParams rp{};
+    rp.k64 = const_cast<unsigned long long *>(keys);
+    rp.topk = ids;
+    rp.p = m;
+    rp.k = k;
+    const size_t base = 2048 * 4 + (kReindexSelectThreads / 32 + 8) * 4;
+    const size_t smem = base + (size_t)m * 8;
+    static const bool ok = set_smem(k_reindex_select<false>, (size_t)max_smem_optin());
+    if (!ok) return CSA2_ERR_CUDA;
+    if (smem <= (size_t)max_smem_optin())
+        launch(k_reindex_select<false>, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
+    else  // keys larger than shared memory: every pass reads them from L2
+        launch(k_reindex_select<true>, dim3(nq), dim3(kReindexSelectThreads), base, stream, rp);
+    return check_launch();
 }
 
 }  // extern "C"

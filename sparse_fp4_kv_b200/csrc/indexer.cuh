@@ -697,6 +697,7 @@ __global__ void __launch_bounds__(kSelThreads) k_sel_emit(SelParams p) {
 // Reindex parameters (kernel in indexer_fused.cuh)
 // ---------------------------------------------------------------------------
 constexpr int kReindexMaxPool = 16384;
+constexpr int kSelectKeysMax = 1 << 20;  // keys per query taken by csa2_select_keys
 
 struct ReindexParams {
     const uint8_t *qidx;
@@ -706,6 +707,7 @@ struct ReindexParams {
     unsigned long long *k64;  // [nq][p] workspace: (score key << 32 | ~id), 0 = empty
     int32_t *topk;   // [nq][k]
     int32_t p, k, hi, q_per_seq;
+    int32_t id_offset;  // added to every id in the keys (entry-range shards)
 };
 
 }  // namespace csa2

@@ -362,7 +362,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 // empty slot) to the workspace; (2) k_reindex_select, one CTA per query:
 // load the pool's keys into shared memory and select the k largest with a
 // radix select that starts at the highest bit in which two keys differ;
-// output in pool order.
+// output in pool order. With G = true the keys stay in global memory (L2)
+// and every pass re-reads them, for key sets larger than shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kReindexScoreThreads = 128;
 constexpr int kReindexSelectThreads = 1024;
@@ -427,17 +428,18 @@ __global__ void __launch_bounds__(kReindexScoreThreads) k_reindex_score(ReindexP
 #pragma unroll
         for (int h = 0; h < kScanN; ++h)
             if (h < p.hi) sc = fmaf(wf[h], fmaxf(dot[h], 0.0f), sc);
-        v = ((unsigned long long)score_key(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)id);
+        v = ((unsigned long long)score_key(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)(id + p.id_offset));
     }
     p.k64[(int64_t)qi * p.p + j] = v;
 }
 
+template <bool G>
 __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(ReindexParams p) {
     constexpr int NT = kReindexSelectThreads;
     extern __shared__ uint8_t smem_raw[];
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                                 // [2048]
     uint32_t *scratch = hist + 2048;                                                         // [NT/32 + 8]
-    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p] (G false)
     __shared__ unsigned long long and_acc, or_acc;
     const int32_t qi = blockIdx.x;
     pdl_trigger();
@@ -450,9 +452,15 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
     uint32_t nvalid_t = 0;
     unsigned long long a_loc = ~0ull, o_loc = 0ull;
     const unsigned long long *src = p.k64 + (int64_t)qi * p.p;
+    auto key = [&](int j) -> uint64_t {
+        if constexpr (G)
+            return __ldcg(src + j);
+        else
+            return k64[j];
+    };
     for (int j = threadIdx.x; j < p.p; j += NT) {
         const unsigned long long v = __ldcg(src + j);
-        k64[j] = v;
+        if constexpr (!G) k64[j] = v;
         if ((uint32_t)v >= 0x80000000u) {
             ++nvalid_t;
             a_loc &= v;
@@ -478,7 +486,7 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
             for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
             __syncthreads();
             for (int j = threadIdx.x; j < p.p; j += NT) {
-                const uint64_t v = k64[j];
+                const uint64_t v = key(j);
                 if ((uint32_t)v >= 0x80000000u && (v & pmask) == prefix)
                     atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
             }
@@ -498,11 +506,14 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
     const int per = (p.p + NT - 1) / NT;
     const int j0 = threadIdx.x * per;
     uint32_t mine = 0;
-    for (int j = j0; j < min(p.p, j0 + per); ++j) mine += (uint32_t)k64[j] >= 0x80000000u && k64[j] >= T;
+    for (int j = j0; j < min(p.p, j0 + per); ++j) {
+        const uint64_t v = key(j);
+        mine += (uint32_t)v >= 0x80000000u && v >= T;
+    }
     uint32_t pos = block_excl_scan<NT>(mine, scratch, nullptr);
     int32_t *out = p.topk + (int64_t)qi * p.k;
     for (int j = j0; j < min(p.p, j0 + per); ++j) {
-        const uint64_t v = k64[j];
+        const uint64_t v = key(j);
         if (!((uint32_t)v >= 0x80000000u && v >= T)) continue;
         if (pos < (uint32_t)p.k) {
             out[pos] = (int32_t)(~(uint32_t)v);
