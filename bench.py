@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sharded", action="store_true", help="skip the entry-range sharded side measurement")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip every side measurement (appends, sharded decode, attention variants)")
     return ap.parse_args()
 
 
@@ -182,6 +184,57 @@ def time_append_e4m3(B, dev, hbm_gbs, reps=20):
         out[name] = {"rows": n, "us_median": us, "algorithmic_bytes": by,
                      "achieved_gbs": by / (us * 1e-6) / 1e9, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs}
     out["note"] = "bf16 in, E4M3 out; events around the call (launch included), median of %d after an L2 flush" % reps
+    return out
+
+
+def time_attn_variants(B, dec, reps=30):
+    """One attention layer of the benchmark step (layer 0's queries, Top-K and
+    window) through the exact call and through the NVFP4 variant (q rounded to
+    NVFP4 for the scores, FP4 block-scaled products on the selected entries);
+    CUDA events around each call (kernel + merge), L2 flushed before each,
+    median of `reps`."""
+    import torch
+    r = dec.r
+    dev = dec.device
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    topk = dec.topk_of(0)
+    o = torch.empty_like(dec.o[0])
+    lse = torch.empty_like(dec.lse[0])
+    ws_nv = B.workspace(B.csa2_sparse_attn_nvfp4_workspace_size(r.nq, r.h, r.k, r.w), dev)
+    args = (dec.q[0], r.q_per_seq, dec.kv, topk, dec.swa[0], dec.swa[0].shape[1], dec.swa_begin, dec.swa_end, r.w,
+            dec.scale, o, lse)
+    calls = {"exact": lambda: B.csa2_sparse_attn_decode(*args, dec.ws_attn),
+             "nvfp4": lambda: B.csa2_sparse_attn_decode_nvfp4(*args, ws_nv)}
+    out = {}
+    stream = torch.cuda.Stream(device=dev)
+    for name, call in calls.items():
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        # the call captured in a CUDA graph, as in the decode step
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call()
+        for mode, run in (("eager", call), ("graph", g.replay)):
+            ts = []
+            for i in range(reps):
+                with torch.cuda.stream(stream):
+                    flush.fill_(i & 0xFF)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    run()
+                    e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            ts.sort()
+            out[f"{name}_{mode}_us"] = ts[len(ts) // 2]
+        del g
+    if B.csa2_device_status() != 0:
+        raise RuntimeError("device error in the attention variants")
+    out["speedup_graph"] = out["exact_graph_us"] / out["nvfp4_graph_us"]
+    out["note"] = (f"{r.name} layer 0: {r.nq} queries x {r.h} heads, Top-K {r.k} + window {r.w}; events around "
+                   f"each call (exact: attention + merge kernels; nvfp4: q quantisation + attention + merge), eager "
+                   f"and replayed from a CUDA graph, median of {reps} after an L2 flush")
     return out
 
 
@@ -550,9 +603,11 @@ def run_ours(args):
     t_roof, t_parts = step_roofline_us(recipe, dec.lens, dec.schedule, hbm_gbs, bf16_sust)
     step_rl = {"t_roof_us": t_roof, "parts_us": t_parts, "step_us": ms * 1e3, "frac": t_roof / (ms * 1e3),
                "peaks": f"{peak_kind}: {hbm_gbs} GB/s HBM, {bf16_sust} TF/s bf16 sustained (FP8 at 2x)"}
-    append_c4 = time_append_chunk512(B, dev, hbm_gbs) if world == 1 else None
-    append_f8 = time_append_e4m3(B, dev, hbm_gbs) if world == 1 else None
-    sharded = time_sharded_hier1m(dev) if world == 1 and not args.no_sharded else None
+    side = world == 1 and not args.no_side
+    append_c4 = time_append_chunk512(B, dev, hbm_gbs) if side else None
+    append_f8 = time_append_e4m3(B, dev, hbm_gbs) if side else None
+    sharded = time_sharded_hier1m(dev) if side and not args.no_sharded else None
+    attn_nv = time_attn_variants(B, dec) if side and recipe.h == 64 else None
     breakdown = {k: 1e3 * statistics.mean(v) for k, v in attn.items()}
     attn_ms = statistics.mean(attn["attention"]) if attn else float("nan")
     achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
@@ -579,6 +634,7 @@ def run_ours(args):
         "append_chunk512": append_c4,
         "append_e4m3": append_f8,
         "sharded_hier1m": sharded,
+        "attention_nvfp4": attn_nv,
         "breakdown_us_per_call": breakdown,
         "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented replay "
                           "of the same step (event nodes between calls prevent launch overlap)",

@@ -241,6 +241,37 @@ csa2_status csa2_sparse_attn_decode_static(const void *q_bf16, int32_t nq, int32
                                            float *lse, cudaStream_t stream);
 
 /*
+ * NVFP4 speed variant of csa2_sparse_attn_decode ([P3] paragraph "V4.1-Flash
+ * also uses FP4 quantization": the FP4 values are restored for computation
+ * on the chip; here the scores of the selected entries are computed from
+ * the FP4 codes directly). Arguments, layouts, workspace rule and errors are
+ * those of csa2_sparse_attn_decode, with h = 64 (other head counts are
+ * refused with CSA2_ERR_UNSUPPORTED) and the workspace
+ * sized by csa2_sparse_attn_nvfp4_workspace_size. What it computes differs
+ * in one step: q is first quantised to NVFP4 with the cache's own block
+ * quantiser (per 16 values one E4M3 scale = RNE(amax / 6), E2M1 codes RNE
+ * of x / scale), and that quantised q (exact in f16) is used for the scores
+ * of every row; the values (P * V), the softmax and the probabilities are as
+ * in csa2_sparse_attn_decode. Its reference is therefore
+ * csa2_sparse_attn_decode's result for the quantised q, within the same
+ * tolerance; against the unquantised q it deviates by the effect of the
+ * quantisation on the scores.
+ * Kernel: tiles made only of selected entries multiply the raw FP4 codes and
+ * E4M3 block scales of the cache against the FP4 q with block-scaled
+ * tensor-core products (no dequantisation before S); the remaining tiles
+ * (a partial last entry tile and the window) take the f16 path.
+ */
+csa2_status csa2_sparse_attn_decode_nvfp4(const void *q_bf16, int32_t nq, int32_t q_per_seq,
+                                          int32_t h, const csa2_kv_desc *kv, const int32_t *topk,
+                                          int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
+                                          const int32_t *swa_begin, const int32_t *swa_end,
+                                          int32_t w_max, float softmax_scale, void *o_bf16,
+                                          float *lse, void *ws, size_t ws_bytes,
+                                          cudaStream_t stream);
+
+size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max);
+
+/*
  * Building blocks of a long sequence decoded with its entries split across
  * GPUs by entry range (one exchange step per layer; the pages put 1M-token
  * contexts on one sequence: [P3] "CSA2 tackles storage", [P4] "How does the

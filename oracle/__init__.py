@@ -242,3 +242,27 @@ def sparse_attn(q_bf16_bits, codes, scales, page_table_seq, page_size, topk, swa
                           _p(sw, ctypes.c_uint8) if sw.shape[0] else None, sw.shape[0],
                           float(softmax_scale), _p(o, ctypes.c_double), _p(lse, ctypes.c_double))
     return o, lse
+
+
+def nvfp4_round(x_bf16_bits):
+    """Rows of bf16 bits [n, d] -> bf16 bits of their NVFP4 quantise-then-
+    dequantise (the block quantiser above, then code value x scale value).
+    Every such value has at most 6 significant bits and lies in
+    [2^-10, 2688], so it is exact in bf16."""
+    x = _c(x_bf16_bits, np.uint16)
+    codes, scales = quantize_rows(x)
+    out = np.zeros_like(x)
+    for i in range(x.shape[0]):
+        v = dequant_row(codes[i], scales[i]).astype(np.float32)
+        bits = v.view(np.uint32)
+        assert np.all((bits & 0xFFFF) == 0), "NVFP4 value not exact in bf16"
+        out[i] = (bits >> 16).astype(np.uint16)
+    return out
+
+
+def sparse_attn_nvfp4(q_bf16_bits, codes, scales, page_table_seq, page_size, topk, swa_rows, softmax_scale):
+    """The NVFP4 variant of the decode attention: the scores of every row use
+    q after NVFP4 quantisation (nvfp4_round); keys, values and softmax as in
+    sparse_attn."""
+    return sparse_attn(nvfp4_round(q_bf16_bits), codes, scales, page_table_seq, page_size, topk, swa_rows,
+                       softmax_scale)

@@ -62,6 +62,9 @@ _SIGS = {
     "csa2_sparse_attn_decode": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
                                        _f32, _vp, _vp, _vp, _sz, _vp]),
     "csa2_sparse_attn_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "csa2_sparse_attn_decode_nvfp4": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
+                                             _f32, _vp, _vp, _vp, _sz, _vp]),
+    "csa2_sparse_attn_nvfp4_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
     "csa2_sparse_attn_decode_static": (_i32, [_vp, _i32, _i32, _i32, _kvp, _vp, _i32, _vp, _i64, _vp, _vp, _i32,
                                               _f32, _vp, _vp, _vp]),
     "csa2_score_ids": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _i32, _kvp, _i32, _vp, _vp]),
@@ -186,6 +189,22 @@ def csa2_sparse_attn_decode_static(q_bf16, q_per_seq, kv: KvCache, topk, swa, sw
         _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
         _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_bf16), _ptr(lse),
         _stream(stream)))
+
+
+def csa2_sparse_attn_nvfp4_workspace_size(nq, h, k, w_max):
+    return _lib.csa2_sparse_attn_nvfp4_workspace_size(nq, h, k, w_max)
+
+
+def csa2_sparse_attn_decode_nvfp4(q_bf16, q_per_seq, kv: KvCache, topk, swa, swa_seq_stride, swa_begin, swa_end,
+                                  w_max, softmax_scale, o_bf16, lse, ws, stream=None):
+    """csa2_sparse_attn_decode with q quantised to NVFP4 for the scores (FP4
+    block-scaled products on the selected entries); h = 64."""
+    nq, h = q_bf16.shape[0], q_bf16.shape[1]
+    k = topk.shape[1] if topk is not None else 0
+    _check("csa2_sparse_attn_decode_nvfp4", _lib.csa2_sparse_attn_decode_nvfp4(
+        _ptr(q_bf16), nq, q_per_seq, h, kv.desc, _ptr(topk), k, _ptr(swa), int(swa_seq_stride),
+        _ptr(swa_begin), _ptr(swa_end), int(w_max), float(softmax_scale), _ptr(o_bf16), _ptr(lse),
+        _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
 
 
 def csa2_append_swa_e4m3(x_bf16, seq, pos, swa, stream=None):

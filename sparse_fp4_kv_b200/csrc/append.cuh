@@ -28,6 +28,33 @@ namespace csa2 {
 
 constexpr int kAppendWarps = 8;
 
+// Quantise one block of 16 values (binary32 copies of bf16 or narrower
+// inputs) with the rule above: returns the E4M3 scale byte and writes the 16
+// E2M1 codes, element i in nibble i of packed[i / 8].
+__device__ __forceinline__ uint32_t quantize_block16(const float (&f)[16], uint32_t (&packed)[2]) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));  // fmaxf drops NaN operands
+    const uint32_t s = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+    const float sv = __half2float(__ushort_as_half((uint16_t)(e4m3x2_to_f16x2((uint16_t)s) & 0xFFFFu)));
+    // decision points of the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}; at an
+    // exact midpoint the even-mantissa neighbour wins ('>' keeps the lower
+    // point, '>=' takes the upper one)
+    const float t1 = 0.25f * sv, t2 = 0.75f * sv, t3 = 1.25f * sv, t4 = 1.75f * sv;
+    const float t5 = 2.5f * sv, t6 = 3.5f * sv, t7 = 5.0f * sv;
+    packed[0] = packed[1] = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(f[i]);
+        uint32_t c = (uint32_t)(a > t1) + (uint32_t)(a >= t2) + (uint32_t)(a > t3) + (uint32_t)(a >= t4) +
+                     (uint32_t)(a > t5) + (uint32_t)(a >= t6) + (uint32_t)(a > t7);
+        c |= (__float_as_uint(f[i]) >> 31) << 3;
+        if (sv == 0.0f) c = 0u;
+        packed[i >> 3] |= c << (4 * (i & 7));
+    }
+    return s;
+}
+
 __global__ void __launch_bounds__(kAppendWarps * 32)
     k_append_fp4(const uint16_t *__restrict__ x, int32_t n, const int32_t *__restrict__ seq,
                  const int64_t *__restrict__ pos, csa2_kv_desc kv) {
@@ -54,26 +81,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
         f[2 * i] = __uint_as_float(wds[i] << 16);
         f[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));  // fmaxf drops NaN operands
-    const uint32_t s = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
-    const float sv = __half2float(__ushort_as_half((uint16_t)(e4m3x2_to_f16x2((uint16_t)s) & 0xFFFFu)));
-    // decision points of the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}; at an
-    // exact midpoint the even-mantissa neighbour wins ('>' keeps the lower
-    // point, '>=' takes the upper one)
-    const float t1 = 0.25f * sv, t2 = 0.75f * sv, t3 = 1.25f * sv, t4 = 1.75f * sv;
-    const float t5 = 2.5f * sv, t6 = 3.5f * sv, t7 = 5.0f * sv;
-    uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float a = fabsf(f[i]);
-        uint32_t c = (uint32_t)(a > t1) + (uint32_t)(a >= t2) + (uint32_t)(a > t3) + (uint32_t)(a >= t4) +
-                     (uint32_t)(a > t5) + (uint32_t)(a >= t6) + (uint32_t)(a > t7);
-        c |= (__float_as_uint(f[i]) >> 31) << 3;
-        if (sv == 0.0f) c = 0u;
-        packed[i >> 3] |= c << (4 * (i & 7));
-    }
+    uint32_t packed[2];
+    const uint32_t s = quantize_block16(f, packed);
     uint2 *dst = reinterpret_cast<uint2 *>(kv.codes + row * (CSA2_D / 2) + lane * 8);
     *dst = make_uint2(packed[0], packed[1]);
     kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;

@@ -37,6 +37,7 @@
 // log-sum-exp values.
 #pragma once
 
+#include "append.cuh"
 #include "common.cuh"
 
 namespace csa2 {
@@ -49,19 +50,32 @@ constexpr uint32_t kBarWork = 5;                      // named barrier of the wo
 constexpr int kAttnTile = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int H>
+template <int H, bool NV = false>
 struct AttnCfg {
     static constexpr int kKvBytes = kAttnTile * CSA2_D * 2;  // 128 KiB f16 tile
     static constexpr int kQBytes = H * CSA2_D * 2;
+    // NVFP4 variant: the Q region holds, in splits of selected entries, the
+    // raw FP4 codes of the tile and of q (K-major, 128B-swizzled) and the
+    // staging of their scale bytes (rows padded to 36 bytes); in window
+    // splits it holds the f16 Q tile as above.
+    static constexpr int kRawBytes = kAttnTile * CSA2_D / 2;
+    static constexpr int kQ4Bytes = H * CSA2_D / 2;
+    static constexpr int kStage = 36;
+    static constexpr int kStageBytes = kAttnTile * kStage;
+    static constexpr int kQStageBytes = H * kStage;
+    static constexpr int kNvBytes = kRawBytes + kQ4Bytes + kStageBytes + kQStageBytes;
+    static constexpr int kQRegion = NV ? ((kNvBytes > kQBytes ? kNvBytes : kQBytes) + 1023) / 1024 * 1024 : kQBytes;
     static constexpr int kPBytes = kAttnTile * H * 2;
     static constexpr int kPGroup = 16 * H;  // bytes of 8 rows of P^T
     static constexpr uint32_t kPSwizzle = H == 64 ? kSw128 : (H == 32 ? kSw64 : kSw32);
     static constexpr int kColS = 0;
     static constexpr int kColO = H;
+    static constexpr int kColSFA = 5 * H;       // NV: scale factors of the tile rows, 4 columns per K step
+    static constexpr int kColSFB = 5 * H + 32;  // NV: scale factors of q, H / 32 columns per K step
     static constexpr uint32_t kTmemCols = H == 64 ? 512u : (H == 32 ? 256u : 128u);
-    static constexpr int kMisc = 8 * 128 * 5 /*resolved rows*/ + 128 * 4 /*valid*/ + 4 * H * 4 /*red*/ +
-                                 3 * H * 4 /*m, alpha, l*/ + 128 /*bars, slot, flags*/;
-    static constexpr size_t kSmem = 1024 + (size_t)kKvBytes + kQBytes + kPBytes + kMisc;
+    static constexpr int kMisc = 8 * 128 * 5 /*resolved rows*/ + (NV ? 2 : 1) * 128 * 4 /*valid*/ +
+                                 4 * H * 4 /*red*/ + 3 * H * 4 /*m, alpha, l*/ + 128 /*bars, slot, flags*/;
+    static constexpr size_t kSmem = 1024 + (size_t)kKvBytes + kQRegion + kPBytes + kMisc;
 };
 
 struct AttnParams {
@@ -82,7 +96,38 @@ struct AttnParams {
     int32_t n_splits;
     int32_t tiles_per_split;
     int32_t out_f32;   // write normalised f32 o (o_part, S = 1) instead of bf16 o
+    // NVFP4 variant: splits [0, e_splits) take tp_e tiles each of the first
+    // e_tiles tiles (selected entries only) with FP4 products for S; the other
+    // splits take tiles_per_split tiles each from tile e_tiles on.
+    int32_t e_splits, e_tiles, tps_e;
+    uint8_t *q4;   // NV: q in NVFP4, codes [nq][H][256] (element i in nibble i & 1 of byte i / 2)
+    uint8_t *q4s;  // NV: its E4M3 block scales [nq][H][32]
 };
+
+// NVFP4 variant, before the attention kernel: every 16-value block of q
+// quantised with the cache's block quantiser, a thread per block.
+constexpr int kQuantThreads = 256;
+__global__ void __launch_bounds__(kQuantThreads)
+    k_quant_rows_nvfp4(const uint16_t *__restrict__ x, int32_t n_blocks, uint8_t *__restrict__ codes,
+                       uint8_t *__restrict__ scales) {
+    pdl_trigger();
+    pdl_wait();
+    const int32_t i = blockIdx.x * kQuantThreads + threadIdx.x;
+    if (i >= n_blocks) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)i * CSA2_BLOCK);
+    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+    const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        f[2 * j] = __uint_as_float(w8[j] << 16);
+        f[2 * j + 1] = __uint_as_float(w8[j] & 0xFFFF0000u);
+    }
+    uint32_t pk[2];
+    const uint32_t sc = quantize_block16(f, pk);
+    *reinterpret_cast<uint2 *>(codes + (int64_t)i * 8) = make_uint2(pk[0], pk[1]);
+    scales[i] = (uint8_t)sc;
+}
 
 __device__ __forceinline__ uint32_t kv_chunk_off(int e, int c64) {
     // f16 KV tile: row e, 16-byte chunk c64 (d = 8*c64 .. 8*c64+7)
@@ -229,7 +274,8 @@ __device__ __forceinline__ void fetch_tile(const AttnParams &p, int32_t b, const
 // (128B-swizzled K-major); chunk 0 also records which rows hold data. Lanes
 // of pieces 4..7 store their second 16-byte half first, so the eight lanes
 // of each store phase hit eight different bank groups.
-__device__ __forceinline__ void store_chunk(const TileRaw &raw, int c, uint8_t *kv_tile, int32_t *valid_s) {
+__device__ __forceinline__ void store_chunk(const TileRaw &raw, int c, uint8_t *kv_tile, int32_t *valid_s,
+                                            bool write_valid = true) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int piece = lane & 7;
 #pragma unroll
@@ -263,7 +309,32 @@ __device__ __forceinline__ void store_chunk(const TileRaw &raw, int c, uint8_t *
         const uint4 second = swap ? make_uint4(h0[0], h0[1], h0[2], h0[3]) : make_uint4(h1[0], h1[1], h1[2], h1[3]);
         *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, c64 + (swap ? 1 : 0))) = first;
         *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, c64 + (swap ? 0 : 1))) = second;
-        if (c == 0 && piece == 0) valid_s[e] = kd != 0u;
+        if (write_valid && c == 0 && piece == 0) valid_s[e] = kd != 0u;
+    }
+}
+
+// NVFP4 variant: the raw FP4 codes of the fetched rows (selected entries or
+// empty) into the K-major 128B-swizzled A tile of the block-scaled product,
+// their scale bytes into the staging rows, and which rows hold data.
+template <int STAGE>
+__device__ __forceinline__ void store_raw(const TileRaw &raw, uint8_t *raw_tile, uint8_t *stage, int32_t *valid_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int piece = lane & 7;
+#pragma unroll
+    for (int j = 0; j < kRowGroups; ++j) {
+        const uint32_t kd = (raw.kinds >> (2 * j)) & 3u;
+        const int e = warp * kRowsPerWarp + 4 * j + (lane >> 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v = raw.v[c * kRowGroups + j];
+            const bool fp4 = kd == 1u;
+            const int blk = 8 * c + piece;
+            const uint32_t off = (uint32_t)((blk >> 4) * 16384 + (e >> 3) * 1024 + (e & 7) * 128 +
+                                            ((((blk & 15) >> 1) ^ (e & 7)) << 4) + (blk & 1) * 8);
+            *reinterpret_cast<uint2 *>(raw_tile + off) = fp4 ? make_uint2(v.x, v.y) : make_uint2(0u, 0u);
+            stage[e * STAGE + blk] = fp4 ? (uint8_t)(v.z & 0xFFu) : (uint8_t)0;
+        }
+        if (piece == 0) valid_s[e] = kd == 1u;
     }
 }
 
@@ -303,20 +374,21 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float scale_log2, bo
     }
 }
 
-template <int H>
+template <int H, bool NV>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
-    using Cfg = AttnCfg<H>;
+    using Cfg = AttnCfg<H, NV>;
+    static_assert(!NV || H == 64, "the NVFP4 variant runs its S product at N = 64");
     constexpr int G = H >= 32 ? 4 : 2;  // softmax head groups (4 warps each, a warp per TMEM lane quarter)
     constexpr int HG = H / G;            // heads per group
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *kv_tile = base;
     uint8_t *q_tile = kv_tile + Cfg::kKvBytes;
-    uint8_t *p_tile = q_tile + Cfg::kQBytes;
+    uint8_t *p_tile = q_tile + Cfg::kQRegion;
     int32_t *rsrc = reinterpret_cast<int32_t *>(p_tile + Cfg::kPBytes);  // [kResolveTiles * 128]
     uint8_t *rkind = reinterpret_cast<uint8_t *>(rsrc + kResolveTiles * kAttnTile);
     int32_t *valid_s = reinterpret_cast<int32_t *>(rkind + kResolveTiles * kAttnTile);
-    float *red = reinterpret_cast<float *>(valid_s + kAttnTile);  // [4][H]
+    float *red = reinterpret_cast<float *>(valid_s + (NV ? 2 : 1) * kAttnTile);  // [4][H]
     float *m_run = red + 4 * H;
     float *alpha = m_run + H;
     float *l_run = alpha + H;
@@ -324,8 +396,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     uint64_t *bar_pv = bar_kv + 4;                               // [4] P*V of chunk c done
     uint64_t *bar_s = bar_pv + 4;                                // S^T of the tile ready
     uint64_t *bar_p = bar_s + 1;                                 // P^T of the tile written
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_p + 1);
+    uint64_t *bar_raw = bar_p + 1;                               // NV: raw FP4 tile + scale factors stored
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_raw + 1);
     int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [4] (per head group)
+
+    uint8_t *raw_tile = q_tile;                 // NV, entry splits
+    uint8_t *q4_tile = q_tile + Cfg::kRawBytes;
+    uint8_t *stage = q4_tile + Cfg::kQ4Bytes;
+    uint8_t *qstage = stage + Cfg::kStageBytes;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t split = blockIdx.x, u = blockIdx.y;
@@ -344,6 +422,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         }
         mbar_init(bar_s, 1);
         mbar_init(bar_p, kAttnWorkThreads);
+        if (NV) mbar_init(bar_raw, kAttnWorkThreads);
         rescale_tile[0] = rescale_tile[1] = rescale_tile[2] = rescale_tile[3] = -1;
         fence_mbar_init();
     }
@@ -361,8 +440,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     }
     const int64_t n_total = (int64_t)p.k + nw;
     const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
-    const int64_t t_begin = (int64_t)split * p.tiles_per_split;
-    const int64_t t_end = min(tiles_total, t_begin + p.tiles_per_split);
+    // NV: an entry split (FP4 products for S) or a split from tile e_tiles on
+    const bool fp4 = NV && split < p.e_splits;
+    int64_t t_begin, t_end;
+    if (fp4) {
+        t_begin = (int64_t)split * p.tps_e;
+        t_end = min((int64_t)p.e_tiles, t_begin + p.tps_e);
+    } else {
+        const int32_t s2 = NV ? split - p.e_splits : split;
+        t_begin = (NV ? (int64_t)p.e_tiles : 0) + (int64_t)s2 * p.tiles_per_split;
+        t_end = min(tiles_total, t_begin + p.tiles_per_split);
+    }
     const int ntiles = (int)max((int64_t)0, t_end - t_begin);
 
     // ---- prologue: Q loads in flight first, then resolve the first rows and
@@ -376,12 +464,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         constexpr int kChunks = H * (CSA2_D / 8);
         constexpr int kPer = kChunks / kAttnWorkThreads;  // 8 / 4 / 2 for H = 64 / 32 / 16
         uint4 qv[kPer];
+        if (NV) {
+            // NVFP4 q from the pre-pass: block b = tid + t * threads (codes, scale)
 #pragma unroll
-        for (int t = 0; t < kPer; ++t) qv[t] = __ldg(qsrc + tid + t * kAttnWorkThreads);
+            for (int t = 0; t < kPer / 2; ++t) {
+                const int bq = tid + t * kAttnWorkThreads;
+                const uint2 cc = *reinterpret_cast<const uint2 *>(p.q4 + ((int64_t)u * H * 32 + bq) * 8);
+                qv[t] = make_uint4(cc.x, cc.y, (uint32_t)p.q4s[(int64_t)u * H * 32 + bq], 0u);
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < kPer; ++t) qv[t] = __ldg(qsrc + tid + t * kAttnWorkThreads);
+        }
         if (ntiles > 0)
             resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile, min(kResolveTiles, ntiles) * kAttnTile, rsrc, rkind);
         named_bar_sync(kBarWork, kAttnWorkThreads);
         if (ntiles > 0) fetch_tile<0, 4>(p, b, rsrc, rkind, 0, raw);
+        if constexpr (NV) {
+            // q in NVFP4: FP4 codes + scale staging for entry splits, its exact
+            // f16 values for window splits
+#pragma unroll
+            for (int t = 0; t < kPer / 2; ++t) {
+                const int bq = tid + t * kAttnWorkThreads;
+                const int h = bq >> 5, blk = bq & 31;
+                const uint32_t pk[2] = {qv[t].x, qv[t].y};
+                const uint32_t sc = qv[t].z;
+                if (fp4) {
+                    const uint32_t off = (uint32_t)((blk >> 4) * (H * 128) + (h >> 3) * 1024 + (h & 7) * 128 +
+                                                    ((((blk & 15) >> 1) ^ (h & 7)) << 4) + (blk & 1) * 8);
+                    *reinterpret_cast<uint2 *>(q4_tile + off) = make_uint2(pk[0], pk[1]);
+                    qstage[h * Cfg::kStage + blk] = (uint8_t)sc;
+                } else {
+                    const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)(sc | (sc << 8)));
+                    uint32_t h0[4], h1[4];
+                    e2m1x8_to_f16x8(pk[0], h0);
+                    e2m1x8_to_f16x8(pk[1], h1);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        h0[i] = hmul2_u32(h0[i], s2);
+                        h1[i] = hmul2_u32(h1[i], s2);
+                    }
+                    *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, 2 * blk)) =
+                        make_uint4(h0[0], h0[1], h0[2], h0[3]);
+                    *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, 2 * blk + 1)) =
+                        make_uint4(h1[0], h1[1], h1[2], h1[3]);
+                }
+            }
+        } else {
 #pragma unroll
         for (int t = 0; t < kPer; ++t) {
             const int i = tid + t * kAttnWorkThreads;
@@ -395,6 +524,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
                 o4[q] = *reinterpret_cast<const uint32_t *>(&hh);
             }
             *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
         }
         fence_proxy_async_smem();
     }
@@ -415,7 +545,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         const uint64_t b_o = make_sdesc(p_addr, 16, Cfg::kPGroup, Cfg::kPSwizzle);
         if (mma_warp) {
             // ---- one elected thread issues every tensor-core product ----
-            if (lane == 0) {
+            if (NV && fp4 && lane == 0) {
+                // S^T = A * B^T with A = the raw FP4 rows, B = q in FP4, one UE4M3
+                // scale per 16 values from TMEM, as soon as the rows are stored;
+                // the P*V products follow as below, chunk by chunk once each f16
+                // chunk is dequantised
+                const uint32_t idesc_s4 = idesc_nvf4_f32(128, H);
+                const uint64_t a_s4 = make_sdesc(smem_u32(raw_tile), 16, 1024, kSw128);
+                const uint64_t b_s4 = make_sdesc(smem_u32(q4_tile), 16, 1024, kSw128);
+                bool ok = true;
+                for (int it = 0; it < ntiles && ok; ++it) {
+                    const uint32_t ph = (uint32_t)it & 1u;
+                    if (!mbar_wait(bar_raw, ph)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kb = 0; kb < CSA2_D / 64; ++kb)
+                        mma_nvf4(tmem + Cfg::kColS, a_s4 + (uint64_t)(((kb >> 2) * 16384 + (kb & 3) * 32) >> 4),
+                                 b_s4 + (uint64_t)(((kb >> 2) * (H * 128) + (kb & 3) * 32) >> 4), idesc_s4,
+                                 tmem + Cfg::kColSFA + 4 * kb, tmem + Cfg::kColSFB + (H / 32) * kb, kb > 0 ? 1u : 0u);
+                    tc_commit(bar_s);
+                    if (!mbar_wait(bar_p, ph)) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int dc = 0; dc < 4; ++dc) {
+                        if (!mbar_wait(&bar_kv[dc], ph)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < kAttnTile / 16; ++kk)
+                            mma_f16(tmem + Cfg::kColO + dc * H, a_o + (uint64_t)((dc * 32768 + kk * 2048) >> 4),
+                                    b_o + (uint64_t)((kk * 2 * Cfg::kPGroup) >> 4), idesc_o,
+                                    (it > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(&bar_pv[dc]);
+                    }
+                }
+            } else if (lane == 0) {
                 bool ok = true;
                 for (int it = 0; it < ntiles && ok; ++it) {
                     const uint32_t ph = (uint32_t)it & 1u;
@@ -465,13 +631,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
 #pragma unroll
         for (int i = 0; i < HG; ++i) l_part[i] = 0.0f;
         bool ok = true;
+        if (NV && fp4 && warp < 4) {
+            // scale factors of q (B), replicated in every TMEM lane quarter: lane l,
+            // column (H / 32) * kb + j holds the four scales of K step kb of head 32 j + l
+            const uint32_t *qs = reinterpret_cast<const uint32_t *>(qstage);
+            const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16) + Cfg::kColSFB;
+            if constexpr (H == 64) {
+                uint32_t r[16];
+#pragma unroll
+                for (int kb = 0; kb < 8; ++kb)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) r[2 * kb + j] = qs[((32 * j + lane) * Cfg::kStage) / 4 + kb];
+                tmem_st16(ta, r);
+            } else {
+                uint32_t r[8];
+#pragma unroll
+                for (int kb = 0; kb < 8; ++kb) r[kb] = qs[(lane * Cfg::kStage) / 4 + kb];
+                tmem_st8(ta, r);
+            }
+        }
         for (int it = 0; it < ntiles; ++it) {
             const int64_t tt = t_begin + it;
+            int32_t *vs = valid_s + ((NV && fp4) ? (it & 1) * kAttnTile : 0);
+            if (NV && fp4) {
+                // 0. raw FP4 rows and their scale factors for S (the previous tile's S is
+                //    complete: this thread waited for it in the softmax)
+                store_raw<Cfg::kStage>(raw, raw_tile, stage, vs);
+                fence_proxy_async_smem();
+                named_bar_sync(kBarWork, kAttnWorkThreads);
+                if (warp < 4) {
+                    // lane l, column 4 kb + j: the four scales of K step kb of row 32 j + l
+                    const uint32_t *st = reinterpret_cast<const uint32_t *>(stage);
+                    uint32_t r[32];
+#pragma unroll
+                    for (int kb = 0; kb < 8; ++kb)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) r[4 * kb + j] = st[((32 * j + lane) * Cfg::kStage) / 4 + kb];
+                    tmem_st32(tmem + ((uint32_t)(warp * 32) << 16) + Cfg::kColSFA, r);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(bar_raw);
+            }
             // 1. dequantise chunk c as soon as the previous tile's P*V on it is done
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 if (it > 0 && ok && !mbar_wait(&bar_pv[c], (uint32_t)(it - 1) & 1u)) ok = false;
-                store_chunk(raw, c, kv_tile, valid_s);
+                store_chunk(raw, c, kv_tile, vs, !(NV && fp4));
                 fence_proxy_async_smem();
                 mbar_arrive(&bar_kv[c]);
             }
@@ -494,7 +700,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
                 if (!got) ok = false;
                 tc_fence_after();
                 const int row = quarter * 32 + lane;
-                const bool row_valid = valid_s[row] != 0 && got;
+                const bool row_valid = vs[row] != 0 && got;
                 const uint32_t s_addr = lane_addr + Cfg::kColS + grp * HG;
                 float v[HG];
                 load_scores<HG>(s_addr, p.scale_log2, row_valid, v);

@@ -212,6 +212,10 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
 
 // Instruction descriptors (kind::f16 with f16 operands, kind::f8f6f4 with
 // E4M3 operands), f32 accumulator. mn_major: 1 = operand is M/N-major.
+// Bit fields (sm_100 instruction descriptor): 4..5 accumulator type (1 = f32),
+// 7..9 / 10..12 A / B type, 15 / 16 A / B major, 17..22 N / 8, 24..28 M / 16;
+// for the block-scaled kinds bits 4..5 and 29..30 select the scale-factor
+// byte of B / A, bit 23 the scale type (0 = UE4M3) and E2M1 is type 1.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major, int b_mn_major) {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -226,6 +230,22 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Block-scaled FP4 product (kind::mxf4nvf4, E2M1 operands, one UE4M3 scale
+// per 16 K values, f32 accumulator); scale factors read from TMEM at sfa /
+// sfb (A: each K step of 64 takes 4 columns at M = 128; B: N / 32 columns).
+__host__ __device__ constexpr uint32_t idesc_nvf4_f32(int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
         : "memory");
 }
 

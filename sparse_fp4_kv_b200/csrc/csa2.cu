@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <numeric>
 #include <cmath>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <cstdint>
@@ -146,6 +147,7 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
 // charge per split for writing and merging the partials.
 struct AttnPlan {
     int32_t tiles, tiles_per_split, splits;
+    int32_t e_tiles = 0, e_splits = 0, tps_e = 0;  // NVFP4 variant: entry splits (see plan_attn_nvfp4)
 };
 
 AttnPlan plan_attn(int32_t nq, int32_t k, int32_t w_max, int sms) {
@@ -174,17 +176,72 @@ AttnPlan plan_attn(int32_t nq, int32_t k, int32_t w_max, int sms) {
     return P;
 }
 
+// NVFP4 variant: the first floor(k / 128) tiles (selected entries only) go
+// to entry splits whose S products are FP4; the rest (the last partial entry
+// tile and the window) to splits on the f16 path. Both split lengths are
+// chosen together with the same cost model, an FP4 tile charged kFp4Tile
+// f16 tiles (measured on the 64-head, 2048 + 512-row step: about 6.3 us per
+// FP4 tile against 5.1 us per f16 tile, from runs of 1 to 16 tiles a CTA).
+AttnPlan plan_attn_nvfp4(int32_t nq, int32_t k, int32_t w_max, int sms) {
+    const int32_t e_tiles = k / kAttnTile;
+    if (e_tiles == 0) return plan_attn(nq, k, w_max, sms);
+    AttnPlan P{};
+    const int64_t rows = (int64_t)k + std::max(0, w_max);
+    P.tiles = (int32_t)((rows + kAttnTile - 1) / kAttnTile);
+    const int32_t w_tiles = P.tiles - e_tiles;
+    // fixed tiles per entry split and per window split, "te,tw" (tuning, tests)
+    if (const char *e = std::getenv("CSA2_ATTN_NV_TILES")) {
+        int te = 1, tw = 1;
+        if (std::sscanf(e, "%d,%d", &te, &tw) == 2 && te > 0 && tw > 0) {
+            P.e_tiles = e_tiles;
+            P.tps_e = std::min(te, e_tiles);
+            P.e_splits = (e_tiles + P.tps_e - 1) / P.tps_e;
+            P.tiles_per_split = w_tiles > 0 ? std::min(tw, w_tiles) : 1;
+            P.splits = P.e_splits + (w_tiles > 0 ? (w_tiles + P.tiles_per_split - 1) / P.tiles_per_split : 0);
+            return P;
+        }
+    }
+    constexpr double kFp4Tile = 1.25, kFixed = 1.2, kMergePerSplit = 0.1;
+    double best = 1e30;
+    for (int32_t te = 1; te <= e_tiles; ++te) {
+        const int32_t se = (e_tiles + te - 1) / te;
+        for (int32_t tw = 1; tw <= std::max(1, w_tiles); ++tw) {
+            const int32_t sw = w_tiles > 0 ? (w_tiles + tw - 1) / tw : 0;
+            const int32_t splits = se + sw;
+            const double waves = (double)(((int64_t)nq * splits + sms - 1) / sms);
+            const double per = std::max(kFp4Tile * te, w_tiles > 0 ? (double)tw : 0.0) + kFixed;
+            const double cost = waves * per + (splits > 1 ? kMergePerSplit * splits : 0.0);
+            if (cost < best - 1e-9) {
+                best = cost;
+                P.e_tiles = e_tiles;
+                P.tps_e = te;
+                P.e_splits = se;
+                P.tiles_per_split = w_tiles > 0 ? tw : 1;
+                P.splits = splits;
+            }
+        }
+    }
+    return P;
+}
+
 struct AttnLayout {
     size_t off_o, off_lse, total;
+    size_t off_q4 = 0, off_q4s = 0;  // NVFP4 variant: q codes [nq][h][256], scales [nq][h][32]
 };
 
 // Split partials: f32 [nq][S][H][512], then the log-sum-exp values [nq][S][H].
-AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P) {
+AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P, bool nvfp4 = false) {
     AttnLayout L{};
-    if (P.splits <= 1) return L;
-    L.off_o = 0;
-    L.off_lse = align_up((size_t)nq * P.splits * h * CSA2_D * 4, 256);
-    L.total = align_up(L.off_lse + (size_t)nq * P.splits * h * 4, 256);
+    if (P.splits > 1) {
+        L.off_o = 0;
+        L.off_lse = align_up((size_t)nq * P.splits * h * CSA2_D * 4, 256);
+        L.total = align_up(L.off_lse + (size_t)nq * P.splits * h * 4, 256);
+    }
+    if (nvfp4) {
+        L.off_q4 = L.total;
+        L.off_q4s = align_up(L.off_q4 + (size_t)nq * h * (CSA2_D / 2), 256);
+        L.total = align_up(L.off_q4s + (size_t)nq * h * (CSA2_D / CSA2_BLOCK), 256);
+    }
     return L;
 }
 
@@ -593,10 +650,13 @@ void launch_combine(int32_t h, int32_t nq, const CombineArgs &ca, cudaStream_t s
 csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h, const csa2_kv_desc *kv,
                       const int32_t *topk, int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
                       const int32_t *swa_begin, const int32_t *swa_end, int32_t w_max, float softmax_scale, void *o,
-                      bool out_f32, float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
+                      bool out_f32, float *lse, void *ws, size_t ws_bytes, cudaStream_t stream, bool nvfp4 = false) {
     csa2_status st = check_kv(kv, false);
     if (st != CSA2_OK) return st;
     if (h != 16 && h != 32 && h != 64) return CSA2_ERR_UNSUPPORTED;
+    // the block-scaled S product runs at N = 64 only (its scale-factor layout in
+    // TMEM is established for that shape)
+    if (nvfp4 && h != 64) return CSA2_ERR_UNSUPPORTED;
     if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
         return CSA2_ERR_INVALID_ARG;
     if (k < 0 || w_max < 0 || (k > 0 && !topk) || (topk && !aligned(topk, 4))) return CSA2_ERR_INVALID_ARG;
@@ -608,8 +668,9 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
         return CSA2_ERR_INVALID_ARG;
     if (!has_swa && w_max > 0) return CSA2_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return CSA2_ERR_INVALID_ARG;
-    const AttnPlan P = plan_attn(nq, k, has_swa ? w_max : 0, num_sms());
-    const AttnLayout L = attn_layout(nq, h, P);
+    const AttnPlan P = nvfp4 ? plan_attn_nvfp4(nq, k, has_swa ? w_max : 0, num_sms())
+                             : plan_attn(nq, k, has_swa ? w_max : 0, num_sms());
+    const AttnLayout L = attn_layout(nq, h, P, nvfp4);
     if (L.total > 0 && (!ws || ws_bytes < L.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
 
@@ -623,8 +684,13 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
     ap.swa_end = has_swa ? swa_end : nullptr;
     ap.o = out_f32 ? nullptr : static_cast<uint16_t *>(o);
     ap.lse = lse;
-    ap.o_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_o) : nullptr;
-    ap.lse_part = L.total ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_lse) : nullptr;
+    const bool parts = P.splits > 1;
+    ap.o_part = parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_o) : nullptr;
+    ap.lse_part = parts ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.off_lse) : nullptr;
+    if (nvfp4) {
+        ap.q4 = static_cast<uint8_t *>(ws) + L.off_q4;
+        ap.q4s = static_cast<uint8_t *>(ws) + L.off_q4s;
+    }
     ap.out_f32 = out_f32 ? 1 : 0;
     if (out_f32 && P.splits == 1) {
         // one split: the kernel's f32 partial is the result
@@ -636,26 +702,40 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
     ap.q_per_seq = q_per_seq;
     ap.n_splits = P.splits;
     ap.tiles_per_split = P.tiles_per_split;
+    ap.e_splits = P.e_splits;
+    ap.e_tiles = P.e_tiles;
+    ap.tps_e = P.tps_e;
     const dim3 grid((unsigned)P.splits, (unsigned)nq);
     auto go = [&](auto kernel, size_t smem) { launch(kernel, grid, dim3(kAttnThreads), smem, stream, ap); };
-    switch (h) {
-        case 64: {
-            static bool ok = set_smem(k_sparse_attn<64>, AttnCfg<64>::kSmem);
-            if (!ok) return CSA2_ERR_CUDA;
-            go(k_sparse_attn<64>, AttnCfg<64>::kSmem);
-            break;
-        }
-        case 32: {
-            static bool ok = set_smem(k_sparse_attn<32>, AttnCfg<32>::kSmem);
-            if (!ok) return CSA2_ERR_CUDA;
-            go(k_sparse_attn<32>, AttnCfg<32>::kSmem);
-            break;
-        }
-        default: {
-            static bool ok = set_smem(k_sparse_attn<16>, AttnCfg<16>::kSmem);
-            if (!ok) return CSA2_ERR_CUDA;
-            go(k_sparse_attn<16>, AttnCfg<16>::kSmem);
-            break;
+    if (nvfp4) {
+        static const bool ok = set_smem(k_sparse_attn<64, true>, AttnCfg<64, true>::kSmem);
+        if (!ok) return CSA2_ERR_CUDA;
+        // q -> NVFP4 once per call (codes and scales into the workspace)
+        const int32_t n_blocks = nq * h * (CSA2_D / CSA2_BLOCK);
+        launch(k_quant_rows_nvfp4, dim3((unsigned)((n_blocks + kQuantThreads - 1) / kQuantThreads)),
+               dim3(kQuantThreads), 0, stream, static_cast<const uint16_t *>(q_bf16), n_blocks, ap.q4, ap.q4s);
+        if ((st = check_launch()) != CSA2_OK) return st;
+        go(k_sparse_attn<64, true>, AttnCfg<64, true>::kSmem);
+    } else {
+        switch (h) {
+            case 64: {
+                static bool ok = set_smem(k_sparse_attn<64, false>, AttnCfg<64>::kSmem);
+                if (!ok) return CSA2_ERR_CUDA;
+                go(k_sparse_attn<64, false>, AttnCfg<64>::kSmem);
+                break;
+            }
+            case 32: {
+                static bool ok = set_smem(k_sparse_attn<32, false>, AttnCfg<32>::kSmem);
+                if (!ok) return CSA2_ERR_CUDA;
+                go(k_sparse_attn<32, false>, AttnCfg<32>::kSmem);
+                break;
+            }
+            default: {
+                static bool ok = set_smem(k_sparse_attn<16, false>, AttnCfg<16>::kSmem);
+                if (!ok) return CSA2_ERR_CUDA;
+                go(k_sparse_attn<16, false>, AttnCfg<16>::kSmem);
+                break;
+            }
         }
     }
     if ((st = check_launch()) != CSA2_OK) return st;
@@ -699,6 +779,21 @@ csa2_status csa2_sparse_attn_partial(const void *q_bf16, int32_t nq, int32_t q_p
                                      size_t ws_bytes, cudaStream_t stream) {
     return attn_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end, w_max,
                      softmax_scale, o_f32, true, lse, ws, ws_bytes, stream);
+}
+
+size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max) {
+    if (nq <= 0 || k < 0 || h != 64) return 0;
+    const AttnPlan P = plan_attn_nvfp4(nq, k, w_max, num_sms());
+    return attn_layout(nq, h, P, true).total;
+}
+
+csa2_status csa2_sparse_attn_decode_nvfp4(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h,
+                                          const csa2_kv_desc *kv, const int32_t *topk, int32_t k, const uint8_t *swa,
+                                          int64_t swa_seq_stride, const int32_t *swa_begin, const int32_t *swa_end,
+                                          int32_t w_max, float softmax_scale, void *o_bf16, float *lse, void *ws,
+                                          size_t ws_bytes, cudaStream_t stream) {
+    return attn_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end, w_max,
+                     softmax_scale, o_bf16, false, lse, ws, ws_bytes, stream, true);
 }
 
 csa2_status csa2_attn_merge(const float *o_parts, const float *lse_parts, int32_t g, int32_t nq, int32_t h,

@@ -431,6 +431,45 @@ def test_attention_padding_and_order_do_not_matter():
     np.testing.assert_allclose(l1, l2, atol=1e-13)
 
 
+# ---- NVFP4 variant of the attention ------------------------------------------
+
+def test_nvfp4_round_is_independent_dequant_of_quantiser_and_idempotent():
+    rng = np.random.default_rng(15)
+    q = _bf16_bits((rng.standard_normal((6, 512)) * np.exp(rng.uniform(-4, 4, (6, 1)))).astype(np.float32))
+    r = oracle.nvfp4_round(q)
+    codes, scales = oracle.quantize_rows(q)
+    want = _bf16_bits(_dequant_indep(codes, scales).astype(np.float32))
+    np.testing.assert_array_equal(r, want)
+    np.testing.assert_array_equal(oracle.nvfp4_round(r), r)       # already NVFP4 values stay put
+    assert np.any(r != q)
+
+
+def test_attention_nvfp4_is_dense_softmax_of_rounded_q():
+    rng = np.random.default_rng(16)
+    d = 64
+    q, codes, scales, pt, topk, swa = _attn_case(rng, d=d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = oracle.sparse_attn_nvfp4(q, codes, scales, pt, 8, topk, swa, scale)
+    # independent: q rounded with the independent dequantisation of its codes,
+    # rows gathered and dequantised by hand, torch softmax + matmul
+    qc, qs = oracle.quantize_rows(q)
+    Qh = torch.from_numpy(_dequant_indep(qc, qs))
+    rows = [pt[t // 8] * 8 + t % 8 for t in topk if t >= 0]
+    V = torch.from_numpy(np.concatenate([_dequant_indep(codes[rows], scales[rows]),
+                                         torch.from_numpy(swa).view(torch.float8_e4m3fn).double().numpy()]))
+    z = scale * Qh @ V.T
+    np.testing.assert_allclose(o, (torch.softmax(z, dim=-1) @ V).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, torch.logsumexp(z, dim=-1).numpy(), rtol=0, atol=1e-12)
+    # the quantised q changes the result; a q that is already NVFP4 does not
+    o_exact, _ = oracle.sparse_attn(q, codes, scales, pt, 8, topk, swa, scale)
+    assert np.abs(o - o_exact).max() > 1e-4
+    qn = oracle.nvfp4_round(q)
+    o1, l1 = oracle.sparse_attn_nvfp4(qn, codes, scales, pt, 8, topk, swa, scale)
+    o2, l2 = oracle.sparse_attn(qn, codes, scales, pt, 8, topk, swa, scale)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
 # ---- FP8 appends (window rows, indexer keys) --------------------------------
 
 def _all_bf16():
