@@ -467,19 +467,28 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
             o_loc |= v;
         }
     }
-    atomicAnd(&and_acc, a_loc);
-    atomicOr(&or_acc, o_loc);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
+        o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicAnd(&and_acc, a_loc);
+        atomicOr(&or_acc, o_loc);
+    }
     uint32_t nvalid;
     block_excl_scan<NT>(nvalid_t, scratch, &nvalid);  // its barriers also publish k64 and the reductions
     const uint32_t r = min((uint32_t)p.k, nvalid);
     uint64_t T = 1ull;  // select keys >= T (every valid key is >= 2^31)
     if (nvalid > (uint32_t)p.k) {
+        // digits of 11 bits from the highest bit in which two keys differ;
+        // bits that are equal in every key are skipped (they decide nothing)
         const unsigned long long diff = and_acc ^ or_acc;
         const int hb = 63 - __clzll((long long)diff);
         uint64_t prefix = hb == 63 ? 0ull : (and_acc & ~((1ull << (hb + 1)) - 1ull));
         uint64_t pmask = hb == 63 ? 0ull : ~((1ull << (hb + 1)) - 1ull);
         uint32_t rem = r;
-        for (int top = hb; top >= 0; top -= 11) {
+        for (int top = hb; top >= 0;) {
             const int nbits = top + 1 < 11 ? top + 1 : 11;
             const int shift = top + 1 - nbits;
             const int nb = 1 << nbits;
@@ -499,8 +508,13 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
             const bool all_taken = hist[bin] == rem;
             __syncthreads();
             if (all_taken) break;
+            const uint64_t below = shift > 0 ? (diff & ((1ull << shift) - 1ull)) : 0ull;
+            if (below == 0ull) break;
+            top = 63 - __clzll((long long)below);
         }
-        T = prefix;
+        // the threshold carries the bits every key shares, so that only the
+        // resolved digits (and the unresolved low bits of the last bin) decide
+        T = prefix | (and_acc & ~diff);
     }
     // ordered emission (pool order)
     const int per = (p.p + NT - 1) / NT;
