@@ -282,11 +282,35 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_source_hash():
+def code_of(src):
+    """C++/CUDA source without comments, trailing blanks and empty lines (what the
+    compiler sees), so that comment edits do not count as kernel changes."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif src[i] == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(src[i])
+            i += 1
+    return "\n".join(ln.rstrip() for ln in "".join(out).split("\n") if ln.strip())
+
+
+def kernel_source_hash(csrc=None):
+    csrc = csrc or os.path.join(ROOT, "sparse_fp4_kv_b200", "csrc")
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(os.path.join(ROOT, "sparse_fp4_kv_b200", "csrc"))):
-        with open(os.path.join(ROOT, "sparse_fp4_kv_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            h.update(code_of(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -35,6 +35,14 @@
 // Probabilities stay below 2^8 and are exact in range for f16.
 // Splits of one query are merged by k_attn_combine with their
 // log-sum-exp values.
+//
+// NVFP4 variant (NV = true, 64 heads): q is rounded to NVFP4 beforehand
+// (k_quant_rows_nvfp4). Splits made only of whole tiles of selected entries
+// store each tile's raw FP4 codes into a K-major A tile and its E4M3 block
+// scales into TMEM as scale factors, and S^T comes from block-scaled FP4
+// products (kind::mxf4nvf4) without waiting for the dequantisation, which
+// still feeds P*V. The remaining tiles (a partial last entry tile, the
+// window) take the path above with the rounded q in f16.
 #pragma once
 
 #include "append.cuh"
