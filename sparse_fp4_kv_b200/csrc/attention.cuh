@@ -803,11 +803,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
             }
             mbar_arrive(bar_p);
         }
-        // the last tile's P*V
-        if (ntiles > 0 && ok && !mbar_wait(&bar_pv[3], (uint32_t)(ntiles - 1) & 1u)) ok = false;
-        tc_fence_after();
-
-        // ---- final denominators: reduce the per-row partials over the 128 rows ----
+        // ---- final denominators: reduce the per-row partials over the 128 rows
+        //      (the last softmax is done; the last tile's P*V may still run) ----
         named_bar_sync(kBarWork, kAttnWorkThreads);
         if (soft) {
             warp_transpose_reduce<HG, false>(l_part);
@@ -821,51 +818,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         }
         named_bar_sync(kBarWork, kAttnWorkThreads);
 
-        // ---- epilogue: O^T (TMEM) -> o = O / l written straight from registers:
-        //      a thread owns latent column d = 128*dc + 32*quarter + lane of its
+        // ---- epilogue: O^T (TMEM) -> o = O / l written straight from registers,
+        //      latent chunk dc as soon as the last tile's P*V on it is done (the
+        //      stores of a chunk run under the products of the next ones): a
+        //      thread owns latent column d = 128*dc + 32*quarter + lane of its
         //      group's heads, so each store instruction of a warp covers 32
-        //      consecutive columns of one head (coalesced); the four TMEM loads
-        //      of a thread are in flight together ----
+        //      consecutive columns of one head (coalesced) ----
         {
             if (soft) {
-                uint32_t vals[4][HG];  // raw f32 bits
-                if (ntiles > 0) {
-#pragma unroll
-                    for (int dc = 0; dc < 4; ++dc) {
+                const int d0 = quarter * 32 + lane;
+                const bool bf16_out = p.n_splits == 1 && !p.out_f32;
+                uint16_t *dst16 = p.o + (int64_t)u * H * CSA2_D;
+                float *dst32 = bf16_out ? nullptr : p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D;
+#pragma unroll 1
+                for (int dc = 0; dc < 4; ++dc) {
+                    uint32_t vals[HG];  // raw f32 bits
+                    if (ntiles > 0) {
+                        if (ok && !mbar_wait(&bar_pv[dc], (uint32_t)(ntiles - 1) & 1u)) ok = false;
+                        tc_fence_after();
                         const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + grp * HG;
                         if (HG == 16) {
-                            tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&vals[dc][0]));
+                            tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&vals[0]));
                         } else {
-                            tmem_ld8(ta, *reinterpret_cast<uint32_t(*)[8]>(&vals[dc][0]));
+                            tmem_ld8(ta, *reinterpret_cast<uint32_t(*)[8]>(&vals[0]));
                         }
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < HG; ++i) vals[i] = 0u;
                     }
-                    tmem_wait_ld();
-                } else {
+                    if (bf16_out) {
 #pragma unroll
-                    for (int dc = 0; dc < 4; ++dc)
+                        for (int i = 0; i < HG; ++i) {
+                            const int h = grp * HG + i;
+                            dst16[(int64_t)h * CSA2_D + dc * 128 + d0] = f32_to_bf16_bits(__uint_as_float(vals[i]) * alpha[h]);
+                        }
+                    } else {
 #pragma unroll
-                        for (int i = 0; i < HG; ++i) vals[dc][i] = 0u;
-                }
-                const int d0 = quarter * 32 + lane;
-                if (p.n_splits == 1 && !p.out_f32) {
-                    uint16_t *dst = p.o + (int64_t)u * H * CSA2_D;
-#pragma unroll
-                    for (int i = 0; i < HG; ++i) {
-                        const int h = grp * HG + i;
-                        const float inv = alpha[h];
-#pragma unroll
-                        for (int dc = 0; dc < 4; ++dc)
-                            dst[(int64_t)h * CSA2_D + dc * 128 + d0] = f32_to_bf16_bits(__uint_as_float(vals[dc][i]) * inv);
-                    }
-                } else {
-                    float *dst = p.o_part + ((int64_t)u * p.n_splits + split) * H * CSA2_D;
-#pragma unroll
-                    for (int i = 0; i < HG; ++i) {
-                        const int h = grp * HG + i;
-                        const float inv = alpha[h];
-#pragma unroll
-                        for (int dc = 0; dc < 4; ++dc)
-                            dst[(int64_t)h * CSA2_D + dc * 128 + d0] = __uint_as_float(vals[dc][i]) * inv;
+                        for (int i = 0; i < HG; ++i) {
+                            const int h = grp * HG + i;
+                            dst32[(int64_t)h * CSA2_D + dc * 128 + d0] = __uint_as_float(vals[i]) * alpha[h];
+                        }
                     }
                 }
             }
