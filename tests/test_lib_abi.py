@@ -104,3 +104,30 @@ def test_host_validation_rejects_before_launch(binding):
                                      0x3000, None, None, 0, None) == 2
     assert L.csa2_sparse_attn_decode(0x1000, 1, 1, 64, _desc(binding), 0x2000, 8, None, 0, None, None, 16, 0.1,
                                      0x3000, None, None, 0, None) == 1
+
+
+def test_host_validation_of_shard_and_variant_calls(binding):
+    L = binding._lib
+    kv = _desc(binding)
+    # NVFP4 attention: 64 heads only; a window size without window rows
+    assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 32, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
+                                           None, None, 0, None) == 2
+    assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 64, kv, 0x2000, 8, None, 0, None, None, 16, 0.1, 0x3000,
+                                           None, None, 0, None) == 1
+    assert binding.csa2_sparse_attn_nvfp4_workspace_size(1, 32, 256, 0) == 0
+    # f32 partials need an lse output
+    assert L.csa2_sparse_attn_partial(0x1000, 1, 1, 64, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
+                                      None, None, 0, None) == 1
+    # merge: head count, part count, alignment
+    assert L.csa2_attn_merge(0x1000, 0x2000, 2, 1, 48, 0x3000, None, None) == 2
+    assert L.csa2_attn_merge(0x1000, 0x2000, 0, 1, 64, 0x3000, None, None) == 1
+    assert L.csa2_attn_merge(0x1004, 0x2000, 2, 1, 64, 0x3000, None, None) == 1
+    # id scoring: indexer heads, empty id list, negative offset, unsupported key width
+    assert L.csa2_score_ids(0x1000, 0x2000, 1, 1, 17, 0x3000, 8, kv, 0, 0x4000, None) == 2
+    assert L.csa2_score_ids(0x1000, 0x2000, 1, 1, 4, 0x3000, 0, kv, 0, 0x4000, None) == 1
+    assert L.csa2_score_ids(0x1000, 0x2000, 1, 1, 4, 0x3000, 8, kv, -1, 0x4000, None) == 1
+    assert L.csa2_score_ids(0x1000, 0x2000, 1, 1, 4, 0x3000, 8, _desc(binding, di=32), 0, 0x4000, None) == 2
+    # key selection: too many keys, k = 0, misaligned keys
+    assert L.csa2_select_keys(0x1000, 1, (1 << 20) + 1, 8, 0x2000, None) == 2
+    assert L.csa2_select_keys(0x1000, 1, 64, 0, 0x2000, None) == 1
+    assert L.csa2_select_keys(0x1004, 1, 64, 8, 0x2000, None) == 1
