@@ -215,20 +215,34 @@ struct TileRaw {
     uint32_t kinds;  // 2 bits per j: 0 empty, 1 FP4 global entry, 2 window row
 };
 
-// Resolve the sources of rows [j0, j0 + n) of the query's attended list into
-// shared memory: physical FP4 row (kind 1), window buffer row (kind 2) or
-// nothing (kind 0). The work warps take part; two dependent loads per row,
-// all rows in flight together.
+// Resolve the sources of rows [j0, j0 + n) (n <= kResolveTiles * 128) of the
+// query's attended list into shared memory: physical FP4 row (kind 1), window
+// buffer row (kind 2) or nothing (kind 0). The work warps take part; thread t
+// takes rows t and t + 512. id_pre (nullable) holds those rows' entry ids
+// already loaded; pt0 is the sequence's page when the cache has one page per
+// sequence (one_page), so that no row waits for a page-table load.
+constexpr int kResolvePerThread = kResolveTiles * kAttnTile / kAttnWorkThreads;  // 2
 __device__ __forceinline__ void resolve_rows(const AttnParams &p, int32_t u, int32_t b, int32_t nw, int32_t wb,
-                                             int64_t j0, int n, int32_t *rsrc, uint8_t *rkind) {
-    for (int i = threadIdx.x; i < n; i += kAttnWorkThreads) {
+                                             int64_t j0, int n, int32_t *rsrc, uint8_t *rkind,
+                                             const int32_t (*id_pre)[kResolvePerThread], bool one_page, int64_t pt0) {
+#pragma unroll
+    for (int r = 0; r < kResolvePerThread; ++r) {
+        const int i = threadIdx.x + r * kAttnWorkThreads;
+        if (i >= n) break;
         const int64_t j = j0 + i;
         int32_t src = 0;
         uint8_t kind = 0;
         if (j < p.k) {
-            const int32_t id = p.topk[(int64_t)u * p.k + j];
+            const int32_t id = id_pre ? (*id_pre)[r] : p.topk[(int64_t)u * p.k + j];
             if (id >= 0) {
-                const int64_t row = physical_row(p.kv, b, id);
+                int64_t row;
+                if (one_page) {
+                    // physical_row with the one page of the sequence already loaded
+                    row = (id < p.kv.page_size && pt0 >= 0) ? pt0 * p.kv.page_size + id : -1;
+                    if (row >= p.kv.rows_cap) row = -1;
+                } else {
+                    row = physical_row(p.kv, b, id);
+                }
                 if (row >= 0) {
                     src = (int32_t)row;
                     kind = 1;
@@ -439,6 +453,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
         l_run[tid] = 0.0f;
     }
     pdl_wait();
+    // NV: an entry split (FP4 products for S) or a split from tile e_tiles on
+    const bool fp4 = NV && split < p.e_splits;
+    const int64_t t_begin = fp4 ? (int64_t)split * p.tps_e
+                                : (NV ? (int64_t)p.e_tiles : 0) +
+                                      (int64_t)(NV ? split - p.e_splits : split) * p.tiles_per_split;
+    // the entry ids of the first resolved rows and, for a cache with one page per
+    // sequence, that page go in flight together with the window bounds
+    const bool one_page = p.kv.max_pages == 1;
+    int64_t pt0 = 0;
+    int32_t id_pre[kResolvePerThread];
+#pragma unroll
+    for (int r = 0; r < kResolvePerThread; ++r) id_pre[r] = -1;
+    if (tid < kAttnWorkThreads) {
+#pragma unroll
+        for (int r = 0; r < kResolvePerThread; ++r) {
+            const int64_t j = t_begin * kAttnTile + tid + r * kAttnWorkThreads;
+            if (j < p.k) id_pre[r] = p.topk[(int64_t)u * p.k + j];
+        }
+        if (one_page) pt0 = p.kv.page_table[b];
+    }
     const int32_t wb = p.swa_begin ? p.swa_begin[u] : 0;
     int32_t nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
     // the window is a run of ring slots: begin in [0, stride), at most stride rows
@@ -448,17 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
     }
     const int64_t n_total = (int64_t)p.k + nw;
     const int64_t tiles_total = (n_total + kAttnTile - 1) / kAttnTile;
-    // NV: an entry split (FP4 products for S) or a split from tile e_tiles on
-    const bool fp4 = NV && split < p.e_splits;
-    int64_t t_begin, t_end;
-    if (fp4) {
-        t_begin = (int64_t)split * p.tps_e;
-        t_end = min((int64_t)p.e_tiles, t_begin + p.tps_e);
-    } else {
-        const int32_t s2 = NV ? split - p.e_splits : split;
-        t_begin = (NV ? (int64_t)p.e_tiles : 0) + (int64_t)s2 * p.tiles_per_split;
-        t_end = min(tiles_total, t_begin + p.tiles_per_split);
-    }
+    const int64_t t_end = fp4 ? min((int64_t)p.e_tiles, t_begin + p.tps_e) : min(tiles_total, t_begin + p.tiles_per_split);
     const int ntiles = (int)max((int64_t)0, t_end - t_begin);
 
     // ---- prologue: Q loads in flight first, then resolve the first rows and
@@ -485,7 +509,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
             for (int t = 0; t < kPer; ++t) qv[t] = __ldg(qsrc + tid + t * kAttnWorkThreads);
         }
         if (ntiles > 0)
-            resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile, min(kResolveTiles, ntiles) * kAttnTile, rsrc, rkind);
+            resolve_rows(p, u, b, nw, wb, t_begin * kAttnTile, min(kResolveTiles, ntiles) * kAttnTile, rsrc, rkind,
+                         &id_pre, one_page, pt0);
         named_bar_sync(kBarWork, kAttnWorkThreads);
         if (ntiles > 0) fetch_tile<0, 4>(p, b, rsrc, rkind, 0, raw);
         if constexpr (NV) {
@@ -696,7 +721,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_sparse_attn(AttnParams p) {
                     // next batch of resolved rows (rare: splits of more than 8 tiles)
                     named_bar_sync(kBarWork, kAttnWorkThreads);
                     resolve_rows(p, u, b, nw, wb, (tt + 1) * kAttnTile,
-                                 (int)min((int64_t)kResolveTiles, t_end - (tt + 1)) * kAttnTile, rsrc, rkind);
+                                 (int)min((int64_t)kResolveTiles, t_end - (tt + 1)) * kAttnTile, rsrc, rkind,
+                                 nullptr, one_page, pt0);
                     named_bar_sync(kBarWork, kAttnWorkThreads);
                 }
                 fetch_tile<0, 4>(p, b, rsrc, rkind, rel * kAttnTile, raw);
