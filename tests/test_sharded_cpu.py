@@ -2,9 +2,10 @@
 ranges, and the sharded decoder (local Full, key exchange, selection from the
 union, Reindex over the owned pool ids, attention partials with the window on
 the first shard, log-sum-exp merge) run with the oracle standing in for the
-library calls, against the unsharded oracle decode. Two gloo ranks for the
-exchange through torch.distributed; several shards in one process for more
-world sizes, an empty shard and a Full layer without a pool."""
+library calls, against the unsharded oracle decode. Two and three gloo ranks
+(uneven ranges) for the exchange through torch.distributed; several shards in
+one process for more world sizes, an empty shard and a Full layer without a
+pool."""
 import os
 import socket
 
@@ -103,11 +104,12 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_match_unsharded_oracle():
-    world, port = 2, _free_port()
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_match_unsharded_oracle(world):
+    port = _free_port()
     out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     exp = _expected(SMALL)
     for rank in range(world):
-        _check(SMALL, exp, *out[rank], f"rank {rank}")
-    assert out[0][0] == out[1][0]          # every rank holds the same selection
+        _check(SMALL, exp, *out[rank], f"rank {rank} of {world}")
+        assert out[rank][0] == out[0][0]   # every rank holds the same selection
