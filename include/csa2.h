@@ -269,6 +269,8 @@ csa2_status csa2_sparse_attn_decode_nvfp4(const void *q_bf16, int32_t nq, int32_
                                           float *lse, void *ws, size_t ws_bytes,
                                           cudaStream_t stream);
 
+/* Workspace bytes of csa2_sparse_attn_decode_nvfp4 (split partials plus q's
+ * FP4 codes and scales); 0 for a head count other than 64. */
 size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max);
 
 /*
@@ -280,20 +282,31 @@ size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, i
  *
  * csa2_score_ids: score the given entry ids (local to kv, -1 = empty) as the
  *   indexer does, into unique 64-bit keys (ordered score key << 32 |
- *   ~(id + id_offset)); empty ids give key 0. ids [nq][m], keys [nq][m].
- *   id + id_offset must stay below 2^31.
+ *   ~(id + id_offset)); empty ids give key 0. ids [nq][m], keys [nq][m]
+ *   (8-byte aligned), qidx / w as in csa2_index_full. Requires
+ *   kv->di in {64, 128} and 1 <= hi <= 16 (else CSA2_ERR_UNSUPPORTED),
+ *   m >= 1 and id_offset >= 0 (else CSA2_ERR_INVALID_ARG); id + id_offset
+ *   must stay below 2^31. An id outside the cache gives key 0 and sets
+ *   CSA2_DEVERR_BAD_ROW. No workspace.
  * csa2_select_keys: the k largest keys of each query's m keys, written as
  *   the ids they carry (~ of the low 32 bits), in key-array order, padded
  *   with -1; key 0 is empty. Because the id is part of the key, equal scores
- *   are taken in ascending id order. m <= 2^20 (up to about 28000 keys are
- *   staged in shared memory, larger sets are re-read from L2 in every radix
- *   pass). keys [nq][m], ids [nq][k].
+ *   are taken in ascending id order. keys [nq][m], ids [nq][k]. Requires
+ *   m, k >= 1 (else CSA2_ERR_INVALID_ARG) and m <= 2^20 (else
+ *   CSA2_ERR_UNSUPPORTED); up to about 28000 keys are staged in shared
+ *   memory, larger sets are re-read from L2 in every radix pass. No
+ *   workspace.
  * csa2_sparse_attn_partial: csa2_sparse_attn_decode over this rank's rows,
- *   writing the normalised f32 o [nq][h][512] and lse [nq][h] (required)
- *   instead of bf16 o; the same workspace.
+ *   writing the normalised f32 o [nq][h][512] and lse [nq][h] instead of
+ *   bf16 o; lse is required (else CSA2_ERR_INVALID_ARG); the same workspace
+ *   rule. A query with no rows gives o = 0 and lse = -inf.
  * csa2_attn_merge: merge g such partials o_parts [g][nq][h][512],
  *   lse_parts [g][nq][h] into bf16 o [nq][h][512] and lse [nq][h]
- *   (nullable): o = sum_r exp(lse_r - M) o_r / sum_r exp(lse_r - M).
+ *   (nullable): o = sum_r exp(lse_r - M) o_r / sum_r exp(lse_r - M) with
+ *   M = max_r lse_r; parts with lse = -inf weigh nothing, and all of them
+ *   -inf give o = 0, lse = -inf. Requires h in {16, 32, 64} (else
+ *   CSA2_ERR_UNSUPPORTED), g >= 1, o_parts / o_bf16 16-byte aligned (else
+ *   CSA2_ERR_INVALID_ARG). No workspace.
  */
 csa2_status csa2_score_ids(const uint8_t *qidx, const float *w, int32_t nq, int32_t q_per_seq,
                            int32_t hi, const int32_t *ids, int32_t m, const csa2_kv_desc *kv,
