@@ -32,6 +32,10 @@
  *     slot in every id list.
  *   - Reuse mode is not a call: a Reuse layer passes its source layer's
  *     Top-k list to csa2_sparse_attn_decode.
+ *   - One device per process: the library sets its kernels' shared-memory
+ *     limits once, on the device current at a kernel's first call; calls on
+ *     another device of the same process may then fail with CSA2_ERR_CUDA.
+ *     (The fixed scratch of csa2_sparse_attn_decode_static is per device.)
  */
 #ifndef CSA2_H
 #define CSA2_H
