@@ -1,23 +1,25 @@
 """Benchmark of the CSA2 decode hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stack20]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|NAME]
     python bench.py --impl reference ...      # the CPU oracle, same metric
 
-A step is one decode step of the workload through the C-ABI: FP4 append of
-the new token of every sequence, then every layer of the static mode schedule
-(Full / Reindex indexer where scheduled, Reuse otherwise) followed by sparse +
-window attention. Default workload: the 20-layer decoder stack, 8 sequences
-x 1 query, 65536 FP4 entries each (Full at 0 and 10, Reindex at 5 and 15,
-Reuse elsewhere, Top-K 2048, 64 heads, window 512).
+A step is one decode step of a workload through the C-ABI: FP4 append of the
+step's new rows, then every layer of the static mode schedule (Full /
+Reindex indexer where scheduled, Reuse otherwise) followed by sparse + window
+attention. Every workload of the benchmark set is measured (tiny_full,
+stack20, hier1m, paged64, chunk512; --workload picks one); the JSON line
+carries one record per workload under "configs", and its headline fields are
+those of the largest single-GPU workload, paged64 (64 paged sequences of
+16K-256K entries, Full + 3 Reuse layers, 32 heads).
 
-Metric: decode query-steps per second per layer = batch * queries * layers /
-step time, with the achieved HBM bandwidth of the step's algorithmic bytes.
-Timing: the step is captured once in a CUDA graph; each of the K timed steps
-is preceded by a 256 MiB L2 flush and bracketed by CUDA events on the
-launching stream; a barrier and a device synchronize bracket the whole timed
-loop; the reported time is the max over ranks. Multi-GPU runs give every rank
-its own independent batch of sequences (weak scaling, no collective on the
-data path).
+Metric: decode query-steps per second per layer = sequences * queries *
+layers / step time, with the achieved HBM bandwidth of the step's
+algorithmic bytes. Timing: each workload's step is captured once in a CUDA
+graph; each of the K timed steps is preceded by a 256 MiB L2 flush and
+bracketed by CUDA events on the launching stream; a barrier and a device
+synchronize bracket each workload's timed loop; the reported time is the max
+over ranks. Multi-GPU runs give every rank its own independent sequences
+(weak scaling, no collective on the data path).
 """
 import argparse
 import datetime
@@ -35,15 +37,18 @@ sys.path.insert(0, ROOT)
 
 METRIC = "CSA2 decode query-steps/s per layer; achieved HBM TB/s vs ~8 TB/s peak"
 UNIT = "query-steps/s/layer"
+WORKLOADS = ("tiny_full", "stack20", "hier1m", "paged64", "chunk512")
+HEADLINE = "paged64"  # the largest workload that fits one GPU
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="stack20")
+    ap.add_argument("--workload", default="all", help="one workload, or 'all' (the default)")
+    ap.add_argument("--headline", default=HEADLINE, help="workload whose record fills the headline fields")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sharded", action="store_true", help="skip the entry-range sharded side measurement")
@@ -55,58 +60,40 @@ def parse():
 # ---------------------------------------------------------------------------
 # algorithmic work (what the method must move / compute)
 # ---------------------------------------------------------------------------
-def algorithmic(recipe, lens, schedule):
-    """(bytes, flops) of one step, and (bytes, flops) of one attention launch."""
+def call_costs(recipe, lens, schedule):
+    """[(kind, layer, bytes, flops, tc)] of the step's C-ABI calls in order:
+    algorithmic bytes (inputs read once, outputs written once) and flops; tc
+    names the tensor-core type of the flops ('fp8' indexer products, 'f16'
+    attention products, None)."""
     nq, h, d = recipe.nq, recipe.h, 512
     n_vis = [int(l) for l in lens.tolist()]
-    by = fl = 0.0
+    out = []
     rows_app = recipe.append if recipe.chunked else recipe.batch
-    by += rows_app * (d * 2 + d // 2 + d // 16)
-    attn_by = attn_fl = 0.0
-    for mode, src in schedule:
-        if mode == "full":
-            for qi in range(nq):
-                n = n_vis[qi // recipe.q_per_seq]
-                by += n * recipe.di
-                fl += 2.0 * recipe.hi * recipe.di * n
-        elif mode == "reindex":
-            by += nq * recipe.p * (recipe.di + 4)
-            fl += 2.0 * nq * recipe.hi * recipe.di * recipe.p
-        rows = recipe.k + recipe.w
-        a_by = nq * (recipe.k * (d // 2 + d // 16 + 4) + recipe.w * d + 2 * 2 * h * d)
-        a_fl = 4.0 * nq * h * rows * d
-        by += a_by
-        fl += a_fl
-        attn_by, attn_fl = a_by, a_fl
-    return by, fl, attn_by, attn_fl
-
-
-def step_roofline_us(recipe, lens, schedule, hbm_gbs, tc_tflops):
-    """t_roof of one step in microseconds: the sum over the step's kernels of
-    max(algorithmic bytes / HBM peak, flops / tensor peak); the indexer's
-    FP8 products are counted at twice the bf16 peak."""
-    nq, h, d = recipe.nq, recipe.h, 512
-    n_vis = [int(l) for l in lens.tolist()]
-    bw, tc = hbm_gbs * 1e9, tc_tflops * 1e12
-    rows_app = recipe.append if recipe.chunked else recipe.batch
-    t = rows_app * (d * 2 + d // 2 + d // 16) / bw
-    parts = {"append": t}
-    for mode, src in schedule:
+    out.append(("append", -1, rows_app * (d * 2 + d // 2 + d // 16), 0.0, None))
+    ql = recipe.q_limit()
+    for l, (mode, src) in enumerate(schedule):
         if mode == "full":
             b = f = 0.0
             for qi in range(nq):
-                n = n_vis[qi // recipe.q_per_seq]
-                b += n * recipe.di
+                n = int(ql[qi]) if ql is not None else n_vis[qi // recipe.q_per_seq]
+                b += n * recipe.di + 4 * (recipe.k + recipe.p)
                 f += 2.0 * recipe.hi * recipe.di * n
-            parts["full"] = parts.get("full", 0.0) + max(b / bw, f / (2 * tc))
+            out.append(("full", l, b, f, "fp8"))
         elif mode == "reindex":
-            b = nq * recipe.p * (recipe.di + 4)
-            f = 2.0 * nq * recipe.hi * recipe.di * recipe.p
-            parts["reindex"] = parts.get("reindex", 0.0) + max(b / bw, f / (2 * tc))
+            out.append(("reindex", l, nq * recipe.p * (recipe.di + 4) + nq * recipe.k * 4,
+                        2.0 * nq * recipe.hi * recipe.di * recipe.p, "fp8"))
         a_by = nq * (recipe.k * (d // 2 + d // 16 + 4) + recipe.w * d + 2 * 2 * h * d)
         a_fl = 4.0 * nq * h * (recipe.k + recipe.w) * d
-        parts["attention"] = parts.get("attention", 0.0) + max(a_by / bw, a_fl / tc)
-    return sum(parts.values()) * 1e6, {k: v * 1e6 for k, v in parts.items()}
+        out.append(("attention", l, a_by, a_fl, "f16"))
+    return out
+
+
+def call_roof_us(by, fl, tc, hbm_gbs, peaks_tf):
+    """max(bytes / HBM peak, flops / tensor peak of the call's type), in us,
+    and which of the two bounds it."""
+    t_b = by / (hbm_gbs * 1e9) * 1e6
+    t_f = fl / (peaks_tf[tc] * 1e12) * 1e6 if tc else 0.0
+    return (t_b, "hbm") if t_b >= t_f else (t_f, "tensor")
 
 
 def time_append_chunk512(B, dev, hbm_gbs, reps=20):
@@ -127,24 +114,35 @@ def time_append_chunk512(B, dev, hbm_gbs, reps=20):
     seq = torch.zeros(n, dtype=torch.int32, device=dev)
     pos = torch.arange(r.prefill, r.prefill + n, dtype=torch.int64, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
     for _ in range(3):
         B.csa2_append_fp4(x, seq, pos, kv)
-    ts = []
-    for i in range(reps):
-        flush.fill_(i & 0xFF)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        B.csa2_append_fp4(x, seq, pos, kv)
-        e1.record()
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) * 1e3)
-    ts.sort()
-    us = ts[len(ts) // 2]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        B.csa2_append_fp4(x, seq, pos, kv, stream)
+    res = {}
+    for mode, run in (("eager", lambda: B.csa2_append_fp4(x, seq, pos, kv, stream)), ("graph", g.replay)):
+        ts = []
+        for i in range(reps):
+            with torch.cuda.stream(stream):
+                flush.fill_(i & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                run()
+                e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        ts.sort()
+        res[mode] = ts[len(ts) // 2]
+    del g
     by = n * (512 * 2 + 256 + 32)
-    return {"rows": n, "us_median": us, "algorithmic_bytes": by, "achieved_gbs": by / (us * 1e-6) / 1e9,
-            "peak_gbs": hbm_gbs, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
-            "note": "bf16 rows in, FP4 codes + E4M3 scales out, 256K-entry cache; CUDA events around the call "
-                    "(launch included), median of %d after an L2 flush" % reps}
+    us = res["graph"]
+    return {"rows": n, "us_median_graph": us, "us_median_eager": res["eager"], "algorithmic_bytes": by,
+            "achieved_gbs": by / (us * 1e-6) / 1e9, "peak_gbs": hbm_gbs, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs,
+            "note": "bf16 rows in, FP4 codes + E4M3 scales out, 256K-entry cache; CUDA events around the call, "
+                    "replayed from a CUDA graph (frac) and eager (launch included), median of %d, L2 flushed "
+                    "before each" % reps}
 
 
 def time_append_e4m3(B, dev, hbm_gbs, reps=20):
@@ -273,13 +271,39 @@ def time_sharded_hier1m(dev, world=2, reps=5):
 
 
 def peaks():
+    """Roofline denominators: the measured copy bandwidth and cuBLAS
+    bf16 rates of this machine's B200s (MEASURED_PEAKS.json), else the fallback
+    figures of the same pool."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
-        return j.get("hbm_gbs", 6650.0), j.get("bf16_tflops", 1590.0), j.get("bf16_tflops_sustained", 1400.0), \
-            "measured"
-    return 6650.0, 1590.0, 1400.0, "fallback"
+        return {"hbm_gbs": float(j.get("hbm_gbs", 6650.0)), "bf16_tflops": float(j.get("bf16_tflops", 1590.0)),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", 1400.0)), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def measure_tc_probe(dev):
+    """Tensor-core rates of this library's own instruction forms (tcgen05.mma
+    kind::f16 and kind::f8f6f4, M = 128, every SM, CUDA events around the
+    grid): TF/s per (kind, N)."""
+    import ctypes
+    import torch
+    lib = ctypes.CDLL(os.path.join(ROOT, "sparse_fp4_kv_b200", "libcsa2_peak.so"))
+    lib.peak_tcgen05.restype = ctypes.c_float
+    lib.peak_tcgen05.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    iters = 1 << 15
+    out = {}
+    for kind, name, kk in ((0, "f16", 16), (1, "fp8_e4m3", 32)):
+        for n in (64, 256):
+            ms = min(lib.peak_tcgen05(kind, n, iters, stream) for _ in range(3))
+            if ms > 0:
+                out[f"{name}_n{n}_tflops"] = 2.0 * 128 * n * kk * iters * sms / (ms * 1e-3) / 1e12
+    out["note"] = ("one CTA per SM issuing tcgen05.mma (M = 128, operands in shared memory) back to back; "
+                   f"{iters} instructions per SM, CUDA events around the grid")
+    return out
 
 
 def code_of(src):
@@ -332,68 +356,95 @@ def recorded_traffic(kernel, workload):
 # clocks sampler
 # ---------------------------------------------------------------------------
 class Clocks:
-    """nvidia-smi samples every 50 ms; only the samples taken between mark()
-    calls (the timed region) are summarised."""
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and throttle reasons of this rank's GPU, read through
+    NVML by a thread every 2 ms (reading only: no setting is touched).
+    summary() describes the samples taken between the last mark(0) and
+    mark(1) (a timed region)."""
+    PERIOD_S = 0.002
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
+    def __init__(self, device):
+        self.device = device
         self.window = [None, None]
+        self.rows = []  # (perf_counter time, sm MHz, max MHz, power W, reasons)
+        self.thread = None
+        self.stop_flag = False
+        self.error = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:
+            bus = torch.cuda.get_device_properties(self.device).pci_bus_id
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(int(self.device.index or 0))
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import threading
+            import pynvml
+            h = self._nvml_handle()
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def loop():
+                while not self.stop_flag:
+                    t = time.perf_counter()
+                    try:
+                        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((t, sm, max_mhz, pw, [n for n, b in bits.items() if rs & b]))
+                    except Exception:
+                        pass
+                    time.sleep(self.PERIOD_S)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+        except Exception as e:  # no NVML: the record says so
+            self.thread = None
+            self.error = str(e)[:80]
 
     def mark(self, which):
-        self.window[which] = datetime.datetime.now()
+        self.window[which] = time.perf_counter()
+
+    def summary(self):
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"no clock source ({self.error})"]}
+        t0, t1 = self.window
+        inside = [r for r in list(self.rows) if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
+        reasons = sorted({n for r in inside for n in r[4]})
+        return {"sm_mhz": statistics.median(r[1] for r in inside) if inside else None,
+                "sm_max_mhz": max(r[2] for r in inside) if inside else None, "reasons": reasons,
+                "samples_in_timed_region": len(inside),
+                "power_w_median": statistics.median(r[3] for r in inside) if inside else None,
+                "source": "NVML every 2 ms"}
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        rows = []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
-                rows.append((ts, float(parts[2]), float(parts[3]),
-                             [n for n, v in zip(names, parts[6:10]) if v.lower() == "active"]))
-            except ValueError:
-                continue
-        t0, t1 = self.window
-        inside = [r for r in rows if t0 is not None and t1 is not None and t0 <= r[0] <= t1]
-        use = inside if inside else rows
-        reasons = sorted({n for r in use for n in r[3]})
-        return {"sm_mhz": statistics.median(r[1] for r in use) if use else None,
-                "sm_max_mhz": max(r[2] for r in use) if use else None, "reasons": reasons,
-                "samples": len(use), "samples_in_timed_region": len(inside),
-                "power_w_note": "50 ms nvidia-smi sampling"}
+        self.stop_flag = True
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
-def oracle_sample(recipe, layers, seq=0):
-    """Time the oracle's step for one sequence over `layers` (cache build and
-    input generation excluded). Returns (seconds, query-layers processed)."""
+def oracle_sample(recipe, layers, seq=0, queries=None):
+    """Time the oracle's step for one sequence over `layers` and the listed
+    queries of that sequence (all of them by default); cache build and input
+    generation are excluded. Returns (seconds, query-layers processed)."""
     import numpy as np
     import torch
     import oracle
     import oracle.stack as ostack
     sched = ostack.schedule(recipe.modes)
     cache = ostack.SeqCache(recipe, seq)
-    qis = [seq * recipe.q_per_seq + j for j in range(recipe.q_per_seq)]
+    js = list(range(recipe.q_per_seq)) if queries is None else list(queries)
+    qis = [seq * recipe.q_per_seq + j for j in js]
     inputs = {}
     for l in layers:
         inputs[l] = (recipe.qidx(l).numpy(), recipe.weights(l).numpy(), recipe.q(l, rows=qis),
@@ -421,13 +472,10 @@ def oracle_sample(recipe, layers, seq=0):
     return time.perf_counter() - t0, len(qis) * len(layers)
 
 
-def reference_layers(recipe):
-    """Layers of the bounded oracle sample: from layer 0 up to the first
-    Reindex layer (so every mode is exercised), capped at 6."""
-    modes = recipe.modes
-    end = modes.find("R")
-    end = len(modes) if end < 0 else end + 1
-    return list(range(min(end, 6)))
+# Bounded oracle samples of each workload (a few seconds of single-threaded
+# CPU work each): (sequence, queries of it or None for all), layers = all.
+CPU_SAMPLE = {"tiny_full": (0, None), "stack20": (0, None), "hier1m": (0, None), "paged64": (0, None),
+              "chunk512": (0, [0, 511])}
 
 
 def cpu_model():
@@ -442,23 +490,43 @@ def cpu_model():
 
 
 def _oracle_worker(job):
-    recipe, seq, layers = job
-    return oracle_sample(recipe, layers, seq)
+    recipe, seq, queries, layers = job
+    return oracle_sample(recipe, layers, seq, queries)
 
 
-def oracle_all_cores(recipe, layers):
-    """The oracle on independent sequences at once, one process each (spawned,
-    no GPU), up to one per core: units of all processes over the longest
-    process's compute time."""
+def oracle_all_cores(recipe, layers, procs):
+    """The oracle on independent units at once, one spawned process each (no
+    GPU): sequences 0..procs-1, or queries of sequence 0 for a one-sequence
+    workload. Units of all processes over the longest process's time."""
     import multiprocessing as mp
-    procs = max(1, min(os.cpu_count() or 1, recipe.batch))
+    if recipe.batch >= procs:
+        jobs = [(recipe, s, [0] if recipe.q_per_seq > 1 else None, layers) for s in range(procs)]
+        what = f"sequences 0..{procs - 1}"
+    else:
+        jobs = [(recipe, 0, [j], layers) for j in range(procs)]
+        what = f"queries 0..{procs - 1} of sequence 0"
     with mp.get_context("spawn").Pool(procs) as pool:
-        res = pool.map(_oracle_worker, [(recipe, s, layers) for s in range(procs)])
+        res = pool.map(_oracle_worker, jobs)
     dt = max(r[0] for r in res)
     n = sum(r[1] for r in res)
     return {"value": n / dt, "unit": UNIT, "cores": procs,
-            "sample": f"sequences 0..{procs - 1}, layers {layers[0]}..{layers[-1]}, one process per sequence "
-                      f"({dt:.1f} s)"}
+            "sample": f"{what}, layers {layers[0]}..{layers[-1]}, one process each ({dt:.1f} s)"}
+
+
+def cpu_baseline(recipe):
+    layers = list(range(recipe.layers))
+    seq, queries = CPU_SAMPLE.get(recipe.name, (0, None))
+    dt, n = oracle_sample(recipe, layers, seq, queries)
+    nq = recipe.q_per_seq if queries is None else len(queries)
+    rec = {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"sequence {seq} ({nq} quer{'y' if nq == 1 else 'ies'}), layers {layers[0]}..{layers[-1]} of "
+                     f"{recipe.name}, single-threaded C oracle ({dt:.1f} s)",
+           "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    units = recipe.batch if recipe.batch > 1 else recipe.q_per_seq
+    procs = max(1, min(os.cpu_count() or 1, 8, units))
+    if procs > 1:
+        rec["all_cores"] = oracle_all_cores(recipe, layers, procs)
+    return rec
 
 
 def run_reference(args):
@@ -466,19 +534,21 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    recipe = RECIPES[args.workload]
-    layers = reference_layers(recipe)
+    name = args.headline if args.workload == "all" else args.workload
+    recipe = RECIPES[name]
+    layers = list(range(recipe.layers))
+    seq, queries = CPU_SAMPLE.get(recipe.name, (0, None))
     times = []
     n_units = 0
     for i in range(args.warmup + args.steps):
-        dt, n_units = oracle_sample(recipe, layers)
+        dt, n_units = oracle_sample(recipe, layers, seq, queries)
         if i >= args.warmup:
             times.append(dt)
     total = sum(times)
     value = n_units * len(times) / total
-    sample = (f"sequence 0 of {recipe.name}, layers {layers[0]}..{layers[-1]} "
-              f"({''.join(recipe.modes[l] for l in layers)}), {recipe.q_per_seq} quer"
-              f"{'y' if recipe.q_per_seq == 1 else 'ies'}, single-threaded C oracle")
+    nq = recipe.q_per_seq if queries is None else len(queries)
+    sample = (f"sequence {seq} of {recipe.name} ({nq} quer{'y' if nq == 1 else 'ies'}), layers "
+              f"{layers[0]}..{layers[-1]} ({recipe.modes}), single-threaded C oracle, per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -491,16 +561,205 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
-def run_ours(args):
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (the library's kernels: the step
+    graph holds nothing else), or None if the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        h = g.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(h, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(h, n)
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
+
+
+def issue_call(dec, kind, l, s):
+    """One C-ABI call of the step on stream s."""
+    from sparse_fp4_kv_b200 import binding as B
+    r = dec.r
+    if kind == "append":
+        dec.append(s)
+    elif kind == "full":
+        B.csa2_index_full(dec.qidx[l], dec.w[l], r.q_per_seq, dec.q_limit, dec.n_max, dec.kv, r.k,
+                          r.p if dec.pool[l] is not None else 0, dec.topk[l], dec.pool[l], dec.ws_full, s)
+    elif kind == "reindex":
+        src = dec.schedule[l][1]
+        B.csa2_index_reindex(dec.qidx[l], dec.w[l], r.q_per_seq, dec.pool[src], dec.kv, r.k, dec.topk[l],
+                             dec.ws_reindex, s)
+    else:
+        B.csa2_sparse_attn_decode(dec.q[l], r.q_per_seq, dec.kv, dec.topk_of(l), dec.swa[l], dec.swa[l].shape[1],
+                                  dec.swa_begin, dec.swa_end, r.w, dec.scale, dec.o[l], dec.lse[l], dec.ws_attn, s)
+
+
+def graph_times_us(g, stream, flush, n):
+    """n replays of graph g, each after an L2 flush, CUDA events on the stream."""
+    import torch
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    out = []
+    for i in range(n):
+        with torch.cuda.stream(stream):
+            flush.fill_(i & 0xFF)
+            st[i].record(stream)
+            g.replay()
+            en[i].record(stream)
+        en[i].synchronize()
+        out.append(st[i].elapsed_time(en[i]) * 1e3)
+    return out
+
+
+def bench_workload(name, args, world, rank, dev, stream, flush, clocks, pk):
+    """One workload: the timed step (value, ms_per_step), the per-call
+    breakdown, the roofline of its dominant call, e2e and the CPU oracle."""
     import torch
     import torch.distributed as dist
     from cuda.bindings import driver as cu
+    from sparse_fp4_kv_b200 import binding as B
+    from sparse_fp4_kv_b200.ranks import job_throughput, max_over_ranks, rank_recipe
+    from sparse_fp4_kv_b200.stack import Csa2Decoder
+    from sparse_fp4_kv_b200.workloads import RECIPES
+
+    recipe = rank_recipe(RECIPES[name], rank, world)
+    dec = Csa2Decoder(recipe, dev)
+    costs = call_costs(recipe, dec.lens, dec.schedule)
+    by = sum(c[2] for c in costs)
+    fl = sum(c[3] for c in costs)
+    calls = [(c[0], c[1]) for c in costs]
+
+    # eager warm-up (first calls set kernel attributes), then the step graph
+    with torch.cuda.stream(stream):
+        dec.step(stream)
+    stream.synchronize()
+    if B.csa2_device_status(stream) != 0:
+        raise RuntimeError(f"{name}: device error during warm-up")
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(graph, stream=stream):
+        dec.step(stream)
+    graph.instantiate()
+    stream.synchronize()
+    launches = graph_kernel_nodes(graph)
+
+    for _ in range(args.warmup):
+        graph_times_us(graph, stream, flush, 1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark(0)
+    per_step = graph_times_us(graph, stream, flush, args.steps)
+    torch.cuda.synchronize(dev)
+    clocks.mark(1)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.summary()
+    if B.csa2_device_status(stream) != 0:
+        raise RuntimeError(f"{name}: device error during the timed steps")
+    total_ms = max_over_ranks(sum(per_step) * 1e-3, dev)
+    value, ms = job_throughput(recipe.nq * recipe.layers, world, total_ms, args.steps)
+
+    # per-call breakdown: external events around every call of a second graph
+    def new_event():
+        err, ev = cu.cuEventCreate(cu.CUevent_flags.CU_EVENT_DEFAULT)
+        assert err == cu.CUresult.CUDA_SUCCESS
+        return ev
+    ev_pairs = [(new_event(), new_event()) for _ in calls]
+    ext = cu.CUevent_record_flags.CU_EVENT_RECORD_EXTERNAL
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
+        h = cu.CUstream(stream.cuda_stream)
+        for (kind, l), (e0, e1) in zip(calls, ev_pairs):
+            cu.cuEventRecordWithFlags(e0, h, ext)
+            issue_call(dec, kind, l, stream)
+            cu.cuEventRecordWithFlags(e1, h, ext)
+    stream.synchronize()
+    per_call = {}
+    for _ in range(max(3, min(args.steps, 20))):
+        graph_times_us(graph_ev, stream, flush, 1)
+        for (kind, l), (a, b) in zip(calls, ev_pairs):
+            err, t = cu.cuEventElapsedTime(a, b)
+            per_call.setdefault(kind, []).append(t * 1e3)
+    n_rep = max(3, min(args.steps, 20))
+    calls_per_step = {k: sum(1 for c in calls if c[0] == k) for k in per_call}
+    breakdown = {k: statistics.mean(v) for k, v in per_call.items()}
+    share = {k: breakdown[k] * calls_per_step[k] for k in breakdown}
+    for e0, e1 in ev_pairs:
+        cu.cuEventDestroy(e0)
+        cu.cuEventDestroy(e1)
+    del graph_ev
+
+    # roofline of the dominant call: that call alone in a graph, L2 flushed
+    # before each replay, CUDA events around it
+    peaks_tf = {"f16": pk["bf16_tflops"], "fp8": pk["fp8_tflops"]}
+    dom = max(share, key=share.get)
+    dom_call = next(c for c in costs if c[0] == dom)
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        issue_call(dec, dom, dom_call[1], stream)
+    stream.synchronize()
+    t1 = graph_times_us(g1, stream, flush, max(args.steps, 10))
+    del g1
+    launch_us = statistics.median(t1)
+    _, bound = call_roof_us(dom_call[2], dom_call[3], dom_call[4], pk["hbm_gbs"], peaks_tf)
+    kernel_of = {"attention": f"k_attn_decode<{recipe.h}>", "full": "k_index_full", "reindex": "k_reindex",
+                 "append": "k_append_fp4"}
+    if bound == "hbm":
+        achieved, peak, unit = dom_call[2] / (launch_us * 1e-6) / 1e9, pk["hbm_gbs"], "GB/s"
+        peak_src = f"{pk['source']} HBM copy bandwidth (burst)"
+    else:
+        tc = dom_call[4]
+        achieved, peak, unit = dom_call[3] / (launch_us * 1e-6) / 1e12, peaks_tf[tc], "TFLOP/s"
+        peak_src = (f"{pk['source']} bf16 dense (burst; f16 runs at the bf16 rate)" if tc == "f16"
+                    else "fp8 e4m3 dense measured by this bench's own tcgen05 kind::f8f6f4 loop")
+    roofline = {"bound": bound, "kernel": kernel_of[dom], "call": dom, "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak, "peak_source": peak_src, "launch_us": launch_us,
+                "launch_note": "median CUDA-event time of the call alone (its kernels) replayed from a graph, "
+                               "L2 flushed before each replay",
+                "bytes_per_launch": dom_call[2], "flops_per_launch": dom_call[3],
+                "traffic": recorded_traffic(kernel_of[dom], name)}
+
+    # the whole step against its roofline (sum over calls of their bound)
+    t_roof = sum(call_roof_us(c[2], c[3], c[4], pk["hbm_gbs"], peaks_tf)[0] for c in costs)
+    step_rl = {"t_roof_us": t_roof, "step_us": ms * 1e3, "frac": t_roof / (ms * 1e3),
+               "peaks": f"{pk['source']}: {pk['hbm_gbs']} GB/s HBM, {pk['bf16_tflops']} TF/s bf16 burst, "
+                        f"{pk['fp8_tflops']:.0f} TF/s fp8 (own tcgen05 loop)"}
+
+    rec = {"value": value, "unit": UNIT, "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup,
+           "config": {"workload": name, "batch": recipe.batch, "queries_per_seq": recipe.q_per_seq,
+                      "layers": recipe.layers, "modes": recipe.modes, "entries_max": int(dec.n_max),
+                      "entries_total": int(dec.lens.sum()), "topk": recipe.k, "pool": recipe.p, "heads": recipe.h,
+                      "window": recipe.w, "indexer": f"{recipe.hi}x{recipe.di}",
+                      "l2": "256 MiB flush before every timed step", "graph": "one CUDA graph per step"},
+           "hbm_tbs": by / (ms * 1e-3) / 1e12, "algorithmic_bytes_per_step": by, "algorithmic_flops_per_step": fl,
+           "roofline": roofline, "step_roofline": step_rl,
+           "breakdown_us_per_call": breakdown, "calls_per_step": calls_per_step,
+           "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented "
+                             f"replay of the same step ({n_rep} replays; event nodes between calls prevent "
+                             "launch overlap)",
+           "gpu_launches": (launches * args.steps) if launches is not None else None,
+           "gpu_launches_per_step": launches, "clocks": clk}
+    if not args.no_e2e:
+        rec["e2e"] = run_e2e(args, dec, stream, flush, world=world, dev=dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_baseline(recipe)
+    extra = {}
+    if name == "stack20" and world == 1 and not args.no_side:
+        extra["attention_nvfp4"] = time_attn_variants(B, dec)
+    del graph
+    del dec
+    torch.cuda.empty_cache()
+    return rec, extra
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
 
     from sparse_fp4_kv_b200 import build
     build.build()
-    from sparse_fp4_kv_b200 import binding as B
-    from sparse_fp4_kv_b200.stack import Csa2Decoder
-    from sparse_fp4_kv_b200.workloads import RECIPES
+    from sparse_fp4_kv_b200 import binding as B  # noqa: F401  (fails loudly without the library)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -511,191 +770,54 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-
-    from sparse_fp4_kv_b200.ranks import job_throughput, max_over_ranks, rank_recipe
-    base = RECIPES[args.workload]
-    recipe = rank_recipe(base, rank, world)
-    dec = Csa2Decoder(recipe, dev)
-    by, fl, attn_by, attn_fl = algorithmic(recipe, dec.lens, dec.schedule)
-
     stream = torch.cuda.Stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    # external timing events around every attention launch inside the graph
-    def new_event():
-        err, ev = cu.cuEventCreate(cu.CUevent_flags.CU_EVENT_DEFAULT)
-        assert err == cu.CUresult.CUDA_SUCCESS
-        return ev
-
-    # external timing events around every C-ABI call inside the graph: the
-    # attention call of every layer (the roofline kernel) and the others
-    # for the per-call breakdown
-    calls = [("append", None)]
-    for l, (mode, _) in enumerate(dec.schedule):
-        if mode in ("full", "reindex"):
-            calls.append((mode, l))
-        calls.append(("attention", l))
-    ev_pairs = [(new_event(), new_event()) for _ in calls]
-    ext = cu.CUevent_record_flags.CU_EVENT_RECORD_EXTERNAL
-
-    def step_with_events(s):
-        h = cu.CUstream(s.cuda_stream)
-        r = dec.r
-        for (kind, l), (e0, e1) in zip(calls, ev_pairs):
-            cu.cuEventRecordWithFlags(e0, h, ext)
-            if kind == "append":
-                dec.append(s)
-            elif kind == "full":
-                B.csa2_index_full(dec.qidx[l], dec.w[l], r.q_per_seq, dec.q_limit, dec.n_max, dec.kv, r.k,
-                                  r.p if dec.pool[l] is not None else 0, dec.topk[l], dec.pool[l], dec.ws_full, s)
-            elif kind == "reindex":
-                src = dec.schedule[l][1]
-                B.csa2_index_reindex(dec.qidx[l], dec.w[l], r.q_per_seq, dec.pool[src], dec.kv, r.k, dec.topk[l],
-                                     dec.ws_reindex, s)
-            else:
-                B.csa2_sparse_attn_decode(dec.q[l], r.q_per_seq, dec.kv, dec.topk_of(l), dec.swa[l],
-                                          dec.swa[l].shape[1], dec.swa_begin, dec.swa_end, r.w, dec.scale, dec.o[l],
-                                          dec.lse[l], dec.ws_attn, s)
-            cu.cuEventRecordWithFlags(e1, h, ext)
-
-    # eager warm-up (first calls set kernel attributes), then capture two
-    # graphs of the step: the plain one that is timed, and one with external
-    # timing events around every call (event nodes sit between the kernels
-    # and stop programmatic launch overlap, so it only feeds the per-call
-    # breakdown and the roofline kernel's duration)
-    with torch.cuda.stream(stream):
-        step_with_events(stream)
-    stream.synchronize()
-    if B.csa2_device_status(stream) != 0:
-        raise RuntimeError("device error during warm-up")
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        dec.step(stream)
-    stream.synchronize()
-    graph_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ev, stream=stream):
-        step_with_events(stream)
-    stream.synchronize()
-
-    def timed_steps(g, n, record):
-        st = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        en = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        per_step, attn = [], {}
-        for i in range(n):
-            with torch.cuda.stream(stream):
-                flush.fill_(i & 0xFF)
-                st[i].record(stream)
-                g.replay()
-                en[i].record(stream)
-            en[i].synchronize()
-            per_step.append(st[i].elapsed_time(en[i]))
-            if record:
-                for (kind, _), (a, b) in zip(calls, ev_pairs):
-                    err, ms = cu.cuEventElapsedTime(a, b)
-                    attn.setdefault(kind, []).append(ms)
-        return per_step, attn
-
-    launches_per_step = count_launches(dec, recipe)
-    for _ in range(args.warmup):
-        timed_steps(graph, 1, False)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    clocks = Clocks(local)
+    pk = peaks()
+    probe = measure_tc_probe(dev)
+    pk["fp8_tflops"] = probe.get("fp8_e4m3_n256_tflops", 2.0 * pk["bf16_tflops"])
+    names = list(WORKLOADS) if args.workload == "all" else [args.workload]
+    headline = args.headline if args.headline in names else names[0]
+    clocks = Clocks(dev)
     clocks.start()
-    time.sleep(0.2)  # the sampler is running
-    clocks.mark(0)
-    per_step, _ = timed_steps(graph, args.steps, False)
-    torch.cuda.synchronize(dev)
-    clocks.mark(1)
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    # instrumented replays right after the timed loop: per-call durations
-    _, attn = timed_steps(graph_ev, args.steps, True)
-    if B.csa2_device_status(stream) != 0:
-        raise RuntimeError("device error during the timed steps")
-    total_ms = max_over_ranks(sum(per_step), dev)
-    value, ms = job_throughput(recipe.nq * recipe.layers, world, total_ms, args.steps)
+    time.sleep(0.05)
+    records, extra = {}, {}
+    for name in names:
+        rec, ex = bench_workload(name, args, world, rank, dev, stream, flush, clocks, pk)
+        records[name] = rec
+        extra.update(ex)
+    clocks.stop()
 
-    # e2e: host buffers in pinned memory, copies inside the timed region
-    e2e = None
-    if not args.no_e2e:
-        e2e = run_e2e(args, dec, stream, flush, world=world, dev=dev)
-
-    hbm_gbs, bf16_burst, bf16_sust, peak_kind = peaks()
-    t_roof, t_parts = step_roofline_us(recipe, dec.lens, dec.schedule, hbm_gbs, bf16_sust)
-    step_rl = {"t_roof_us": t_roof, "parts_us": t_parts, "step_us": ms * 1e3, "frac": t_roof / (ms * 1e3),
-               "peaks": f"{peak_kind}: {hbm_gbs} GB/s HBM, {bf16_sust} TF/s bf16 sustained (FP8 at 2x)"}
     side = world == 1 and not args.no_side
-    append_c4 = time_append_chunk512(B, dev, hbm_gbs) if side else None
-    append_f8 = time_append_e4m3(B, dev, hbm_gbs) if side else None
-    sharded = time_sharded_hier1m(dev) if side and not args.no_sharded else None
-    attn_nv = time_attn_variants(B, dec) if side and recipe.h == 64 else None
-    breakdown = {k: 1e3 * statistics.mean(v) for k, v in attn.items()}
-    attn_ms = statistics.mean(attn["attention"]) if attn else float("nan")
-    achieved_tf = attn_fl / (attn_ms * 1e-3) / 1e12
-    kernel = f"k_sparse_attn<{recipe.h}>"
+    hbm = pk["hbm_gbs"]
+    if side:
+        extra["append_chunk512"] = time_append_chunk512(B, dev, hbm)
+        extra["append_e4m3"] = time_append_e4m3(B, dev, hbm)
+        if not args.no_sharded:
+            extra["sharded_hier1m"] = time_sharded_hier1m(dev)
+    h = records[headline]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": h["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16+e4m3 tensor-core, f32 accumulate", "data": "synthetic",
-        "config": {"workload": recipe.name, "batch": recipe.batch, "queries_per_seq": recipe.q_per_seq,
-                   "layers": recipe.layers, "modes": recipe.modes, "entries": int(dec.n_max),
-                   "topk": recipe.k, "pool": recipe.p, "heads": recipe.h, "window": recipe.w,
-                   "indexer": f"{recipe.hi}x{recipe.di}", "l2": "256 MiB flush before every timed step",
-                   "graph": "one CUDA graph per step", "parallelism": f"dp{world} (independent sequences)"},
-        "hbm_tbs": by / (ms * 1e-3) / 1e12,
-        "algorithmic_bytes_per_step": by, "algorithmic_flops_per_step": fl,
-        "roofline": {"bound": "tensor", "kernel": kernel, "achieved": achieved_tf, "peak": bf16_sust,
-                     "unit": "TFLOP/s", "frac": achieved_tf / bf16_sust,
-                     "peak_source": f"{peak_kind} bf16 dense sustained (f16 runs at the bf16 rate)",
-                     "launch_us": attn_ms * 1e3, "launch_note": "event-timed attention call (attention kernel + "
-                     "split combine) in the instrumented replay", "flops_per_launch": attn_fl, "bytes_per_launch": attn_by,
-                     "hbm_frac": attn_by / (attn_ms * 1e-3) / (hbm_gbs * 1e9),
-                     "traffic": recorded_traffic(kernel, recipe.name)},
-        "step_roofline": step_rl,
-        "append_chunk512": append_c4,
-        "append_e4m3": append_f8,
-        "sharded_hier1m": sharded,
-        "attention_nvfp4": attn_nv,
-        "breakdown_us_per_call": breakdown,
-        "breakdown_note": "CUDA-event durations of each C-ABI call in a separately captured, instrumented replay "
-                          "of the same step (event nodes between calls prevent launch overlap)",
-        "breakdown_calls_per_step": {k: len(v) // args.steps for k, v in attn.items()},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
+        "config": dict(h["config"], parallelism=f"dp{world} (independent sequences)"),
+        "hbm_tbs": h["hbm_tbs"], "roofline": h["roofline"], "step_roofline": h["step_roofline"],
+        "gpu_launches": h["gpu_launches"], "clocks": h["clocks"],
+        "breakdown_us_per_call": h["breakdown_us_per_call"],
     }
-    if e2e is not None:
-        line["e2e"] = e2e
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        layers = list(range(recipe.layers))
-        dt, n = oracle_sample(recipe, layers)
-        line["cpu_baseline"] = {
-            "value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"sequence 0, layers {layers[0]}..{layers[-1]} of {recipe.name}, single-threaded C oracle "
-                      f"({dt:.1f} s)", "cpu_model": cpu_model(), "nproc": os.cpu_count(),
-            "all_cores": oracle_all_cores(recipe, layers)}
+    if "e2e" in h:
+        line["e2e"] = h["e2e"]
+    if "cpu_baseline" in h:
+        line["cpu_baseline"] = h["cpu_baseline"]
+    line["peaks"] = {"hbm_gbs": hbm, "bf16_tflops": pk["bf16_tflops"], "source": pk["source"],
+                     "fp8_tflops": pk["fp8_tflops"], "tc_probe": probe}
+    line["configs"] = records
+    line.update(extra)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_ev
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-
-
-def count_launches(dec, recipe):
-    """Kernels of this library launched by one step (the memset of the Full
-    layer's histograms is a runtime call, not counted)."""
-    from sparse_fp4_kv_b200 import binding as B
-    n = 1  # append
-    for mode, _ in dec.schedule:
-        if mode == "full":
-            n += 5
-        elif mode == "reindex":
-            n += 2
-        n += 1 + (1 if B.csa2_sparse_attn_workspace_size(recipe.nq, recipe.h, recipe.k, recipe.w) > 0 else 0)
-    return n
 
 
 def run_e2e(args, dec, stream, flush, world, dev):

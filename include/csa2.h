@@ -32,10 +32,10 @@
  *     slot in every id list.
  *   - Reuse mode is not a call: a Reuse layer passes its source layer's
  *     Top-k list to csa2_sparse_attn_decode.
- *   - One device per process: the library sets its kernels' shared-memory
- *     limits once, on the device current at a kernel's first call; calls on
- *     another device of the same process may then fail with CSA2_ERR_CUDA.
- *     (The fixed scratch of csa2_sparse_attn_decode_static is per device.)
+ *   - Devices: a call runs on the device current on the calling thread.
+ *     Kernel attributes (shared-memory limits) are set up once per device,
+ *     at the first call on that device that needs the kernel, so one process
+ *     may use several devices.
  */
 #ifndef CSA2_H
 #define CSA2_H
@@ -197,9 +197,13 @@ size_t csa2_index_reindex_workspace_size(int32_t nq, int32_t p);
  *   o_h = sum_j softmax_j(softmax_scale * <q_h, v_j>) v_j
  * written as bf16 o [nq][h][d]; lse [nq][h] (nullable) gets the natural-log
  * sum of exp of the scaled scores. An empty S gives o = 0, lse = -inf.
- * Arithmetic: q converted to f16 (|q| must be finite in f16), f16 tensor-core
+ * Arithmetic: q converted to f16 (round to nearest), f16 tensor-core
  * products with f32 accumulation, f32 online softmax, probabilities rounded
- * to f16 for the P*V product. h in {16, 32, 64}.
+ * to f16 for the P*V product. h in {16, 32, 64}. Range of q: a bf16 value of
+ * magnitude 65536 or more (or an infinity or NaN) has no finite f16 value;
+ * the kernel records CSA2_DEVERR_Q_RANGE and that query's o and lse are
+ * undefined (other queries are unaffected). Magnitudes below 2^-14 become
+ * f16 subnormals: absolute error at most 2^-25 per element.
  * ws: at least csa2_sparse_attn_workspace_size(nq, h, k, w) bytes, with
  * w = w_max when a window is given and w = 0 when swa_begin is NULL (the
  * split plan follows the rows the call really has; the size is not monotone
@@ -229,8 +233,12 @@ size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t
  * csa2_sparse_attn_decode with a caller-owned workspace instead.
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress with that device current); make that first call
- * before any stream capture begins. No part of the array has to start at
- * zero: each call writes every partial it reads back.
+ * before any stream capture begins. The address belongs to the device's
+ * context: when that context is replaced (cudaDeviceReset, or a context
+ * destroyed and created again), the next call looks it up again, so make
+ * the first call after such a change outside stream capture as well. No part
+ * of the array has to start at zero: each call writes every partial it reads
+ * back.
  * Concurrency: all calls on one device share the one array, so two calls
  * whose kernels can overlap (different streams, or different host threads,
  * without ordering between them) race on it and give wrong results. Order
@@ -333,7 +341,20 @@ csa2_status csa2_attn_merge(const float *o_parts, const float *lse_parts, int32_
 #define CSA2_DEVERR_BAD_ROW 1u       /* id / page / position outside the cache */
 #define CSA2_DEVERR_WAIT_TIMEOUT 2u  /* a bounded barrier wait gave up         */
 #define CSA2_DEVERR_SELECT 4u        /* selection produced more ids than asked  */
+#define CSA2_DEVERR_Q_RANGE 8u       /* attention q outside f16's finite range  */
 csa2_status csa2_device_status(cudaStream_t stream, uint32_t *code);
+
+/*
+ * Self-check of the device-side failure detection (no counterpart in the
+ * pages). Every barrier wait in the library's kernels is bounded (one second
+ * of device time); a wait that runs out records CSA2_DEVERR_WAIT_TIMEOUT,
+ * skips the rest of its work and lets the kernel end, so the context stays
+ * usable. This call launches one thread that waits, with a limit of
+ * limit_us microseconds (1 ... 1000000, else CSA2_ERR_INVALID_ARG), on a
+ * barrier that nothing arrives at; afterwards csa2_device_status() reports
+ * CSA2_DEVERR_WAIT_TIMEOUT. Nothing else is touched.
+ */
+csa2_status csa2_check_wait_timeout(uint32_t limit_us, cudaStream_t stream);
 
 const char *csa2_status_string(csa2_status status);
 

@@ -73,6 +73,7 @@ _SIGS = {
                                         _f32, _vp, _vp, _vp, _sz, _vp]),
     "csa2_attn_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "csa2_device_status": (_i32, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "csa2_check_wait_timeout": (_i32, [ctypes.c_uint32, _vp]),
     "csa2_status_string": (ctypes.c_char_p, [_i32]),
     "csa2_version": (_i32, []),
 }
@@ -256,6 +257,11 @@ def csa2_device_status(stream=None):
     if st not in (0, 5):
         raise Csa2Error("csa2_device_status", st)
     return code.value
+
+
+def csa2_check_wait_timeout(limit_us, stream=None):
+    """Launch the bounded-wait self-check (a wait that runs out after limit_us)."""
+    _check("csa2_check_wait_timeout", _lib.csa2_check_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def csa2_status_string(status):

@@ -55,37 +55,59 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&f)[16], uint3
     return s;
 }
 
+// A warp walks rows r, r + W, r + 2W, ... (W = warps in the grid). The
+// loads of its next row (input values and destination lookup) are issued
+// before the current row is quantised and stored, so every warp keeps two
+// rows in flight; the grid fills every SM.
+__device__ __forceinline__ int64_t append_dest(const csa2_kv_desc &kv, const int32_t *__restrict__ seq,
+                                               const int64_t *__restrict__ pos, int64_t r) {
+    const int32_t b = seq[r];
+    return (b >= 0 && b < kv.batch) ? physical_row(kv, b, pos[r]) : -1;
+}
+
 __global__ void __launch_bounds__(kAppendWarps * 32)
     k_append_fp4(const uint16_t *__restrict__ x, int32_t n, const int32_t *__restrict__ seq,
                  const int64_t *__restrict__ pos, csa2_kv_desc kv) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+    const int64_t stride = (int64_t)gridDim.x * kAppendWarps;
+    int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
     if (r >= n) return;
-    // the row's values are loaded first, in flight while its destination is
-    // looked up (sequence, position, page table)
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16);
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    const int32_t b = seq[r];
-    int64_t row = -1;
-    if (b >= 0 && b < kv.batch) row = physical_row(kv, b, pos[r]);
-    if (row < 0) {
-        if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
-        return;
-    }
-    const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float f[16];
+    uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16));
+    uint4 v1 = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16) + 1);
+    int64_t row = append_dest(kv, seq, pos, r);
+    for (; r < n; r += stride) {
+        // the next row's values and destination go in flight first
+        const int64_t rn = r + stride;
+        uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+        int64_t row_n = -1;
+        if (rn < n) {
+            n0 = __ldg(reinterpret_cast<const uint4 *>(x + rn * CSA2_D + lane * 16));
+            n1 = __ldg(reinterpret_cast<const uint4 *>(x + rn * CSA2_D + lane * 16) + 1);
+            row_n = append_dest(kv, seq, pos, rn);
+        }
+        if (row < 0) {
+            if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
+        } else {
+            const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float f[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        f[2 * i] = __uint_as_float(wds[i] << 16);
-        f[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+            for (int i = 0; i < 8; ++i) {
+                f[2 * i] = __uint_as_float(wds[i] << 16);
+                f[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
+            }
+            uint32_t packed[2];
+            const uint32_t s = quantize_block16(f, packed);
+            // codes: 8 bytes per lane (256 contiguous bytes per warp); scales: one
+            // byte per lane (the row's 32-byte sector in one warp store)
+            *reinterpret_cast<uint2 *>(kv.codes + row * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
+            kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
+        }
+        v0 = n0;
+        v1 = n1;
+        row = row_n;
     }
-    uint32_t packed[2];
-    const uint32_t s = quantize_block16(f, packed);
-    uint2 *dst = reinterpret_cast<uint2 *>(kv.codes + row * (CSA2_D / 2) + lane * 8);
-    *dst = make_uint2(packed[0], packed[1]);
-    kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
 }
 
 // ---------------------------------------------------------------------------

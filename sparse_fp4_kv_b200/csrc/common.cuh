@@ -84,26 +84,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Gives up after
-// about one second of global-timer time (a few hundred fast polls first,
-// then polls spaced by short sleeps), records the timeout in the device
-// error word and returns false so the caller can unwind.
+// limit_ns of global-timer time (a few hundred fast polls first, then polls
+// spaced by short sleeps) or, should the timer not advance, after 2^26
+// sleeping polls; records the timeout in the device error word and returns
+// false so the caller can unwind. Every wait of the library's kernels uses a
+// one-second limit.
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kWaitMaxPolls = 1u << 26;
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    while (global_ns() - t0 < kWaitNs) {
+#pragma unroll 1
+    for (uint32_t n = 0; n < kWaitMaxPolls && global_ns() - t0 < limit_ns; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         __nanosleep(64);
     }
     set_error(CSA2_DEVERR_WAIT_TIMEOUT);
     return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) { return mbar_wait_for(bar, parity, kWaitNs); }
+
+// Self-check of the bounded wait: one thread initialises an mbarrier that
+// nothing ever arrives at and waits for its first phase with the given limit.
+// The wait runs out, the device error word gets CSA2_DEVERR_WAIT_TIMEOUT and
+// the kernel returns normally.
+__global__ void k_wait_selfcheck(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_for(&bar, 0, limit_ns);
 }
 
 // ---------------------------------------------------------------------------
@@ -156,6 +173,26 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *t
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
 }
+
+// cp.async (16 bytes, L2 only) into shared memory, its commit and wait.
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Bulk asynchronous copy shared -> global (no tensor map), tracked by the
+// issuing thread's bulk async-group: size a multiple of 16, both addresses
+// 16-byte aligned. wait_read: the shared-memory source may be reused;
+// wait_all: the writes are complete.
+__device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst), "r"(smem_u32(smem_src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Programmatic dependent launch: let the next kernel on the stream start
 // launching, and wait until the previous kernel has completed and its memory

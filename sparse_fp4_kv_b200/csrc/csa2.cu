@@ -12,13 +12,18 @@
 #include <cstdlib>
 #include <cstring>
 #include <cstdint>
+#include <array>
+#include <map>
 #include <mutex>
+#include <set>
 #include <utility>
 
 #include "append.cuh"
 #include "attention.cuh"
+#include "attn_decode.cuh"
 #include "indexer.cuh"
 #include "indexer_fused.cuh"
+#include "indexer_batch.cuh"
 
 using namespace csa2;
 
@@ -36,16 +41,23 @@ int max_smem_optin() {
     return n;
 }
 
-// CSA2_FULL_PATH=multipass forces the multi-launch Full indexer even where the
-// single-launch cluster path applies (both are complete implementations; the
-// switch lets tests exercise both at small sizes).
-bool force_multipass() {
-    static const bool v = [] {
+// CSA2_FULL_PATH picks the Full indexer path where several apply: "multipass"
+// (the multi-launch path), "fused" (never the batched path) or "batch" (the
+// batched path whenever it applies); all are complete implementations and the
+// switch lets tests exercise each at small sizes. Unset: the automatic choice.
+enum FullPath { kPathAuto, kPathMultipass, kPathFused, kPathBatch };
+FullPath full_path_env() {
+    static const FullPath v = [] {
         const char *e = std::getenv("CSA2_FULL_PATH");
-        return e != nullptr && std::strcmp(e, "multipass") == 0;
+        if (!e) return kPathAuto;
+        if (std::strcmp(e, "multipass") == 0) return kPathMultipass;
+        if (std::strcmp(e, "fused") == 0) return kPathFused;
+        if (std::strcmp(e, "batch") == 0) return kPathBatch;
+        return kPathAuto;
     }();
     return v;
 }
+bool force_multipass() { return full_path_env() == kPathMultipass; }
 
 int num_sms() {
     int dev = 0, n = 148;
@@ -116,6 +128,8 @@ struct FullLayout {
     int64_t key_stride;
     int32_t n_sel_chunks;
     size_t off_keys, off_hist0, off_hist1, off_hist2, off_state, off_cnt, total;
+    size_t b_hist, b_state, b_sure, b_cand;  // batched path
+    int64_t b_cap;
 };
 
 FullLayout full_layout(int32_t nq, int64_t n_max) {
@@ -135,7 +149,18 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
     off = align_up(off + (size_t)nq * kStateWords * 4, 256);
     L.off_cnt = off;
     off = align_up(off + (size_t)nq * 2 * L.n_sel_chunks * 2 * 4, 256);
-    L.total = off;
+    // the batched path's region (the same bytes: one path runs per call)
+    size_t b = 0;
+    L.b_hist = b;
+    b = align_up(b + (size_t)nq * kBatchBins * 4, 256);
+    L.b_state = b;
+    b = align_up(b + (size_t)nq * 4 * 4, 256);
+    L.b_sure = b;
+    b = align_up(b + (size_t)nq * kBatchMaxK * 4, 256);
+    L.b_cand = b;
+    L.b_cap = std::max<int64_t>(n_max, 1);
+    b = align_up(b + (size_t)nq * L.b_cap * 8, 256);
+    L.total = std::max(off, b);
     return L;
 }
 
@@ -245,6 +270,32 @@ AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P, bool nvfp4 = fa
     return L;
 }
 
+// Persistent decode attention: tiles per query, tiles per CTA (each CTA
+// one SM) and the number of partial slots of the split.
+struct DecPlan {
+    int32_t tpq, per, ctas, slots;
+    size_t off_o, off_lse, off_qslot, total;
+};
+
+DecPlan plan_decode(int32_t nq, int32_t h, int32_t k, int32_t w_max, int sms) {
+    DecPlan P{};
+    const int64_t rows = (int64_t)k + std::max(0, w_max);
+    P.tpq = (int32_t)std::max<int64_t>(1, (rows + kAttnTile - 1) / kAttnTile);
+    const int64_t T = (int64_t)nq * P.tpq;
+    int64_t per = (T + sms - 1) / sms;
+    if (const char *e = std::getenv("CSA2_ATTN_PER")) per = std::max<int64_t>(1, std::atoll(e));  // tuning, tests
+    P.per = (int32_t)std::min<int64_t>(per, INT32_MAX);
+    P.ctas = (int32_t)((T + P.per - 1) / P.per);
+    const DecSplit sp{T, P.per, P.tpq};
+    P.slots = 0;
+    for (int32_t g = 0; g < P.ctas; ++g) P.slots += sp.nparts(g);
+    P.off_o = 0;
+    P.off_lse = align_up((size_t)P.slots * h * CSA2_D * 4, 256);
+    P.off_qslot = align_up(P.off_lse + (size_t)P.slots * h * 4, 256);
+    P.total = P.slots > 0 ? align_up(P.off_qslot + (size_t)nq * 4, 256) : 0;
+    return P;
+}
+
 // Dynamic shared memory limit of a kernel, and the maximal shared-memory
 // carveout, which every kernel of the library requests so that consecutive
 // launches do not change the L1 / shared split of the SMs.
@@ -308,16 +359,52 @@ cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Kernel attributes belong to a device: every (device, kernel) pair is set up
+// once, with that device current, the first time a call on that device needs
+// the kernel. `key` names the set-up (a kernel's address or another tag).
+std::mutex g_attr_mu;
+std::set<std::pair<int, const void *>> g_attr_done;
+
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return dev;
+}
+
+template <typename F>
+bool once_per_device(const void *key, F &&setup) {
+    const int dev = current_device();
+    if (dev < 0) return false;
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (g_attr_done.count({dev, key})) return true;
+    if (!setup()) return false;
+    g_attr_done.insert({dev, key});
+    return true;
+}
+
+// set_smem once per device for this kernel.
+template <typename K>
+bool smem_attr(K kernel, size_t bytes) {
+    return once_per_device(reinterpret_cast<const void *>(kernel), [&] { return set_smem(kernel, bytes); });
+}
+
 // Attributes of the single-launch Full kernel (maximal dynamic shared
-// memory; clusters above 8 CTAs need the non-portable size), set once, and
-// how many clusters of each size the device holds at once (0: not possible).
+// memory; clusters above 8 CTAs need the non-portable size), set once per
+// device, and how many clusters of each size that device holds at once
+// (0: not possible).
 template <int DI>
 const int *fused_cluster_caps() {
-    static int caps[kFusedClusterMax + 1];
-    static std::once_flag once;
-    std::call_once(once, [] {
-        for (int c = 0; c <= kFusedClusterMax; ++c) caps[c] = 0;
-        if (!set_smem(k_index_full_fused<DI>, (size_t)max_smem_optin())) return;
+    static std::mutex mu;
+    static std::map<int, std::array<int, kFusedClusterMax + 1>> per_dev;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = per_dev.find(dev);
+    if (it != per_dev.end()) return it->second.data();
+    std::array<int, kFusedClusterMax + 1> caps{};
+    if (dev >= 0 && set_smem(k_index_full_fused<DI>, (size_t)max_smem_optin())) {
         if (cudaFuncSetAttribute(k_index_full_fused<DI>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
             cudaSuccess)
             cudaGetLastError();
@@ -340,8 +427,8 @@ const int *fused_cluster_caps() {
             }
             caps[c] = n;
         }
-    });
-    return caps;
+    }
+    return per_dev.emplace(dev, caps).first->second.data();
 }
 
 // CTAs per query for the single-launch Full kernel: the largest size whose
@@ -364,15 +451,22 @@ bool prefer_shared(K kernel) {
                                 (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
-// One-time attribute set-up of the kernels without large dynamic shared memory.
+// Attribute set-up of the kernels without large dynamic shared memory, once
+// per device.
 bool init_small_kernels() {
-    static const bool ok = prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_hist<1>) &&
-                           prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
-                           prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
-                           prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
-                           prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
-                           prefer_shared(k_attn_combine<32, true>) && prefer_shared(k_attn_combine<64, true>);
-    return ok;
+    static const char key = 0;
+    return once_per_device(&key, [] {
+        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_hist<1>) &&
+               prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
+               prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
+               prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
+               prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
+               prefer_shared(k_attn_combine<32, true>) && prefer_shared(k_attn_combine<64, true>) &&
+               prefer_shared(k_attn_merge_parts<16, false>) && prefer_shared(k_attn_merge_parts<32, false>) &&
+               prefer_shared(k_attn_merge_parts<64, false>) && prefer_shared(k_attn_merge_parts<16, true>) &&
+               prefer_shared(k_attn_merge_parts<32, true>) && prefer_shared(k_attn_merge_parts<64, true>) &&
+               prefer_shared(k_wait_selfcheck);
+    });
 }
 
 }  // namespace
@@ -403,6 +497,12 @@ csa2_status csa2_device_status(cudaStream_t stream, uint32_t *code) {
     return v ? CSA2_ERR_DEVICE : CSA2_OK;
 }
 
+csa2_status csa2_check_wait_timeout(uint32_t limit_us, cudaStream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return CSA2_ERR_INVALID_ARG;
+    k_wait_selfcheck<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull);
+    return check_launch();
+}
+
 csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, const int64_t *pos,
                             const csa2_kv_desc *kv, cudaStream_t stream) {
     csa2_status st = check_kv(kv, false);
@@ -412,7 +512,10 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
     if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
         return CSA2_ERR_INVALID_ARG;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
-    const unsigned grid = (unsigned)((n + kAppendWarps - 1) / kAppendWarps);
+    // every SM holds 8 CTAs of 8 warps; each warp walks rows with a stride and
+    // keeps two in flight
+    const int64_t want = (int64_t)num_sms() * 8;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, ((int64_t)n + kAppendWarps - 1) / kAppendWarps);
     launch(k_append_fp4, dim3(grid), dim3(kAppendWarps * 32), 0, stream, static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
     return check_launch();
 }
@@ -478,6 +581,71 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     const int tile_entries = 128 * epr;
     CUtensorMap tm;
     if (!make_kidx_map(&tm, kv, box_rows)) return CSA2_ERR_CUDA;
+
+    // Batched: many queries of one sequence share each key tile in one
+    // tensor-core product (groups of 16 queries with up to 4 indexer heads, 8
+    // with up to 8), two scans of the keys and an exact select per query.
+    {
+        const int hp = hi <= 4 ? 4 : 8;
+        const int qg = batch_qg(hp);
+        const FullPath fp = full_path_env();
+        const bool applies = p == 0 && hi <= 8 && k <= kBatchMaxK && q_per_seq % qg == 0;
+        if (applies && (fp == kPathBatch || (fp == kPathAuto && q_per_seq >= 64))) {
+            CUtensorMap bm;
+            if (!make_kidx_map(&bm, kv, box_rows)) return CSA2_ERR_CUDA;
+            BatchParams bp{};
+            bp.qidx = qidx;
+            bp.w = w;
+            bp.q_limit = q_limit;
+            bp.kv = *kv;
+            bp.hist = reinterpret_cast<uint32_t *>(wsb + L.b_hist);
+            bp.state = reinterpret_cast<uint32_t *>(wsb + L.b_state);
+            bp.sure = reinterpret_cast<int32_t *>(wsb + L.b_sure);
+            bp.cand = reinterpret_cast<unsigned long long *>(wsb + L.b_cand);
+            bp.topk = topk;
+            bp.cap = L.b_cap;
+            bp.k = k;
+            bp.q_per_seq = q_per_seq;
+            bp.hi = hi;
+            bp.hi_pad = hp;
+            bp.nq = nq;
+            bp.box_rows = box_rows;
+            const int ngroups = (nq + qg - 1) / qg;
+            const int64_t tiles = std::max<int64_t>(1, (n_max + tile_entries - 1) / tile_entries);
+            const int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>(tiles, num_sms() / ngroups));
+            bp.chunk = (tiles + nchunks - 1) / nchunks * tile_entries;
+            if (bp.chunk / kv->page_size + 2 > kMaxScanPages) return CSA2_ERR_UNSUPPORTED;
+            const dim3 sgrid((unsigned)((std::max<int64_t>(n_max, 1) + bp.chunk - 1) / bp.chunk), (unsigned)ngroups);
+            if (cudaMemsetAsync(bp.hist, 0, (size_t)nq * kBatchBins * 4, stream) != cudaSuccess) return CSA2_ERR_CUDA;
+            auto scan = [&](auto k0, auto k1, size_t sm0, size_t sm1) -> csa2_status {
+                if (!smem_attr(k0, sm0) || !smem_attr(k1, sm1)) return CSA2_ERR_CUDA;
+                launch(k0, sgrid, dim3(kBatchThreads), sm0, stream, bm, bp);
+                launch(k_batch_thresh, dim3((unsigned)nq), dim3(kBatchThreshThreads), 0, stream, bp);
+                launch(k1, sgrid, dim3(kBatchThreads), sm1, stream, bm, bp);
+                return CSA2_OK;
+            };
+            csa2_status bs;
+            if (kv->di == 64 && hp == 4)
+                bs = scan(k_batch_scan<64, 4, 0>, k_batch_scan<64, 4, 1>, BatchCfg<64, 4, 0>::kSmem,
+                          BatchCfg<64, 4, 1>::kSmem);
+            else if (kv->di == 64)
+                bs = scan(k_batch_scan<64, 8, 0>, k_batch_scan<64, 8, 1>, BatchCfg<64, 8, 0>::kSmem,
+                          BatchCfg<64, 8, 1>::kSmem);
+            else if (hp == 4)
+                bs = scan(k_batch_scan<128, 4, 0>, k_batch_scan<128, 4, 1>, BatchCfg<128, 4, 0>::kSmem,
+                          BatchCfg<128, 4, 1>::kSmem);
+            else
+                bs = scan(k_batch_scan<128, 8, 0>, k_batch_scan<128, 8, 1>, BatchCfg<128, 8, 0>::kSmem,
+                          BatchCfg<128, 8, 1>::kSmem);
+            if (bs != CSA2_OK) return bs;
+            const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
+            if (!smem_attr(k_batch_final, fsm)) return CSA2_ERR_CUDA;
+            const size_t ffixed = 2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + (size_t)kBatchMaxK * 4;
+            const int32_t smem_keys = (int32_t)((fsm - ffixed) / 8);
+            launch(k_batch_final, dim3((unsigned)nq), dim3(kBatchFinalThreads), fsm, stream, bp, smem_keys);
+            return check_launch();
+        }
+    }
 
     // Single launch: one cluster per query, every score kept in shared
     // memory, when a query's entries fit. Clusters of 16 CTAs when the device
@@ -546,12 +714,10 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sp.chunk_tiles = (int32_t)chunk;
     const dim3 sgrid((unsigned)((tiles_max + chunk - 1) / chunk), (unsigned)nq);
     if (kv->di == 64) {
-        static bool ok = set_smem(k_index_scan<64>, ScanCfg<64>::kSmem);
-        if (!ok) return CSA2_ERR_CUDA;
+        if (!smem_attr(k_index_scan<64>, ScanCfg<64>::kSmem)) return CSA2_ERR_CUDA;
         launch(k_index_scan<64>, sgrid, dim3(kScanThreads), ScanCfg<64>::kSmem, stream, tm, sp);
     } else {
-        static bool ok = set_smem(k_index_scan<128>, ScanCfg<128>::kSmem);
-        if (!ok) return CSA2_ERR_CUDA;
+        if (!smem_attr(k_index_scan<128>, ScanCfg<128>::kSmem)) return CSA2_ERR_CUDA;
         launch(k_index_scan<128>, sgrid, dim3(kScanThreads), ScanCfg<128>::kSmem, stream, tm, sp);
     }
     if ((st = check_launch()) != CSA2_OK) return st;
@@ -610,6 +776,21 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     rp.k = k;
     rp.hi = hi;
     rp.q_per_seq = q_per_seq;
+    // one launch per query when its pool's keys fit shared memory (always up to
+    // the largest pool the call accepts); the two-launch path otherwise
+    {
+        const size_t fsm = kv->di == 64 ? RfCfg<64>::smem(p) : RfCfg<128>::smem(p);
+        if (fsm + 1024 <= (size_t)max_smem_optin() && !force_multipass()) {
+            if (kv->di == 64) {
+                if (!smem_attr(k_reindex_fused<64>, (size_t)max_smem_optin() - 1024)) return CSA2_ERR_CUDA;
+                launch(k_reindex_fused<64>, dim3((unsigned)nq), dim3(kRfThreads), fsm, stream, rp);
+            } else {
+                if (!smem_attr(k_reindex_fused<128>, (size_t)max_smem_optin() - 1024)) return CSA2_ERR_CUDA;
+                launch(k_reindex_fused<128>, dim3((unsigned)nq), dim3(kRfThreads), fsm, stream, rp);
+            }
+            return check_launch();
+        }
+    }
     const dim3 grid((unsigned)((p + kReindexScoreThreads - 1) / kReindexScoreThreads), (unsigned)nq);
     if (kv->di == 64)
         launch(k_reindex_score<64>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
@@ -617,8 +798,7 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
         launch(k_reindex_score<128>, grid, dim3(kReindexScoreThreads), 0, stream, rp);
     if ((st = check_launch()) != CSA2_OK) return st;
     const size_t smem = 2048 * 4 + (kReindexSelectThreads / 32 + 8) * 4 + (size_t)p * 8;
-    static bool ok = set_smem(k_reindex_select<false>, (size_t)max_smem_optin());
-    if (!ok) return CSA2_ERR_CUDA;
+    if (!smem_attr(k_reindex_select<false>, (size_t)max_smem_optin())) return CSA2_ERR_CUDA;
     launch(k_reindex_select<false>, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
     return check_launch();
 }
@@ -626,8 +806,7 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
 size_t csa2_sparse_attn_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max) {
     if (nq <= 0 || h <= 0 || k < 0) return 0;
     if (h != 16 && h != 32 && h != 64) return 0;
-    const AttnPlan P = plan_attn(nq, k, w_max, num_sms());
-    return attn_layout(nq, h, P).total;
+    return plan_decode(nq, h, k, w_max, num_sms()).total;
 }
 
 }  // extern "C"
@@ -643,6 +822,65 @@ void launch_combine(int32_t h, int32_t nq, const CombineArgs &ca, cudaStream_t s
         case 32: launch(k_attn_combine<32, F32>, cgrid, dim3(kCombineThreads), csmem, stream, ca); break;
         default: launch(k_attn_combine<16, F32>, cgrid, dim3(kCombineThreads), csmem, stream, ca); break;
     }
+}
+
+template <int H>
+void launch_decode(const DecParams &dp, const DecPlan &P, bool out_f32, cudaStream_t stream) {
+    launch(k_attn_decode<H>, dim3((unsigned)P.ctas), dim3(kDecThreads), DecCfg<H>::kSmem, stream, dp);
+    if (P.slots > 0) {
+        const dim3 mgrid((unsigned)H, (unsigned)dp.nq);
+        if (out_f32)
+            launch(k_attn_merge_parts<H, true>, mgrid, dim3(kMergeThreads), 0, stream, dp);
+        else
+            launch(k_attn_merge_parts<H, false>, mgrid, dim3(kMergeThreads), 0, stream, dp);
+    }
+}
+
+// The exact decode attention (arguments already checked by attn_impl):
+// the persistent kernel, then the merge of the queries split across CTAs.
+csa2_status decode_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h, const csa2_kv_desc *kv,
+                        const int32_t *topk, int32_t k, const uint8_t *swa, int64_t swa_seq_stride,
+                        const int32_t *swa_begin, const int32_t *swa_end, int32_t w_max, float softmax_scale, void *o,
+                        bool out_f32, float *lse, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const DecPlan P = plan_decode(nq, h, k, w_max, num_sms());
+    if (P.total > 0 && (!ws || ws_bytes < P.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
+    if (!init_small_kernels()) return CSA2_ERR_CUDA;
+    DecParams dp{};
+    dp.q = static_cast<const uint16_t *>(q_bf16);
+    dp.kv = *kv;
+    dp.topk = topk;
+    dp.swa = swa;
+    dp.swa_seq_stride = swa_seq_stride;
+    dp.swa_begin = swa_begin;
+    dp.swa_end = swa_end;
+    dp.o = out_f32 ? nullptr : static_cast<uint16_t *>(o);
+    dp.o32 = out_f32 ? static_cast<float *>(o) : nullptr;
+    dp.lse = lse;
+    dp.o_part = P.slots > 0 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + P.off_o) : nullptr;
+    dp.lse_part = P.slots > 0 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + P.off_lse) : nullptr;
+    dp.qslot = P.slots > 0 ? reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + P.off_qslot) : nullptr;
+    dp.scale_log2 = softmax_scale * 1.4426950408889634f;
+    dp.k = k;
+    dp.w_max = w_max;
+    dp.q_per_seq = q_per_seq;
+    dp.nq = nq;
+    dp.tpq = P.tpq;
+    dp.per = P.per;
+    switch (h) {
+        case 64:
+            if (!smem_attr(k_attn_decode<64>, DecCfg<64>::kSmem)) return CSA2_ERR_CUDA;
+            launch_decode<64>(dp, P, out_f32, stream);
+            break;
+        case 32:
+            if (!smem_attr(k_attn_decode<32>, DecCfg<32>::kSmem)) return CSA2_ERR_CUDA;
+            launch_decode<32>(dp, P, out_f32, stream);
+            break;
+        default:
+            if (!smem_attr(k_attn_decode<16>, DecCfg<16>::kSmem)) return CSA2_ERR_CUDA;
+            launch_decode<16>(dp, P, out_f32, stream);
+            break;
+    }
+    return check_launch();
 }
 
 // Shared body of the decode entry points: o is bf16 (out_f32 false) or the
@@ -668,8 +906,10 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
         return CSA2_ERR_INVALID_ARG;
     if (!has_swa && w_max > 0) return CSA2_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return CSA2_ERR_INVALID_ARG;
-    const AttnPlan P = nvfp4 ? plan_attn_nvfp4(nq, k, has_swa ? w_max : 0, num_sms())
-                             : plan_attn(nq, k, has_swa ? w_max : 0, num_sms());
+    if (!nvfp4) return decode_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, has_swa ? swa_begin : nullptr,
+                                   has_swa ? swa_end : nullptr, has_swa ? w_max : 0, softmax_scale, o, out_f32, lse,
+                                   ws, ws_bytes, stream);
+    const AttnPlan P = plan_attn_nvfp4(nq, k, has_swa ? w_max : 0, num_sms());
     const AttnLayout L = attn_layout(nq, h, P, nvfp4);
     if (L.total > 0 && (!ws || ws_bytes < L.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
@@ -708,35 +948,13 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
     const dim3 grid((unsigned)P.splits, (unsigned)nq);
     auto go = [&](auto kernel, size_t smem) { launch(kernel, grid, dim3(kAttnThreads), smem, stream, ap); };
     if (nvfp4) {
-        static const bool ok = set_smem(k_sparse_attn<64, true>, AttnCfg<64, true>::kSmem);
-        if (!ok) return CSA2_ERR_CUDA;
+        if (!smem_attr(k_sparse_attn<64, true>, AttnCfg<64, true>::kSmem)) return CSA2_ERR_CUDA;
         // q -> NVFP4 once per call (codes and scales into the workspace)
         const int32_t n_blocks = nq * h * (CSA2_D / CSA2_BLOCK);
         launch(k_quant_rows_nvfp4, dim3((unsigned)((n_blocks + kQuantThreads - 1) / kQuantThreads)),
                dim3(kQuantThreads), 0, stream, static_cast<const uint16_t *>(q_bf16), n_blocks, ap.q4, ap.q4s);
         if ((st = check_launch()) != CSA2_OK) return st;
         go(k_sparse_attn<64, true>, AttnCfg<64, true>::kSmem);
-    } else {
-        switch (h) {
-            case 64: {
-                static bool ok = set_smem(k_sparse_attn<64, false>, AttnCfg<64>::kSmem);
-                if (!ok) return CSA2_ERR_CUDA;
-                go(k_sparse_attn<64, false>, AttnCfg<64>::kSmem);
-                break;
-            }
-            case 32: {
-                static bool ok = set_smem(k_sparse_attn<32, false>, AttnCfg<32>::kSmem);
-                if (!ok) return CSA2_ERR_CUDA;
-                go(k_sparse_attn<32, false>, AttnCfg<32>::kSmem);
-                break;
-            }
-            default: {
-                static bool ok = set_smem(k_sparse_attn<16, false>, AttnCfg<16>::kSmem);
-                if (!ok) return CSA2_ERR_CUDA;
-                go(k_sparse_attn<16, false>, AttnCfg<16>::kSmem);
-                break;
-            }
-        }
     }
     if ((st = check_launch()) != CSA2_OK) return st;
     if (P.splits > 1) {
@@ -862,8 +1080,7 @@ csa2_status csa2_select_keys(const unsigned long long *keys, int32_t nq, int32_t
     rp.k = k;
     const size_t base = 2048 * 4 + (kReindexSelectThreads / 32 + 8) * 4;
     const size_t smem = base + (size_t)m * 8;
-    static const bool ok = set_smem(k_reindex_select<false>, (size_t)max_smem_optin());
-    if (!ok) return CSA2_ERR_CUDA;
+    if (!smem_attr(k_reindex_select<false>, (size_t)max_smem_optin())) return CSA2_ERR_CUDA;
     if (smem <= (size_t)max_smem_optin())
         launch(k_reindex_select<false>, dim3(nq), dim3(kReindexSelectThreads), smem, stream, rp);
     else  // keys larger than shared memory: every pass reads them from L2
@@ -890,22 +1107,49 @@ static __device__ __align__(256) uint8_t g_attn_scratch[CSA2_ATTN_STATIC_SCRATCH
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_attn_scratch_mu;
 void *g_attn_scratch_ptr[kMaxScratchDevices] = {};
+CUcontext g_attn_scratch_ctx[kMaxScratchDevices] = {};
+
+// cuCtxGetCurrent, fetched through the runtime like cuTensorMapEncodeTiled.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
 
 // Device address of this device's copy of g_attn_scratch, or null on error.
+// The address belongs to the context the module was loaded into: it is looked
+// up again whenever the device's current context is not the one it was
+// looked up in (after cudaDeviceReset, for example, the module is loaded
+// anew and the old address is gone).
 void *attn_scratch_of_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) {
         cudaGetLastError();
         return nullptr;
     }
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return nullptr;
+    CUcontext ctx = nullptr;  // stays null while no context is current on this thread
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
     std::lock_guard<std::mutex> lock(g_attn_scratch_mu);
-    if (!g_attn_scratch_ptr[dev]) {
+    if (!g_attn_scratch_ptr[dev] || ctx == nullptr || g_attn_scratch_ctx[dev] != ctx) {
         void *ptr = nullptr;
+        // with the device current; makes the runtime's context current if none was
         if (cudaGetSymbolAddress(&ptr, g_attn_scratch) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
         g_attn_scratch_ptr[dev] = ptr;
+        g_attn_scratch_ctx[dev] = ctx;
     }
     return g_attn_scratch_ptr[dev];
 }

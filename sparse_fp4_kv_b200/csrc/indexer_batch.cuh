@@ -1,0 +1,438 @@
+// indexer_batch.cuh -- Full-mode indexer for many queries of one sequence
+// (the chunked-prefill workload: hundreds of causal queries over one cache),
+// with the key tiles shared by a group of queries in each tensor-core
+// product.
+//
+// Same method as indexer.cuh (DeepSeek V4.1-Flash Cuts KV Cache by 437x,
+// paragraph "CSA2 assigns each layer one of three static operating modes":
+// Full mode scores the whole visible context and keeps its Top-K):
+//     score(t) = sum_h w_h * max(0, <q_h, kidx_t>),
+// order score descending, entry id ascending on ties; output ids ascending.
+//
+// The queries are taken in groups of QG (16 with up to 4 indexer heads, 8
+// with up to 8; all of one sequence). One
+// product per tile of 128 key rows scores every entry of the tile for every
+// query of the group: B holds the group's heads (kEpr copies side by side
+// as in the single-query scan, so that a 128-byte key row can hold two
+// 64-byte entries), N = kEpr * QG * HP = 128 / (DI / 64). The selection runs in
+// two scans of the keys plus two small per-query kernels:
+//   1. k_batch_scan<0>: the score keys' top 11 bits counted per query
+//      (histograms in shared memory, added to a global histogram);
+//   2. k_batch_thresh: per query, the bin b0 holding its k-th largest key and
+//      how many keys of b0 are still needed;
+//   3. k_batch_scan<1>: the scores again (the same products, so the same
+//      keys): entries above b0 go to the query's "sure" list, entries in b0
+//      to its candidate list as unique 64-bit keys (score key << 32 | ~id);
+//   4. k_batch_final: the needed number of largest candidates by an exact
+//      radix select, merged with the sure ids and sorted ascending.
+#pragma once
+
+#include "indexer.cuh"
+
+namespace csa2 {
+
+constexpr int kBatchBins = 2048;   // digit 0: the key's top 11 bits
+constexpr int kBatchShift = 21;
+constexpr int kBatchEpiWarps = 16;  // 4 per TMEM lane quarter
+constexpr int kBatchThreads = 64 + kBatchEpiWarps * 32;
+constexpr int kBatchFinalThreads = 1024;
+constexpr int kBatchMaxK = 4096;   // ids staged and sorted in shared memory
+constexpr uint32_t kBatchAll = 0xFFFFFFFFu;  // b0 marker: every visible entry is taken
+
+struct BatchParams {
+    const uint8_t *qidx;  // [nq][hi][DI] E4M3
+    const float *w;       // [nq][hi]
+    const int32_t *q_limit;
+    csa2_kv_desc kv;
+    uint32_t *hist;             // [nq][kBatchBins]
+    uint32_t *state;            // [nq][4]: b0, rem, n_sure, n_cand
+    int32_t *sure;              // [nq][k]
+    unsigned long long *cand;   // [nq][cap]
+    int32_t *topk;              // [nq][k]
+    int64_t cap;
+    int64_t chunk;              // entries per CTA (a multiple of the tile)
+    int32_t k, q_per_seq, hi, hi_pad, nq, box_rows;
+};
+
+template <int DI>
+struct BatchGeom {
+    static constexpr int kEpr = 128 / DI;   // entries per 128-byte key row
+    static constexpr int kTile = 128 * kEpr;
+    static constexpr int kStageBytes = 128 * 128;
+};
+
+// Queries per group for HP padded heads (N = kEpr * QG * HP stays 64 or 128).
+__host__ __device__ constexpr int batch_qg(int hp) { return hp == 4 ? 16 : 8; }
+
+// Queries of group gq: [gq * QG, min(nq, (gq + 1) * QG)); the largest visible
+// limit among them bounds the group's scan.
+template <int QG>
+__device__ __forceinline__ int64_t group_limit(const BatchParams &p, int32_t gq, int32_t *lim /*[QG]*/) {
+    int64_t mx = 0;
+    for (int j = 0; j < QG; ++j) {
+        const int32_t qi = gq * QG + j;
+        const int64_t l = qi < p.nq ? query_limit(p.q_limit, p.kv, qi, p.q_per_seq) : 0;
+        if (lim) lim[j] = (int32_t)min(l, (int64_t)INT32_MAX);
+        mx = max(mx, l);
+    }
+    return mx;
+}
+
+// HP: indexer heads padded to 4 or 8.
+template <int DI, int HP, int PASS>
+struct BatchCfg {
+    using G = BatchGeom<DI>;
+    static constexpr int QG = batch_qg(HP);
+    static constexpr int N = G::kEpr * QG * HP;
+    static constexpr int kStages = PASS == 0 ? 4 : 8;
+    static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128u : 256u;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * G::kStageBytes + (size_t)N * 128 +
+                                    (PASS == 0 ? (size_t)QG * kBatchBins * 4 : 0) + 16 * 16 * 4 + 16 * 4 * 2 +
+                                    (size_t)kMaxScanPages * 4 + 256;
+};
+
+template <int DI, int HP, int PASS>
+__global__ void __launch_bounds__(kBatchThreads, 1)
+    k_batch_scan(const __grid_constant__ CUtensorMap tm, BatchParams p) {
+    using G = BatchGeom<DI>;
+    using Cfg = BatchCfg<DI, HP, PASS>;
+    static_assert(HP == 4 || HP == 8, "heads padded to 4 or 8");
+    constexpr int QG = Cfg::QG, N = Cfg::N, kStages = Cfg::kStages;
+    constexpr uint32_t tcols = Cfg::kTmemCols;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = base;
+    uint8_t *btile = stages + kStages * G::kStageBytes;  // N rows x 128 B
+    uint32_t *hist = reinterpret_cast<uint32_t *>(btile + N * 128);          // PASS 0: [QG][bins]
+    float *wq = reinterpret_cast<float *>(hist + (PASS == 0 ? QG * kBatchBins : 0));  // [16][16]
+    int32_t *lim = reinterpret_cast<int32_t *>(wq + 16 * 16);                 // [16]
+    uint32_t *b0s = reinterpret_cast<uint32_t *>(lim + 16);                   // [16] (PASS 1)
+    int32_t *ptab = reinterpret_cast<int32_t *>(b0s + 16);                    // [kMaxScanPages]
+    uint64_t *full_b = reinterpret_cast<uint64_t *>(ptab + kMaxScanPages);
+    uint64_t *empty_b = full_b + kStages;
+    uint64_t *tfull = empty_b + kStages;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t gq = blockIdx.y;
+    const int32_t q0 = gq * QG;
+    const int32_t b = q0 / p.q_per_seq;
+
+    pdl_trigger();
+    if (PASS == 0)
+        for (int i = tid; i < QG * kBatchBins; i += kBatchThreads) hist[i] = 0u;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty_b[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], kBatchEpiWarps);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, tcols);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    if (tid == 0) group_limit<QG>(p, gq, lim);
+    __syncthreads();
+    int64_t gl = 0;
+    for (int j = 0; j < QG; ++j) gl = max(gl, (int64_t)lim[j]);
+    const int64_t start = (int64_t)blockIdx.x * p.chunk;
+    const int64_t n_loc = max((int64_t)0, min(gl, start + p.chunk) - start);
+    const int ntiles = (int)((n_loc + G::kTile - 1) / G::kTile);
+    // B: rows (u, j, h) = u * QG * HP + j * HP + h hold query j's head h
+    // in the 64-byte half u of a 128-byte row (DI = 64), zero elsewhere
+    for (int i = tid; i < N * 8; i += kBatchThreads) {
+        const int r = i / 8, c = i % 8;
+        const int u = r / (QG * HP), jh = r % (QG * HP);
+        const int j = jh / HP, h = jh % HP;
+        const int32_t qi = q0 + j;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (qi < p.nq && h < p.hi) {
+            const uint8_t *q = p.qidx + ((int64_t)qi * p.hi + h) * DI;
+            if (DI == 128)
+                v = *reinterpret_cast<const uint4 *>(q + c * 16);
+            else if (c / 4 == u)
+                v = *reinterpret_cast<const uint4 *>(q + (c % 4) * 16);
+        }
+        *reinterpret_cast<uint4 *>(btile + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
+    for (int i = tid; i < QG * 16; i += kBatchThreads) {
+        const int j = i / 16, h = i % 16;
+        const int32_t qi = q0 + j;
+        wq[i] = (qi < p.nq && h < p.hi) ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
+    }
+    if (PASS == 1 && tid < QG) b0s[tid] = q0 + tid < p.nq ? __ldcg(p.state + (int64_t)(q0 + tid) * 4) : 0u;
+    if (ntiles > 0) stage_pages(p.kv, b, start, n_loc, ptab, kBatchThreads);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        scan_tma_loop<DI>(p.kv, ptab, start, gl, ntiles, kStages, p.box_rows, stages, &tm, full_b, empty_b);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_e4m3_f32(128, N);
+            const uint32_t qaddr = smem_u32(btile);
+            int s = 0;
+            uint32_t phase = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int a = i & 1;
+                if (!mbar_wait(&tempty[a], ((i >> 1) & 1) ^ 1)) break;
+                if (!mbar_wait(&full_b[s], phase)) break;
+                tc_fence_after();
+                const uint32_t aaddr = smem_u32(stages + (size_t)s * G::kStageBytes);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_e4m3(tmem + (uint32_t)(a * N), make_sdesc(aaddr + kk * 32, 16, 1024, kSw128),
+                             make_sdesc(qaddr + kk * 32, 16, 1024, kSw128), idesc, kk > 0 ? 1u : 0u);
+                tc_commit(&empty_b[s]);
+                tc_commit(&tfull[a]);
+                if (++s == kStages) {
+                    s = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // epilogue: TMEM lane quarter (warp & 3), queries [sub * QW, sub * QW + QW)
+        constexpr int QW = QG / 4;  // queries of one warp: QW * HP = 16 columns per half row
+        const int ew = warp - 2;
+        const int quarter = warp & 3, sub = ew >> 2;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        for (int i = 0; i < ntiles; ++i) {
+            const int a = i & 1;
+            const bool got = mbar_wait(&tfull[a], (i >> 1) & 1);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int u = 0; u < G::kEpr; ++u) {
+                // the 16 columns of this warp's queries in half u
+                uint32_t r[16];
+                const uint32_t col = (uint32_t)(a * N + u * QG * HP + sub * QW * HP);
+                tmem_ld16(lane_base + col, r);
+                tmem_wait_ld();
+                const int64_t t = start + (int64_t)i * G::kTile + (int64_t)G::kEpr * (quarter * 32 + lane) + u;
+#pragma unroll
+                for (int jj = 0; jj < QW; ++jj) {
+                    const int j = sub * QW + jj;
+                    float sc = 0.0f;
+#pragma unroll
+                    for (int h = 0; h < HP; ++h)
+                        sc = fmaf(wq[j * 16 + h], fmaxf(__uint_as_float(r[jj * HP + h]), 0.0f), sc);
+                    const uint32_t key = score_key(sc + 0.0f);
+                    const bool vis = t < (int64_t)lim[j];
+                    const int32_t qi = q0 + j;
+                    if (PASS == 0) {
+                        if (vis) atomicAdd(&hist[j * kBatchBins + (key >> kBatchShift)], 1u);
+                    } else {
+                        const uint32_t b0 = b0s[j];
+                        const uint32_t d = key >> kBatchShift;
+                        const bool sure = vis && (b0 == kBatchAll || d > b0);
+                        const bool cand = vis && b0 != kBatchAll && d == b0;
+                        const uint32_t ms = __ballot_sync(0xFFFFFFFFu, sure);
+                        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, cand);
+                        const uint32_t lt = (1u << lane) - 1u;
+                        if (ms) {
+                            uint32_t base0 = 0;
+                            if (lane == 0) base0 = atomicAdd(p.state + (int64_t)qi * 4 + 2, (uint32_t)__popc(ms));
+                            base0 = __shfl_sync(0xFFFFFFFFu, base0, 0);
+                            if (sure) {
+                                const uint32_t at = base0 + __popc(ms & lt);
+                                if (at < (uint32_t)p.k)
+                                    p.sure[(int64_t)qi * p.k + at] = (int32_t)t;
+                                else
+                                    set_error(CSA2_DEVERR_SELECT);
+                            }
+                        }
+                        if (mc) {
+                            uint32_t base0 = 0;
+                            if (lane == 0) base0 = atomicAdd(p.state + (int64_t)qi * 4 + 3, (uint32_t)__popc(mc));
+                            base0 = __shfl_sync(0xFFFFFFFFu, base0, 0);
+                            if (cand) {
+                                const uint32_t at = base0 + __popc(mc & lt);
+                                if ((int64_t)at < p.cap)
+                                    p.cand[(int64_t)qi * p.cap + at] =
+                                        ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)t);
+                                else
+                                    set_error(CSA2_DEVERR_SELECT);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[a]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tcols);
+    }
+    if (PASS == 0) {
+        for (int i = tid; i < QG * kBatchBins; i += kBatchThreads) {
+            const int j = i / kBatchBins;
+            const uint32_t v = hist[i];
+            if (v && q0 + j < p.nq) atomicAdd(p.hist + (int64_t)(q0 + j) * kBatchBins + (i % kBatchBins), v);
+        }
+    }
+}
+
+// Per query: the digit-0 bin of its k-th largest key, how many keys of that
+// bin are needed, and zeroed list counts (or "take all" when k covers every
+// visible entry).
+constexpr int kBatchThreshThreads = 256;
+__global__ void __launch_bounds__(kBatchThreshThreads) k_batch_thresh(BatchParams p) {
+    __shared__ uint32_t scratch[kBatchThreshThreads / 32 + 4];
+    pdl_trigger();
+    pdl_wait();
+    const int32_t qi = blockIdx.x;
+    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+    uint32_t bin = kBatchAll, rem = 0;
+    if ((int64_t)p.k < limit)
+        find_rank_bin<kBatchThreshThreads, kBatchBins / kBatchThreshThreads, true>(
+            p.hist + (int64_t)qi * kBatchBins, kBatchBins, (uint32_t)p.k, scratch, bin, rem);
+    if (threadIdx.x == 0) {
+        uint32_t *st = p.state + (int64_t)qi * 4;
+        st[0] = bin;
+        st[1] = rem;
+        st[2] = 0u;
+        st[3] = 0u;
+    }
+}
+
+// Per query: the rem largest of its n_cand candidate keys (unique 64-bit
+// keys, kept in shared memory when they fit, else re-read from L2 in every
+// radix pass), merged with its sure ids, sorted ascending, padded with -1.
+__global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchParams p, int32_t smem_keys) {
+    constexpr int NT = kBatchFinalThreads;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);            // [2048]
+    uint32_t *scratch = hist + 2048;                                    // [NT/32 + 8]
+    int32_t *ids = reinterpret_cast<int32_t *>(scratch + NT / 32 + 8);   // [kBatchMaxK]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(ids + kBatchMaxK);  // [smem_keys]
+    __shared__ unsigned long long and_acc, or_acc;
+    __shared__ uint32_t n_out;
+    const int32_t qi = blockIdx.x;
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        and_acc = ~0ull;
+        or_acc = 0ull;
+        n_out = 0u;
+    }
+    pdl_wait();
+    const uint32_t *st = p.state + (int64_t)qi * 4;
+    const uint32_t b0 = __ldcg(st), need = __ldcg(st + 1);
+    const uint32_t n_sure = min(__ldcg(st + 2), (uint32_t)p.k);
+    const uint32_t n_cand = (uint32_t)min((int64_t)__ldcg(st + 3), p.cap);
+    const unsigned long long *src = p.cand + (int64_t)qi * p.cap;
+    __syncthreads();
+    // the sure ids first
+    for (uint32_t j = threadIdx.x; j < n_sure; j += NT) ids[j] = p.sure[(int64_t)qi * p.k + j];
+    uint32_t take = 0;
+    if (b0 != kBatchAll && need > 0 && n_cand > 0) {
+        take = min(need, n_cand);
+        const bool G = n_cand > (uint32_t)smem_keys;  // candidates re-read from L2 in every pass
+        unsigned long long a_loc = ~0ull, o_loc = 0ull;
+        for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
+            const unsigned long long v = __ldcg(src + j);
+            if (!G) k64[j] = v;
+            a_loc &= v;
+            o_loc |= v;
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
+            o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
+        }
+        if ((threadIdx.x & 31) == 0) {
+            atomicAnd(&and_acc, a_loc);
+            atomicOr(&or_acc, o_loc);
+        }
+        __syncthreads();
+        auto key = [&](uint32_t j) -> unsigned long long { return G ? __ldcg(src + j) : k64[j]; };
+        unsigned long long T = 0ull;  // take the keys >= T
+        if (take < n_cand) {
+            const unsigned long long diff = and_acc ^ or_acc;  // keys are unique: diff != 0
+            int top = 63 - __clzll((long long)diff);
+            unsigned long long prefix = and_acc & ~((2ull << top) - 1ull);
+            unsigned long long pmask = ~((2ull << top) - 1ull);
+            if (top == 63) {
+                prefix = 0ull;
+                pmask = 0ull;
+            }
+            uint32_t rem = take;
+            while (true) {
+                const int nbits = top + 1 < 11 ? top + 1 : 11;
+                const int shift = top + 1 - nbits;
+                const int nb = 1 << nbits;
+                for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
+                __syncthreads();
+                for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
+                    const unsigned long long v = key(j);
+                    if ((v & pmask) == prefix) atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
+                }
+                __syncthreads();
+                uint32_t bin, inbin;
+                find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
+                prefix |= (unsigned long long)bin << shift;
+                pmask |= (unsigned long long)(nb - 1) << shift;
+                rem = inbin;
+                const bool all_taken = hist[bin] == rem;
+                __syncthreads();
+                if (all_taken || shift == 0) break;
+                const unsigned long long below = diff & ((1ull << shift) - 1ull);
+                if (below == 0ull) break;
+                top = 63 - __clzll((long long)below);
+            }
+            T = prefix | (and_acc & ~diff & ~pmask);
+        }
+        for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
+            const unsigned long long v = key(j);
+            if (v >= T) {
+                const uint32_t at = n_sure + atomicAdd(&n_out, 1u);
+                if (at < (uint32_t)kBatchMaxK && at < (uint32_t)p.k)
+                    ids[at] = (int32_t)(~(uint32_t)v);
+                else
+                    set_error(CSA2_DEVERR_SELECT);
+            }
+        }
+    }
+    __syncthreads();
+    const uint32_t total = min(n_sure + min(n_out, take), (uint32_t)p.k);
+    // bitonic sort of the ids ascending (padding above total sorts last)
+    int P2 = 1;
+    while (P2 < p.k) P2 <<= 1;
+    for (int j = (int)total + threadIdx.x; j < P2; j += NT) ids[j] = INT32_MAX;
+    __syncthreads();
+    for (int size = 2; size <= P2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < P2 / 2; i += NT) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int32_t x = ids[lo], y = ids[hi];
+                if ((x > y) == up) {
+                    ids[lo] = y;
+                    ids[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    int32_t *out = p.topk + (int64_t)qi * p.k;
+    for (int j = threadIdx.x; j < p.k; j += NT) out[j] = j < (int)total ? ids[j] : -1;
+}
+
+}  // namespace csa2

@@ -433,54 +433,24 @@ __global__ void __launch_bounds__(kReindexScoreThreads) k_reindex_score(ReindexP
     p.k64[(int64_t)qi * p.p + j] = v;
 }
 
-template <bool G>
-__global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(ReindexParams p) {
-    constexpr int NT = kReindexSelectThreads;
-    extern __shared__ uint8_t smem_raw[];
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                                 // [2048]
-    uint32_t *scratch = hist + 2048;                                                         // [NT/32 + 8]
-    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p] (G false)
-    __shared__ unsigned long long and_acc, or_acc;
-    const int32_t qi = blockIdx.x;
-    pdl_trigger();
-    if (threadIdx.x == 0) {
-        and_acc = ~0ull;
-        or_acc = 0ull;
-    }
-    pdl_wait();
-    __syncthreads();
-    uint32_t nvalid_t = 0;
-    unsigned long long a_loc = ~0ull, o_loc = 0ull;
-    const unsigned long long *src = p.k64 + (int64_t)qi * p.p;
+// Select the k largest of the m unique 64-bit keys of query qi (0 = empty;
+// in shared memory k64 unless G, then read through L2 from src) and write the
+// ids they carry in key-array order, padded with -1. nvalid, and_acc and
+// or_acc: the count and the AND / OR of the valid keys (made visible to all
+// threads by the caller). Block-wide (NT threads, a power of two).
+template <bool G, int NT>
+__device__ __forceinline__ void select_k64(const unsigned long long *k64, const unsigned long long *src, int32_t m,
+                                           int32_t k, int32_t *out, uint32_t nvalid, unsigned long long and_acc,
+                                           unsigned long long or_acc, uint32_t *hist, uint32_t *scratch) {
     auto key = [&](int j) -> uint64_t {
         if constexpr (G)
             return __ldcg(src + j);
         else
             return k64[j];
     };
-    for (int j = threadIdx.x; j < p.p; j += NT) {
-        const unsigned long long v = __ldcg(src + j);
-        if constexpr (!G) k64[j] = v;
-        if ((uint32_t)v >= 0x80000000u) {
-            ++nvalid_t;
-            a_loc &= v;
-            o_loc |= v;
-        }
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
-        o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
-    }
-    if ((threadIdx.x & 31) == 0) {
-        atomicAnd(&and_acc, a_loc);
-        atomicOr(&or_acc, o_loc);
-    }
-    uint32_t nvalid;
-    block_excl_scan<NT>(nvalid_t, scratch, &nvalid);  // its barriers also publish k64 and the reductions
-    const uint32_t r = min((uint32_t)p.k, nvalid);
+    const uint32_t r = min((uint32_t)k, nvalid);
     uint64_t T = 1ull;  // select keys >= T (every valid key is >= 2^31)
-    if (nvalid > (uint32_t)p.k) {
+    if (nvalid > (uint32_t)k) {
         // digits of 11 bits from the highest bit in which two keys differ;
         // bits that are equal in every key are skipped (they decide nothing)
         const unsigned long long diff = and_acc ^ or_acc;
@@ -494,7 +464,7 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
             const int nb = 1 << nbits;
             for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
             __syncthreads();
-            for (int j = threadIdx.x; j < p.p; j += NT) {
+            for (int j = threadIdx.x; j < m; j += NT) {
                 const uint64_t v = key(j);
                 if ((uint32_t)v >= 0x80000000u && (v & pmask) == prefix)
                     atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
@@ -516,27 +486,255 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
         // resolved digits (and the unresolved low bits of the last bin) decide
         T = prefix | (and_acc & ~diff);
     }
-    // ordered emission (pool order)
-    const int per = (p.p + NT - 1) / NT;
+    // ordered emission (key-array order)
+    const int per = (m + NT - 1) / NT;
     const int j0 = threadIdx.x * per;
     uint32_t mine = 0;
-    for (int j = j0; j < min(p.p, j0 + per); ++j) {
+    for (int j = j0; j < min(m, j0 + per); ++j) {
         const uint64_t v = key(j);
         mine += (uint32_t)v >= 0x80000000u && v >= T;
     }
     uint32_t pos = block_excl_scan<NT>(mine, scratch, nullptr);
-    int32_t *out = p.topk + (int64_t)qi * p.k;
-    for (int j = j0; j < min(p.p, j0 + per); ++j) {
+    for (int j = j0; j < min(m, j0 + per); ++j) {
         const uint64_t v = key(j);
         if (!((uint32_t)v >= 0x80000000u && v >= T)) continue;
-        if (pos < (uint32_t)p.k) {
+        if (pos < (uint32_t)k) {
             out[pos] = (int32_t)(~(uint32_t)v);
         } else {
             set_error(CSA2_DEVERR_SELECT);
         }
         ++pos;
     }
-    for (int j = (int)r + threadIdx.x; j < p.k; j += NT) out[j] = -1;
+    for (int j = (int)r + threadIdx.x; j < k; j += NT) out[j] = -1;
+}
+
+template <bool G>
+__global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(ReindexParams p) {
+    constexpr int NT = kReindexSelectThreads;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                                 // [2048]
+    uint32_t *scratch = hist + 2048;                                                         // [NT/32 + 8]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p] (G false)
+    __shared__ unsigned long long and_acc, or_acc;
+    const int32_t qi = blockIdx.x;
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        and_acc = ~0ull;
+        or_acc = 0ull;
+    }
+    pdl_wait();
+    __syncthreads();
+    uint32_t nvalid_t = 0;
+    unsigned long long a_loc = ~0ull, o_loc = 0ull;
+    const unsigned long long *src = p.k64 + (int64_t)qi * p.p;
+    for (int j = threadIdx.x; j < p.p; j += NT) {
+        const unsigned long long v = __ldcg(src + j);
+        if constexpr (!G) k64[j] = v;
+        if ((uint32_t)v >= 0x80000000u) {
+            ++nvalid_t;
+            a_loc &= v;
+            o_loc |= v;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
+        o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicAnd(&and_acc, a_loc);
+        atomicOr(&or_acc, o_loc);
+    }
+    uint32_t nvalid;
+    block_excl_scan<NT>(nvalid_t, scratch, &nvalid);  // its barriers also publish k64 and the reductions
+    select_k64<G, NT>(k64, src, p.p, p.k, p.topk + (int64_t)qi * p.k, nvalid, and_acc, or_acc, hist, scratch);
+}
+
+// ---------------------------------------------------------------------------
+// Reindex in one launch, one CTA per query: the pool's indexer keys are
+// gathered by cp.async (16-byte pieces, a ring of 128-row tiles laid out as
+// the scan's 128B-swizzled A operand, two 64-byte entries per row when
+// di = 64), scored by tcgen05 FP8 products against the query's heads (as in
+// the Full scan, so the same exact scores), and the unique 64-bit keys
+// (score key << 32 | ~id) kept in shared memory for select_k64.
+// Warps 0..7 gather, warps 8..11 (TMEM lane quarters 0..3) read the scores
+// back, warp 12 issues the products; then every thread selects.
+// ---------------------------------------------------------------------------
+constexpr int kRfStages = 4;
+constexpr int kRfThreads = 512;
+constexpr int kRfGatherThreads = 256;
+constexpr int kRfMmaWarp = 12;
+
+template <int DI>
+struct RfCfg {
+    using G = ScanGeom<DI>;
+    static size_t smem(int p) {
+        return 1024 + (size_t)kRfStages * G::kStageBytes + 4096 /*q tile*/ + 2048 * 4 + (NT32 + 8) * 4 +
+               (size_t)p * 8 + ((size_t)p / 32 + 2) * 4 + 256;
+    }
+    static constexpr int NT32 = kRfThreads / 32;
+};
+
+template <int DI>
+__global__ void __launch_bounds__(kRfThreads, 1) k_reindex_fused(ReindexParams p) {
+    using G = ScanGeom<DI>;
+    constexpr int NT = kRfThreads;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = base;
+    uint8_t *qt = stages + kRfStages * G::kStageBytes;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(qt + 4096);  // [2048]
+    uint32_t *scratch = hist + 2048;                            // [NT/32 + 8]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p]
+    uint32_t *vbits = reinterpret_cast<uint32_t *>(k64 + p.p);  // [p / 32 + 1]: valid pool slots
+    uint64_t *full_b = reinterpret_cast<uint64_t *>(vbits + (p.p / 32 + 2) / 2 * 2);
+    uint64_t *empty_b = full_b + kRfStages;
+    uint64_t *tfull = empty_b + kRfStages;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    __shared__ unsigned long long and_acc, or_acc;
+    __shared__ uint32_t nvalid_s;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t qi = blockIdx.x;
+    const int32_t b = qi / p.q_per_seq;
+    const int ntiles = (p.p + G::kTile - 1) / G::kTile;
+    pdl_trigger();
+    for (int i = tid; i < p.p / 32 + 1; i += NT) vbits[i] = 0u;
+    if (tid == 0) {
+        and_acc = ~0ull;
+        or_acc = 0ull;
+        nvalid_s = 0u;
+        for (int s = 0; s < kRfStages; ++s) {
+            mbar_init(&full_b[s], kRfGatherThreads);
+            mbar_init(&empty_b[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        fence_mbar_init();
+    }
+    if (warp == kRfMmaWarp) {
+        tmem_alloc(tmem_slot, 2 * kScanBatch * G::kN);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    build_q_tile<DI>(qt, p.qidx + (int64_t)qi * p.hi * DI, p.hi, NT);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int32_t *pool = p.pool + (int64_t)qi * p.p;
+
+    if (tid < kRfGatherThreads) {
+        // tile t, stage t % S: entry e of the tile -> row e / kEpr, 64-byte half
+        // e % kEpr (di = 64), 16-byte pieces; an empty slot or a bad id is
+        // zero-filled (a bad id is reported). Up to kRfStages tiles of this
+        // thread's pieces are in flight: tile t is published to the products
+        // once the pieces of tile t are complete, kRfStages - 1 tiles later.
+        constexpr int kPieces = DI / 16;                             // per entry
+        constexpr int kPer = G::kTile * kPieces / kRfGatherThreads;  // per thread and tile (4)
+        int s = 0;
+        uint32_t phase = 0;
+        int s_pub = 0;
+        auto publish = [&]() {
+            fence_proxy_async_smem();
+            mbar_arrive(&full_b[s_pub]);
+            if (++s_pub == kRfStages) s_pub = 0;
+        };
+        bool ok = true;
+        int issued = 0;
+        for (int t = 0; t < ntiles; ++t) {
+            if (!mbar_wait(&empty_b[s], phase ^ 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t *st = stages + (size_t)s * G::kStageBytes;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int idx = tid + i * kRfGatherThreads;  // piece index in the tile
+                const int e = idx / kPieces, c = idx % kPieces;
+                const int j = t * G::kTile + e;              // pool position
+                const int32_t id = j < p.p ? pool[j] : -1;
+                const int64_t row = id >= 0 ? physical_row(p.kv, b, id) : -1;
+                if (c == 0 && row >= 0) atomicOr(&vbits[j >> 5], 1u << (j & 31));
+                if (c == 0 && id >= 0 && row < 0) set_error(CSA2_DEVERR_BAD_ROW);
+                const int r = e / G::kEpr, u = e % G::kEpr;
+                const int chunk = u * kPieces + c;
+                uint8_t *dst = st + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+                const uint8_t *srcp = row >= 0 ? p.kv.kidx + row * DI + c * 16 : p.kv.kidx;
+                const uint32_t bytes = row >= 0 ? 16u : 0u;  // 0: zero fill
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(srcp),
+                             "r"(bytes)
+                             : "memory");
+            }
+            cp_async_commit();
+            ++issued;
+            if (issued >= kRfStages) {
+                asm volatile("cp.async.wait_group 3;" ::: "memory");  // kRfStages - 1 groups may stay in flight
+                publish();
+            }
+            if (++s == kRfStages) {
+                s = 0;
+                phase ^= 1u;
+            }
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        if (ok)
+            for (int t = max(0, issued - (kRfStages - 1)); t < issued; ++t) publish();
+    } else if (warp == kRfMmaWarp) {
+        if (lane == 0)
+            scan_mma_loop<DI>(ntiles, kRfStages, stages, smem_u32(qt), full_b, empty_b, tfull, tempty, tmem);
+        __syncwarp();
+    } else if (warp >= 8 && warp < 12) {
+        float wv[kScanN];
+#pragma unroll
+        for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
+        scan_epilogue_loop<DI>(ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3, [&](int i, int e_in, uint32_t key) {
+            const int j = i * G::kTile + e_in;
+            if (j < p.p)
+                k64[j] = ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)(pool[j] + p.id_offset));
+        });
+    }
+    tc_fence_before();
+    __syncthreads();
+    // empty or bad slots (no valid bit) become key 0; the valid keys' count,
+    // AND and OR for the select
+    {
+        uint32_t nv = 0;
+        unsigned long long a_loc = ~0ull, o_loc = 0ull;
+        for (int j = tid; j < p.p; j += NT) {
+            if ((vbits[j >> 5] >> (j & 31)) & 1u) {
+                const unsigned long long v = k64[j];
+                ++nv;
+                a_loc &= v;
+                o_loc |= v;
+            } else {
+                k64[j] = 0ull;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
+            o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
+            nv += __shfl_xor_sync(0xFFFFFFFFu, nv, o);
+        }
+        if (lane == 0) {
+            atomicAnd(&and_acc, a_loc);
+            atomicOr(&or_acc, o_loc);
+            atomicAdd(&nvalid_s, nv);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kRfMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * kScanBatch * G::kN);
+    }
+    select_k64<false, NT>(k64, nullptr, p.p, p.k, p.topk + (int64_t)qi * p.k, nvalid_s, and_acc, or_acc, hist,
+                          scratch);
 }
 
 }  // namespace csa2

@@ -10,14 +10,23 @@ ATTN_TOL = 2e-3  # max |o_gpu - o_oracle| where |o| <= 0.5 (bf16 output)
 
 
 def attn_excess(o_gpu, o_ref):
-    """Largest ratio |o_gpu - o_ref| / tol over the outputs; <= 1 passes.
-    tol = 2e-3 where |o_ref| <= 0.5 (the acceptance bar, meaningful for the
-    N(0,1) workloads). Above 0.5 the bf16 rounding of the output alone can
-    exceed 2e-3 (half an ulp is up to |o|/512), so there the bar is
-    2e-3 + |o_ref|/256: twice that half ulp on top of the absolute bar."""
+    """Largest ratio of an output's error to its bound over the outputs; <= 1
+    passes. Where |o_ref| <= 0.5 the bound is the acceptance bar 2e-3 on
+    |o_gpu - o_ref| (meaningful for the N(0,1) workloads, where |o| stays far
+    below 0.5). Above 0.5 half a bf16 ulp of the output alone can exceed
+    2e-3, so there the kernel's bf16 value must lie within one bf16 ulp of the
+    bf16 rounding of the oracle's value: the kernel's own error may only move
+    the rounding to a neighbouring bf16 value."""
+    o_gpu = np.asarray(o_gpu, np.float64)
+    o_ref = np.asarray(o_ref, np.float64)
     a = np.abs(o_ref)
-    tol = np.where(a <= 0.5, ATTN_TOL, ATTN_TOL + a / 256.0)
-    return float((np.abs(o_gpu - o_ref) / tol).max())
+    big = a > 0.5
+    ratio = np.abs(o_gpu - o_ref) / ATTN_TOL
+    if big.any():
+        rb = torch.from_numpy(o_ref[big]).to(torch.bfloat16).double().numpy()
+        ulp = np.exp2(np.floor(np.log2(np.abs(rb))) - 7.0)
+        ratio[big] = np.abs(o_gpu[big] - rb) / ulp
+    return float(ratio.max()) if ratio.size else 0.0
 
 
 def bf16_bits(t):

@@ -89,14 +89,18 @@ def test_single_query_many_tiles_split(B, cuda_device):
     _run(B, cuda_device, [70000], 128, 64, 2048, 512, seed=1)
 
 
-@pytest.mark.parametrize("splits", ["1", "3", "7", "auto"])
-def test_several_queries_split_ragged(B, cuda_device, monkeypatch, splits):
-    # several queries with ragged row counts, 32 and 16 heads, the split
-    # count fixed (1: no merge; 3, 7: ragged last split) or chosen by the plan
-    if splits != "auto":
-        monkeypatch.setenv("CSA2_ATTN_SPLITS", splits)
+@pytest.mark.parametrize("per", ["1", "3", "7", "12", "20", "40", "auto"])
+def test_several_queries_split_ragged(B, cuda_device, monkeypatch, per):
+    # several queries with ragged row counts, 32 and 16 heads, the tiles per
+    # CTA fixed or chosen by the plan: 1, 3: every query split over several
+    # CTAs; 7: CTAs that end one query and start the next (partial first and
+    # last segments); 12: one whole query per CTA; 20, 40: CTAs holding whole
+    # queries and parts of others, or every query (no merge)
+    if per != "auto":
+        monkeypatch.setenv("CSA2_ATTN_PER", per)
     _run(B, cuda_device, [9000, 5000, 3000], 64, 32, 1300, 200, seed=21)
     _run(B, cuda_device, [9000, 7000], 64, 16, 1800, 300, seed=22)
+    _run(B, cuda_device, [4000, 4000, 4000, 4000], 64, 64, 1000, 120, seed=23)
 
 
 def test_many_queries_single_split(B, cuda_device):
@@ -148,3 +152,56 @@ def test_running_max_raised_in_later_tiles(B, cuda_device):
     assert np.any(tmax[-1] > tmax[0] + 8), "case does not reach the rescale path"
     assert attn_excess(o.float().cpu().numpy()[0], oo) <= 1.0
     np.testing.assert_allclose(lse.cpu().numpy()[0], ol, atol=1e-3, rtol=0)
+
+
+def test_window_longer_than_w_max_is_dropped(B, cuda_device):
+    # a window of w_max + 5 rows (still inside its ring) breaks the call's
+    # contract: the window is dropped, the device error word records it, and
+    # the query attends its selected entries only
+    rng = np.random.default_rng(31)
+    lens, ps, h, k, w = [2000, 2000], 64, 32, 256, 100
+    pt, cap, codes, scales = _cache(rng, lens, ps, 31)
+    topk = np.stack([rng.permutation(2000)[:k].astype(np.int32) for _ in range(2)])
+    swa_rows = 160
+    swa = synth.normal_e4m3(31, 4, 0, 2 * swa_rows * 512).view(2, swa_rows, 512).numpy()
+    begin = np.array([0, 10], np.int32)
+    end = np.array([w, 10 + w + 5], np.int32)  # query 1: w_max + 5 rows
+    q = synth.normal_bf16(31, 3, 0, 2 * h * 512).view(2, h, 512)
+    scale = 1.0 / math.sqrt(512)
+    kv = kv_from_numpy(codes, scales, None, pt, lens, ps, cuda_device)
+    d = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(cuda_device)
+    o = torch.full((2, h, 512), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.full((2, h), float("nan"), dtype=torch.float32, device=cuda_device)
+    ws = B.workspace(B.csa2_sparse_attn_workspace_size(2, h, k, w), cuda_device)
+    B.csa2_sparse_attn_decode(q.to(cuda_device), 1, kv, d(topk), d(swa), swa_rows, d(begin), d(end), w, scale, o,
+                              lse, ws)
+    torch.cuda.synchronize()
+    assert B.csa2_device_status() == 1  # CSA2_DEVERR_BAD_ROW
+    go = o.float().cpu().numpy()
+    o0, _ = oracle.sparse_attn(bf16_bits(q[0]), codes, scales, pt[0], ps, topk[0], swa[0][0:w], scale)
+    o1, _ = oracle.sparse_attn(bf16_bits(q[1]), codes, scales, pt[1], ps, topk[1], None, scale)
+    assert attn_excess(go[0], o0) <= 1.0
+    assert attn_excess(go[1], o1) <= 1.0
+
+
+def test_query_outside_f16_range_is_reported(B, cuda_device):
+    # q is converted to f16 for the tensor-core products: a value whose
+    # magnitude rounds beyond f16's largest finite value sets
+    # CSA2_DEVERR_Q_RANGE; the other queries are unaffected
+    rng = np.random.default_rng(32)
+    lens, ps, h, k = [1500, 1500], 64, 16, 128
+    pt, cap, codes, scales = _cache(rng, lens, ps, 32)
+    topk = np.stack([rng.permutation(1500)[:k].astype(np.int32) for _ in range(2)])
+    q = synth.normal_bf16(32, 3, 0, 2 * h * 512).view(2, h, 512).clone()
+    q[1, 3, 17] = 70000.0
+    scale = 1.0 / math.sqrt(512)
+    kv = kv_from_numpy(codes, scales, None, pt, lens, ps, cuda_device)
+    o = torch.full((2, h, 512), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.full((2, h), float("nan"), dtype=torch.float32, device=cuda_device)
+    ws = B.workspace(B.csa2_sparse_attn_workspace_size(2, h, k, 0), cuda_device)
+    B.csa2_sparse_attn_decode(q.to(cuda_device), 1, kv, torch.from_numpy(topk).to(cuda_device), None, 0, None, None,
+                              0, scale, o, lse, ws)
+    torch.cuda.synchronize()
+    assert B.csa2_device_status() == 8  # CSA2_DEVERR_Q_RANGE
+    o0, _ = oracle.sparse_attn(bf16_bits(q[0]), codes, scales, pt[0], ps, topk[0], None, scale)
+    assert attn_excess(o.float().cpu().numpy()[0], o0) <= 1.0

@@ -184,3 +184,46 @@ def test_reindex_ties_and_short_pool(B, cuda_device):
     torch.cuda.synchronize()
     g = out2.cpu().numpy()[0]
     assert sorted(g[:9]) == sorted(pool[0][pool[0] >= 0]) and list(g[9:]) == [-1, -1, -1]
+
+
+# ---- many queries of one sequence: the batched path (16 queries per key tile
+# with up to 4 indexer heads, 8 with up to 8), chosen for 64 or more queries
+# per sequence without a pool ----
+def _causal(total, nqs, first=None):
+    first = total - nqs if first is None else first
+    return [min(total, first + j + 1) for j in range(nqs)]
+
+
+def test_full_batched_causal_di64(B, cuda_device):
+    total = 5000
+    _run_full(B, cuda_device, [total], 5120, 64, 4, 300, 0, q_per_seq=64, q_limit=_causal(total, 64), seed=21,
+              shuffle=False)
+
+
+def test_full_batched_two_sequences_paged_di128(B, cuda_device):
+    # two sequences of 64 queries each, eight indexer heads (8 queries per
+    # tile), a shuffled 64-entry page table; each query sees all of its sequence
+    _run_full(B, cuda_device, [3000, 2600], 64, 128, 8, 400, 0, q_per_seq=64, seed=22)
+
+
+def test_full_batched_limits_below_k(B, cuda_device):
+    # the first queries see fewer entries than k: all of them, then -1 padding
+    total = 2000
+    _run_full(B, cuda_device, [total], 2048, 64, 3, 500, 0, q_per_seq=128, q_limit=_causal(total, 128, first=100),
+              seed=23, shuffle=False)
+
+
+def test_full_batched_all_ties(B, cuda_device):
+    same = lambda cap, di: np.full((cap, di), 0x38, np.uint8)  # every key = 1.0
+    topk, _, _ = _run_full(B, cuda_device, [3000], 3072, 64, 4, 700, 0, q_per_seq=64, kidx_fn=same, seed=24,
+                           shuffle=False)
+    for qi in range(64):
+        assert list(topk[qi]) == list(range(700))
+
+
+def test_full_batched_largest_dot_products(B, cuda_device):
+    def extreme(cap, di):
+        rng = np.random.default_rng(25)
+        v = np.where(rng.random((cap, di)) < 0.97, 8.0, -8.0).astype(np.float32)
+        return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    _run_full(B, cuda_device, [4000], 4096, 128, 8, 333, 0, q_per_seq=64, kidx_fn=extreme, seed=25, shuffle=False)

@@ -131,3 +131,9 @@ def test_host_validation_of_shard_and_variant_calls(binding):
     assert L.csa2_select_keys(0x1000, 1, (1 << 20) + 1, 8, 0x2000, None) == 2
     assert L.csa2_select_keys(0x1000, 1, 64, 0, 0x2000, None) == 1
     assert L.csa2_select_keys(0x1004, 1, 64, 8, 0x2000, None) == 1
+
+
+def test_wait_selfcheck_limits_refused_on_host(binding):
+    L = binding._lib
+    assert L.csa2_check_wait_timeout(0, None) == 1
+    assert L.csa2_check_wait_timeout(1000001, None) == 1
