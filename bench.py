@@ -371,12 +371,14 @@ class Clocks:
         self.error = None
 
     def _nvml_handle(self):
+        """NVML handle of this process's CUDA device: by UUID (NVML does not
+        follow CUDA_VISIBLE_DEVICES), else by index."""
         import pynvml
         import torch
         pynvml.nvmlInit()
         try:
-            bus = torch.cuda.get_device_properties(self.device).pci_bus_id
-            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
         except Exception:
             return pynvml.nvmlDeviceGetHandleByIndex(int(self.device.index or 0))
 
@@ -563,16 +565,29 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 def graph_kernel_nodes(g):
     """Kernel nodes of a captured CUDA graph (the library's kernels: the step
-    graph holds nothing else), or None if the graph cannot be inspected."""
+    graph holds nothing else), counted through the driver API, or None if the
+    graph cannot be inspected."""
+    import ctypes
     try:
-        from cuda.bindings import runtime as rt
-        h = g.raw_cuda_graph()
-        err, _, n = rt.cudaGraphGetNodes(h, 0)
-        if err != rt.cudaError_t.cudaSuccess:
+        cuda = ctypes.CDLL("libcuda.so.1")
+        cuda.cuGraphGetNodes.restype = ctypes.c_int
+        cuda.cuGraphGetNodes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]
+        cuda.cuGraphNodeGetType.restype = ctypes.c_int
+        cuda.cuGraphNodeGetType.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+        h = ctypes.c_void_p(int(g.raw_cuda_graph()))
+        n = ctypes.c_size_t(0)
+        if cuda.cuGraphGetNodes(h, None, ctypes.byref(n)) != 0:
             return None
-        err, nodes, n = rt.cudaGraphGetNodes(h, n)
-        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
-        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+        nodes = (ctypes.c_void_p * max(1, n.value))()
+        if cuda.cuGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+            return None
+        kernels = 0
+        for i in range(n.value):
+            t = ctypes.c_int(-1)
+            if cuda.cuGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) != 0:
+                return None
+            kernels += t.value == 0  # CU_GRAPH_NODE_TYPE_KERNEL
+        return kernels
     except Exception:
         return None
 
@@ -915,6 +930,8 @@ def run_e2e(args, dec, stream, flush, world, dev):
 
 
 def main():
+    import faulthandler
+    faulthandler.enable()  # a crash in native code prints the Python stack
     args = parse()
     if args.impl == "reference":
         run_reference(args)

@@ -151,7 +151,8 @@ csa2_status csa2_append_kidx_e4m3(const void *x_bf16, int32_t n, const int32_t *
  * order and padded with -1 when fewer entries are visible; topk is a subset
  * of pool. Scores are exact (hence the ids bit-exact) whenever every
  * partial sum is an integer below 2^24, as with small-integer E4M3 data.
- * Requires 1 <= hi <= 16, di in {64, 128}, 1 <= k, 0 <= p, k <= p if p > 0.
+ * Requires 1 <= hi <= 16, di in {64, 128}, 1 <= k <= 8192, 0 <= p <= 8192,
+ * k <= p if p > 0 (CSA2_ERR_UNSUPPORTED for larger ranks).
  * ws: at least csa2_index_full_workspace_size(nq, n_max) bytes.
  */
 csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq,

@@ -625,18 +625,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
             const bool whole = seg_start == u * p.tpq && x == (u + 1) * p.tpq - 1;
             int32_t slot = 0;
             if (!whole) slot = sp.slot(g, u, part_base);
-            // o (bf16 or f32) or the f32 partial of this segment, one latent chunk
-            // at a time as its P*V completes, into the KV tile (free once the
-            // chunk's product is done) as [h][128] rows, then out by bulk copies
+            // o (bf16 or f32) or the f32 partial of this segment: once the last
+            // P*V is done the whole KV tile is free; O / l goes there as [h][512]
+            // rows (the layout of the destination), then out in four bulk copies
             const bool f32 = !whole || p.o32 != nullptr;
             const int es = f32 ? 4 : 2;
             if (soft) {
                 const int d0 = quarter * 32 + lane;
+                // the commit of the last chunk follows every product of the tile
+                if (ok && !mbar_wait(&bar_pv[3], (uint32_t)i & 1u)) ok = false;
+                tc_fence_after();
 #pragma unroll 1
                 for (int dc = 0; dc < 4; ++dc) {
                     uint32_t vals[HG];
-                    if (ok && !mbar_wait(&bar_pv[dc], (uint32_t)i & 1u)) ok = false;
-                    tc_fence_after();
                     const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + grp * HG;
                     if (HG == 16) {
                         tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&vals[0]));
@@ -644,18 +645,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
                         tmem_ld8(ta, *reinterpret_cast<uint32_t(*)[8]>(&vals[0]));
                     }
                     tmem_wait_ld();
-                    uint8_t *stg = kv_tile + dc * 32768;
                     if (f32) {
 #pragma unroll
                         for (int j = 0; j < HG; ++j) {
                             const int h = grp * HG + j;
-                            reinterpret_cast<float *>(stg)[h * 128 + d0] = __uint_as_float(vals[j]) * alpha[h];
+                            reinterpret_cast<float *>(kv_tile)[h * CSA2_D + dc * 128 + d0] =
+                                __uint_as_float(vals[j]) * alpha[h];
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < HG; ++j) {
                             const int h = grp * HG + j;
-                            reinterpret_cast<uint16_t *>(stg)[h * 128 + d0] =
+                            reinterpret_cast<uint16_t *>(kv_tile)[h * CSA2_D + dc * 128 + d0] =
                                 f32_to_bf16_bits(__uint_as_float(vals[j]) * alpha[h]);
                         }
                     }
@@ -665,16 +666,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
             tc_fence_before();
             named_bar_sync(kBarWork, kDecWorkThreads);
             if (warp == 0) {
-                // 4 * H row pieces of 128 values, spread over the lanes
                 uint8_t *dst = whole ? (p.o32 ? reinterpret_cast<uint8_t *>(p.o32 + u * H * CSA2_D)
                                               : reinterpret_cast<uint8_t *>(p.o + u * H * CSA2_D))
                                      : reinterpret_cast<uint8_t *>(p.o_part + (int64_t)slot * H * CSA2_D);
-                for (int r = lane; r < 4 * H; r += 32) {
-                    const int dc = r / H, h = r % H;
-                    bulk_store(dst + ((int64_t)h * CSA2_D + dc * 128) * es, kv_tile + dc * 32768 + h * 128 * es,
-                               (uint32_t)(128 * es));
+                const uint32_t quarter_bytes = (uint32_t)(H * CSA2_D * es / 4);
+                if (lane < 4) {
+                    bulk_store(dst + lane * quarter_bytes, kv_tile + lane * quarter_bytes, quarter_bytes);
+                    bulk_commit();
                 }
-                bulk_commit();
                 if (!whole && seg_start == u * p.tpq && lane == 0) p.qslot[u] = slot;  // the first part of u
             }
             tc_fence_before();

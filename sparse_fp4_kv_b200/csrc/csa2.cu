@@ -59,6 +59,17 @@ FullPath full_path_env() {
 }
 bool force_multipass() { return full_path_env() == kPathMultipass; }
 
+// The one-launch Reindex (one CTA per query) is kept as an alternative
+// behind CSA2_REINDEX=fused: its gathers run on one SM per query and measured
+// slower than the two-launch path, which spreads them over the whole GPU.
+bool reindex_fused_enabled() {
+    static const bool v = [] {
+        const char *e = std::getenv("CSA2_REINDEX");
+        return e != nullptr && std::strcmp(e, "fused") == 0;
+    }();
+    return v;
+}
+
 int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -126,40 +137,84 @@ bool make_kidx_map(CUtensorMap *tm, const csa2_kv_desc *kv, int box_rows) {
 // ---- Full indexer workspace ------------------------------------------------
 struct FullLayout {
     int64_t key_stride;
-    int32_t n_sel_chunks;
-    size_t off_keys, off_hist0, off_hist1, off_hist2, off_state, off_cnt, total;
-    size_t b_hist, b_state, b_sure, b_cand;  // batched path
-    int64_t b_cap;
+    int64_t c_chunk;       // keys per collecting CTA (part) of the multi-launch path
+    int32_t c_parts;       // parts per query
+    int32_t c_sure_stride;
+    size_t off_keys, off_hist0, off_state, off_cnt, off_sure, off_cand, total;
+    size_t b_hist, b_state, b_cnt, b_sure, b_cand;  // batched path
 };
+
+// Split of the batched Full path: query groups of qg queries, chunks of
+// whole tiles per group (one CTA each, about one CTA per SM in total). The
+// workspace is sized with the bound over both group sizes (qg = 8 or 16) and
+// both tile sizes (128 or 256 entries).
+struct BatchSplit {
+    int64_t nchunks, chunk;          // for a given qg and tile size
+    int64_t max_chunks, max_span;    // bounds over every qg and tile size of chunks and chunks * chunk
+};
+BatchSplit batch_split(int32_t nq, int64_t n_max, int tile_entries, int sms, int qg = 16) {
+    BatchSplit s{};
+    auto one = [&](int q, int te, int64_t &nch, int64_t &chunk) {
+        const int64_t ngroups = (nq + q - 1) / q;
+        const int64_t tiles = std::max<int64_t>(1, (n_max + te - 1) / te);
+        nch = std::max<int64_t>(1, std::min<int64_t>(tiles, std::min<int64_t>(kBatchMaxChunks, sms / ngroups)));
+        chunk = (tiles + nch - 1) / nch * te;
+    };
+    one(qg, tile_entries, s.nchunks, s.chunk);
+    s.max_chunks = 0;
+    s.max_span = 0;
+    for (int q : {8, 16})
+        for (int te : {128, 256}) {
+            int64_t a, c;
+            one(q, te, a, c);
+            s.max_chunks = std::max(s.max_chunks, a);
+            s.max_span = std::max(s.max_span, a * c);
+        }
+    return s;
+}
+
+// Parts of the multi-launch path's selection: about two collecting CTAs per
+// SM over all queries, parts of whole 2048-key steps, at most
+// kBatchMaxChunks parts per query.
+void collect_split(int32_t nq, int64_t n_max, int sms, int64_t &chunk, int32_t &parts) {
+    const int64_t n = std::max<int64_t>(n_max, 1);
+    chunk = std::max<int64_t>((int64_t)nq * n / (2 * sms), (n + kBatchMaxChunks - 1) / kBatchMaxChunks);
+    chunk = std::max<int64_t>(2048, (chunk + 2047) / 2048 * 2048);
+    parts = (int32_t)((n + chunk - 1) / chunk);
+}
 
 FullLayout full_layout(int32_t nq, int64_t n_max) {
     FullLayout L{};
     L.key_stride = (int64_t)align_up((size_t)std::max<int64_t>(n_max, 1), 128);
-    L.n_sel_chunks = (int32_t)((std::max<int64_t>(n_max, 1) + kSelChunk - 1) / kSelChunk);
+    collect_split(nq, n_max, num_sms(), L.c_chunk, L.c_parts);
+    L.c_sure_stride = (int32_t)std::min<int64_t>(kBatchMaxK, L.c_chunk);  // a part holds < rank sure ids
     size_t off = 0;
     L.off_keys = off;
     off = align_up(off + (size_t)nq * L.key_stride * 4, 256);
     L.off_hist0 = off;
     off = align_up(off + (size_t)nq * kHist0Bins * 4, 256);
-    L.off_hist1 = off;
-    off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
-    L.off_hist2 = off;
-    off = align_up(off + (size_t)nq * 2 * kHistBins * 4, 256);
     L.off_state = off;
     off = align_up(off + (size_t)nq * kStateWords * 4, 256);
     L.off_cnt = off;
-    off = align_up(off + (size_t)nq * 2 * L.n_sel_chunks * 2 * 4, 256);
-    // the batched path's region (the same bytes: one path runs per call)
+    off = align_up(off + (size_t)nq * L.c_parts * 2 * 4, 256);
+    L.off_sure = off;
+    off = align_up(off + (size_t)nq * L.c_parts * L.c_sure_stride * 4, 256);
+    L.off_cand = off;
+    off = align_up(off + (size_t)nq * L.c_parts * L.c_chunk * 8, 256);
+    // the batched path's region (the same bytes: one path runs per call),
+    // sized for its largest split: chunks per query group, entries per chunk
+    const BatchSplit bs = batch_split(nq, n_max, 256, num_sms());
     size_t b = 0;
     L.b_hist = b;
     b = align_up(b + (size_t)nq * kBatchBins * 4, 256);
     L.b_state = b;
-    b = align_up(b + (size_t)nq * 4 * 4, 256);
+    b = align_up(b + (size_t)nq * 2 * 4, 256);
+    L.b_cnt = b;
+    b = align_up(b + (size_t)nq * bs.max_chunks * 2 * 4, 256);
     L.b_sure = b;
-    b = align_up(b + (size_t)nq * kBatchMaxK * 4, 256);
+    b = align_up(b + (size_t)nq * bs.max_chunks * kBatchMaxK * 4, 256);
     L.b_cand = b;
-    L.b_cap = std::max<int64_t>(n_max, 1);
-    b = align_up(b + (size_t)nq * L.b_cap * 8, 256);
+    b = align_up(b + (size_t)nq * bs.max_span * 8, 256);
     L.total = std::max(off, b);
     return L;
 }
@@ -456,8 +511,7 @@ bool prefer_shared(K kernel) {
 bool init_small_kernels() {
     static const char key = 0;
     return once_per_device(&key, [] {
-        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_hist<1>) &&
-               prefer_shared(k_sel_hist<2>) && prefer_shared(k_sel_count) && prefer_shared(k_sel_emit) &&
+        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) &&
                prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
                prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
                prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
@@ -565,6 +619,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
         return CSA2_ERR_INVALID_ARG;
     if (hi < 1 || hi > kScanN) return CSA2_ERR_UNSUPPORTED;
     if (k < 1 || p < 0 || (p > 0 && p < k) || n_max < 0) return CSA2_ERR_INVALID_ARG;
+    if (k > kBatchMaxK || p > kBatchMaxK) return CSA2_ERR_UNSUPPORTED;
     if (n_max > (int64_t)kv->max_pages * kv->page_size) return CSA2_ERR_INVALID_ARG;
     if (!qidx || !w || !topk || !aligned(qidx, 16) || !aligned(w, 4) || !aligned(topk, 4))
         return CSA2_ERR_INVALID_ARG;
@@ -600,22 +655,25 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
             bp.kv = *kv;
             bp.hist = reinterpret_cast<uint32_t *>(wsb + L.b_hist);
             bp.state = reinterpret_cast<uint32_t *>(wsb + L.b_state);
+            bp.state_stride = 2;
+            bp.state_off = 0;
+            bp.cnt = reinterpret_cast<uint32_t *>(wsb + L.b_cnt);
             bp.sure = reinterpret_cast<int32_t *>(wsb + L.b_sure);
             bp.cand = reinterpret_cast<unsigned long long *>(wsb + L.b_cand);
             bp.topk = topk;
-            bp.cap = L.b_cap;
             bp.k = k;
+            bp.sure_stride = k;
             bp.q_per_seq = q_per_seq;
             bp.hi = hi;
             bp.hi_pad = hp;
             bp.nq = nq;
             bp.box_rows = box_rows;
             const int ngroups = (nq + qg - 1) / qg;
-            const int64_t tiles = std::max<int64_t>(1, (n_max + tile_entries - 1) / tile_entries);
-            const int64_t nchunks = std::max<int64_t>(1, std::min<int64_t>(tiles, num_sms() / ngroups));
-            bp.chunk = (tiles + nchunks - 1) / nchunks * tile_entries;
+            const BatchSplit bsp = batch_split(nq, n_max, tile_entries, num_sms(), qg);
+            bp.chunk = bsp.chunk;
+            bp.nchunks = (int32_t)((std::max<int64_t>(n_max, 1) + bp.chunk - 1) / bp.chunk);
             if (bp.chunk / kv->page_size + 2 > kMaxScanPages) return CSA2_ERR_UNSUPPORTED;
-            const dim3 sgrid((unsigned)((std::max<int64_t>(n_max, 1) + bp.chunk - 1) / bp.chunk), (unsigned)ngroups);
+            const dim3 sgrid((unsigned)bp.nchunks, (unsigned)ngroups);
             if (cudaMemsetAsync(bp.hist, 0, (size_t)nq * kBatchBins * 4, stream) != cudaSuccess) return CSA2_ERR_CUDA;
             auto scan = [&](auto k0, auto k1, size_t sm0, size_t sm1) -> csa2_status {
                 if (!smem_attr(k0, sm0) || !smem_attr(k1, sm1)) return CSA2_ERR_CUDA;
@@ -640,7 +698,8 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
             if (bs != CSA2_OK) return bs;
             const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
             if (!smem_attr(k_batch_final, fsm)) return CSA2_ERR_CUDA;
-            const size_t ffixed = 2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + (size_t)kBatchMaxK * 4;
+            const size_t ffixed =
+                2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + 4 * kBatchMaxChunks * 4 + (size_t)kBatchMaxK * 4;
             const int32_t smem_keys = (int32_t)((fsm - ffixed) / 8);
             launch(k_batch_final, dim3((unsigned)nq), dim3(kBatchFinalThreads), fsm, stream, bp, smem_keys);
             return check_launch();
@@ -707,8 +766,11 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sp.hi = hi;
     sp.box_rows = box_rows;
     const int64_t tiles_max = std::max<int64_t>(1, (n_max + tile_entries - 1) / tile_entries);
-    const int64_t target = (int64_t)num_sms() * 2;  // about two resident CTAs per SM, one wave
-    int64_t chunk = std::max<int64_t>(4, ((int64_t)nq * tiles_max + target - 1) / target);
+    // several waves of two resident CTAs per SM when every query had n_max
+    // entries: queries of ragged lengths then leave short CTAs behind instead
+    // of a few long ones, and the hardware scheduler evens the SMs out
+    const int64_t target = (int64_t)num_sms() * 2 * 4;
+    int64_t chunk = std::max<int64_t>(16, ((int64_t)nq * tiles_max + target - 1) / target);
     chunk = std::min<int64_t>(chunk, 256);
     chunk = std::min<int64_t>(chunk, std::max<int64_t>(1, ((int64_t)(kMaxScanPages - 2) * kv->page_size) / tile_entries));
     sp.chunk_tiles = (int32_t)chunk;
@@ -722,26 +784,36 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     }
     if ((st = check_launch()) != CSA2_OK) return st;
 
-    SelParams sel{};
-    sel.keys = sp.keys;
-    sel.q_limit = q_limit;
-    sel.kv = *kv;
-    sel.state = sp.state;
-    sel.hist1 = reinterpret_cast<uint32_t *>(wsb + L.off_hist1);
-    sel.hist2 = reinterpret_cast<uint32_t *>(wsb + L.off_hist2);
-    sel.cnt = reinterpret_cast<uint32_t *>(wsb + L.off_cnt);
-    sel.out[0] = topk;
-    sel.out[1] = pool;
-    sel.rank[0] = k;
-    sel.rank[1] = p;
-    sel.key_stride = L.key_stride;
-    sel.q_per_seq = q_per_seq;
-    sel.n_chunks = L.n_sel_chunks;
-    const dim3 grid((unsigned)L.n_sel_chunks, (unsigned)nq);
-    launch(k_sel_hist<1>, dim3(grid), dim3(kSelThreads), 0, stream, sel);
-    launch(k_sel_hist<2>, dim3(grid), dim3(kSelThreads), 0, stream, sel);
-    launch(k_sel_count, dim3(grid), dim3(kSelThreads), 0, stream, sel);
-    launch(k_sel_emit, dim3(grid), dim3(kSelThreads), 0, stream, sel);
+    // per target (Top-K, then the pool): collect each query's sure ids and
+    // threshold-bin candidates in parts, then the exact select and sort of
+    // the batched path
+    BatchParams cp{};
+    cp.q_limit = q_limit;
+    cp.kv = *kv;
+    cp.state = sp.state;
+    cp.state_stride = kStateWords;
+    cp.cnt = reinterpret_cast<uint32_t *>(wsb + L.off_cnt);
+    cp.sure = reinterpret_cast<int32_t *>(wsb + L.off_sure);
+    cp.cand = reinterpret_cast<unsigned long long *>(wsb + L.off_cand);
+    cp.chunk = L.c_chunk;
+    cp.nchunks = L.c_parts;
+    cp.sure_stride = L.c_sure_stride;
+    cp.q_per_seq = q_per_seq;
+    cp.nq = nq;
+    const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
+    if (!smem_attr(k_batch_final, fsm)) return CSA2_ERR_CUDA;
+    const size_t ffixed = 2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + 4 * kBatchMaxChunks * 4 + (size_t)kBatchMaxK * 4;
+    const int32_t smem_keys = (int32_t)((fsm - ffixed) / 8);
+    for (int tau = 0; tau < 2; ++tau) {
+        const int32_t rank = tau == 0 ? k : p;
+        if (rank <= 0) continue;
+        cp.state_off = 8 * tau;
+        cp.k = rank;
+        cp.topk = tau == 0 ? topk : pool;
+        launch(k_sel_collect, dim3((unsigned)L.c_parts, (unsigned)nq), dim3(kCollectThreads), 0, stream, cp,
+               (const uint32_t *)sp.keys, L.key_stride, rank);
+        launch(k_batch_final, dim3((unsigned)nq), dim3(kBatchFinalThreads), fsm, stream, cp, smem_keys);
+    }
     return check_launch();
 }
 
@@ -776,11 +848,11 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     rp.k = k;
     rp.hi = hi;
     rp.q_per_seq = q_per_seq;
-    // one launch per query when its pool's keys fit shared memory (always up to
-    // the largest pool the call accepts); the two-launch path otherwise
+    // one launch per query (CSA2_REINDEX=fused, when its pool's keys fit shared
+    // memory); by default the two-launch path
     {
         const size_t fsm = kv->di == 64 ? RfCfg<64>::smem(p) : RfCfg<128>::smem(p);
-        if (fsm + 1024 <= (size_t)max_smem_optin() && !force_multipass()) {
+        if (fsm + 1024 <= (size_t)max_smem_optin() && reindex_fused_enabled()) {
             if (kv->di == 64) {
                 if (!smem_attr(k_reindex_fused<64>, (size_t)max_smem_optin() - 1024)) return CSA2_ERR_CUDA;
                 launch(k_reindex_fused<64>, dim3((unsigned)nq), dim3(kRfThreads), fsm, stream, rp);

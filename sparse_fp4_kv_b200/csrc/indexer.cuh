@@ -22,10 +22,12 @@
 // of every score and histogram its top 12 bits. HBM-bound: di bytes per
 // entry.
 //
-// Selection: exact radix select on the 32-bit key in three digits
-// (12 + 10 + 10 bits) with global histograms, then an ordered emission in
-// which equal keys are taken in ascending id order, so the output lists are
-// sorted by id. Reindex (indexer_fused.cuh) keeps the pool's 64-bit keys
+// Selection (indexer_batch.cuh): the scan's last CTA of a query finds the
+// digit-0 bin of each target rank; k_sel_collect then splits the query's
+// keys into ids certainly selected and candidates in that bin, and
+// k_batch_final selects among the candidates on the unique 64-bit key
+// (score key, ~id), so equal scores go to the lower id, and sorts the ids.
+// Reindex (indexer_fused.cuh) keeps the pool's 64-bit keys
 // (score key, ~id), which are unique, in shared memory.
 #pragma once
 
@@ -37,10 +39,6 @@ constexpr int kScanTile = 128;
 constexpr int kScanThreads = 192;
 constexpr int kScanN = 16;  // MMA N: indexer heads padded to 16
 constexpr int kHist0Bins = 4096;
-constexpr int kHistBins = 1024;
-constexpr int kSelThreads = 512;
-constexpr int kSelChunk = 8192;  // entries per selection CTA
-constexpr int kSelPer = kSelChunk / kSelThreads;
 
 // Scan geometry. The indexer keys reach the tensor cores as 128-byte
 // shared-memory rows (128B swizzle). With di = 64 a row holds two
@@ -477,218 +475,6 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_consta
                 p.state[(int64_t)qi * kStateWords + 8 * tau + 0] = bin;
                 p.state[(int64_t)qi * kStateWords + 8 * tau + 1] = rem;
             }
-        }
-    }
-}
-
-struct SelParams {
-    const uint32_t *keys;
-    const int32_t *q_limit;
-    csa2_kv_desc kv;
-    uint32_t *hist1;  // [nq][2][1024]
-    uint32_t *hist2;  // [nq][2][1024]
-    uint32_t *cnt;    // [nq][2][n_chunks][2]
-    uint32_t *state;  // [nq][kStateWords]
-    int32_t *out[2];  // topk [nq][k], pool [nq][p]
-    int32_t rank[2];  // k, p (0 = no pool)
-    int64_t key_stride;
-    int32_t q_per_seq;
-    int32_t n_chunks;
-};
-
-// A target needs a threshold only when fewer than all visible entries are
-// asked for; otherwise every visible entry is taken.
-__device__ __forceinline__ bool sel_active(const SelParams &p, int tau, int64_t limit) {
-    return p.rank[tau] > 0 && (int64_t)p.rank[tau] < limit;
-}
-
-// The kSelPer consecutive keys t0 .. t0+kSelPer-1 of this thread (64-byte
-// aligned; keys at or beyond `end` read as 0 and must be masked by the
-// caller), loaded with four 16-byte loads in flight together.
-__device__ __forceinline__ void load_key_slice(const uint32_t *keys, int64_t t0, int64_t end,
-                                               uint32_t (&k)[kSelPer]) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(keys + t0);
-    uint4 v[kSelPer / 4];
-#pragma unroll
-    for (int i = 0; i < kSelPer / 4; ++i) v[i] = t0 + 4 * i < end ? __ldcg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int i = 0; i < kSelPer / 4; ++i) {
-        k[4 * i + 0] = v[i].x;
-        k[4 * i + 1] = v[i].y;
-        k[4 * i + 2] = v[i].z;
-        k[4 * i + 3] = v[i].w;
-    }
-}
-
-// PASS 1: histogram of digit 1 (bits 19..10) among keys whose digit 0 is the
-// threshold bin; PASS 2: digit 2 (bits 9..0) among keys matching digits 0
-// and 1. The last CTA of each query then locates the next threshold digit.
-template <int PASS>
-__global__ void __launch_bounds__(kSelThreads) k_sel_hist(SelParams p) {
-    pdl_trigger();
-    pdl_wait();
-    __shared__ uint32_t nh[2][kHistBins];
-    __shared__ uint32_t scratch[kSelThreads / 32 + 4];
-    const int32_t qi = blockIdx.y;
-    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
-    const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
-    if (c0 >= limit) return;
-    const int64_t c1 = min(limit, c0 + kSelChunk);
-    const uint32_t *st = p.state + (int64_t)qi * kStateWords;
-    bool act[2];
-    uint32_t b0[2], b1[2];
-    for (int tau = 0; tau < 2; ++tau) {
-        act[tau] = sel_active(p, tau, limit);
-        b0[tau] = act[tau] ? __ldcg(st + 8 * tau + 0) : 0u;
-        b1[tau] = act[tau] ? __ldcg(st + 8 * tau + 2) : 0u;
-    }
-    if (!act[0] && !act[1]) return;
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += kSelThreads) (&nh[0][0])[i] = 0u;
-    __syncthreads();
-    const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
-    const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
-    uint32_t kreg[kSelPer];
-    load_key_slice(keys, s0, c1, kreg);
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j) {
-        const uint32_t key = kreg[j];
-        const bool in = s0 + j < c1;
-#pragma unroll
-        for (int tau = 0; tau < 2; ++tau) {
-            if (!act[tau]) continue;
-            bool match = in && (key >> 20) == b0[tau];
-            if (PASS == 2) match = match && ((key >> 10) & 1023u) == b1[tau];
-            hist_add_warp(nh[tau], match ? (PASS == 1 ? (key >> 10) & 1023u : key & 1023u) : 0xFFFFFFFFu);
-        }
-    }
-    __syncthreads();
-    uint32_t *dst = (PASS == 1 ? p.hist1 : p.hist2) + (int64_t)qi * 2 * kHistBins;
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += kSelThreads) {
-        const uint32_t v = (&nh[0][0])[i];
-        if (v) atomicAdd(&dst[i], v);
-    }
-    const uint32_t n_part = (uint32_t)((limit + kSelChunk - 1) / kSelChunk);
-    if (last_block(p.state + (int64_t)qi * kStateWords + kCtrScan + PASS, n_part, scratch + kSelThreads / 32 + 3)) {
-        uint32_t *stw = p.state + (int64_t)qi * kStateWords;
-        for (int tau = 0; tau < 2; ++tau) {
-            if (!act[tau]) continue;
-            const uint32_t r = __ldcg(stw + 8 * tau + (PASS == 1 ? 1 : 3));
-            uint32_t bin, rem;
-            find_rank_bin<kSelThreads, kHistBins / kSelThreads, true>(dst + tau * kHistBins, kHistBins, r, scratch, bin, rem);
-            if (threadIdx.x == 0) {
-                if (PASS == 1) {
-                    stw[8 * tau + 2] = bin;
-                    stw[8 * tau + 3] = rem;
-                } else {
-                    stw[8 * tau + 4] = bin;
-                    stw[8 * tau + 5] = rem;
-                    stw[8 * tau + 6] = (b0[tau] << 20) | (b1[tau] << 10) | bin;
-                }
-            }
-        }
-    }
-}
-
-// Counts, per chunk, the keys above and equal to each target's threshold.
-__global__ void __launch_bounds__(kSelThreads) k_sel_count(SelParams p) {
-    pdl_trigger();
-    pdl_wait();
-    __shared__ uint32_t scratch[kSelThreads / 32 + 4];
-    const int32_t qi = blockIdx.y;
-    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
-    const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
-    const int64_t c1 = min(limit, c0 + kSelChunk);
-    const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
-    const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
-    uint32_t kreg[kSelPer];
-    if (sel_active(p, 0, limit) || sel_active(p, 1, limit)) load_key_slice(keys, s0, c1, kreg);
-    for (int tau = 0; tau < 2; ++tau) {
-        if (!sel_active(p, tau, limit)) continue;
-        const uint32_t T = __ldcg(p.state + (int64_t)qi * kStateWords + 8 * tau + 6);
-        uint32_t gt = 0, eq = 0;
-#pragma unroll
-        for (int j = 0; j < kSelPer; ++j) {
-            const bool in = s0 + j < c1;
-            gt += in && kreg[j] > T;
-            eq += in && kreg[j] == T;
-        }
-        uint32_t tgt, teq;
-        block_excl_scan<kSelThreads>(gt, scratch, &tgt);
-        block_excl_scan<kSelThreads>(eq, scratch, &teq);
-        if (threadIdx.x == 0) {
-            uint32_t *c = p.cnt + (((int64_t)qi * 2 + tau) * p.n_chunks + blockIdx.x) * 2;
-            c[0] = tgt;
-            c[1] = teq;
-        }
-    }
-}
-
-// Writes the selected ids of each target in ascending id order.
-__global__ void __launch_bounds__(kSelThreads) k_sel_emit(SelParams p) {
-    pdl_trigger();
-    pdl_wait();
-    __shared__ uint32_t scratch[kSelThreads / 32 + 4];
-    const int32_t qi = blockIdx.y;
-    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
-    const int64_t c0 = (int64_t)blockIdx.x * kSelChunk;
-    const int64_t c1 = min(limit, c0 + kSelChunk);
-    const uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
-    // this thread's contiguous slice of the chunk
-    const int64_t s0 = c0 + (int64_t)threadIdx.x * kSelPer;
-    uint32_t kreg[kSelPer];
-    load_key_slice(keys, s0, c1, kreg);
-    for (int tau = 0; tau < 2; ++tau) {
-        const int32_t r_out = p.rank[tau];
-        if (r_out <= 0 || p.out[tau] == nullptr) continue;
-        int32_t *out = p.out[tau] + (int64_t)qi * r_out;
-        if (blockIdx.x == 0) {
-            const int64_t nsel = min((int64_t)r_out, limit);
-            for (int64_t j = nsel + threadIdx.x; j < r_out; j += kSelThreads) out[j] = -1;
-        }
-        if (!sel_active(p, tau, limit)) {
-            // no more visible entries than requested: take every visible entry
-            for (int j = 0; j < kSelPer; ++j)
-                if (s0 + j < c1) out[s0 + j] = (int32_t)(s0 + j);
-            continue;
-        }
-        const uint32_t *st = p.state + (int64_t)qi * kStateWords + 8 * tau;
-        const uint32_t T = __ldcg(st + 6);
-        const uint32_t need = __ldcg(st + 5);
-        // counts of the chunks before this one
-        const uint32_t *cnt = p.cnt + ((int64_t)qi * 2 + tau) * p.n_chunks * 2;
-        uint32_t bgt = 0, beq = 0;
-        for (int c = threadIdx.x; c < (int)blockIdx.x; c += kSelThreads) {
-            bgt += __ldcg(cnt + 2 * c);
-            beq += __ldcg(cnt + 2 * c + 1);
-        }
-        uint32_t base_gt, base_eq;
-        block_excl_scan<kSelThreads>(bgt, scratch, &base_gt);
-        block_excl_scan<kSelThreads>(beq, scratch, &base_eq);
-        uint32_t myeq = 0;
-        for (int j = 0; j < kSelPer; ++j) myeq += (s0 + j < c1) && kreg[j] == T;
-        uint32_t eq_rank = base_eq + block_excl_scan<kSelThreads>(myeq, scratch, nullptr);
-        uint32_t selmask = 0, nsel = 0;
-        for (int j = 0; j < kSelPer; ++j) {
-            if (s0 + j >= c1) break;
-            bool sel = kreg[j] > T;
-            if (kreg[j] == T) {
-                sel = eq_rank < need;
-                ++eq_rank;
-            }
-            if (sel) {
-                selmask |= 1u << j;
-                ++nsel;
-            }
-        }
-        uint32_t pos = base_gt + min(base_eq, need) + block_excl_scan<kSelThreads>(nsel, scratch, nullptr);
-        for (int j = 0; j < kSelPer; ++j) {
-            if (!(selmask & (1u << j))) continue;
-            if (pos < (uint32_t)r_out) {
-                out[pos] = (int32_t)(s0 + j);
-            } else {
-                set_error(CSA2_DEVERR_SELECT);
-            }
-            ++pos;
         }
     }
 }

@@ -23,6 +23,8 @@
 //   3. k_batch_scan<1>: the scores again (the same products, so the same
 //      keys): entries above b0 go to the query's "sure" list, entries in b0
 //      to its candidate list as unique 64-bit keys (score key << 32 | ~id);
+//      every CTA fills its own part of each list (shared-memory counters)
+//      and records how many it wrote;
 //   4. k_batch_final: the needed number of largest candidates by an exact
 //      radix select, merged with the sure ids and sorted ascending.
 #pragma once
@@ -36,7 +38,7 @@ constexpr int kBatchShift = 21;
 constexpr int kBatchEpiWarps = 16;  // 4 per TMEM lane quarter
 constexpr int kBatchThreads = 64 + kBatchEpiWarps * 32;
 constexpr int kBatchFinalThreads = 1024;
-constexpr int kBatchMaxK = 4096;   // ids staged and sorted in shared memory
+constexpr int kBatchMaxK = 8192;   // ids staged and sorted in shared memory
 constexpr uint32_t kBatchAll = 0xFFFFFFFFu;  // b0 marker: every visible entry is taken
 
 struct BatchParams {
@@ -45,12 +47,15 @@ struct BatchParams {
     const int32_t *q_limit;
     csa2_kv_desc kv;
     uint32_t *hist;             // [nq][kBatchBins]
-    uint32_t *state;            // [nq][4]: b0, rem, n_sure, n_cand
-    int32_t *sure;              // [nq][k]
-    unsigned long long *cand;   // [nq][cap]
-    int32_t *topk;              // [nq][k]
-    int64_t cap;
-    int64_t chunk;              // entries per CTA (a multiple of the tile)
+    uint32_t *state;            // b0, rem of query qi at state[qi * state_stride + state_off + 0 / 1]
+    int32_t state_stride, state_off;
+    int32_t *sure;              // [nq][nchunks][sure_stride]: ids above b0 found by each CTA (part)
+    unsigned long long *cand;   // [nq][nchunks][chunk]: keys in b0 found by each part
+    uint32_t *cnt;              // [nq][nchunks][2]: how many of each
+    int32_t *topk;              // [nq][k]: the selected ids, ascending, -1 padded
+    int64_t chunk;              // entries per part
+    int32_t nchunks;            // parts per query (gridDim.x of the collecting kernel)
+    int32_t sure_stride;        // >= min(k, chunk): a part holds fewer than k sure ids
     int32_t k, q_per_seq, hi, hi_pad, nq, box_rows;
 };
 
@@ -87,7 +92,7 @@ struct BatchCfg {
     static constexpr int kStages = PASS == 0 ? 4 : 8;
     static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128u : 256u;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * G::kStageBytes + (size_t)N * 128 +
-                                    (PASS == 0 ? (size_t)QG * kBatchBins * 4 : 0) + 16 * 16 * 4 + 16 * 4 * 2 +
+                                    (PASS == 0 ? (size_t)QG * kBatchBins * 4 : 0) + 16 * 16 * 4 + 16 * 4 * 4 +
                                     (size_t)kMaxScanPages * 4 + 256;
 };
 
@@ -107,7 +112,8 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
     float *wq = reinterpret_cast<float *>(hist + (PASS == 0 ? QG * kBatchBins : 0));  // [16][16]
     int32_t *lim = reinterpret_cast<int32_t *>(wq + 16 * 16);                 // [16]
     uint32_t *b0s = reinterpret_cast<uint32_t *>(lim + 16);                   // [16] (PASS 1)
-    int32_t *ptab = reinterpret_cast<int32_t *>(b0s + 16);                    // [kMaxScanPages]
+    uint32_t *lcnt = b0s + 16;                                                // [16][2] (PASS 1)
+    int32_t *ptab = reinterpret_cast<int32_t *>(lcnt + 32);                   // [kMaxScanPages]
     uint64_t *full_b = reinterpret_cast<uint64_t *>(ptab + kMaxScanPages);
     uint64_t *empty_b = full_b + kStages;
     uint64_t *tfull = empty_b + kStages;
@@ -167,7 +173,10 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
         const int32_t qi = q0 + j;
         wq[i] = (qi < p.nq && h < p.hi) ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
     }
-    if (PASS == 1 && tid < QG) b0s[tid] = q0 + tid < p.nq ? __ldcg(p.state + (int64_t)(q0 + tid) * 4) : 0u;
+    if (PASS == 1 && tid < QG) {
+        b0s[tid] = q0 + tid < p.nq ? __ldcg(p.state + (int64_t)(q0 + tid) * p.state_stride + p.state_off) : 0u;
+        lcnt[2 * tid] = lcnt[2 * tid + 1] = 0u;
+    }
     if (ntiles > 0) stage_pages(p.kv, b, start, n_loc, ptab, kBatchThreads);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -241,26 +250,27 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
                         const uint32_t ms = __ballot_sync(0xFFFFFFFFu, sure);
                         const uint32_t mc = __ballot_sync(0xFFFFFFFFu, cand);
                         const uint32_t lt = (1u << lane) - 1u;
+                        const int64_t part = (int64_t)qi * p.nchunks + blockIdx.x;  // this CTA's part
                         if (ms) {
                             uint32_t base0 = 0;
-                            if (lane == 0) base0 = atomicAdd(p.state + (int64_t)qi * 4 + 2, (uint32_t)__popc(ms));
+                            if (lane == 0) base0 = atomicAdd(&lcnt[2 * j], (uint32_t)__popc(ms));
                             base0 = __shfl_sync(0xFFFFFFFFu, base0, 0);
                             if (sure) {
                                 const uint32_t at = base0 + __popc(ms & lt);
-                                if (at < (uint32_t)p.k)
-                                    p.sure[(int64_t)qi * p.k + at] = (int32_t)t;
+                                if (at < (uint32_t)p.sure_stride)
+                                    p.sure[part * p.sure_stride + at] = (int32_t)t;
                                 else
                                     set_error(CSA2_DEVERR_SELECT);
                             }
                         }
                         if (mc) {
                             uint32_t base0 = 0;
-                            if (lane == 0) base0 = atomicAdd(p.state + (int64_t)qi * 4 + 3, (uint32_t)__popc(mc));
+                            if (lane == 0) base0 = atomicAdd(&lcnt[2 * j + 1], (uint32_t)__popc(mc));
                             base0 = __shfl_sync(0xFFFFFFFFu, base0, 0);
                             if (cand) {
                                 const uint32_t at = base0 + __popc(mc & lt);
-                                if ((int64_t)at < p.cap)
-                                    p.cand[(int64_t)qi * p.cap + at] =
+                                if ((int64_t)at < p.chunk)
+                                    p.cand[part * p.chunk + at] =
                                         ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)t);
                                 else
                                     set_error(CSA2_DEVERR_SELECT);
@@ -279,6 +289,11 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, tcols);
+    }
+    if (PASS == 1 && tid < QG && q0 + tid < p.nq) {
+        uint32_t *c = p.cnt + ((int64_t)(q0 + tid) * p.nchunks + blockIdx.x) * 2;
+        c[0] = min(lcnt[2 * tid], (uint32_t)p.sure_stride);
+        c[1] = lcnt[2 * tid + 1];
     }
     if (PASS == 0) {
         for (int i = tid; i < QG * kBatchBins; i += kBatchThreads) {
@@ -304,27 +319,30 @@ __global__ void __launch_bounds__(kBatchThreshThreads) k_batch_thresh(BatchParam
         find_rank_bin<kBatchThreshThreads, kBatchBins / kBatchThreshThreads, true>(
             p.hist + (int64_t)qi * kBatchBins, kBatchBins, (uint32_t)p.k, scratch, bin, rem);
     if (threadIdx.x == 0) {
-        uint32_t *st = p.state + (int64_t)qi * 4;
+        uint32_t *st = p.state + (int64_t)qi * p.state_stride + p.state_off;
         st[0] = bin;
         st[1] = rem;
-        st[2] = 0u;
-        st[3] = 0u;
     }
 }
 
-// Per query: the rem largest of its n_cand candidate keys (unique 64-bit
-// keys, kept in shared memory when they fit, else re-read from L2 in every
-// radix pass), merged with its sure ids, sorted ascending, padded with -1.
+// Per query: the rem largest of its candidate keys (unique 64-bit keys, in
+// the parts its group's CTAs wrote; copied into shared memory when they fit,
+// else re-read from those parts through L2 in every radix pass), merged with
+// its sure ids, sorted ascending, padded with -1.
+constexpr int kBatchMaxChunks = 256;
 __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchParams p, int32_t smem_keys) {
     constexpr int NT = kBatchFinalThreads;
     extern __shared__ uint8_t smem_raw[];
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);            // [2048]
-    uint32_t *scratch = hist + 2048;                                    // [NT/32 + 8]
-    int32_t *ids = reinterpret_cast<int32_t *>(scratch + NT / 32 + 8);   // [kBatchMaxK]
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);              // [2048]
+    uint32_t *scratch = hist + 2048;                                      // [NT/32 + 8]
+    uint32_t *pcnt = scratch + NT / 32 + 8;                               // [kBatchMaxChunks][2]
+    uint32_t *poff = pcnt + 2 * kBatchMaxChunks;                          // [kBatchMaxChunks][2] exclusive prefixes
+    int32_t *ids = reinterpret_cast<int32_t *>(poff + 2 * kBatchMaxChunks);  // [kBatchMaxK]
     unsigned long long *k64 = reinterpret_cast<unsigned long long *>(ids + kBatchMaxK);  // [smem_keys]
     __shared__ unsigned long long and_acc, or_acc;
-    __shared__ uint32_t n_out;
+    __shared__ uint32_t n_out, tot[2];
     const int32_t qi = blockIdx.x;
+    const int nch = min(p.nchunks, kBatchMaxChunks);
     pdl_trigger();
     if (threadIdx.x == 0) {
         and_acc = ~0ull;
@@ -332,24 +350,55 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
         n_out = 0u;
     }
     pdl_wait();
-    const uint32_t *st = p.state + (int64_t)qi * 4;
-    const uint32_t b0 = __ldcg(st), need = __ldcg(st + 1);
-    const uint32_t n_sure = min(__ldcg(st + 2), (uint32_t)p.k);
-    const uint32_t n_cand = (uint32_t)min((int64_t)__ldcg(st + 3), p.cap);
-    const unsigned long long *src = p.cand + (int64_t)qi * p.cap;
+    for (int c = threadIdx.x; c < nch; c += NT) {
+        const uint32_t *cc = p.cnt + ((int64_t)qi * p.nchunks + c) * 2;
+        pcnt[2 * c] = __ldcg(cc);
+        pcnt[2 * c + 1] = __ldcg(cc + 1);
+    }
     __syncthreads();
+    if (threadIdx.x < 2) {
+        uint32_t acc = 0;
+        for (int c = 0; c < nch; ++c) {
+            poff[2 * c + threadIdx.x] = acc;
+            acc += pcnt[2 * c + threadIdx.x];
+        }
+        tot[threadIdx.x] = acc;
+    }
+    __syncthreads();
+    const uint32_t *stq = p.state + (int64_t)qi * p.state_stride + p.state_off;
+    const uint32_t b0 = __ldcg(stq), need = __ldcg(stq + 1);
+    const uint32_t n_sure = min(tot[0], (uint32_t)p.k);
+    const uint32_t n_cand = tot[1];
     // the sure ids first
-    for (uint32_t j = threadIdx.x; j < n_sure; j += NT) ids[j] = p.sure[(int64_t)qi * p.k + j];
+    for (int c = 0; c < nch; ++c) {
+        const int32_t *src = p.sure + ((int64_t)qi * p.nchunks + c) * p.sure_stride;
+        for (uint32_t j = threadIdx.x; j < pcnt[2 * c]; j += NT)
+            if (poff[2 * c] + j < n_sure) ids[poff[2 * c] + j] = src[j];
+    }
     uint32_t take = 0;
     if (b0 != kBatchAll && need > 0 && n_cand > 0) {
         take = min(need, n_cand);
-        const bool G = n_cand > (uint32_t)smem_keys;  // candidates re-read from L2 in every pass
+        const bool G = n_cand > (uint32_t)smem_keys;  // re-read the parts from L2 in every pass
+        // fn(key) over every candidate, each once, spread over the threads
+        auto each = [&](auto fn) {
+            if (!G) {
+                for (uint32_t j = threadIdx.x; j < n_cand; j += NT) fn(k64[j]);
+            } else {
+                for (int c = 0; c < nch; ++c) {
+                    const unsigned long long *src = p.cand + ((int64_t)qi * p.nchunks + c) * p.chunk;
+                    for (uint32_t j = threadIdx.x; j < pcnt[2 * c + 1]; j += NT) fn(__ldcg(src + j));
+                }
+            }
+        };
         unsigned long long a_loc = ~0ull, o_loc = 0ull;
-        for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
-            const unsigned long long v = __ldcg(src + j);
-            if (!G) k64[j] = v;
-            a_loc &= v;
-            o_loc |= v;
+        for (int c = 0; c < nch; ++c) {
+            const unsigned long long *src = p.cand + ((int64_t)qi * p.nchunks + c) * p.chunk;
+            for (uint32_t j = threadIdx.x; j < pcnt[2 * c + 1]; j += NT) {
+                const unsigned long long v = __ldcg(src + j);
+                if (!G) k64[poff[2 * c + 1] + j] = v;
+                a_loc &= v;
+                o_loc |= v;
+            }
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) {
@@ -361,17 +410,12 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
             atomicOr(&or_acc, o_loc);
         }
         __syncthreads();
-        auto key = [&](uint32_t j) -> unsigned long long { return G ? __ldcg(src + j) : k64[j]; };
         unsigned long long T = 0ull;  // take the keys >= T
         if (take < n_cand) {
             const unsigned long long diff = and_acc ^ or_acc;  // keys are unique: diff != 0
             int top = 63 - __clzll((long long)diff);
-            unsigned long long prefix = and_acc & ~((2ull << top) - 1ull);
-            unsigned long long pmask = ~((2ull << top) - 1ull);
-            if (top == 63) {
-                prefix = 0ull;
-                pmask = 0ull;
-            }
+            unsigned long long prefix = top == 63 ? 0ull : (and_acc & ~((2ull << top) - 1ull));
+            unsigned long long pmask = top == 63 ? 0ull : ~((2ull << top) - 1ull);
             uint32_t rem = take;
             while (true) {
                 const int nbits = top + 1 < 11 ? top + 1 : 11;
@@ -379,10 +423,9 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
                 const int nb = 1 << nbits;
                 for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
                 __syncthreads();
-                for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
-                    const unsigned long long v = key(j);
+                each([&](unsigned long long v) {
                     if ((v & pmask) == prefix) atomicAdd(&hist[(uint32_t)(v >> shift) & (uint32_t)(nb - 1)], 1u);
-                }
+                });
                 __syncthreads();
                 uint32_t bin, inbin;
                 find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
@@ -398,8 +441,7 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
             }
             T = prefix | (and_acc & ~diff & ~pmask);
         }
-        for (uint32_t j = threadIdx.x; j < n_cand; j += NT) {
-            const unsigned long long v = key(j);
+        each([&](unsigned long long v) {
             if (v >= T) {
                 const uint32_t at = n_sure + atomicAdd(&n_out, 1u);
                 if (at < (uint32_t)kBatchMaxK && at < (uint32_t)p.k)
@@ -407,7 +449,7 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
                 else
                     set_error(CSA2_DEVERR_SELECT);
             }
-        }
+        });
     }
     __syncthreads();
     const uint32_t total = min(n_sure + min(n_out, take), (uint32_t)p.k);
@@ -433,6 +475,88 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
     }
     int32_t *out = p.topk + (int64_t)qi * p.k;
     for (int j = threadIdx.x; j < p.k; j += NT) out[j] = j < (int)total ? ids[j] : -1;
+}
+
+// ---------------------------------------------------------------------------
+// Selection of the multi-launch Full path (one query per sequence, its score
+// keys in the workspace after k_index_scan): part c of query qi reads keys
+// [c * part, (c + 1) * part) of the query's visible range; keys whose
+// digit 0 (top 12 bits) is above the target's threshold bin go to the
+// part's sure list, keys in the bin to its candidates, as in the batched
+// path, whose k_batch_final then selects and sorts. Every key is read once
+// per target.
+// ---------------------------------------------------------------------------
+constexpr int kCollectThreads = 512;
+
+__global__ void __launch_bounds__(kCollectThreads) k_sel_collect(BatchParams p, const uint32_t *keys,
+                                                                 int64_t key_stride, int32_t rank) {
+    __shared__ uint32_t lcnt[2];
+    pdl_trigger();
+    if (threadIdx.x < 2) lcnt[threadIdx.x] = 0u;
+    pdl_wait();
+    const int32_t qi = blockIdx.y;
+    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+    const bool all = (int64_t)rank >= limit;  // every visible entry is taken
+    uint32_t *stq = p.state + (int64_t)qi * p.state_stride + p.state_off;
+    const uint32_t b0 = all ? kBatchAll : __ldcg(stq);
+    if (all && blockIdx.x == 0 && threadIdx.x == 0) {
+        stq[0] = kBatchAll;
+        stq[1] = 0u;
+    }
+    __syncthreads();
+    const int64_t c0 = (int64_t)blockIdx.x * p.chunk;
+    const int64_t c1 = min(limit, c0 + p.chunk);
+    const int64_t part = (int64_t)qi * p.nchunks + blockIdx.x;
+    const uint32_t *kq = keys + (int64_t)qi * key_stride;
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    // 4 consecutive keys per thread and step (one 16-byte load); the trip
+    // count is the same for every thread (warp-wide ballots inside)
+    for (int64_t base4 = c0; base4 < c1; base4 += 4 * kCollectThreads) {
+        const int64_t t0 = base4 + 4 * threadIdx.x;
+        const uint4 k4 = t0 < c1 ? __ldcg(reinterpret_cast<const uint4 *>(kq + t0)) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t t = t0 + j;
+            const bool in = t < c1;
+            const uint32_t d = kk[j] >> 20;
+            const bool sure = in && (all || d > b0);
+            const bool cand = in && !all && d == b0;
+            const uint32_t ms = __ballot_sync(0xFFFFFFFFu, sure);
+            const uint32_t mc = __ballot_sync(0xFFFFFFFFu, cand);
+            if (ms) {
+                uint32_t b = 0;
+                if (lane == 0) b = atomicAdd(&lcnt[0], (uint32_t)__popc(ms));
+                b = __shfl_sync(0xFFFFFFFFu, b, 0);
+                if (sure) {
+                    const uint32_t at = b + __popc(ms & lt);
+                    if (at < (uint32_t)p.sure_stride)
+                        p.sure[part * p.sure_stride + at] = (int32_t)t;
+                    else
+                        set_error(CSA2_DEVERR_SELECT);
+                }
+            }
+            if (mc) {
+                uint32_t b = 0;
+                if (lane == 0) b = atomicAdd(&lcnt[1], (uint32_t)__popc(mc));
+                b = __shfl_sync(0xFFFFFFFFu, b, 0);
+                if (cand) {
+                    const uint32_t at = b + __popc(mc & lt);
+                    if ((int64_t)at < p.chunk)
+                        p.cand[part * p.chunk + at] = ((unsigned long long)kk[j] << 32) | (unsigned long long)(~(uint32_t)t);
+                    else
+                        set_error(CSA2_DEVERR_SELECT);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t *c = p.cnt + part * 2;
+        c[0] = min(lcnt[0], (uint32_t)p.sure_stride);
+        c[1] = lcnt[1];
+    }
 }
 
 }  // namespace csa2

@@ -1,7 +1,7 @@
 """The Full indexer has two complete implementations: a single launch per
 query cluster (used whenever a query's entries fit its shared memory) and a
-multi-launch path (scan + radix passes through global memory, used for
-longer sequences). This runs the Full-indexer parity tests once more with
+multi-launch path (scan, then per target a collecting pass and a per-query
+select, used for longer sequences). This runs the Full-indexer parity tests once more with
 the multi-launch path forced (CSA2_FULL_PATH=multipass, read by the library
 at load time, hence the separate process); there the score keys left in the
 workspace are also compared with the oracle's exact scores."""
