@@ -59,13 +59,13 @@ FullPath full_path_env() {
 }
 bool force_multipass() { return full_path_env() == kPathMultipass; }
 
-// The one-launch Reindex (one CTA per query) is kept as an alternative
-// behind CSA2_REINDEX=fused: its gathers run on one SM per query and measured
-// slower than the two-launch path, which spreads them over the whole GPU.
-bool reindex_fused_enabled() {
+// CSA2_REINDEX=two: the two-launch Reindex (scores to global memory, then a
+// select CTA per query) even where the one-launch cluster path applies
+// (tests of both paths, tuning).
+bool reindex_two_launch() {
     static const bool v = [] {
         const char *e = std::getenv("CSA2_REINDEX");
-        return e != nullptr && std::strcmp(e, "fused") == 0;
+        return e != nullptr && std::strcmp(e, "two") == 0;
     }();
     return v;
 }
@@ -140,7 +140,7 @@ struct FullLayout {
     int64_t c_chunk;       // keys per collecting CTA (part) of the multi-launch path
     int32_t c_parts;       // parts per query
     int32_t c_sure_stride;
-    size_t off_keys, off_hist0, off_state, off_cnt, off_sure, off_cand, total;
+    size_t off_keys, off_hist0, off_state, off_hist1, off_cnt, off_sure, off_cand, total;
     size_t b_hist, b_state, b_cnt, b_sure, b_cand;  // batched path
 };
 
@@ -195,6 +195,8 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
     off = align_up(off + (size_t)nq * kHist0Bins * 4, 256);
     L.off_state = off;
     off = align_up(off + (size_t)nq * kStateWords * 4, 256);
+    L.off_hist1 = off;  // [2 targets][nq][2048]
+    off = align_up(off + (size_t)2 * nq * 2048 * 4, 256);
     L.off_cnt = off;
     off = align_up(off + (size_t)nq * L.c_parts * 2 * 4, 256);
     L.off_sure = off;
@@ -335,7 +337,7 @@ struct DecPlan {
 DecPlan plan_decode(int32_t nq, int32_t h, int32_t k, int32_t w_max, int sms) {
     DecPlan P{};
     const int64_t rows = (int64_t)k + std::max(0, w_max);
-    P.tpq = (int32_t)std::max<int64_t>(1, (rows + kAttnTile - 1) / kAttnTile);
+    P.tpq = (int32_t)std::max<int64_t>(1, (rows + kDecRows - 1) / kDecRows);
     const int64_t T = (int64_t)nq * P.tpq;
     int64_t per = (T + sms - 1) / sms;
     if (const char *e = std::getenv("CSA2_ATTN_PER")) per = std::max<int64_t>(1, std::atoll(e));  // tuning, tests
@@ -798,6 +800,8 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     cp.chunk = L.c_chunk;
     cp.nchunks = L.c_parts;
     cp.sure_stride = L.c_sure_stride;
+    cp.shift1 = kCollectShift1;
+    cp.parts_sorted = 1;
     cp.q_per_seq = q_per_seq;
     cp.nq = nq;
     const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
@@ -808,6 +812,7 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
         const int32_t rank = tau == 0 ? k : p;
         if (rank <= 0) continue;
         cp.state_off = 8 * tau;
+        cp.hist1 = reinterpret_cast<uint32_t *>(wsb + L.off_hist1) + (size_t)tau * nq * 2048;
         cp.k = rank;
         cp.topk = tau == 0 ? topk : pool;
         launch(k_sel_collect, dim3((unsigned)L.c_parts, (unsigned)nq), dim3(kCollectThreads), 0, stream, cp,
@@ -848,20 +853,21 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     rp.k = k;
     rp.hi = hi;
     rp.q_per_seq = q_per_seq;
-    // one launch per query (CSA2_REINDEX=fused, when its pool's keys fit shared
-    // memory); by default the two-launch path
-    {
-        const size_t fsm = kv->di == 64 ? RfCfg<64>::smem(p) : RfCfg<128>::smem(p);
-        if (fsm + 1024 <= (size_t)max_smem_optin() && reindex_fused_enabled()) {
-            if (kv->di == 64) {
-                if (!smem_attr(k_reindex_fused<64>, (size_t)max_smem_optin() - 1024)) return CSA2_ERR_CUDA;
-                launch(k_reindex_fused<64>, dim3((unsigned)nq), dim3(kRfThreads), fsm, stream, rp);
-            } else {
-                if (!smem_attr(k_reindex_fused<128>, (size_t)max_smem_optin() - 1024)) return CSA2_ERR_CUDA;
-                launch(k_reindex_fused<128>, dim3((unsigned)nq), dim3(kRfThreads), fsm, stream, rp);
-            }
-            return check_launch();
+    // one launch: a cluster of CTAs per query scores the pool into the first
+    // CTA's shared memory, which selects; pools of more than 8 * 1024 ids take
+    // the two-launch path
+    const int cl = (p + kRcThreads - 1) / kRcThreads;
+    if (cl <= kRcMaxCluster && !reindex_two_launch()) {
+        const size_t rsm = 2048 * 4 + (kRcThreads / 32 + 8) * 4 + (size_t)p * 8;
+        const dim3 rgrid((unsigned)cl, (unsigned)nq);
+        if (kv->di == 64) {
+            if (!smem_attr(k_reindex_cluster<64>, (size_t)max_smem_optin())) return CSA2_ERR_CUDA;
+            launch_cluster(k_reindex_cluster<64>, rgrid, dim3(kRcThreads), rsm, stream, (unsigned)cl, rp);
+        } else {
+            if (!smem_attr(k_reindex_cluster<128>, (size_t)max_smem_optin())) return CSA2_ERR_CUDA;
+            launch_cluster(k_reindex_cluster<128>, rgrid, dim3(kRcThreads), rsm, stream, (unsigned)cl, rp);
         }
+        return check_launch();
     }
     const dim3 grid((unsigned)((p + kReindexScoreThreads - 1) / kReindexScoreThreads), (unsigned)nq);
     if (kv->di == 64)
@@ -897,8 +903,14 @@ void launch_combine(int32_t h, int32_t nq, const CombineArgs &ca, cudaStream_t s
 }
 
 template <int H>
-void launch_decode(const DecParams &dp, const DecPlan &P, bool out_f32, cudaStream_t stream) {
-    launch(k_attn_decode<H>, dim3((unsigned)P.ctas), dim3(kDecThreads), DecCfg<H>::kSmem, stream, dp);
+csa2_status launch_decode(const DecParams &dp, const DecPlan &P, bool out_f32, cudaStream_t stream) {
+    // the merge reads slot numbers the decode kernel writes: it is not
+    // launched after a failed launch of that kernel
+    if (launch(k_attn_decode<H>, dim3((unsigned)P.ctas), dim3(kDecThreads), DecCfg<H>::kSmem, stream, dp) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return CSA2_ERR_CUDA;
+    }
     if (P.slots > 0) {
         const dim3 mgrid((unsigned)H, (unsigned)dp.nq);
         if (out_f32)
@@ -906,6 +918,7 @@ void launch_decode(const DecParams &dp, const DecPlan &P, bool out_f32, cudaStre
         else
             launch(k_attn_merge_parts<H, false>, mgrid, dim3(kMergeThreads), 0, stream, dp);
     }
+    return CSA2_OK;
 }
 
 // The exact decode attention (arguments already checked by attn_impl):
@@ -938,18 +951,19 @@ csa2_status decode_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32
     dp.nq = nq;
     dp.tpq = P.tpq;
     dp.per = P.per;
+    dp.nslots = P.slots;
     switch (h) {
         case 64:
             if (!smem_attr(k_attn_decode<64>, DecCfg<64>::kSmem)) return CSA2_ERR_CUDA;
-            launch_decode<64>(dp, P, out_f32, stream);
+            if (launch_decode<64>(dp, P, out_f32, stream) != CSA2_OK) return CSA2_ERR_CUDA;
             break;
         case 32:
             if (!smem_attr(k_attn_decode<32>, DecCfg<32>::kSmem)) return CSA2_ERR_CUDA;
-            launch_decode<32>(dp, P, out_f32, stream);
+            if (launch_decode<32>(dp, P, out_f32, stream) != CSA2_OK) return CSA2_ERR_CUDA;
             break;
         default:
             if (!smem_attr(k_attn_decode<16>, DecCfg<16>::kSmem)) return CSA2_ERR_CUDA;
-            launch_decode<16>(dp, P, out_f32, stream);
+            if (launch_decode<16>(dp, P, out_f32, stream) != CSA2_OK) return CSA2_ERR_CUDA;
             break;
     }
     return check_launch();

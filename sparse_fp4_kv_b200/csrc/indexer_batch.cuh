@@ -56,6 +56,9 @@ struct BatchParams {
     int64_t chunk;              // entries per part
     int32_t nchunks;            // parts per query (gridDim.x of the collecting kernel)
     int32_t sure_stride;        // >= min(k, chunk): a part holds fewer than k sure ids
+    uint32_t *hist1;            // [nq][2048] digit-1 histogram of the candidates, or null
+    int32_t shift1;             // digit 1 = bits shift1 .. shift1 + 10 of the score key
+    int32_t parts_sorted;       // every part's lists are in ascending id order
     int32_t k, q_per_seq, hi, hi_pad, nq, box_rows;
 };
 
@@ -326,10 +329,45 @@ __global__ void __launch_bounds__(kBatchThreshThreads) k_batch_thresh(BatchParam
 }
 
 // Per query: the rem largest of its candidate keys (unique 64-bit keys, in
-// the parts its group's CTAs wrote; copied into shared memory when they fit,
-// else re-read from those parts through L2 in every radix pass), merged with
-// its sure ids, sorted ascending, padded with -1.
+// the parts the collecting CTAs wrote; copied into shared memory when they
+// fit, else re-read from those parts through L2 in every radix pass), merged
+// with its sure ids in ascending order, padded with -1. Parts are read with
+// flattened indices (a binary search over the parts' offsets), so that every
+// thread's loads are in flight at once whatever the number of parts. With a
+// digit-1 histogram of the candidates (p.hist1), the radix select starts
+// below digit 1. With p.parts_sorted, every part lists its ids in ascending
+// order and the parts cover ascending id ranges, so the sure ids and the
+// taken candidates are two sorted runs that are merged; otherwise they are
+// sorted (bitonic) in shared memory.
 constexpr int kBatchMaxChunks = 256;
+
+// Largest part c in [0, nch) whose exclusive offset poff[2c + w] is <= j:
+// the part holding flattened item j.
+__device__ __forceinline__ int find_part(const uint32_t *poff, int nch, int w, uint32_t j) {
+    int lo = 0, hi = nch - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (poff[2 * mid + w] <= j)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Number of elements of the ascending run a[0..n) below x.
+__device__ __forceinline__ uint32_t count_below(const int32_t *a, uint32_t n, int32_t x) {
+    uint32_t lo = 0, hi = n;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (a[mid] < x)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchParams p, int32_t smem_keys) {
     constexpr int NT = kBatchFinalThreads;
     extern __shared__ uint8_t smem_raw[];
@@ -337,23 +375,23 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
     uint32_t *scratch = hist + 2048;                                      // [NT/32 + 8]
     uint32_t *pcnt = scratch + NT / 32 + 8;                               // [kBatchMaxChunks][2]
     uint32_t *poff = pcnt + 2 * kBatchMaxChunks;                          // [kBatchMaxChunks][2] exclusive prefixes
-    int32_t *ids = reinterpret_cast<int32_t *>(poff + 2 * kBatchMaxChunks);  // [kBatchMaxK]
+    int32_t *ids = reinterpret_cast<int32_t *>(poff + 2 * kBatchMaxChunks);  // [kBatchMaxK]: sure, then taken
     unsigned long long *k64 = reinterpret_cast<unsigned long long *>(ids + kBatchMaxK);  // [smem_keys]
     __shared__ unsigned long long and_acc, or_acc;
-    __shared__ uint32_t n_out, tot[2];
+    __shared__ uint32_t tot[2];
     const int32_t qi = blockIdx.x;
     const int nch = min(p.nchunks, kBatchMaxChunks);
     pdl_trigger();
     if (threadIdx.x == 0) {
         and_acc = ~0ull;
         or_acc = 0ull;
-        n_out = 0u;
     }
     pdl_wait();
     for (int c = threadIdx.x; c < nch; c += NT) {
+        // clamped to the parts' capacities: no read outside them whatever the counts say
         const uint32_t *cc = p.cnt + ((int64_t)qi * p.nchunks + c) * 2;
-        pcnt[2 * c] = __ldcg(cc);
-        pcnt[2 * c + 1] = __ldcg(cc + 1);
+        pcnt[2 * c] = min(__ldcg(cc), (uint32_t)p.sure_stride);
+        pcnt[2 * c + 1] = (uint32_t)min((int64_t)__ldcg(cc + 1), p.chunk);
     }
     __syncthreads();
     if (threadIdx.x < 2) {
@@ -369,35 +407,60 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
     const uint32_t b0 = __ldcg(stq), need = __ldcg(stq + 1);
     const uint32_t n_sure = min(tot[0], (uint32_t)p.k);
     const uint32_t n_cand = tot[1];
-    // the sure ids first
-    for (int c = 0; c < nch; ++c) {
-        const int32_t *src = p.sure + ((int64_t)qi * p.nchunks + c) * p.sure_stride;
-        for (uint32_t j = threadIdx.x; j < pcnt[2 * c]; j += NT)
-            if (poff[2 * c] + j < n_sure) ids[poff[2 * c] + j] = src[j];
+    const int64_t part0 = (int64_t)qi * p.nchunks;
+    // the sure ids first, flattened over the parts
+    for (uint32_t j0 = threadIdx.x; j0 < n_sure; j0 += 4 * NT) {
+        int32_t v[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t j = j0 + r * NT;
+            v[r] = 0;
+            if (j < n_sure) {
+                const int c = find_part(poff, nch, 0, j);
+                v[r] = __ldcg(p.sure + (part0 + c) * p.sure_stride + (j - poff[2 * c]));
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            if (j0 + r * NT < n_sure) ids[j0 + r * NT] = v[r];
     }
+    // candidate j, flattened over the parts
+    auto cand_at = [&](uint32_t j) -> unsigned long long {
+        const int c = find_part(poff, nch, 1, j);
+        return __ldcg(p.cand + (part0 + c) * p.chunk + (j - poff[2 * c + 1]));
+    };
     uint32_t take = 0;
+    const bool G = n_cand > (uint32_t)smem_keys;  // re-read the parts from L2 in every pass
     if (b0 != kBatchAll && need > 0 && n_cand > 0) {
         take = min(need, n_cand);
-        const bool G = n_cand > (uint32_t)smem_keys;  // re-read the parts from L2 in every pass
-        // fn(key) over every candidate, each once, spread over the threads
+        // fn(key) over every candidate, each once, four loads in flight per thread
         auto each = [&](auto fn) {
             if (!G) {
                 for (uint32_t j = threadIdx.x; j < n_cand; j += NT) fn(k64[j]);
             } else {
-                for (int c = 0; c < nch; ++c) {
-                    const unsigned long long *src = p.cand + ((int64_t)qi * p.nchunks + c) * p.chunk;
-                    for (uint32_t j = threadIdx.x; j < pcnt[2 * c + 1]; j += NT) fn(__ldcg(src + j));
+                for (uint32_t j0 = threadIdx.x; j0 < n_cand; j0 += 4 * NT) {
+                    unsigned long long v[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) v[r] = j0 + r * NT < n_cand ? cand_at(j0 + r * NT) : 0ull;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        if (j0 + r * NT < n_cand) fn(v[r]);
                 }
             }
         };
         unsigned long long a_loc = ~0ull, o_loc = 0ull;
-        for (int c = 0; c < nch; ++c) {
-            const unsigned long long *src = p.cand + ((int64_t)qi * p.nchunks + c) * p.chunk;
-            for (uint32_t j = threadIdx.x; j < pcnt[2 * c + 1]; j += NT) {
-                const unsigned long long v = __ldcg(src + j);
-                if (!G) k64[poff[2 * c + 1] + j] = v;
-                a_loc &= v;
-                o_loc |= v;
+        for (uint32_t j0 = threadIdx.x; j0 < n_cand; j0 += 4 * NT) {
+            unsigned long long v[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) v[r] = j0 + r * NT < n_cand ? cand_at(j0 + r * NT) : 0ull;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t j = j0 + r * NT;
+                if (j < n_cand) {
+                    if (!G) k64[j] = v[r];
+                    a_loc &= v[r];
+                    o_loc |= v[r];
+                }
             }
         }
 #pragma unroll
@@ -417,7 +480,23 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
             unsigned long long prefix = top == 63 ? 0ull : (and_acc & ~((2ull << top) - 1ull));
             unsigned long long pmask = top == 63 ? 0ull : ~((2ull << top) - 1ull);
             uint32_t rem = take;
-            while (true) {
+            bool done = false;
+            if (p.hist1 != nullptr) {
+                // digits 0 and 1 of the key's top word from the collecting pass's
+                // histogram of the candidates' digit 1
+                uint32_t b1, r1;
+                find_rank_bin<NT, 2048 / NT, true>(p.hist1 + (int64_t)qi * 2048, 2048, take, scratch, b1, r1);
+                const int lo = 32 + p.shift1;
+                pmask = ~0ull << lo;
+                prefix = (and_acc & pmask & ~(2047ull << lo)) | ((unsigned long long)b1 << lo);
+                rem = r1;
+                const unsigned long long below = diff & ((1ull << lo) - 1ull);
+                if (below == 0ull)
+                    done = true;
+                else
+                    top = 63 - __clzll((long long)below);
+            }
+            while (!done) {
                 const int nbits = top + 1 < 11 ? top + 1 : 11;
                 const int shift = top + 1 - nbits;
                 const int nb = 1 << nbits;
@@ -441,18 +520,61 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
             }
             T = prefix | (and_acc & ~diff & ~pmask);
         }
-        each([&](unsigned long long v) {
-            if (v >= T) {
-                const uint32_t at = n_sure + atomicAdd(&n_out, 1u);
-                if (at < (uint32_t)kBatchMaxK && at < (uint32_t)p.k)
-                    ids[at] = (int32_t)(~(uint32_t)v);
-                else
-                    set_error(CSA2_DEVERR_SELECT);
+        // the taken candidates after the sure ids: in candidate order (each
+        // thread a contiguous run) when the parts are sorted
+        const uint32_t per = (n_cand + NT - 1) / NT;
+        const uint32_t j0 = min(n_cand, threadIdx.x * per), j1 = min(n_cand, j0 + per);
+        // fn(key) over candidates j0 .. j1-1 in order; from L2 eight loads at a
+        // time, the part index walked forward
+        auto run = [&](auto fn) {
+            if (!G) {
+                for (uint32_t j = j0; j < j1; ++j) fn(k64[j]);
+                return;
             }
+            int c = j0 < j1 ? find_part(poff, nch, 1, j0) : 0;
+            for (uint32_t jb = j0; jb < j1; jb += 8) {
+                unsigned long long v[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const uint32_t j = jb + r;
+                    v[r] = 0ull;
+                    if (j < j1) {
+                        while (c + 1 < nch && poff[2 * (c + 1) + 1] <= j) ++c;
+                        v[r] = __ldcg(p.cand + (part0 + c) * p.chunk + (j - poff[2 * c + 1]));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+                    if (jb + r < j1) fn(v[r]);
+            }
+        };
+        uint32_t mine = 0;
+        run([&](unsigned long long v) { mine += v >= T; });
+        uint32_t pos = n_sure + block_excl_scan<NT>(mine, scratch, nullptr);
+        run([&](unsigned long long v) {
+            if (v < T) return;
+            if (pos < (uint32_t)kBatchMaxK && pos < (uint32_t)p.k)
+                ids[pos] = (int32_t)(~(uint32_t)v);
+            else
+                set_error(CSA2_DEVERR_SELECT);
+            ++pos;
         });
     }
     __syncthreads();
-    const uint32_t total = min(n_sure + min(n_out, take), (uint32_t)p.k);
+    const uint32_t n_take = min(take, (uint32_t)p.k - n_sure);
+    const uint32_t total = n_sure + n_take;
+    int32_t *out = p.topk + (int64_t)qi * p.k;
+    if (p.parts_sorted) {
+        // two ascending runs: ids[0, n_sure) and ids[n_sure, total)
+        for (uint32_t i = threadIdx.x; i < total; i += NT) {
+            const int32_t x = ids[i];
+            const uint32_t at = i < n_sure ? i + count_below(ids + n_sure, n_take, x)
+                                           : (i - n_sure) + count_below(ids, n_sure, x);
+            out[at] = x;
+        }
+        for (int j = (int)total + threadIdx.x; j < p.k; j += NT) out[j] = -1;
+        return;
+    }
     // bitonic sort of the ids ascending (padding above total sorts last)
     int P2 = 1;
     while (P2 < p.k) P2 <<= 1;
@@ -473,26 +595,31 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
             __syncthreads();
         }
     }
-    int32_t *out = p.topk + (int64_t)qi * p.k;
     for (int j = threadIdx.x; j < p.k; j += NT) out[j] = j < (int)total ? ids[j] : -1;
 }
 
 // ---------------------------------------------------------------------------
 // Selection of the multi-launch Full path (one query per sequence, its score
 // keys in the workspace after k_index_scan): part c of query qi reads keys
-// [c * part, (c + 1) * part) of the query's visible range; keys whose
+// [c * chunk, (c + 1) * chunk) of the query's visible range; keys whose
 // digit 0 (top 12 bits) is above the target's threshold bin go to the
-// part's sure list, keys in the bin to its candidates, as in the batched
-// path, whose k_batch_final then selects and sorts. Every key is read once
-// per target.
+// part's sure list, keys in the bin to its candidates (64-bit keys) and to a
+// histogram of their digit 1 (the next 11 bits), as in the batched path,
+// whose k_batch_final then selects and merges. Every key is read once per
+// target; each thread takes 16 consecutive keys per round, and one block
+// scan per round places them, so every part's lists are in ascending id
+// order.
 // ---------------------------------------------------------------------------
 constexpr int kCollectThreads = 512;
+constexpr int kCollectShift1 = 9;  // digit 1: bits 19..9 of the score key
 
 __global__ void __launch_bounds__(kCollectThreads) k_sel_collect(BatchParams p, const uint32_t *keys,
                                                                  int64_t key_stride, int32_t rank) {
-    __shared__ uint32_t lcnt[2];
+    constexpr int NT = kCollectThreads;
+    __shared__ uint32_t h1[2048];
+    __shared__ uint32_t scratch[NT / 32 + 4];
     pdl_trigger();
-    if (threadIdx.x < 2) lcnt[threadIdx.x] = 0u;
+    for (int i = threadIdx.x; i < 2048; i += NT) h1[i] = 0u;
     pdl_wait();
     const int32_t qi = blockIdx.y;
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
@@ -503,59 +630,68 @@ __global__ void __launch_bounds__(kCollectThreads) k_sel_collect(BatchParams p, 
         stq[0] = kBatchAll;
         stq[1] = 0u;
     }
-    __syncthreads();
     const int64_t c0 = (int64_t)blockIdx.x * p.chunk;
     const int64_t c1 = min(limit, c0 + p.chunk);
     const int64_t part = (int64_t)qi * p.nchunks + blockIdx.x;
     const uint32_t *kq = keys + (int64_t)qi * key_stride;
-    const int lane = threadIdx.x & 31;
-    const uint32_t lt = (1u << lane) - 1u;
-    // 4 consecutive keys per thread and step (one 16-byte load); the trip
-    // count is the same for every thread (warp-wide ballots inside)
-    for (int64_t base4 = c0; base4 < c1; base4 += 4 * kCollectThreads) {
-        const int64_t t0 = base4 + 4 * threadIdx.x;
-        const uint4 k4 = t0 < c1 ? __ldcg(reinterpret_cast<const uint4 *>(kq + t0)) : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+    uint32_t n_s = 0, n_c = 0;  // written so far (block-uniform)
+    for (int64_t base = c0; base < c1; base += 16 * NT) {
+        const int64_t t0 = base + 16 * threadIdx.x;
+        uint4 k4[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int64_t t = t0 + j;
-            const bool in = t < c1;
-            const uint32_t d = kk[j] >> 20;
-            const bool sure = in && (all || d > b0);
-            const bool cand = in && !all && d == b0;
-            const uint32_t ms = __ballot_sync(0xFFFFFFFFu, sure);
-            const uint32_t mc = __ballot_sync(0xFFFFFFFFu, cand);
-            if (ms) {
-                uint32_t b = 0;
-                if (lane == 0) b = atomicAdd(&lcnt[0], (uint32_t)__popc(ms));
-                b = __shfl_sync(0xFFFFFFFFu, b, 0);
-                if (sure) {
-                    const uint32_t at = b + __popc(ms & lt);
-                    if (at < (uint32_t)p.sure_stride)
-                        p.sure[part * p.sure_stride + at] = (int32_t)t;
-                    else
-                        set_error(CSA2_DEVERR_SELECT);
-                }
+        for (int r = 0; r < 4; ++r)
+            k4[r] = t0 + 4 * r < c1 ? __ldcg(reinterpret_cast<const uint4 *>(kq + t0 + 4 * r)) : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t ms = 0, mc = 0;  // bit i: key t0 + i is sure / a candidate
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = 4 * r + j;
+                const bool in = t0 + i < c1;
+                const uint32_t d = kk[j] >> 20;
+                ms |= (uint32_t)(in && (all || d > b0)) << i;
+                mc |= (uint32_t)(in && !all && d == b0) << i;
             }
-            if (mc) {
-                uint32_t b = 0;
-                if (lane == 0) b = atomicAdd(&lcnt[1], (uint32_t)__popc(mc));
-                b = __shfl_sync(0xFFFFFFFFu, b, 0);
-                if (cand) {
-                    const uint32_t at = b + __popc(mc & lt);
-                    if ((int64_t)at < p.chunk)
-                        p.cand[part * p.chunk + at] = ((unsigned long long)kk[j] << 32) | (unsigned long long)(~(uint32_t)t);
+        }
+        // counts packed as sure | cand << 16 (each below 2^16 per round)
+        uint32_t tot_r;
+        const uint32_t ex = block_excl_scan<NT>((uint32_t)__popc(ms) | ((uint32_t)__popc(mc) << 16), scratch, &tot_r);
+        uint32_t ps = n_s + (ex & 0xFFFFu), pc = n_c + (ex >> 16);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = 4 * r + j;
+                const int64_t t = t0 + i;
+                if (ms & (1u << i)) {
+                    if (ps < (uint32_t)p.sure_stride)
+                        p.sure[part * p.sure_stride + ps] = (int32_t)t;
                     else
                         set_error(CSA2_DEVERR_SELECT);
+                    ++ps;
+                } else if (mc & (1u << i)) {
+                    if ((int64_t)pc < p.chunk)
+                        p.cand[part * p.chunk + pc] = ((unsigned long long)kk[j] << 32) | (unsigned long long)(~(uint32_t)t);
+                    else
+                        set_error(CSA2_DEVERR_SELECT);
+                    atomicAdd(&h1[(kk[j] >> kCollectShift1) & 2047u], 1u);
+                    ++pc;
                 }
             }
         }
+        n_s += tot_r & 0xFFFFu;
+        n_c += tot_r >> 16;
     }
     __syncthreads();
+    if (p.hist1 != nullptr && n_c > 0)
+        for (int i = threadIdx.x; i < 2048; i += NT)
+            if (h1[i]) atomicAdd(p.hist1 + (int64_t)qi * 2048 + i, h1[i]);
     if (threadIdx.x == 0) {
         uint32_t *c = p.cnt + part * 2;
-        c[0] = min(lcnt[0], (uint32_t)p.sure_stride);
-        c[1] = lcnt[1];
+        c[0] = min(n_s, (uint32_t)p.sure_stride);
+        c[1] = n_c;
     }
 }
 

@@ -368,69 +368,88 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 constexpr int kReindexScoreThreads = 128;
 constexpr int kReindexSelectThreads = 1024;
 
+// Pool slot j of query qi: its id's indexer key row gathered (all its loads
+// in flight before the query is staged by the caller), returned in kv.
+template <int DI>
+__device__ __forceinline__ int32_t reindex_gather(const ReindexParams &p, int32_t qi, int32_t j, uint4 (&kv)[DI / 16]) {
+    const int32_t b = qi / p.q_per_seq;
+    int32_t id = (j < p.p) ? p.pool[(int64_t)qi * p.p + j] : -1;
+    const int64_t row = id >= 0 ? physical_row(p.kv, b, id) : -1;
+    if (id >= 0 && row < 0) {
+        set_error(CSA2_DEVERR_BAD_ROW);
+        id = -1;
+    }
+#pragma unroll
+    for (int c = 0; c < DI / 16; ++c)
+        kv[c] = id >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.kv.kidx + row * DI) + c) : make_uint4(0u, 0u, 0u, 0u);
+    return id;
+}
+
+// The query's heads (E4M3 -> f32) and weights into shared memory.
+template <int DI, int NT>
+__device__ __forceinline__ void reindex_stage_query(const ReindexParams &p, int32_t qi, float *qf, float *wf) {
+    for (int i = threadIdx.x; i < p.hi * DI; i += NT)
+        qf[i] = e4m3x2_to_float2((uint16_t)p.qidx[(int64_t)qi * p.hi * DI + i]).x;
+    if (threadIdx.x < p.hi) wf[threadIdx.x] = p.w[(int64_t)qi * p.hi + threadIdx.x];
+}
+
+// The unique 64-bit key of a gathered row (score key << 32 | ~id), 0 for an
+// empty slot (a valid key has ~id >= 2^31). CUDA-core products, exact for
+// small-integer E4M3 data like the tensor-core path.
+template <int DI>
+__device__ __forceinline__ unsigned long long reindex_key(const ReindexParams &p, int32_t id, const uint4 (&kv)[DI / 16],
+                                                          const float *qf, const float *wf) {
+    if (id < 0) return 0ull;
+    float dot[kScanN];
+#pragma unroll
+    for (int h = 0; h < kScanN; ++h) dot[h] = 0.0f;
+#pragma unroll
+    for (int c = 0; c < DI / 16; ++c) {
+        const uint32_t wv[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
+        float kf[16];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float2 lo = e4m3x2_to_float2((uint16_t)(wv[t] & 0xFFFFu));
+            const float2 hi2 = e4m3x2_to_float2((uint16_t)(wv[t] >> 16));
+            kf[t * 4 + 0] = lo.x;
+            kf[t * 4 + 1] = lo.y;
+            kf[t * 4 + 2] = hi2.x;
+            kf[t * 4 + 3] = hi2.y;
+        }
+#pragma unroll
+        for (int h = 0; h < kScanN; ++h) {
+            if (h >= p.hi) break;
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 q4 = *reinterpret_cast<const float4 *>(&qf[h * DI + c * 16 + i]);
+                dot[h] = fmaf(q4.x, kf[i], dot[h]);
+                dot[h] = fmaf(q4.y, kf[i + 1], dot[h]);
+                dot[h] = fmaf(q4.z, kf[i + 2], dot[h]);
+                dot[h] = fmaf(q4.w, kf[i + 3], dot[h]);
+            }
+        }
+    }
+    float sc = 0.0f;
+#pragma unroll
+    for (int h = 0; h < kScanN; ++h)
+        if (h < p.hi) sc = fmaf(wf[h], fmaxf(dot[h], 0.0f), sc);
+    return ((unsigned long long)score_key(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)(id + p.id_offset));
+}
+
 template <int DI>
 __global__ void __launch_bounds__(kReindexScoreThreads) k_reindex_score(ReindexParams p) {
     __shared__ __align__(16) float qf[kScanN * DI];
     __shared__ float wf[kScanN];
     const int32_t qi = blockIdx.y;
-    const int32_t b = qi / p.q_per_seq;
     pdl_trigger();
     pdl_wait();
     const int32_t j = blockIdx.x * kReindexScoreThreads + threadIdx.x;
-    // this thread's row goes out before the query is staged
-    int32_t id = (j < p.p) ? p.pool[(int64_t)qi * p.p + j] : -1;
-    int64_t row = id >= 0 ? physical_row(p.kv, b, id) : -1;
-    if (id >= 0 && row < 0) {
-        set_error(CSA2_DEVERR_BAD_ROW);
-        id = -1;
-    }
     uint4 kv[DI / 16];
-#pragma unroll
-    for (int c = 0; c < DI / 16; ++c)
-        kv[c] = row >= 0 ? __ldg(reinterpret_cast<const uint4 *>(p.kv.kidx + row * DI) + c) : make_uint4(0u, 0u, 0u, 0u);
-    for (int i = threadIdx.x; i < p.hi * DI; i += kReindexScoreThreads)
-        qf[i] = e4m3x2_to_float2((uint16_t)p.qidx[(int64_t)qi * p.hi * DI + i]).x;
-    if (threadIdx.x < p.hi) wf[threadIdx.x] = p.w[(int64_t)qi * p.hi + threadIdx.x];
+    const int32_t id = reindex_gather<DI>(p, qi, j, kv);  // out before the query is staged
+    reindex_stage_query<DI, kReindexScoreThreads>(p, qi, qf, wf);
     __syncthreads();
     if (j >= p.p) return;
-    unsigned long long v = 0ull;  // 0 marks an empty slot (a valid key has ~id >= 2^31)
-    if (id >= 0) {
-        float dot[kScanN];
-#pragma unroll
-        for (int h = 0; h < kScanN; ++h) dot[h] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < DI / 16; ++c) {
-            const uint32_t wv[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
-            float kf[16];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const float2 lo = e4m3x2_to_float2((uint16_t)(wv[t] & 0xFFFFu));
-                const float2 hi2 = e4m3x2_to_float2((uint16_t)(wv[t] >> 16));
-                kf[t * 4 + 0] = lo.x;
-                kf[t * 4 + 1] = lo.y;
-                kf[t * 4 + 2] = hi2.x;
-                kf[t * 4 + 3] = hi2.y;
-            }
-#pragma unroll
-            for (int h = 0; h < kScanN; ++h) {
-                if (h >= p.hi) break;
-#pragma unroll
-                for (int i = 0; i < 16; i += 4) {
-                    const float4 q4 = *reinterpret_cast<const float4 *>(&qf[h * DI + c * 16 + i]);
-                    dot[h] = fmaf(q4.x, kf[i], dot[h]);
-                    dot[h] = fmaf(q4.y, kf[i + 1], dot[h]);
-                    dot[h] = fmaf(q4.z, kf[i + 2], dot[h]);
-                    dot[h] = fmaf(q4.w, kf[i + 3], dot[h]);
-                }
-            }
-        }
-        float sc = 0.0f;
-#pragma unroll
-        for (int h = 0; h < kScanN; ++h)
-            if (h < p.hi) sc = fmaf(wf[h], fmaxf(dot[h], 0.0f), sc);
-        v = ((unsigned long long)score_key(sc + 0.0f) << 32) | (unsigned long long)(~(uint32_t)(id + p.id_offset));
-    }
-    p.k64[(int64_t)qi * p.p + j] = v;
+    p.k64[(int64_t)qi * p.p + j] = reindex_key<DI>(p, id, kv, qf, wf);
 }
 
 // Select the k largest of the m unique 64-bit keys of query qi (0 = empty;
@@ -551,190 +570,69 @@ __global__ void __launch_bounds__(kReindexSelectThreads, 1) k_reindex_select(Rei
 }
 
 // ---------------------------------------------------------------------------
-// Reindex in one launch, one CTA per query: the pool's indexer keys are
-// gathered by cp.async (16-byte pieces, a ring of 128-row tiles laid out as
-// the scan's 128B-swizzled A operand, two 64-byte entries per row when
-// di = 64), scored by tcgen05 FP8 products against the query's heads (as in
-// the Full scan, so the same exact scores), and the unique 64-bit keys
-// (score key << 32 | ~id) kept in shared memory for select_k64.
-// Warps 0..7 gather, warps 8..11 (TMEM lane quarters 0..3) read the scores
-// back, warp 12 issues the products; then every thread selects.
+// Reindex in one launch: a cluster of ceil(p / 1024) CTAs per query (at most
+// 8, the portable cluster size). Thread j of the cluster gathers and scores
+// pool slot j as k_reindex_score does and stores its key straight into the
+// shared memory of the cluster's first CTA (distributed shared memory); after
+// a cluster barrier that CTA selects the k largest with select_k64, as
+// k_reindex_select does, with no round trip through global memory and no
+// second launch.
 // ---------------------------------------------------------------------------
-constexpr int kRfStages = 4;
-constexpr int kRfThreads = 512;
-constexpr int kRfGatherThreads = 256;
-constexpr int kRfMmaWarp = 12;
+constexpr int kRcThreads = 1024;
+constexpr int kRcMaxCluster = 8;
 
 template <int DI>
-struct RfCfg {
-    using G = ScanGeom<DI>;
-    static size_t smem(int p) {
-        return 1024 + (size_t)kRfStages * G::kStageBytes + 4096 /*q tile*/ + 2048 * 4 + (NT32 + 8) * 4 +
-               (size_t)p * 8 + ((size_t)p / 32 + 2) * 4 + 256;
-    }
-    static constexpr int NT32 = kRfThreads / 32;
-};
-
-template <int DI>
-__global__ void __launch_bounds__(kRfThreads, 1) k_reindex_fused(ReindexParams p) {
-    using G = ScanGeom<DI>;
-    constexpr int NT = kRfThreads;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *stages = base;
-    uint8_t *qt = stages + kRfStages * G::kStageBytes;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(qt + 4096);  // [2048]
-    uint32_t *scratch = hist + 2048;                            // [NT/32 + 8]
-    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p]
-    uint32_t *vbits = reinterpret_cast<uint32_t *>(k64 + p.p);  // [p / 32 + 1]: valid pool slots
-    uint64_t *full_b = reinterpret_cast<uint64_t *>(vbits + (p.p / 32 + 2) / 2 * 2);
-    uint64_t *empty_b = full_b + kRfStages;
-    uint64_t *tfull = empty_b + kRfStages;
-    uint64_t *tempty = tfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+__global__ void __launch_bounds__(kRcThreads, 1) k_reindex_cluster(ReindexParams p) {
+    constexpr int NT = kRcThreads;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem_raw);                                 // [2048]
+    uint32_t *scratch = hist + 2048;                                                         // [NT/32 + 8]
+    unsigned long long *k64 = reinterpret_cast<unsigned long long *>(scratch + NT / 32 + 8);  // [p], first CTA
+    __shared__ __align__(16) float qf[kScanN * DI];
+    __shared__ float wf[kScanN];
     __shared__ unsigned long long and_acc, or_acc;
-    __shared__ uint32_t nvalid_s;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int32_t qi = blockIdx.x;
-    const int32_t b = qi / p.q_per_seq;
-    const int ntiles = (p.p + G::kTile - 1) / G::kTile;
+    const uint32_t rank = cluster_rank();
+    const int32_t qi = blockIdx.y;
     pdl_trigger();
-    for (int i = tid; i < p.p / 32 + 1; i += NT) vbits[i] = 0u;
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
         and_acc = ~0ull;
         or_acc = 0ull;
-        nvalid_s = 0u;
-        for (int s = 0; s < kRfStages; ++s) {
-            mbar_init(&full_b[s], kRfGatherThreads);
-            mbar_init(&empty_b[s], 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);
-        }
-        fence_mbar_init();
-    }
-    if (warp == kRfMmaWarp) {
-        tmem_alloc(tmem_slot, 2 * kScanBatch * G::kN);
-        tmem_relinquish();
     }
     pdl_wait();
-    build_q_tile<DI>(qt, p.qidx + (int64_t)qi * p.hi * DI, p.hi, NT);
-    fence_proxy_async_smem();
-    tc_fence_before();
+    const int32_t j = (int32_t)rank * NT + threadIdx.x;
+    uint4 kv[DI / 16];
+    const int32_t id = reindex_gather<DI>(p, qi, j, kv);
+    reindex_stage_query<DI, NT>(p, qi, qf, wf);
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const int32_t *pool = p.pool + (int64_t)qi * p.p;
-
-    if (tid < kRfGatherThreads) {
-        // tile t, stage t % S: entry e of the tile -> row e / kEpr, 64-byte half
-        // e % kEpr (di = 64), 16-byte pieces; an empty slot or a bad id is
-        // zero-filled (a bad id is reported). Up to kRfStages tiles of this
-        // thread's pieces are in flight: tile t is published to the products
-        // once the pieces of tile t are complete, kRfStages - 1 tiles later.
-        constexpr int kPieces = DI / 16;                             // per entry
-        constexpr int kPer = G::kTile * kPieces / kRfGatherThreads;  // per thread and tile (4)
-        int s = 0;
-        uint32_t phase = 0;
-        int s_pub = 0;
-        auto publish = [&]() {
-            fence_proxy_async_smem();
-            mbar_arrive(&full_b[s_pub]);
-            if (++s_pub == kRfStages) s_pub = 0;
-        };
-        bool ok = true;
-        int issued = 0;
-        for (int t = 0; t < ntiles; ++t) {
-            if (!mbar_wait(&empty_b[s], phase ^ 1)) {
-                ok = false;
-                break;
-            }
-            uint8_t *st = stages + (size_t)s * G::kStageBytes;
-#pragma unroll
-            for (int i = 0; i < kPer; ++i) {
-                const int idx = tid + i * kRfGatherThreads;  // piece index in the tile
-                const int e = idx / kPieces, c = idx % kPieces;
-                const int j = t * G::kTile + e;              // pool position
-                const int32_t id = j < p.p ? pool[j] : -1;
-                const int64_t row = id >= 0 ? physical_row(p.kv, b, id) : -1;
-                if (c == 0 && row >= 0) atomicOr(&vbits[j >> 5], 1u << (j & 31));
-                if (c == 0 && id >= 0 && row < 0) set_error(CSA2_DEVERR_BAD_ROW);
-                const int r = e / G::kEpr, u = e % G::kEpr;
-                const int chunk = u * kPieces + c;
-                uint8_t *dst = st + (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
-                const uint8_t *srcp = row >= 0 ? p.kv.kidx + row * DI + c * 16 : p.kv.kidx;
-                const uint32_t bytes = row >= 0 ? 16u : 0u;  // 0: zero fill
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(srcp),
-                             "r"(bytes)
-                             : "memory");
-            }
-            cp_async_commit();
-            ++issued;
-            if (issued >= kRfStages) {
-                asm volatile("cp.async.wait_group 3;" ::: "memory");  // kRfStages - 1 groups may stay in flight
-                publish();
-            }
-            if (++s == kRfStages) {
-                s = 0;
-                phase ^= 1u;
-            }
-        }
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        if (ok)
-            for (int t = max(0, issued - (kRfStages - 1)); t < issued; ++t) publish();
-    } else if (warp == kRfMmaWarp) {
-        if (lane == 0)
-            scan_mma_loop<DI>(ntiles, kRfStages, stages, smem_u32(qt), full_b, empty_b, tfull, tempty, tmem);
-        __syncwarp();
-    } else if (warp >= 8 && warp < 12) {
-        float wv[kScanN];
-#pragma unroll
-        for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
-        scan_epilogue_loop<DI>(ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3, [&](int i, int e_in, uint32_t key) {
-            const int j = i * G::kTile + e_in;
-            if (j < p.p)
-                k64[j] = ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)(pool[j] + p.id_offset));
-        });
+    if (j < p.p) {
+        const unsigned long long v = reindex_key<DI>(p, id, kv, qf, wf);
+        const uint32_t addr = cluster_smem_addr(k64 + j, 0);
+        asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
     }
-    tc_fence_before();
-    __syncthreads();
-    // empty or bad slots (no valid bit) become key 0; the valid keys' count,
-    // AND and OR for the select
-    {
-        uint32_t nv = 0;
-        unsigned long long a_loc = ~0ull, o_loc = 0ull;
-        for (int j = tid; j < p.p; j += NT) {
-            if ((vbits[j >> 5] >> (j & 31)) & 1u) {
-                const unsigned long long v = k64[j];
-                ++nv;
-                a_loc &= v;
-                o_loc |= v;
-            } else {
-                k64[j] = 0ull;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
-            o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
-            nv += __shfl_xor_sync(0xFFFFFFFFu, nv, o);
-        }
-        if (lane == 0) {
-            atomicAnd(&and_acc, a_loc);
-            atomicOr(&or_acc, o_loc);
-            atomicAdd(&nvalid_s, nv);
+    cluster_sync_all();  // release / acquire: the first CTA sees every key
+    if (rank != 0) return;
+    uint32_t nvalid_t = 0;
+    unsigned long long a_loc = ~0ull, o_loc = 0ull;
+    for (int i = threadIdx.x; i < p.p; i += NT) {
+        const unsigned long long v = k64[i];
+        if ((uint32_t)v >= 0x80000000u) {
+            ++nvalid_t;
+            a_loc &= v;
+            o_loc |= v;
         }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == kRfMmaWarp) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 2 * kScanBatch * G::kN);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        a_loc &= __shfl_xor_sync(0xFFFFFFFFu, a_loc, o);
+        o_loc |= __shfl_xor_sync(0xFFFFFFFFu, o_loc, o);
     }
-    select_k64<false, NT>(k64, nullptr, p.p, p.k, p.topk + (int64_t)qi * p.k, nvalid_s, and_acc, or_acc, hist,
-                          scratch);
+    if ((threadIdx.x & 31) == 0) {
+        atomicAnd(&and_acc, a_loc);
+        atomicOr(&or_acc, o_loc);
+    }
+    uint32_t nvalid;
+    block_excl_scan<NT>(nvalid_t, scratch, &nvalid);  // its barriers also publish the reductions
+    select_k64<false, NT>(k64, nullptr, p.p, p.k, p.topk + (int64_t)qi * p.k, nvalid, and_acc, or_acc, hist, scratch);
 }
 
 }  // namespace csa2

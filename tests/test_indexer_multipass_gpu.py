@@ -22,3 +22,14 @@ def test_full_indexer_multipass_path(cuda_device):
                         os.path.join(HERE, "test_indexer_gpu.py"), "-k", "full"],
                        env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+def test_reindex_two_launch_path(cuda_device):
+    """The Reindex parity tests once more on the two-launch path (scores to
+    global memory, then a select CTA per query; CSA2_REINDEX=two) instead of
+    the one-launch cluster kernel."""
+    env = dict(os.environ, CSA2_REINDEX="two")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        os.path.join(HERE, "test_indexer_gpu.py"), "-k", "reindex"],
+                       env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
