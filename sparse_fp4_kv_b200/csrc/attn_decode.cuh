@@ -10,80 +10,59 @@
 //     o_h = sum_j softmax_j(scale * <q_h, v_j>) v_j.
 //
 // Work list. Query u's attended rows (its selected global entries, then its
-// window rows) are cut into tpq tiles of 64 rows, tpq = ceil((k + w_max) /
-// 64); the call's T = nq * tpq tiles form one list, query-major. CTA g
+// window rows) are cut into tpq tiles of 128 rows, tpq = ceil((k + w_max) /
+// 128); the call's T = nq * tpq tiles form one list, query-major. CTA g
 // takes tiles [g*per, (g+1)*per) with per = ceil(T / SMs): a run of whole
-// queries plus possibly a part of a query at either end. A run of one query
-// inside a CTA is a segment; a segment that covers its whole query writes o
-// (bf16, or f32 for the partial-output call) directly, the others write an
-// f32 partial (o normalised by its own denominators, and its log-sum-exp)
-// that k_attn_merge_parts combines. Consecutive tiles of a CTA go through
-// one pipeline regardless of segment boundaries.
+// queries plus possibly a part of a query at either end. A run of one query inside a CTA is a
+// segment; a segment that covers its whole query writes o (bf16, or f32 for
+// the partial-output call) directly, the others write an f32 partial (o
+// normalised by its own denominators, and its log-sum-exp) that
+// k_attn_merge_parts combines. Consecutive tiles of a CTA go through one
+// pipeline regardless of segment boundaries.
 //
-// Pipeline. Two f16 tiles (64 rows x 512, 64 KiB each) in shared memory,
-// two S^T accumulators and two P^T tiles, so that the dequantisation of
-// tile t+1, the products of tile t and the softmax of tile t overlap:
+// Warps:
 //   * resolver (1 warp): runs up to kResRing tiles ahead: entry ids ->
 //     physical rows through the page table (or window ring slots), into a
-//     shared-memory ring, with an L2 prefetch of every resolved row and of
-//     the next query's q;
-//   * 8 dequantising warps: gather the next tile's rows into registers with
+//     shared-memory ring, and an L2 prefetch of every resolved row;
+//   * 16 work warps: gather the next tile's rows into registers with
 //     16-byte loads (FP4 codes: four 16-byte pieces of a row per lane, its
 //     scale bytes as one 8-byte piece; window rows: eight 16-byte pieces),
-//     widen them into the free f16 tile (exact: an E2M1 value times an E4M3
-//     block scale has at most five significant bits), and at a query change
-//     write the new q (f16) once the last product reading the old one is done;
-//   * 1 MMA warp: one elected thread issues S^T(t) = KV(t) * Q^T
-//     (tcgen05.mma kind::f16, M = 64 rows, N = H heads, K = 512), then
-//     O^T += V(t-1)^T * P^T(t-1) (M = 128 latent columns per chunk, four
-//     chunks, K = 64 rows) -- S of a tile goes out before P*V of the one
-//     before, so the softmax of tile t-1 runs under S(t);
-//   * 8 softmax warps (two head groups of four TMEM lane quarters): the
-//     online softmax in base 2 on S^T from TMEM, P^T (f16) into shared
-//     memory, and the segment epilogue (o straight from TMEM to global
-//     memory, one coalesced store per head and 32 latent columns). The
-//     running maximum is only raised when a score exceeds it by more than
-//     2^8, so the common case needs no tile maximum: one vote per head group
-//     decides; a raise takes the full path (tile maximum, rescale of O^T in
-//     TMEM after the previous P*V is done).
-// Probabilities stay below 2^8 and are exact in range for f16.
+//     dequantise chunk by chunk into the f16 tile (exact), run the online
+//     softmax (a thread per row) and the segment epilogue;
+//   * 1 MMA warp: one elected thread issues S^T = KV * Q^T (tcgen05.mma
+//     kind::f16, M = 128 rows, N = H heads) chunk by chunk as chunks are
+//     stored, then O^T += V^T * P^T chunk by chunk.
+// The f16 tile (128 KiB) is handled in four 128-column chunks, so the
+// dequantisation of chunk c of tile t+1 starts as soon as the P*V product
+// of tile t on chunk c is done and the tensor pipe runs PV(t) and S(t+1)
+// back to back.
 #pragma once
 
 #include "attention.cuh"
 
 namespace csa2 {
 
-constexpr int kDecRows = 64;  // rows per tile
-constexpr int kDecDqWarps = 8;
-constexpr int kDecSmWarps = 8;
-constexpr int kDecDqThreads = kDecDqWarps * 32;
-constexpr int kDecSmThreads = kDecSmWarps * 32;
-constexpr int kDecSmWarp0 = kDecDqWarps;
-constexpr int kDecMmaWarp = kDecDqWarps + kDecSmWarps;
-constexpr int kDecResWarp = kDecMmaWarp + 1;
-constexpr int kDecThreads = (kDecResWarp + 1) * 32;
-constexpr int kResRing = 8;             // resolved tiles in flight
-constexpr uint32_t kBarSmGroup = 1;     // + head group (0, 1): the four warps of a group
-constexpr uint32_t kBarSm = 3;          // the softmax warps
-constexpr uint32_t kBarDq = 4;          // the dequantising warps
+constexpr int kDecWorkWarps = 16;
+constexpr int kDecWorkThreads = kDecWorkWarps * 32;
+constexpr int kDecMmaWarp = kDecWorkWarps;
+constexpr int kDecResWarp = kDecWorkWarps + 1;
+constexpr int kDecThreads = kDecWorkThreads + 64;
+constexpr int kResRing = 4;  // resolved tiles in flight
 
 template <int H>
 struct DecCfg {
-    static constexpr int kHG = H / 2;                        // heads per softmax group
-    static constexpr int kBufBytes = kDecRows * CSA2_D * 2;  // one f16 tile
+    static constexpr int kKvBytes = kAttnTile * CSA2_D * 2;
     static constexpr int kQBytes = H * CSA2_D * 2;
-    static constexpr int kPBytes = kDecRows * H * 2;  // one P^T tile
-    static constexpr int kPGroup = 16 * H;            // bytes of 8 rows of P^T
+    static constexpr int kPBytes = kAttnTile * H * 2;
+    static constexpr int kPGroup = 16 * H;
     static constexpr uint32_t kPSwizzle = H == 64 ? kSw128 : (H == 32 ? kSw64 : kSw32);
-    static constexpr int kColS = 0;      // S^T of tile buffer b: columns kColS + b * H
-    static constexpr int kColO = 2 * H;  // O^T, latent chunk dc: columns kColO + dc * H
+    static constexpr int kColS = 0;
+    static constexpr int kColO = H;
     static constexpr uint32_t kTmemCols = H == 64 ? 512u : (H == 32 ? 256u : 128u);
-    static constexpr int kMisc = kResRing * kDecRows * 5 /*rsrc, rkind*/ + 2 * kDecRows * 4 /*valid*/ +
-                                 4 * H * 4 /*red*/ + 3 * H * 4 /*m, alpha, 1/l*/ + 512 /*bars, slot, flags*/;
-    static constexpr size_t kSmem = 1024 + 2 * (size_t)kBufBytes + kQBytes + 2 * (size_t)kPBytes + kMisc;
+    static constexpr int kMisc = kResRing * kAttnTile * 5 /*rsrc, rkind*/ + kAttnTile * 4 /*valid*/ +
+                                 4 * H * 4 /*red*/ + 3 * H * 4 /*m, alpha, l*/ + 256 /*bars, slot, flags*/;
+    static constexpr size_t kSmem = 1024 + (size_t)kKvBytes + kQBytes + kPBytes + kMisc;
 };
-static_assert(DecCfg<64>::kSmem <= 227 * 1024, "shared memory of the 64-head kernel");
-static_assert(DecCfg<64>::kQBytes <= DecCfg<64>::kBufBytes, "q is staged in a tile buffer");
 
 struct DecParams {
     const uint16_t *q;  // bf16 [nq][H][512]
@@ -151,8 +130,8 @@ __device__ __forceinline__ int32_t block_part_base(const DecSplit &sp, int32_t g
     return *red_word;
 }
 
-// One tile's raw rows in registers. Lane l of dequantising warp w holds row
-// 8w + l%8 of the tile, part m = l / 8: FP4 rows: v[c] = the 16 code bytes 64c + 16m
+// One tile's raw rows in registers. Lane l of work warp w holds row 8w + l%8
+// of the tile, part m = l / 8: FP4 rows: v[c] = the 16 code bytes 64c + 16m
 // (values 128c + 32m .. + 31) for c = 0..3, v[4].xy = scale bytes 8m .. 8m+7
 // (the scales of chunk m); window rows: v[2c], v[2c+1] = the 32 E4M3 bytes
 // 128c + 32m .. + 31.
@@ -180,15 +159,8 @@ __device__ __forceinline__ void gather_row(const DecParams &p, const uint8_t *sw
     }
 }
 
-// f16 tile of 64 rows, K-major with 128B swizzle: eight column blocks of 64
-// latent values (8 KiB each), rows at 128 B, 16-byte piece c64 of row e
-// (values 8*c64 .. 8*c64+7) at:
-__device__ __forceinline__ uint32_t dec_kv_off(int e, int c64) {
-    return (uint32_t)((c64 >> 3) * 8192 + (e >> 3) * 1024 + (e & 7) * 128 + (((c64 & 7) ^ (e & 7)) << 4));
-}
-
-// Dequantise latent chunk c of this lane's row into the f16 tile: 32
-// values, four 16-byte stores. The scale bytes of the
+// Dequantise latent chunk c of this lane's row into the f16 tile (K-major,
+// 128B swizzle): 32 values, four 16-byte stores. The scale bytes of the
 // chunk come from the lane of the same row that loaded chunk c's scales.
 // Each quarter warp stores the same piece of eight consecutive rows, which
 // the swizzle spreads over the eight 16-byte bank groups.
@@ -230,7 +202,7 @@ __device__ __forceinline__ void dequant_chunk(const RawRow &raw, int c, uint8_t 
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-        *reinterpret_cast<uint4 *>(kv_tile + dec_kv_off(e, 16 * c + 4 * m + j)) =
+        *reinterpret_cast<uint4 *>(kv_tile + kv_chunk_off(e, 16 * c + 4 * m + j)) =
             make_uint4(h[j][0], h[j][1], h[j][2], h[j][3]);
 }
 
@@ -255,59 +227,49 @@ __device__ __forceinline__ void store_q_piece(uint8_t *q_tile, int i, const uint
     *reinterpret_cast<uint4 *>(q_tile + q_chunk_off<H>(h, c64)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
 }
 
-// q of query u (bf16 [H][512]) staged into `stage` by cp.async, kPer 16-byte
-// pieces per dequantising thread, and each thread's own pieces converted into
-// the f16 Q tile once they have landed.
+// Q of query u into the Q tile by the work threads, four 16-byte pieces per
+// thread in flight at a time.
 template <int H>
-__device__ __forceinline__ void stage_q(const DecParams &p, int64_t u, uint8_t *stage) {
-    constexpr int kPer = H * (CSA2_D / 8) / kDecDqThreads;
+__device__ __forceinline__ void load_q(const DecParams &p, int64_t u, uint8_t *q_tile) {
+    constexpr int kPer = H * (CSA2_D / 8) / kDecWorkThreads;  // 16-byte pieces per thread
+    constexpr int kBatch = kPer < 4 ? kPer : 4;
     const uint4 *src = reinterpret_cast<const uint4 *>(p.q + u * H * CSA2_D);
 #pragma unroll
-    for (int t = 0; t < kPer; ++t)
-        cp_async_16(stage + (size_t)(threadIdx.x + t * kDecDqThreads) * 16, src + threadIdx.x + t * kDecDqThreads);
-    cp_async_commit();
-}
-template <int H>
-__device__ __forceinline__ void convert_q(const uint8_t *stage, uint8_t *q_tile) {
-    constexpr int kPer = H * (CSA2_D / 8) / kDecDqThreads;
-    cp_async_wait_all();
+    for (int t0 = 0; t0 < kPer; t0 += kBatch) {
+        uint4 v[kBatch];
 #pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-        const int i = threadIdx.x + t * kDecDqThreads;
-        store_q_piece<H>(q_tile, i, *reinterpret_cast<const uint4 *>(stage + (size_t)i * 16));
+        for (int t = 0; t < kBatch; ++t) v[t] = __ldg(src + threadIdx.x + (t0 + t) * kDecWorkThreads);
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) store_q_piece<H>(q_tile, threadIdx.x + (t0 + t) * kDecWorkThreads, v[t]);
     }
 }
-
-// Row of the 64-row S^T accumulator (tcgen05.mma M = 64, cta_group::1) held
-// by TMEM lane 32 * quarter + l, or -1: rows 16 * quarter .. + 15 sit in
-// lanes 0..15 of each lane quarter.
-__device__ __forceinline__ int s_row_of(int quarter, int l) { return l < 16 ? 16 * quarter + l : -1; }
 
 template <int H>
 __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
     using Cfg = DecCfg<H>;
-    constexpr int HG = Cfg::kHG;
+    constexpr int G4 = H >= 32 ? 4 : 2;  // softmax head groups (4 warps each)
+    constexpr int HG = H / G4;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *kvb = base;                             // [2][kBufBytes]
-    uint8_t *q_tile = kvb + 2 * Cfg::kBufBytes;
-    uint8_t *pb = q_tile + Cfg::kQBytes;            // [2][kPBytes]
-    int32_t *rsrc = reinterpret_cast<int32_t *>(pb + 2 * Cfg::kPBytes);  // [kResRing][64]
-    uint8_t *rkind = reinterpret_cast<uint8_t *>(rsrc + kResRing * kDecRows);
-    int32_t *valid_s = reinterpret_cast<int32_t *>(rkind + kResRing * kDecRows);  // [2][64]
-    float *red = reinterpret_cast<float *>(valid_s + 2 * kDecRows);  // [4][H]
+    uint8_t *kv_tile = base;
+    uint8_t *q_tile = kv_tile + Cfg::kKvBytes;
+    uint8_t *p_tile = q_tile + Cfg::kQBytes;
+    int32_t *rsrc = reinterpret_cast<int32_t *>(p_tile + Cfg::kPBytes);  // [kResRing][128]
+    uint8_t *rkind = reinterpret_cast<uint8_t *>(rsrc + kResRing * kAttnTile);
+    int32_t *valid_s = reinterpret_cast<int32_t *>(rkind + kResRing * kAttnTile);
+    float *red = reinterpret_cast<float *>(valid_s + kAttnTile);  // [4][H]
     float *m_run = red + 4 * H;
     float *alpha = m_run + H;
-    float *inv_l = alpha + H;
-    uint64_t *kv_full = reinterpret_cast<uint64_t *>(inv_l + H);  // [2]: tile b stored (and q, at a query change)
-    uint64_t *kv_empty = kv_full + 2;                              // [2]: P*V of tile buffer b done
-    uint64_t *s_full = kv_empty + 2;                               // [2]: S^T of buffer b done
-    uint64_t *p_full = s_full + 2;                                 // [2]: P^T of buffer b stored
-    uint64_t *res_full = p_full + 2;                               // [kResRing]
-    uint64_t *res_empty = res_full + kResRing;                     // [kResRing]
+    float *l_run = alpha + H;
+    uint64_t *bar_kv = reinterpret_cast<uint64_t *>(l_run + H);  // [4]
+    uint64_t *bar_pv = bar_kv + 4;                               // [4]
+    uint64_t *bar_s = bar_pv + 4;
+    uint64_t *bar_p = bar_s + 1;
+    uint64_t *res_full = bar_p + 1;            // [kResRing]
+    uint64_t *res_empty = res_full + kResRing;  // [kResRing]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(res_empty + kResRing);
-    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [2]
-    int32_t *part_word = rescale_tile + 2;
+    int32_t *rescale_tile = reinterpret_cast<int32_t *>(tmem_slot + 1);  // [4]
+    int32_t *part_word = rescale_tile + 4;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const DecSplit sp{(int64_t)p.nq * p.tpq, p.per, p.tpq};
@@ -316,25 +278,29 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
     const int n = (int)max((int64_t)0, x1 - x0);
 
     pdl_trigger();
-    if (warp == kDecMmaWarp) {
+    if (warp == 0) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&kv_full[b], kDecDqWarps);  // one arrival per warp (lane 0, after __syncwarp)
-            mbar_init(&kv_empty[b], 1);
-            mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], kDecSmWarps);
+        // the work warps arrive once per warp (lane 0, after __syncwarp)
+        for (int c = 0; c < 4; ++c) {
+            mbar_init(&bar_kv[c], kDecWorkWarps);
+            mbar_init(&bar_pv[c], 1);
         }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_p, kDecWorkWarps);
         for (int r = 0; r < kResRing; ++r) {
             mbar_init(&res_full[r], 32);
-            mbar_init(&res_empty[r], kDecDqWarps);
+            mbar_init(&res_empty[r], kDecWorkWarps);
         }
-        rescale_tile[0] = rescale_tile[1] = -1;
+        rescale_tile[0] = rescale_tile[1] = rescale_tile[2] = rescale_tile[3] = -1;
         fence_mbar_init();
     }
-    if (tid < H) m_run[tid] = -INFINITY;
+    if (tid < H) {
+        m_run[tid] = -INFINITY;
+        l_run[tid] = 0.0f;
+    }
     const int32_t part_base = block_part_base(sp, g, part_word);  // its barriers publish the set-up above
     tc_fence_before();
     __syncthreads();
@@ -367,20 +333,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
                 }
                 one_page_pt = one_page ? p.kv.page_table[b] : -1;
                 swa_seq = p.swa ? p.swa + (int64_t)b * p.swa_seq_stride * CSA2_D : nullptr;
-                // q of a later query is read at its first tile: into L2 now
-                if (i > 0) {
-                    const uint8_t *qb = reinterpret_cast<const uint8_t *>(p.q + u * H * CSA2_D);
-                    for (int o = lane * 128; o < H * CSA2_D * 2; o += 32 * 128)
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(qb + o));
-                }
             }
             // the tile's entry ids, then their pages, then the rows: every load of
             // a phase is in flight at once
-            constexpr int kR = kDecRows / 32;
+            constexpr int kR = kAttnTile / 32;
             int32_t id[kR];
 #pragma unroll
             for (int rr = 0; rr < kR; ++rr) {
-                const int64_t j = t * kDecRows + lane + 32 * rr;
+                const int64_t j = t * kAttnTile + lane + 32 * rr;
                 id[rr] = j < p.k ? p.topk[u * p.k + j] : -1;
             }
             int32_t phys[kR];
@@ -399,7 +359,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
 #pragma unroll
             for (int rr = 0; rr < kR; ++rr) {
                 const int r = lane + 32 * rr;
-                const int64_t j = t * kDecRows + r;
+                const int64_t j = t * kAttnTile + r;
                 int32_t src = 0;
                 uint32_t kind = 0;
                 if (j < p.k) {
@@ -426,132 +386,123 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
 #pragma unroll
                     for (int o = 0; o < CSA2_D; o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(wr + o));
                 }
-                rsrc[slot * kDecRows + r] = src;
-                rkind[slot * kDecRows + r] = (uint8_t)kind;
+                rsrc[slot * kAttnTile + r] = src;
+                rkind[slot * kAttnTile + r] = (uint8_t)kind;
             }
             mbar_arrive(&res_full[slot]);
         }
     } else if (warp == kDecMmaWarp) {
         // ---- one elected thread issues every tensor-core product ----
         if (lane == 0) {
-            const uint32_t kv_addr = smem_u32(kvb), q_addr = smem_u32(q_tile), p_addr = smem_u32(pb);
-            const uint32_t idesc_s = idesc_f16_f32(64, H, 0, 0);
+            const uint32_t kv_addr = smem_u32(kv_tile), q_addr = smem_u32(q_tile), p_addr = smem_u32(p_tile);
+            const uint32_t idesc_s = idesc_f16_f32(128, H, 0, 0);
             const uint32_t idesc_o = idesc_f16_f32(128, H, 1, 1);
             const uint64_t a_s = make_sdesc(kv_addr, 16, 1024, kSw128);
             const uint64_t b_s = make_sdesc(q_addr, 16, 1024, kSw128);
-            const uint64_t a_o = make_sdesc(kv_addr, 8192, 1024, kSw128);
+            const uint64_t a_o = make_sdesc(kv_addr, 16384, 1024, kSw128);
             const uint64_t b_o = make_sdesc(p_addr, 16, Cfg::kPGroup, Cfg::kPSwizzle);
-            // S^T(i): tile i against q, into S buffer i & 1
-            auto s_mma = [&](int i) {
-                const int bi = i & 1;
-                const uint64_t a = a_s + (uint64_t)((bi * Cfg::kBufBytes) >> 4);
+            bool ok = true;
+            for (int i = 0; i < n && ok; ++i) {
+                const uint32_t ph = (uint32_t)i & 1u;
+                const int64_t x = x0 + i;
+                const bool first = i == 0 || x % p.tpq == 0;
 #pragma unroll 1
-                for (int kb = 0; kb < CSA2_D / 64; ++kb)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(tmem + Cfg::kColS + bi * H, a + (uint64_t)((kb * 8192 + kk * 32) >> 4),
-                                b_s + (uint64_t)((kb * (H * 128) + kk * 32) >> 4), idesc_s, (kb | kk) ? 1u : 0u);
-                tc_commit(&s_full[bi]);
-            };
-            // O^T += V(j)^T * P^T(j), then tile buffer j & 1 is free again
-            auto pv_mma = [&](int j) {
-                const int bj = j & 1;
-                const bool first = j == 0 || (x0 + j) % p.tpq == 0;
-                const uint64_t a = a_o + (uint64_t)((bj * Cfg::kBufBytes) >> 4);
-                const uint64_t bb = b_o + (uint64_t)((bj * Cfg::kPBytes) >> 4);
-#pragma unroll 1
-                for (int dc = 0; dc < 4; ++dc)
-#pragma unroll
-                    for (int kk = 0; kk < kDecRows / 16; ++kk)
-                        mma_f16(tmem + Cfg::kColO + dc * H, a + (uint64_t)((dc * 16384 + kk * 2048) >> 4),
-                                bb + (uint64_t)((kk * 2 * Cfg::kPGroup) >> 4), idesc_o, (!first || kk > 0) ? 1u : 0u);
-                tc_commit(&kv_empty[bj]);
-            };
-            // Products are issued as their inputs become ready, P*V first: S of
-            // tile ns once that tile is stored and its S buffer is free (the
-            // softmax of tile ns-2 is done, which P*V of ns-2 having been issued
-            // shows); P*V of tile np once its P is stored. The tensor pipe
-            // then never waits for a product whose inputs were ready behind one
-            // whose inputs were not. A second without progress ends the loop
-            // with the wait-timeout error.
-            int ns = 0, np = 0;
-            uint64_t idle0 = 0;
-#pragma unroll 1
-            while (np < n) {
-                if (np < ns && mbar_test(&p_full[np & 1], (uint32_t)(np >> 1) & 1u)) {
-                    tc_fence_after();
-                    pv_mma(np++);
-                    idle0 = 0;
-                } else if (ns < n && ns <= np + 1 && mbar_test(&kv_full[ns & 1], (uint32_t)(ns >> 1) & 1u)) {
-                    tc_fence_after();
-                    s_mma(ns++);
-                    idle0 = 0;
-                } else {
-                    const uint64_t now = global_ns();
-                    if (idle0 == 0) {
-                        idle0 = now;
-                    } else if (now - idle0 > kWaitNs) {
-                        set_error(CSA2_DEVERR_WAIT_TIMEOUT);
+                for (int c = 0; c < 4 && ok; ++c) {
+                    if (!mbar_wait(&bar_kv[c], ph)) {
+                        ok = false;
                         break;
                     }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kb = 2 * c; kb < 2 * c + 2; ++kb)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16(tmem + Cfg::kColS, a_s + (uint64_t)((kb * 16384 + kk * 32) >> 4),
+                                    b_s + (uint64_t)((kb * (H * 128) + kk * 32) >> 4), idesc_s, (kb | kk) ? 1u : 0u);
+                }
+                if (!ok) break;
+                tc_commit(bar_s);
+                if (!mbar_wait(bar_p, ph)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int dc = 0; dc < 4; ++dc) {
+#pragma unroll
+                    for (int kk = 0; kk < kAttnTile / 16; ++kk)
+                        mma_f16(tmem + Cfg::kColO + dc * H, a_o + (uint64_t)((dc * 32768 + kk * 2048) >> 4),
+                                b_o + (uint64_t)((kk * 2 * Cfg::kPGroup) >> 4), idesc_o,
+                                (!first || kk > 0) ? 1u : 0u);
+                    tc_commit(&bar_pv[dc]);
                 }
             }
         }
         __syncwarp();
-    } else if (warp < kDecDqWarps) {
-        // ---- dequantising warps ----
+    } else {
+        // ---- work warps ----
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const int quarter = warp & 3, grp = warp >> 2;
+        const bool soft = grp < G4;
         const int m = lane >> 3;
         const int row_e = warp * 8 + (lane & 7);  // this lane's row in the gather / dequantisation
+        float l_part[HG];
+#pragma unroll
+        for (int i = 0; i < HG; ++i) l_part[i] = 0.0f;
         bool ok = true;
         RawRow raw;
         raw.kind = 0;
+        // tile 0's rows, then Q of its query
+        int64_t u_cur = x0 / p.tpq;
+        const uint8_t *swa_seq = p.swa ? p.swa + (u_cur / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
         if (n > 0) {
-            // q of the first query does not depend on the resolved rows: its bf16
-            // bytes go into buffer 1 (unused until tile 1) by cp.async while the
-            // first tile's rows are gathered
-            const int64_t u0 = x0 / p.tpq;
-            stage_q<H>(p, u0, kvb + Cfg::kBufBytes);
+            // Q of the first query does not depend on the resolved rows: its bf16
+            // bytes go into the (still unused) KV tile by cp.async first, the first
+            // tile's rows are gathered, then each thread converts the pieces it
+            // copied into the f16 Q tile
+            constexpr int kQPer = H * (CSA2_D / 8) / kDecWorkThreads;
+            const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + u_cur * H * CSA2_D);
+#pragma unroll
+            for (int t = 0; t < kQPer; ++t)
+                cp_async_16(kv_tile + (size_t)(tid + t * kDecWorkThreads) * 16, qsrc + tid + t * kDecWorkThreads);
+            cp_async_commit();
             if (mbar_wait(&res_full[0], 0)) {
                 const int32_t src = rsrc[row_e];
                 const uint32_t kd = rkind[row_e];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&res_empty[0]);
-                const uint8_t *sw0 = p.swa ? p.swa + (u0 / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
-                gather_row(p, sw0, src, kd, m, raw);
+                gather_row(p, swa_seq, src, kd, m, raw);
             } else {
                 ok = false;
             }
-            convert_q<H>(kvb + Cfg::kBufBytes, q_tile);
-            named_bar_sync(kBarDq, kDecDqThreads);  // every staged piece is read before buffer 1 is reused
-        }
-        for (int t = 0; t < n; ++t) {
-            const int b = t & 1;
-            const int64_t x = x0 + t;
-            uint8_t *buf = kvb + b * Cfg::kBufBytes;
-            // buffer b is free once P*V of tile t-2 is done
-            if (t >= 2 && ok && !mbar_wait(&kv_empty[b], (uint32_t)((t - 2) >> 1) & 1u)) ok = false;
-            if (t > 0 && x % p.tpq == 0) {
-                // a new query: its q replaces the last one's once S^T of tile t-1
-                // (the last product that reads it) is done
-                if (ok && !mbar_wait(&s_full[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u)) ok = false;
-                stage_q<H>(p, x / p.tpq, buf);
-                convert_q<H>(buf, q_tile);
-                named_bar_sync(kBarDq, kDecDqThreads);
-            }
+            cp_async_wait_all();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) dequant_chunk(raw, c, buf);
-            if (m == 0) valid_s[b * kDecRows + row_e] = raw.kind != 0u;
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&kv_full[b]);
-            // the next tile's rows go in flight under this tile's products
-            if (t + 1 < n) {
-                const int slot = (t + 1) % kResRing;
+            for (int t = 0; t < kQPer; ++t) {
+                const int i = tid + t * kDecWorkThreads;
+                const uint4 w = *reinterpret_cast<const uint4 *>(kv_tile + (size_t)i * 16);
+                store_q_piece<H>(q_tile, i, w);
+            }
+            named_bar_sync(kBarWork, kDecWorkThreads);  // the KV tile is free for the first dequantisation
+        }
+        for (int i = 0; i < n; ++i) {
+            const int64_t x = x0 + i;
+            const int64_t u = x / p.tpq;
+            const bool last = i == n - 1 || (x + 1) % p.tpq == 0;
+            // 1. dequantise chunk c once the previous tile's P*V on it is done
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (i > 0 && ok && !mbar_wait(&bar_pv[c], (uint32_t)(i - 1) & 1u)) ok = false;
+                dequant_chunk(raw, c, kv_tile);
+                if (c == 0 && m == 0) valid_s[row_e] = raw.kind != 0u;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_kv[c]);
+            }
+            // 2. the next tile's rows go in flight under this tile's products
+            if (i + 1 < n) {
+                const int slot = (i + 1) % kResRing;
                 int32_t src = 0;
                 uint32_t kd = 0;
-                if (ok && mbar_wait(&res_full[slot], (uint32_t)((t + 1) / kResRing) & 1u)) {
-                    src = rsrc[slot * kDecRows + row_e];
-                    kd = rkind[slot * kDecRows + row_e];
+                if (ok && mbar_wait(&res_full[slot], (uint32_t)((i + 1) / kResRing) & 1u)) {
+                    src = rsrc[slot * kAttnTile + row_e];
+                    kd = rkind[slot * kAttnTile + row_e];
                 } else {
                     ok = false;
                 }
@@ -561,169 +512,197 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
                 const uint8_t *sn = p.swa ? p.swa + (un / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
                 gather_row(p, sn, src, kd, m, raw);
             }
-        }
-    } else {
-        // ---- softmax warps: lane quarter q of TMEM, head group grp ----
-        // A thread holds the scores of one row (lanes 0..15) for the group's
-        // HG heads; the row sums are reduced over the warp every tile, so a
-        // lane keeps one running sum, of head grp * HG + lane / R.
-        constexpr int R = HG >= 32 ? 1 : 32 / HG;  // lanes holding the same head's sum
-        const int sw = warp - kDecSmWarp0;
-        const int quarter = warp & 3, grp = sw >> 2;
-        const int stid = tid - kDecSmWarp0 * 32;
-        const int srow = s_row_of(quarter, lane);
-        const int hl = grp * HG + lane / R;  // the head of this lane's running sum
-        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-        float l_acc = 0.0f;
-        bool ok = true;
-        for (int t = 0; t < n; ++t) {
-            const int b = t & 1;
-            const int64_t x = x0 + t;
-            const int64_t u = x / p.tpq;
-            const bool last = t == n - 1 || (x + 1) % p.tpq == 0;
-            const bool got = ok && mbar_wait(&s_full[b], (uint32_t)(t >> 1) & 1u);
-            if (!got) ok = false;
-            tc_fence_after();
-            const bool row_valid = got && srow >= 0 && valid_s[b * kDecRows + srow] != 0;
-            const uint32_t s_addr = lane_addr + Cfg::kColS + b * H + grp * HG;
-            float v[HG];
-            load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
-            bool raise = false;
+            // 3. online softmax: thread = row (TMEM lane), warps 4g..4g+3 take
+            //    heads [g*HG, (g+1)*HG)
+            if (soft) {
+                const bool got = ok && mbar_wait(bar_s, (uint32_t)i & 1u);
+                if (!got) ok = false;
+                tc_fence_after();
+                const int row = quarter * 32 + lane;
+                const bool row_valid = valid_s[row] != 0 && got;
+                float v[HG];
+                load_scores<HG>(lane_addr + Cfg::kColS + grp * HG, p.scale_log2, row_valid, v);
+                bool raise = false;
 #pragma unroll
-            for (int gg = 0; gg < HG / 4; ++gg) {
-                const float4 mm = *reinterpret_cast<const float4 *>(m_run + grp * HG + 4 * gg);
-                raise |= v[4 * gg] > mm.x + kRescaleThreshold;
-                raise |= v[4 * gg + 1] > mm.y + kRescaleThreshold;
-                raise |= v[4 * gg + 2] > mm.z + kRescaleThreshold;
-                raise |= v[4 * gg + 3] > mm.w + kRescaleThreshold;
-            }
-            raise = named_bar_or(kBarSmGroup + grp, 128, raise);
-            if (raise) {
-                // the tile maximum per head (the scores are read again afterwards)
-                warp_transpose_reduce<HG, true>(v);
-                store_warp_reduced<HG>(red + quarter * H + grp * HG, v);
-                named_bar_sync(kBarSmGroup + grp, 128);
-                if (quarter == 0 && lane < HG) {
-                    const int h = grp * HG + lane;
-                    const float mt = fmaxf(fmaxf(red[h], red[H + h]), fmaxf(red[2 * H + h], red[3 * H + h]));
-                    const float mo = m_run[h];
-                    float a = 1.0f, mn = mo;
-                    if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt > -INFINITY)) {
-                        mn = mt;
-                        a = (mo == -INFINITY) ? 0.0f : exp2f(mo - mt);
-                        if (mo != -INFINITY) rescale_tile[grp] = t;
+                for (int gg = 0; gg < HG / 4; ++gg) {
+                    const float4 mm = *reinterpret_cast<const float4 *>(m_run + grp * HG + 4 * gg);
+                    raise |= v[4 * gg] > mm.x + kRescaleThreshold;
+                    raise |= v[4 * gg + 1] > mm.y + kRescaleThreshold;
+                    raise |= v[4 * gg + 2] > mm.z + kRescaleThreshold;
+                    raise |= v[4 * gg + 3] > mm.w + kRescaleThreshold;
+                }
+                raise = named_bar_or(1 + grp, 128, raise);
+                if (raise) {
+                    float mx[HG];
+#pragma unroll
+                    for (int j = 0; j < HG; ++j) mx[j] = v[j];
+                    warp_transpose_reduce<HG, true>(mx);
+                    store_warp_reduced<HG>(red + quarter * H + grp * HG, mx);
+                    named_bar_sync(1 + grp, 128);
+                    if (quarter == 0 && lane < HG) {
+                        const int h = grp * HG + lane;
+                        const float mt = fmaxf(fmaxf(red[h], red[H + h]), fmaxf(red[2 * H + h], red[3 * H + h]));
+                        const float mo = m_run[h];
+                        float a = 1.0f, mn = mo;
+                        if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt > -INFINITY)) {
+                            mn = mt;
+                            a = (mo == -INFINITY) ? 0.0f : exp2f(mo - mt);
+                            if (mo != -INFINITY) rescale_tile[grp] = i;
+                        }
+                        m_run[h] = mn;
+                        alpha[h] = a;
                     }
-                    m_run[h] = mn;
-                    alpha[h] = a;
+                    named_bar_sync(1 + grp, 128);
                 }
-                named_bar_sync(kBarSmGroup + grp, 128);
-                load_scores<HG>(s_addr, p.scale_log2, row_valid, v);
-            }
-            // P = exp2(s - m) in place, stored as f16 P^T
 #pragma unroll
-            for (int gg = 0; gg < HG / 8; ++gg) {
-                const int h0 = grp * HG + 8 * gg;
-                const float4 ma = *reinterpret_cast<const float4 *>(m_run + h0);
-                const float4 mb = *reinterpret_cast<const float4 *>(m_run + h0 + 4);
-                const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-                uint32_t pk[4];
+                for (int gg = 0; gg < HG / 8; ++gg) {
+                    const int h0 = grp * HG + 8 * gg;
+                    const float4 ma = *reinterpret_cast<const float4 *>(m_run + h0);
+                    const float4 mb = *reinterpret_cast<const float4 *>(m_run + h0 + 4);
+                    const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+                    float al[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+                    if (raise) {
+                        const float4 aa = *reinterpret_cast<const float4 *>(alpha + h0);
+                        const float4 ab = *reinterpret_cast<const float4 *>(alpha + h0 + 4);
+                        al[0] = aa.x, al[1] = aa.y, al[2] = aa.z, al[3] = aa.w;
+                        al[4] = ab.x, al[5] = ab.y, al[6] = ab.z, al[7] = ab.w;
+                    }
+                    uint32_t pk[4];
 #pragma unroll
-                for (int t2 = 0; t2 < 4; ++t2) {
-                    const int j = 8 * gg + 2 * t2;
-                    v[j] = (mm[2 * t2] == -INFINITY) ? 0.0f : exp2f(v[j] - mm[2 * t2]);
-                    v[j + 1] = (mm[2 * t2 + 1] == -INFINITY) ? 0.0f : exp2f(v[j + 1] - mm[2 * t2 + 1]);
-                    const __half2 h2 = __floats2half2_rn(v[j], v[j + 1]);
-                    pk[t2] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                if (srow >= 0)
-                    *reinterpret_cast<uint4 *>(pb + b * Cfg::kPBytes + p_chunk_off<H>(srow, h0 >> 3)) =
+                    for (int t = 0; t < 4; ++t) {
+                        const int j = 8 * gg + 2 * t;
+                        const float p0 = (mm[2 * t] == -INFINITY) ? 0.0f : exp2f(v[j] - mm[2 * t]);
+                        const float p1 = (mm[2 * t + 1] == -INFINITY) ? 0.0f : exp2f(v[j + 1] - mm[2 * t + 1]);
+                        l_part[j] = fmaf(l_part[j], al[2 * t], p0);
+                        l_part[j + 1] = fmaf(l_part[j + 1], al[2 * t + 1], p1);
+                        const __half2 h2 = __floats2half2_rn(p0, p1);
+                        pk[t] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    *reinterpret_cast<uint4 *>(p_tile + p_chunk_off<H>(row, h0 >> 3)) =
                         make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+                // a raise of the running maximum rescales this group's O^T columns
+                // (every earlier P*V is complete: this tile's S commit came after)
+                if (raise && rescale_tile[grp] == i) {
+#pragma unroll 1
+                    for (int dc = 0; dc < 4; ++dc) {
+#pragma unroll
+                        for (int c = 0; c < HG; c += 8) {
+                            uint32_t r8[8];
+                            const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
+                            tmem_ld8(ta, r8);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                r8[j] = __float_as_uint(__uint_as_float(r8[j]) * alpha[grp * HG + c + j]);
+                            tmem_st8(ta, r8);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
             }
-            // the tile's row sums, reduced over the warp's rows
-            warp_transpose_reduce<HG, false>(v);
-            l_acc = fmaf(l_acc, raise ? alpha[hl] : 1.0f, v[0]);
-            // a raise of the running maximum rescales this group's O^T columns once
-            // the P*V of the previous tile (issued after this tile's S) is done
-            if (raise && rescale_tile[grp] == t) {
-                if (ok && !mbar_wait(&kv_empty[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u)) ok = false;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p);
+
+            if (!last) continue;
+            // ---- 4. end of a segment: Q of the next one (this tile's S is done,
+            //      so the Q tile is free), then o of this one ----
+            const bool has_next = i + 1 < n;
+            named_bar_sync(kBarWork, kDecWorkThreads);
+            if (soft) {
+                warp_transpose_reduce<HG, false>(l_part);
+                store_warp_reduced<HG>(red + quarter * H + grp * HG, l_part);
+            }
+            named_bar_sync(kBarWork, kDecWorkThreads);
+            if (tid < H) {
+                const float l = (red[tid] + red[H + tid]) + (red[2 * H + tid] + red[3 * H + tid]);
+                l_run[tid] = l;
+                alpha[tid] = l > 0.0f ? 1.0f / l : 0.0f;  // reused as 1 / l
+            }
+            named_bar_sync(kBarWork, kDecWorkThreads);
+            const int64_t seg_start = (i == 0 || x0 > u * p.tpq) ? x0 : u * p.tpq;  // first tile of the segment
+            const bool whole = seg_start == u * p.tpq && x == (u + 1) * p.tpq - 1;
+            int32_t slot = 0;
+            if (!whole) slot = sp.slot(g, u, part_base);
+            // o (bf16 or f32) or the f32 partial of this segment: once the last
+            // P*V is done the whole KV tile is free; O / l goes there as [h][512]
+            // rows (the layout of the destination), then out in four bulk copies
+            const bool f32 = !whole || p.o32 != nullptr;
+            const int es = f32 ? 4 : 2;
+            if (soft) {
+                const int d0 = quarter * 32 + lane;
+                // the commit of the last chunk follows every product of the tile
+                if (ok && !mbar_wait(&bar_pv[3], (uint32_t)i & 1u)) ok = false;
                 tc_fence_after();
 #pragma unroll 1
                 for (int dc = 0; dc < 4; ++dc) {
-#pragma unroll
-                    for (int c = 0; c < HG; c += 8) {
-                        uint32_t r8[8];
-                        const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
-                        tmem_ld8(ta, r8);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) r8[j] = __float_as_uint(__uint_as_float(r8[j]) * alpha[grp * HG + c + j]);
-                        tmem_st8(ta, r8);
-                    }
-                }
-                tmem_wait_st();
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[b]);
-            if (!last) continue;
-
-            // ---- end of a segment: o of its query (or its partial) ----
-            const int64_t seg_start = max(x0, u * p.tpq);
-            const bool whole = seg_start == u * p.tpq && x == (u + 1) * p.tpq - 1;
-            const int32_t slot = whole ? 0 : sp.slot(g, u, part_base);
-            const bool f32 = !whole || p.o32 != nullptr;
-            if (lane % R == 0) red[quarter * H + hl] = l_acc;
-            l_acc = 0.0f;
-            named_bar_sync(kBarSm, kDecSmThreads);
-            if (stid < H) {
-                const float l = (red[stid] + red[H + stid]) + (red[2 * H + stid] + red[3 * H + stid]);
-                inv_l[stid] = l > 0.0f ? 1.0f / l : 0.0f;
-                const float lse = l > 0.0f ? (m_run[stid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                if (whole) {
-                    if (p.lse) p.lse[u * H + stid] = lse;
-                } else {
-                    p.lse_part[(int64_t)slot * H + stid] = lse;
-                }
-                m_run[stid] = -INFINITY;  // the next segment starts afresh
-            }
-            if (!whole && seg_start == u * p.tpq && stid == 0) p.qslot[u] = slot;  // the first part of u
-            named_bar_sync(kBarSm, kDecSmThreads);
-            // the P*V of this tile is the last product into O^T
-            if (ok && !mbar_wait(&kv_empty[b], (uint32_t)(t >> 1) & 1u)) ok = false;
-            tc_fence_after();
-            const int dl = quarter * 32 + lane;  // latent column within a chunk (TMEM lane)
-            float *o32 = whole ? (p.o32 ? p.o32 + u * H * CSA2_D : nullptr) : p.o_part + (int64_t)slot * H * CSA2_D;
-            uint16_t *o16 = p.o + u * H * CSA2_D;
-#pragma unroll 1
-            for (int dc = 0; dc < 4; ++dc) {
-#pragma unroll
-                for (int c = 0; c < HG; c += (HG >= 16 ? 16 : 8)) {
-                    uint32_t vals[16];
-                    const uint32_t ta = lane_addr + Cfg::kColO + dc * H + grp * HG + c;
-                    if (HG >= 16)
-                        tmem_ld16(ta, vals);
-                    else
+                    uint32_t vals[HG];
+                    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + Cfg::kColO + dc * H + grp * HG;
+                    if (HG == 16) {
+                        tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(&vals[0]));
+                    } else {
                         tmem_ld8(ta, *reinterpret_cast<uint32_t(*)[8]>(&vals[0]));
+                    }
                     tmem_wait_ld();
+                    if (f32) {
 #pragma unroll
-                    for (int j = 0; j < (HG >= 16 ? 16 : 8); ++j) {
-                        const int h = grp * HG + c + j;
-                        const float val = __uint_as_float(vals[j]) * inv_l[h];
-                        const int64_t at = (int64_t)h * CSA2_D + dc * 128 + dl;
-                        if (f32)
-                            o32[at] = val;
-                        else
-                            o16[at] = f32_to_bf16_bits(val);
+                        for (int j = 0; j < HG; ++j) {
+                            const int h = grp * HG + j;
+                            reinterpret_cast<float *>(kv_tile)[h * CSA2_D + dc * 128 + d0] =
+                                __uint_as_float(vals[j]) * alpha[h];
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < HG; ++j) {
+                            const int h = grp * HG + j;
+                            reinterpret_cast<uint16_t *>(kv_tile)[h * CSA2_D + dc * 128 + d0] =
+                                f32_to_bf16_bits(__uint_as_float(vals[j]) * alpha[h]);
+                        }
                     }
                 }
+                fence_proxy_async_smem();
             }
             tc_fence_before();
+            named_bar_sync(kBarWork, kDecWorkThreads);
+            if (warp == 0) {
+                uint8_t *dst = whole ? (p.o32 ? reinterpret_cast<uint8_t *>(p.o32 + u * H * CSA2_D)
+                                              : reinterpret_cast<uint8_t *>(p.o + u * H * CSA2_D))
+                                     : reinterpret_cast<uint8_t *>(p.o_part + (int64_t)slot * H * CSA2_D);
+                const uint32_t quarter_bytes = (uint32_t)(H * CSA2_D * es / 4);
+                if (lane < 4) {
+                    bulk_store(dst + lane * quarter_bytes, kv_tile + lane * quarter_bytes, quarter_bytes);
+                    bulk_commit();
+                }
+                if (!whole && seg_start == u * p.tpq && lane == 0) p.qslot[u] = slot;  // the first part of u
+            }
+            tc_fence_before();
+            if (tid < H) {
+                const float l = l_run[tid];
+                const float lse = l > 0.0f ? (m_run[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                if (whole) {
+                    if (p.lse) p.lse[u * H + tid] = lse;
+                } else {
+                    p.lse_part[(int64_t)slot * H + tid] = lse;
+                }
+                m_run[tid] = -INFINITY;  // the next segment starts afresh
+                l_run[tid] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < HG; ++j) l_part[j] = 0.0f;
+            if (has_next) load_q<H>(p, u + 1, q_tile);
+            if (warp == 0) bulk_wait_read();  // the KV tile may be overwritten again
+            // m_run is reset, the Q tile rewritten and the staging read before any
+            // thread starts the next tile (its dequantisation is followed by the
+            // fences and arrivals the tensor-core products wait for)
+            named_bar_sync(kBarWork, kDecWorkThreads);
         }
     }
+    if (warp == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
-    if (warp == kDecMmaWarp) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }

@@ -59,13 +59,14 @@ FullPath full_path_env() {
 }
 bool force_multipass() { return full_path_env() == kPathMultipass; }
 
-// CSA2_REINDEX=two: the two-launch Reindex (scores to global memory, then a
-// select CTA per query) even where the one-launch cluster path applies
-// (tests of both paths, tuning).
-bool reindex_two_launch() {
+// CSA2_REINDEX=cluster: the one-launch Reindex (a cluster of CTAs per query
+// scores into the first CTA's shared memory, which selects). It is correct
+// and tested but measured slower than the two-launch path (22 against about
+// 15 us cold on eight queries with 4096-id pools), so it is opt-in.
+bool reindex_cluster() {
     static const bool v = [] {
         const char *e = std::getenv("CSA2_REINDEX");
-        return e != nullptr && std::strcmp(e, "two") == 0;
+        return e != nullptr && std::strcmp(e, "cluster") == 0;
     }();
     return v;
 }
@@ -337,7 +338,7 @@ struct DecPlan {
 DecPlan plan_decode(int32_t nq, int32_t h, int32_t k, int32_t w_max, int sms) {
     DecPlan P{};
     const int64_t rows = (int64_t)k + std::max(0, w_max);
-    P.tpq = (int32_t)std::max<int64_t>(1, (rows + kDecRows - 1) / kDecRows);
+    P.tpq = (int32_t)std::max<int64_t>(1, (rows + kAttnTile - 1) / kAttnTile);
     const int64_t T = (int64_t)nq * P.tpq;
     int64_t per = (T + sms - 1) / sms;
     if (const char *e = std::getenv("CSA2_ATTN_PER")) per = std::max<int64_t>(1, std::atoll(e));  // tuning, tests
@@ -853,11 +854,10 @@ csa2_status csa2_index_reindex(const uint8_t *qidx, const float *w, int32_t nq, 
     rp.k = k;
     rp.hi = hi;
     rp.q_per_seq = q_per_seq;
-    // one launch: a cluster of CTAs per query scores the pool into the first
-    // CTA's shared memory, which selects; pools of more than 8 * 1024 ids take
-    // the two-launch path
+    // one launch (opt-in, see reindex_cluster): a cluster of CTAs per query
+    // scores the pool into the first CTA's shared memory, which selects
     const int cl = (p + kRcThreads - 1) / kRcThreads;
-    if (cl <= kRcMaxCluster && !reindex_two_launch()) {
+    if (cl <= kRcMaxCluster && reindex_cluster()) {
         const size_t rsm = 2048 * 4 + (kRcThreads / 32 + 8) * 4 + (size_t)p * 8;
         const dim3 rgrid((unsigned)cl, (unsigned)nq);
         if (kv->di == 64) {

@@ -641,39 +641,48 @@ __global__ void __launch_bounds__(kCollectThreads) k_sel_collect(BatchParams p, 
 #pragma unroll
         for (int r = 0; r < 4; ++r)
             k4[r] = t0 + 4 * r < c1 ? __ldcg(reinterpret_cast<const uint4 *>(kq + t0 + 4 * r)) : make_uint4(0u, 0u, 0u, 0u);
-        uint32_t ms = 0, mc = 0;  // bit i: key t0 + i is sure / a candidate
+        // bit i: key t0 + i is sure / a candidate
+        const int64_t left = c1 - t0;
+        const uint32_t inmask = left >= 16 ? 0xFFFFu : (left > 0 ? (1u << left) - 1u : 0u);
+        uint32_t ms = 0, mc = 0;
+        if (all) {
+            ms = inmask;
+        } else {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = 4 * r + j;
-                const bool in = t0 + i < c1;
-                const uint32_t d = kk[j] >> 20;
-                ms |= (uint32_t)(in && (all || d > b0)) << i;
-                mc |= (uint32_t)(in && !all && d == b0) << i;
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t d = kk[j] >> 20;
+                    ms |= (uint32_t)(d > b0) << (4 * r + j);
+                    mc |= (uint32_t)(d == b0) << (4 * r + j);
+                }
             }
+            ms &= inmask;
+            mc &= inmask;
         }
         // counts packed as sure | cand << 16 (each below 2^16 per round)
         uint32_t tot_r;
         const uint32_t ex = block_excl_scan<NT>((uint32_t)__popc(ms) | ((uint32_t)__popc(mc) << 16), scratch, &tot_r);
         uint32_t ps = n_s + (ex & 0xFFFFu), pc = n_c + (ex >> 16);
+        const int32_t tl = (int32_t)t0;
+        for (uint32_t m = ms; m; m &= m - 1u) {
+            if (ps < (uint32_t)p.sure_stride)
+                p.sure[part * p.sure_stride + ps] = tl + (int32_t)(__ffs(m) - 1);
+            else
+                set_error(CSA2_DEVERR_SELECT);
+            ++ps;
+        }
+        if (mc) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t kk[4] = {k4[r].x, k4[r].y, k4[r].z, k4[r].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = 4 * r + j;
-                const int64_t t = t0 + i;
-                if (ms & (1u << i)) {
-                    if (ps < (uint32_t)p.sure_stride)
-                        p.sure[part * p.sure_stride + ps] = (int32_t)t;
-                    else
-                        set_error(CSA2_DEVERR_SELECT);
-                    ++ps;
-                } else if (mc & (1u << i)) {
+                for (int j = 0; j < 4; ++j) {
+                    if (!(mc & (1u << (4 * r + j)))) continue;
+                    const uint32_t t = (uint32_t)(tl + 4 * r + j);
                     if ((int64_t)pc < p.chunk)
-                        p.cand[part * p.chunk + pc] = ((unsigned long long)kk[j] << 32) | (unsigned long long)(~(uint32_t)t);
+                        p.cand[part * p.chunk + pc] = ((unsigned long long)kk[j] << 32) | (unsigned long long)(~t);
                     else
                         set_error(CSA2_DEVERR_SELECT);
                     atomicAdd(&h1[(kk[j] >> kCollectShift1) & 2047u], 1u);

@@ -24,11 +24,10 @@ def test_full_indexer_multipass_path(cuda_device):
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
-def test_reindex_two_launch_path(cuda_device):
-    """The Reindex parity tests once more on the two-launch path (scores to
-    global memory, then a select CTA per query; CSA2_REINDEX=two) instead of
-    the one-launch cluster kernel."""
-    env = dict(os.environ, CSA2_REINDEX="two")
+def test_reindex_cluster_path(cuda_device):
+    """The Reindex parity tests once more on the one-launch cluster kernel
+    (CSA2_REINDEX=cluster) instead of the default two-launch path."""
+    env = dict(os.environ, CSA2_REINDEX="cluster")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
                         os.path.join(HERE, "test_indexer_gpu.py"), "-k", "reindex"],
                        env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
