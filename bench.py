@@ -73,11 +73,17 @@ def call_costs(recipe, lens, schedule):
     ql = recipe.q_limit()
     for l, (mode, src) in enumerate(schedule):
         if mode == "full":
+            # keys of a sequence are read once for all its queries (the widest
+            # visible range); every query scores each visible key
             b = f = 0.0
+            seq_n = {}
             for qi in range(nq):
                 n = int(ql[qi]) if ql is not None else n_vis[qi // recipe.q_per_seq]
-                b += n * recipe.di + 4 * (recipe.k + recipe.p)
+                sq = qi // recipe.q_per_seq
+                seq_n[sq] = max(seq_n.get(sq, 0), n)
+                b += 4 * (recipe.k + recipe.p) + recipe.hi * (recipe.di + 4)
                 f += 2.0 * recipe.hi * recipe.di * n
+            b += sum(seq_n.values()) * recipe.di
             out.append(("full", l, b, f, "fp8"))
         elif mode == "reindex":
             out.append(("reindex", l, nq * recipe.p * (recipe.di + 4) + nq * recipe.k * 4,

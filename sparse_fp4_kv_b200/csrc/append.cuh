@@ -14,12 +14,8 @@
 // codes and 1 scale byte, so a warp moves 1 KiB in and 288 B out with fully
 // coalesced 16-byte loads. HBM-bound: 1312 algorithmic bytes per row.
 //
-// The E2M1 rounding compares |x| against the seven decision points of the
-// grid scaled by value(s) instead of dividing. The products t * value(s)
-// are exact in binary32 (at most 3 + 4 significant bits), and for bf16 x
-// (8 significant bits) the quotient x / value(s) cannot land within half a
-// binary32 ulp of a decision point without being equal to it, so the
-// comparison gives the same code as rounding the binary32 quotient.
+// The E2M1 rounding is the hardware conversion of the correctly rounded
+// binary32 quotient x / value(s) (see quantize_block16).
 #pragma once
 
 #include "common.cuh"
@@ -31,34 +27,67 @@ constexpr int kAppendWarps = 8;
 // Quantise one block of 16 values (binary32 copies of bf16 or narrower
 // inputs) with the rule above: returns the E4M3 scale byte and writes the 16
 // E2M1 codes, element i in nibble i of packed[i / 8].
+// The code of x is the E2M1 rounding (cvt.rn.satfinite.e2m1x2, ties to the
+// even mantissa, saturating to 6) of the correctly rounded binary32 quotient
+// x / value(s): q0 = x * r with r ~ 1 / value(s) (rcp.approx), the remainder
+// x - q0 * value(s) by one fma, and q = q0 + remainder * r by another (the
+// fma remainder correction of Markstein's division). For bf16 x a quotient
+// that is not exactly a decision point of the grid is at least 2^-9 (relative)
+// away from one, far beyond the correction's error, and an exact decision
+// point is reproduced exactly, so the codes equal those of the exact quotient.
+// NaN inputs give a zero code with their sign, infinite ones the largest
+// code with their sign; value(s) = 0 gives all-zero codes.
+__device__ __forceinline__ uint32_t e2m1x2_of_f32(float hi, float lo) {
+    uint16_t out;
+    asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u16.u8 %0, b;\n\t}"
+        : "=h"(out)
+        : "f"(hi), "f"(lo));
+    return out & 0xFFu;
+}
+// Hardware reciprocal approximation (rcp.approx.f32: within a few ulps).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+// a / b for a finite a >= 0 and b > 0 with r ~ 1 / b (a few ulps): the
+// remainder correction above, which reproduces an exactly representable
+// quotient exactly; the scale needs it because amax / 6 can be an exact
+// E4M3 rounding midpoint. amax = +inf stays +inf.
+__device__ __forceinline__ float quotient_rn(float a, float b, float r) {
+    const float q0 = a * r;
+    const float q = fmaf(fmaf(-q0, b, a), r, q0);
+    return q == q ? q : q0;
+}
 __device__ __forceinline__ uint32_t quantize_block16(const float (&f)[16], uint32_t (&packed)[2]) {
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));  // fmaxf drops NaN operands
-    const uint32_t s = f32_to_e4m3_satfinite(__fdiv_rn(amax, 6.0f));
+    const uint32_t s = f32_to_e4m3_satfinite(quotient_rn(amax, 6.0f, 1.0f / 6.0f));
     const float sv = __half2float(__ushort_as_half((uint16_t)(e4m3x2_to_f16x2((uint16_t)s) & 0xFFFFu)));
-    // decision points of the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}; at an
-    // exact midpoint the even-mantissa neighbour wins ('>' keeps the lower
-    // point, '>=' takes the upper one)
-    const float t1 = 0.25f * sv, t2 = 0.75f * sv, t3 = 1.25f * sv, t4 = 1.75f * sv;
-    const float t5 = 2.5f * sv, t6 = 3.5f * sv, t7 = 5.0f * sv;
     packed[0] = packed[1] = 0u;
+    if (sv == 0.0f) return s;
+    const float r = rcp_approx(sv);
+    float q[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const float a = fabsf(f[i]);
-        uint32_t c = (uint32_t)(a > t1) + (uint32_t)(a >= t2) + (uint32_t)(a > t3) + (uint32_t)(a >= t4) +
-                     (uint32_t)(a > t5) + (uint32_t)(a >= t6) + (uint32_t)(a > t7);
-        c |= (__float_as_uint(f[i]) >> 31) << 3;
-        if (sv == 0.0f) c = 0u;
-        packed[i >> 3] |= c << (4 * (i & 7));
+        const float q0 = f[i] * r;
+        const float rem = fmaf(-q0, sv, f[i]);
+        const float qq = fmaf(rem, r, q0);
+        // an infinite x leaves q0 infinite (it saturates to 6) and a NaN remainder
+        q[i] = qq == qq ? qq : (f[i] == f[i] ? q0 : copysignf(0.0f, f[i]));
     }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) packed[j >> 2] |= e2m1x2_of_f32(q[2 * j + 1], q[2 * j]) << (8 * (j & 3));
     return s;
 }
 
-// A warp walks rows r, r + W, r + 2W, ... (W = warps in the grid). The
-// loads of its next row (input values and destination lookup) are issued
-// before the current row is quantised and stored, so every warp keeps two
-// rows in flight; the grid fills every SM.
+// A warp walks rows r, r + W, r + 2W, ... (W = warps in the grid) in batches
+// of kAppendBatch rows: the input values and destination lookups of a whole
+// batch are issued before any of its rows is quantised and stored, so every
+// warp has kAppendBatch rows in flight; the grid is one wave of resident CTAs.
+constexpr int kAppendBatch = 4;
+
 __device__ __forceinline__ int64_t append_dest(const csa2_kv_desc &kv, const int32_t *__restrict__ seq,
                                                const int64_t *__restrict__ pos, int64_t r) {
     const int32_t b = seq[r];
@@ -72,25 +101,28 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * kAppendWarps;
-    int64_t r = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
-    if (r >= n) return;
-    uint4 v0 = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16));
-    uint4 v1 = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16) + 1);
-    int64_t row = append_dest(kv, seq, pos, r);
-    for (; r < n; r += stride) {
-        // the next row's values and destination go in flight first
-        const int64_t rn = r + stride;
-        uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
-        int64_t row_n = -1;
-        if (rn < n) {
-            n0 = __ldg(reinterpret_cast<const uint4 *>(x + rn * CSA2_D + lane * 16));
-            n1 = __ldg(reinterpret_cast<const uint4 *>(x + rn * CSA2_D + lane * 16) + 1);
-            row_n = append_dest(kv, seq, pos, rn);
+    for (int64_t r0 = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5); r0 < n; r0 += kAppendBatch * stride) {
+        uint4 v[kAppendBatch][2];
+        int64_t row[kAppendBatch];
+#pragma unroll
+        for (int j = 0; j < kAppendBatch; ++j) {
+            const int64_t r = r0 + j * stride;
+            row[j] = -2;  // no row
+            if (r < n) {
+                v[j][0] = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16));
+                v[j][1] = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16) + 1);
+                row[j] = append_dest(kv, seq, pos, r);
+            }
         }
-        if (row < 0) {
-            if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
-        } else {
-            const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int j = 0; j < kAppendBatch; ++j) {
+            if (row[j] == -2) continue;
+            if (row[j] < 0) {
+                if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
+                continue;
+            }
+            const uint32_t wds[8] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w,
+                                     v[j][1].x, v[j][1].y, v[j][1].z, v[j][1].w};
             float f[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -101,12 +133,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
             const uint32_t s = quantize_block16(f, packed);
             // codes: 8 bytes per lane (256 contiguous bytes per warp); scales: one
             // byte per lane (the row's 32-byte sector in one warp store)
-            *reinterpret_cast<uint2 *>(kv.codes + row * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
-            kv.scales[row * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
+            *reinterpret_cast<uint2 *>(kv.codes + row[j] * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
+            kv.scales[row[j] * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
         }
-        v0 = n0;
-        v1 = n1;
-        row = row_n;
     }
 }
 

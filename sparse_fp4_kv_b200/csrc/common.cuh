@@ -35,7 +35,8 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 // lookup leaves the page table or the cache.
 __device__ __forceinline__ int64_t physical_row(const csa2_kv_desc &kv, int32_t b, int64_t t) {
     if (t < 0) return -1;
-    int64_t page = t / kv.page_size;
+    // 32-bit division when the position fits (always for int32 ids)
+    int64_t page = t < 0x80000000ll ? (int64_t)((uint32_t)t / (uint32_t)kv.page_size) : t / kv.page_size;
     if (page >= kv.max_pages) return -1;
     int64_t phys = kv.page_table[(int64_t)b * kv.max_pages + page];
     int64_t row = phys * kv.page_size + (t - page * kv.page_size);

@@ -174,13 +174,16 @@ BatchSplit batch_split(int32_t nq, int64_t n_max, int tile_entries, int sms, int
     return s;
 }
 
-// Parts of the multi-launch path's selection: about two collecting CTAs per
-// SM over all queries, parts of whole 2048-key steps, at most
-// kBatchMaxChunks parts per query.
+// Parts of the multi-launch path's selection: one round of the collecting
+// CTA (16 keys per thread, 8192 keys) per part, so that parts are short and
+// many, whatever the spread of the queries' lengths; more keys per part only
+// beyond kBatchMaxChunks parts per query.
 void collect_split(int32_t nq, int64_t n_max, int sms, int64_t &chunk, int32_t &parts) {
+    (void)nq;
+    (void)sms;
+    constexpr int64_t kRound = 16 * kCollectThreads;
     const int64_t n = std::max<int64_t>(n_max, 1);
-    chunk = std::max<int64_t>((int64_t)nq * n / (2 * sms), (n + kBatchMaxChunks - 1) / kBatchMaxChunks);
-    chunk = std::max<int64_t>(2048, (chunk + 2047) / 2048 * 2048);
+    chunk = std::max<int64_t>(kRound, ((n + kBatchMaxChunks - 1) / kBatchMaxChunks + kRound - 1) / kRound * kRound);
     parts = (int32_t)((n + chunk - 1) / chunk);
 }
 
@@ -569,10 +572,17 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
     if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
         return CSA2_ERR_INVALID_ARG;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
-    // every SM holds 8 CTAs of 8 warps; each warp walks rows with a stride and
-    // keeps two in flight
-    const int64_t want = (int64_t)num_sms() * 8;
-    const unsigned grid = (unsigned)std::min<int64_t>(want, ((int64_t)n + kAppendWarps - 1) / kAppendWarps);
+    // one wave of resident CTAs (each warp walks rows with a stride, a batch
+    // of rows in flight at a time), fewer when there are not enough rows
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_append_fp4, kAppendWarps * 32, 0) != cudaSuccess ||
+        per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const int64_t want = (int64_t)num_sms() * per_sm;
+    const int64_t rows_per_cta = (int64_t)kAppendWarps * kAppendBatch;
+    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, ((int64_t)n + rows_per_cta - 1) / rows_per_cta));
     launch(k_append_fp4, dim3(grid), dim3(kAppendWarps * 32), 0, stream, static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
     return check_launch();
 }
