@@ -59,6 +59,22 @@ FullPath full_path_env() {
 }
 bool force_multipass() { return full_path_env() == kPathMultipass; }
 
+// Batched Full path: CSA2_BATCH_MODE=exact skips the sampled threshold path
+// (two exact passes for every query), =redo runs it and hands every query to
+// the exact passes anyway (tests of the fallback). Default: sampled, with the
+// exact passes for the queries it cannot settle.
+enum BatchMode { kBatchSampled, kBatchExact, kBatchRedo };
+BatchMode batch_mode_env() {
+    static const BatchMode v = [] {
+        const char *e = std::getenv("CSA2_BATCH_MODE");
+        if (e == nullptr) return kBatchSampled;
+        if (std::strcmp(e, "exact") == 0) return kBatchExact;
+        if (std::strcmp(e, "redo") == 0) return kBatchRedo;
+        return kBatchSampled;
+    }();
+    return v;
+}
+
 // CSA2_REINDEX=cluster: the one-launch Reindex (a cluster of CTAs per query
 // scores into the first CTA's shared memory, which selects). It is correct
 // and tested but measured slower than the two-launch path (22 against about
@@ -143,6 +159,8 @@ struct FullLayout {
     int32_t c_sure_stride;
     size_t off_keys, off_hist0, off_state, off_hist1, off_cnt, off_sure, off_cand, total;
     size_t b_hist, b_state, b_cnt, b_sure, b_cand;  // batched path
+    size_t b_sstate, b_redo, b_samples;             // its sampled threshold path
+    int64_t sample_stride;
 };
 
 // Split of the batched Full path: query groups of qg queries, chunks of
@@ -221,6 +239,14 @@ FullLayout full_layout(int32_t nq, int64_t n_max) {
     b = align_up(b + (size_t)nq * bs.max_chunks * kBatchMaxK * 4, 256);
     L.b_cand = b;
     b = align_up(b + (size_t)nq * bs.max_span * 8, 256);
+    L.b_sstate = b;
+    b = align_up(b + (size_t)nq * 2 * 4, 256);
+    L.b_redo = b;
+    b = align_up(b + (size_t)nq * 4, 256);
+    L.b_samples = b;
+    // every kSampleStride-th tile of 256 (di = 64) or 128 entries; sized for 256
+    L.sample_stride = ((std::max<int64_t>(n_max, 1) + (int64_t)kSampleStride * 128 - 1) / ((int64_t)kSampleStride * 128) + 1) * 256;
+    b = align_up(b + (size_t)nq * L.sample_stride * 4, 256);
     L.total = std::max(off, b);
     return L;
 }
@@ -517,7 +543,7 @@ bool prefer_shared(K kernel) {
 bool init_small_kernels() {
     static const char key = 0;
     return once_per_device(&key, [] {
-        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) &&
+        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) && prefer_shared(k_batch_sthresh) && prefer_shared(k_batch_thresh) &&
                prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
                prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
                prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
@@ -687,6 +713,52 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
             bp.nchunks = (int32_t)((std::max<int64_t>(n_max, 1) + bp.chunk - 1) / bp.chunk);
             if (bp.chunk / kv->page_size + 2 > kMaxScanPages) return CSA2_ERR_UNSUPPORTED;
             const dim3 sgrid((unsigned)bp.nchunks, (unsigned)ngroups);
+            const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
+            if (!smem_attr(k_batch_final, fsm)) return CSA2_ERR_CUDA;
+            const size_t ffixed =
+                2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + 4 * kBatchMaxChunks * 4 + (size_t)kBatchMaxK * 4;
+            const int32_t smem_keys = (int32_t)((fsm - ffixed) / 8);
+            const BatchMode mode = batch_mode_env();
+            // Sampled threshold path: sample pass (every kSampleStride-th tile),
+            // per-query threshold, one collecting pass (every key at or above
+            // the threshold), exact select; queries with too few candidates are
+            // marked for the exact passes that follow.
+            uint32_t *redo = reinterpret_cast<uint32_t *>(wsb + L.b_redo);
+            if (mode != kBatchExact) {
+                BatchParams sp = bp;
+                sp.state = reinterpret_cast<uint32_t *>(wsb + L.b_sstate);
+                sp.samples = reinterpret_cast<uint32_t *>(wsb + L.b_samples);
+                sp.sample_stride = L.sample_stride;
+                sp.tile_stride = kSampleStride;
+                sp.sample_rank = (int32_t)((3 * (int64_t)k + 2 * kSampleStride - 1) / (2 * kSampleStride)) + 32;
+                if (cudaMemsetAsync(redo, 0, (size_t)nq * 4, stream) != cudaSuccess) return CSA2_ERR_CUDA;
+                auto spass = [&](auto k2, auto k3, size_t sm2, size_t sm3) -> csa2_status {
+                    if (!smem_attr(k2, sm2) || !smem_attr(k3, sm3)) return CSA2_ERR_CUDA;
+                    launch(k2, sgrid, dim3(kBatchThreads), sm2, stream, bm, sp);
+                    launch(k_batch_sthresh, dim3((unsigned)nq), dim3(kSthreshThreads), 0, stream, sp);
+                    launch(k3, sgrid, dim3(kBatchThreads), sm3, stream, bm, sp);
+                    return CSA2_OK;
+                };
+                csa2_status ss;
+                if (kv->di == 64 && hp == 4)
+                    ss = spass(k_batch_scan<64, 4, 2>, k_batch_scan<64, 4, 3>, BatchCfg<64, 4, 2>::kSmem,
+                               BatchCfg<64, 4, 3>::kSmem);
+                else if (kv->di == 64)
+                    ss = spass(k_batch_scan<64, 8, 2>, k_batch_scan<64, 8, 3>, BatchCfg<64, 8, 2>::kSmem,
+                               BatchCfg<64, 8, 3>::kSmem);
+                else if (hp == 4)
+                    ss = spass(k_batch_scan<128, 4, 2>, k_batch_scan<128, 4, 3>, BatchCfg<128, 4, 2>::kSmem,
+                               BatchCfg<128, 4, 3>::kSmem);
+                else
+                    ss = spass(k_batch_scan<128, 8, 2>, k_batch_scan<128, 8, 3>, BatchCfg<128, 8, 2>::kSmem,
+                               BatchCfg<128, 8, 3>::kSmem);
+                if (ss != CSA2_OK) return ss;
+                sp.redo = redo;
+                sp.redo_mark = mode == kBatchRedo ? 2 : 1;
+                launch(k_batch_final, dim3((unsigned)nq), dim3(kBatchFinalThreads), fsm, stream, sp, smem_keys);
+                bp.redo = redo;  // the exact passes below take only the marked queries
+            }
+            // Exact path: two scans with a digit-0 histogram and threshold bin.
             if (cudaMemsetAsync(bp.hist, 0, (size_t)nq * kBatchBins * 4, stream) != cudaSuccess) return CSA2_ERR_CUDA;
             auto scan = [&](auto k0, auto k1, size_t sm0, size_t sm1) -> csa2_status {
                 if (!smem_attr(k0, sm0) || !smem_attr(k1, sm1)) return CSA2_ERR_CUDA;
@@ -709,11 +781,6 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
                 bs = scan(k_batch_scan<128, 8, 0>, k_batch_scan<128, 8, 1>, BatchCfg<128, 8, 0>::kSmem,
                           BatchCfg<128, 8, 1>::kSmem);
             if (bs != CSA2_OK) return bs;
-            const size_t fsm = (size_t)max_smem_optin() - 1024;  // leaves room for the static shared words
-            if (!smem_attr(k_batch_final, fsm)) return CSA2_ERR_CUDA;
-            const size_t ffixed =
-                2048 * 4 + (kBatchFinalThreads / 32 + 8) * 4 + 4 * kBatchMaxChunks * 4 + (size_t)kBatchMaxK * 4;
-            const int32_t smem_keys = (int32_t)((fsm - ffixed) / 8);
             launch(k_batch_final, dim3((unsigned)nq), dim3(kBatchFinalThreads), fsm, stream, bp, smem_keys);
             return check_launch();
         }

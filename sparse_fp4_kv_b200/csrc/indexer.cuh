@@ -239,12 +239,45 @@ template <int DI>
 __device__ __forceinline__ void scan_tma_loop(const csa2_kv_desc &kv, const int32_t *ptab, int64_t start,
                                               int64_t limit, int ntiles, int nstages, int box_rows,
                                               uint8_t *stage_base, const CUtensorMap *tm, uint64_t *full_b,
-                                              uint64_t *empty_b) {
+                                              uint64_t *empty_b, int tile_stride = 1,
+                                              const int32_t *pt_row = nullptr) {
     using G = ScanGeom<DI>;
     const bool leader = (threadIdx.x & 31) == 0;
     const int nbox = 128 / box_rows;
     const int32_t step = box_rows * G::kEpr;  // entries per box
     const int32_t ps = kv.page_size;
+    if (tile_stride > 1) {
+        // every tile_stride-th tile from start (a sample of the range): the
+        // page of each box is read from the sequence's page-table row
+        int s = 0;
+        uint32_t phase = 0;
+        const int64_t lim = limit;
+        for (int i = 0; i < ntiles; ++i) {
+            if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
+            const int64_t t0 = start + (int64_t)i * tile_stride * G::kTile;
+            int nvalid = 0;
+            for (int j = 0; j < nbox; ++j) nvalid += (t0 + (int64_t)j * step < lim);
+            if (leader) mbar_arrive_expect_tx(&full_b[s], (uint32_t)(nvalid * box_rows * 128));
+            for (int j = 0; j < nvalid; ++j) {
+                if (!leader) break;
+                const int64_t pos = t0 + (int64_t)j * step;
+                const int64_t pg = pos / ps;
+                const int64_t phys = pg < kv.max_pages ? (int64_t)pt_row[pg] : -1;
+                int64_t row = phys * ps + pos % ps;
+                if (phys < 0 || row + step > kv.rows_cap) {
+                    set_error(CSA2_DEVERR_BAD_ROW);
+                    row = 0;
+                }
+                tma_load_2d(stage_base + (size_t)s * G::kStageBytes + j * box_rows * 128, tm, &full_b[s], 0,
+                            (int32_t)(row / G::kEpr));
+            }
+            if (++s == nstages) {
+                s = 0;
+                phase ^= 1u;
+            }
+        }
+        return;
+    }
     // entry positions fit in 32 bits (sequence lengths are int32)
     int32_t pi = 0, off = (int32_t)(start % ps);
     int32_t t = (int32_t)start;

@@ -39,6 +39,7 @@ constexpr int kBatchEpiWarps = 16;  // 4 per TMEM lane quarter
 constexpr int kBatchThreads = 64 + kBatchEpiWarps * 32;
 constexpr int kBatchFinalThreads = 1024;
 constexpr int kBatchMaxK = 8192;   // ids staged and sorted in shared memory
+constexpr int kSampleStride = 32;  // the sampled threshold path reads every 32nd tile first
 constexpr uint32_t kBatchAll = 0xFFFFFFFFu;  // b0 marker: every visible entry is taken
 
 struct BatchParams {
@@ -59,6 +60,13 @@ struct BatchParams {
     uint32_t *hist1;            // [nq][2048] digit-1 histogram of the candidates, or null
     int32_t shift1;             // digit 1 = bits shift1 .. shift1 + 10 of the score key
     int32_t parts_sorted;       // every part's lists are in ascending id order
+    // sampled threshold path
+    uint32_t *samples;          // [nq][sample_stride]: score keys of every tile_stride-th tile (0: not visible)
+    int64_t sample_stride;
+    int32_t tile_stride;
+    int32_t sample_rank;        // the threshold is the sample_rank-th largest sampled key
+    uint32_t *redo;             // [nq]: 1 where the sampled path could not settle the query, or null
+    int32_t redo_mark;          // final: mark (instead of writing) queries with too few candidates
     int32_t k, q_per_seq, hi, hi_pad, nq, box_rows;
 };
 
@@ -92,7 +100,7 @@ struct BatchCfg {
     using G = BatchGeom<DI>;
     static constexpr int QG = batch_qg(HP);
     static constexpr int N = G::kEpr * QG * HP;
-    static constexpr int kStages = PASS == 0 ? 4 : 8;
+    static constexpr int kStages = PASS == 0 || PASS == 2 ? 4 : 8;
     static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128u : 256u;
     static constexpr size_t kSmem = 1024 + (size_t)kStages * G::kStageBytes + (size_t)N * 128 +
                                     (PASS == 0 ? (size_t)QG * kBatchBins * 4 : 0) + 16 * 16 * 4 + 16 * 4 * 4 +
@@ -148,12 +156,19 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
     }
     pdl_wait();
     if (tid == 0) group_limit<QG>(p, gq, lim);
+    if (p.redo != nullptr && tid < QG) {
+        // fallback run of the exact passes: only the queries the sampled path
+        // could not settle are scanned (the others look empty)
+        if (q0 + tid >= p.nq || __ldcg(p.redo + q0 + tid) == 0u) lim[tid] = 0;
+    }
     __syncthreads();
     int64_t gl = 0;
     for (int j = 0; j < QG; ++j) gl = max(gl, (int64_t)lim[j]);
+    // PASS 2 takes every tile_stride-th tile of its range (a sample)
+    const int tstride = PASS == 2 ? p.tile_stride : 1;
     const int64_t start = (int64_t)blockIdx.x * p.chunk;
     const int64_t n_loc = max((int64_t)0, min(gl, start + p.chunk) - start);
-    const int ntiles = (int)((n_loc + G::kTile - 1) / G::kTile);
+    const int ntiles = (int)((n_loc + (int64_t)tstride * G::kTile - 1) / ((int64_t)tstride * G::kTile));
     // B: rows (u, j, h) = u * QG * HP + j * HP + h hold query j's head h
     // in the 64-byte half u of a 128-byte row (DI = 64), zero elsewhere
     for (int i = tid; i < N * 8; i += kBatchThreads) {
@@ -176,11 +191,11 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
         const int32_t qi = q0 + j;
         wq[i] = (qi < p.nq && h < p.hi) ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
     }
-    if (PASS == 1 && tid < QG) {
+    if ((PASS == 1 || PASS == 3) && tid < QG) {
         b0s[tid] = q0 + tid < p.nq ? __ldcg(p.state + (int64_t)(q0 + tid) * p.state_stride + p.state_off) : 0u;
         lcnt[2 * tid] = lcnt[2 * tid + 1] = 0u;
     }
-    if (ntiles > 0) stage_pages(p.kv, b, start, n_loc, ptab, kBatchThreads);
+    if (ntiles > 0 && PASS != 2) stage_pages(p.kv, b, start, n_loc, ptab, kBatchThreads);
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -188,7 +203,8 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        scan_tma_loop<DI>(p.kv, ptab, start, gl, ntiles, kStages, p.box_rows, stages, &tm, full_b, empty_b);
+        scan_tma_loop<DI>(p.kv, ptab, start, gl, ntiles, kStages, p.box_rows, stages, &tm, full_b, empty_b, tstride,
+                          p.kv.page_table + (int64_t)b * p.kv.max_pages);
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_e4m3_f32(128, N);
@@ -220,6 +236,19 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
         const int ew = warp - 2;
         const int quarter = warp & 3, sub = ew >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        // this warp's queries: head weights, visible limits (relative to the
+        // CTA's range) and thresholds in registers for the whole loop
+        float wr[QW][HP];
+        int32_t limr[QW];
+        uint32_t b0r[QW];
+#pragma unroll
+        for (int jj = 0; jj < QW; ++jj) {
+            const int j = sub * QW + jj;
+#pragma unroll
+            for (int h = 0; h < HP; ++h) wr[jj][h] = wq[j * 16 + h];
+            limr[jj] = (int32_t)max((int64_t)-1, min((int64_t)lim[j] - start, (int64_t)INT32_MAX));
+            b0r[jj] = PASS == 1 || PASS == 3 ? b0s[j] : 0u;
+        }
         for (int i = 0; i < ntiles; ++i) {
             const int a = i & 1;
             const bool got = mbar_wait(&tfull[a], (i >> 1) & 1);
@@ -232,21 +261,46 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
                 const uint32_t col = (uint32_t)(a * N + u * QG * HP + sub * QW * HP);
                 tmem_ld16(lane_base + col, r);
                 tmem_wait_ld();
-                const int64_t t = start + (int64_t)i * G::kTile + (int64_t)G::kEpr * (quarter * 32 + lane) + u;
+                const int64_t tile0 = start + (int64_t)i * tstride * G::kTile;
+                const int64_t t = tile0 + (int64_t)G::kEpr * (quarter * 32 + lane) + u;
+                const int32_t trel = (int32_t)(t - start);  // < chunk
 #pragma unroll
                 for (int jj = 0; jj < QW; ++jj) {
                     const int j = sub * QW + jj;
                     float sc = 0.0f;
 #pragma unroll
-                    for (int h = 0; h < HP; ++h)
-                        sc = fmaf(wq[j * 16 + h], fmaxf(__uint_as_float(r[jj * HP + h]), 0.0f), sc);
+                    for (int h = 0; h < HP; ++h) sc = fmaf(wr[jj][h], fmaxf(__uint_as_float(r[jj * HP + h]), 0.0f), sc);
                     const uint32_t key = score_key(sc + 0.0f);
-                    const bool vis = t < (int64_t)lim[j];
+                    const bool vis = trel < limr[jj];
                     const int32_t qi = q0 + j;
                     if (PASS == 0) {
                         if (vis) atomicAdd(&hist[j * kBatchBins + (key >> kBatchShift)], 1u);
+                    } else if (PASS == 2) {
+                        // sample slot: sample tile (tile0 / kTile / tstride), entry in tile;
+                        // 0 (no score has it) where the entry is not visible
+                        if (qi < p.nq) {
+                            const int64_t js = tile0 / ((int64_t)tstride * G::kTile);
+                            p.samples[(int64_t)qi * p.sample_stride + js * G::kTile + (t - tile0)] = vis ? key : 0u;
+                        }
+                    } else if (PASS == 3) {
+                        const bool cand = vis && key >= b0r[jj];
+                        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, cand);
+                        if (mc) {
+                            const int64_t part = (int64_t)qi * p.nchunks + blockIdx.x;
+                            uint32_t base0 = 0;
+                            if (lane == 0) base0 = atomicAdd(&lcnt[2 * j + 1], (uint32_t)__popc(mc));
+                            base0 = __shfl_sync(0xFFFFFFFFu, base0, 0);
+                            if (cand) {
+                                const uint32_t at = base0 + __popc(mc & ((1u << lane) - 1u));
+                                if ((int64_t)at < p.chunk)
+                                    p.cand[part * p.chunk + at] =
+                                        ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)t);
+                                else
+                                    set_error(CSA2_DEVERR_SELECT);
+                            }
+                        }
                     } else {
-                        const uint32_t b0 = b0s[j];
+                        const uint32_t b0 = b0r[jj];
                         const uint32_t d = key >> kBatchShift;
                         const bool sure = vis && (b0 == kBatchAll || d > b0);
                         const bool cand = vis && b0 != kBatchAll && d == b0;
@@ -293,7 +347,8 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, tcols);
     }
-    if (PASS == 1 && tid < QG && q0 + tid < p.nq) {
+    if ((PASS == 1 || PASS == 3) && tid < QG && q0 + tid < p.nq &&
+        (p.redo == nullptr || __ldcg(p.redo + q0 + tid) != 0u)) {
         uint32_t *c = p.cnt + ((int64_t)(q0 + tid) * p.nchunks + blockIdx.x) * 2;
         c[0] = min(lcnt[2 * tid], (uint32_t)p.sure_stride);
         c[1] = lcnt[2 * tid + 1];
@@ -316,6 +371,7 @@ __global__ void __launch_bounds__(kBatchThreshThreads) k_batch_thresh(BatchParam
     pdl_trigger();
     pdl_wait();
     const int32_t qi = blockIdx.x;
+    if (p.redo != nullptr && __ldcg(p.redo + qi) == 0u) return;  // settled by the sampled path
     const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
     uint32_t bin = kBatchAll, rem = 0;
     if ((int64_t)p.k < limit)
@@ -325,6 +381,65 @@ __global__ void __launch_bounds__(kBatchThreshThreads) k_batch_thresh(BatchParam
         uint32_t *st = p.state + (int64_t)qi * p.state_stride + p.state_off;
         st[0] = bin;
         st[1] = rem;
+    }
+}
+
+// Sampled threshold path, per query: the sample_rank-th largest of the keys
+// the sampling pass recorded (every tile_stride-th tile of the query's
+// range), by an exact radix select in three digits (11, 11, 10 bits) over
+// those keys (read through L2 in every pass). Every visible entry whose key
+// is at least that threshold becomes a candidate in the collecting pass, so
+// about sample_rank * tile_stride entries do; with fewer sampled keys than
+// sample_rank the threshold is 0 and every visible entry is a candidate.
+// state: [0] the threshold, [1] k.
+constexpr int kSthreshThreads = 512;
+__global__ void __launch_bounds__(kSthreshThreads) k_batch_sthresh(BatchParams p) {
+    constexpr int NT = kSthreshThreads;
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t scratch[NT / 32 + 4];
+    pdl_trigger();
+    pdl_wait();
+    const int32_t qi = blockIdx.x;
+    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+    const int64_t tile = 128 * (128 / p.kv.di);
+    const int64_t span = (int64_t)p.tile_stride * tile;
+    const int64_t ns = min((limit + span - 1) / span * tile, p.sample_stride);
+    const uint32_t *src = p.samples + (int64_t)qi * p.sample_stride;
+    uint32_t prefix = 0u, pmask = 0u, rem = (uint32_t)p.sample_rank;
+    bool enough = true;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    for (int d = 0; d < 3 && enough; ++d) {
+        const int sh = shifts[d], nb = 1 << widths[d];
+        for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0u;
+        __syncthreads();
+        for (int64_t i0 = threadIdx.x; i0 < ns; i0 += 4 * NT) {
+            uint32_t v[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) v[r] = i0 + r * NT < ns ? __ldcg(src + i0 + r * NT) : 0u;
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                if (v[r] != 0u && (v[r] & pmask) == prefix) atomicAdd(&hist[(v[r] >> sh) & (uint32_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        if (d == 0) {
+            uint32_t c = 0;
+            for (int i = threadIdx.x; i < nb; i += NT) c += hist[i];
+            uint32_t total;
+            block_excl_scan<NT>(c, scratch, &total);
+            enough = total >= rem;
+            if (!enough) break;
+        }
+        uint32_t bin, inbin;
+        find_rank_bin<NT, 2048 / NT, false>(hist, nb, rem, scratch, bin, inbin);
+        prefix |= bin << sh;
+        pmask |= (uint32_t)(nb - 1) << sh;
+        rem = inbin;
+    }
+    if (threadIdx.x == 0) {
+        uint32_t *st = p.state + (int64_t)qi * p.state_stride + p.state_off;
+        st[0] = enough ? prefix : 0u;
+        st[1] = (uint32_t)p.k;
     }
 }
 
@@ -382,6 +497,10 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
     const int32_t qi = blockIdx.x;
     const int nch = min(p.nchunks, kBatchMaxChunks);
     pdl_trigger();
+    if (p.redo != nullptr && !p.redo_mark) {
+        pdl_wait();
+        if (__ldcg(p.redo + qi) == 0u) return;  // settled by the sampled path
+    }
     if (threadIdx.x == 0) {
         and_acc = ~0ull;
         or_acc = 0ull;
@@ -407,6 +526,15 @@ __global__ void __launch_bounds__(kBatchFinalThreads, 1) k_batch_final(BatchPara
     const uint32_t b0 = __ldcg(stq), need = __ldcg(stq + 1);
     const uint32_t n_sure = min(tot[0], (uint32_t)p.k);
     const uint32_t n_cand = tot[1];
+    if (p.redo_mark) {
+        // sampled path: fewer candidates than the query needs (the sample put
+        // the threshold too high) -> left to the exact passes
+        const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+        if ((int64_t)(n_sure + n_cand) < min((int64_t)p.k, limit) || p.redo_mark > 1) {
+            if (threadIdx.x == 0) p.redo[qi] = 1u;
+            return;
+        }
+    }
     const int64_t part0 = (int64_t)qi * p.nchunks;
     // the sure ids first, flattened over the parts
     for (uint32_t j0 = threadIdx.x; j0 < n_sure; j0 += 4 * NT) {

@@ -227,3 +227,24 @@ def test_full_batched_largest_dot_products(B, cuda_device):
         v = np.where(rng.random((cap, di)) < 0.97, 8.0, -8.0).astype(np.float32)
         return torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     _run_full(B, cuda_device, [4000], 4096, 128, 8, 333, 0, q_per_seq=64, kidx_fn=extreme, seed=25, shuffle=False)
+
+
+def test_full_batched_sample_misses_leave_it_to_the_exact_passes(B, cuda_device):
+    # the batched path first samples every 32nd tile of 256 entries (entries
+    # [8192 j, 8192 j + 256)) and takes the keys at or above a threshold from
+    # that sample; here exactly those tiles hold the largest scores, so the
+    # threshold leaves fewer than k candidates and the exact passes must take
+    # over (the result is checked against the oracle as usual)
+    total = 40000
+
+    def sampled_high(cap, di):
+        rng = np.random.default_rng(26)
+        v = np.where(rng.random(di) < 0.5, 1.0, -1.0).astype(np.float32)
+        t = np.arange(cap)
+        high = (t % 8192) < 256
+        mag = np.where(high, rng.choice([4.0, 6.0], cap), rng.choice([0.5, 1.0], cap)).astype(np.float32)
+        x = mag[:, None] * v[None, :]
+        return torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    _run_full(B, cuda_device, [total], 40960, 64, 4, 600, 0, q_per_seq=64, kidx_fn=sampled_high, seed=26,
+              shuffle=False)

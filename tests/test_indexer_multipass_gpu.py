@@ -32,3 +32,16 @@ def test_reindex_cluster_path(cuda_device):
                         os.path.join(HERE, "test_indexer_gpu.py"), "-k", "reindex"],
                        env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("mode", ["exact", "redo"])
+def test_batched_full_modes(cuda_device, mode):
+    """The batched Full parity tests once more with the exact two-pass path
+    alone (CSA2_BATCH_MODE=exact) and with every query handed from the sampled
+    threshold path to the exact passes (=redo), the fallback the sampled path
+    takes when its threshold leaves too few candidates."""
+    env = dict(os.environ, CSA2_BATCH_MODE=mode)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        os.path.join(HERE, "test_indexer_gpu.py"), "-k", "batched"],
+                       env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
