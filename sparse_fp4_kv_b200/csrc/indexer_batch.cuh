@@ -101,7 +101,10 @@ struct BatchCfg {
     static constexpr int QG = batch_qg(HP);
     static constexpr int N = G::kEpr * QG * HP;
     static constexpr int kStages = PASS == 0 || PASS == 2 ? 4 : 8;
-    static constexpr uint32_t kTmemCols = 2 * N <= 128 ? 128u : 256u;
+    // TMEM accumulators: the products run up to three tiles ahead (two for the
+    // sample pass, two of whose CTAs can share an SM)
+    static constexpr int kAcc = PASS == 2 ? 2 : 4;
+    static constexpr uint32_t kTmemCols = kAcc * N <= 128 ? 128u : (kAcc * N <= 256 ? 256u : 512u);
     static constexpr size_t kSmem = 1024 + (size_t)kStages * G::kStageBytes + (size_t)N * 128 +
                                     (PASS == 0 ? (size_t)QG * kBatchBins * 4 : 0) + 16 * 16 * 4 + 16 * 4 * 4 +
                                     (size_t)kMaxScanPages * 4 + 256;
@@ -128,8 +131,8 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
     uint64_t *full_b = reinterpret_cast<uint64_t *>(ptab + kMaxScanPages);
     uint64_t *empty_b = full_b + kStages;
     uint64_t *tfull = empty_b + kStages;
-    uint64_t *tempty = tfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint64_t *tempty = tfull + Cfg::kAcc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + Cfg::kAcc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int32_t gq = blockIdx.y;
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
             mbar_init(&full_b[s], 1);
             mbar_init(&empty_b[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < Cfg::kAcc; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], kBatchEpiWarps);
         }
@@ -212,8 +215,8 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
             int s = 0;
             uint32_t phase = 0;
             for (int i = 0; i < ntiles; ++i) {
-                const int a = i & 1;
-                if (!mbar_wait(&tempty[a], ((i >> 1) & 1) ^ 1)) break;
+                const int a = i % Cfg::kAcc;
+                if (!mbar_wait(&tempty[a], ((i / Cfg::kAcc) & 1) ^ 1)) break;
                 if (!mbar_wait(&full_b[s], phase)) break;
                 tc_fence_after();
                 const uint32_t aaddr = smem_u32(stages + (size_t)s * G::kStageBytes);
@@ -250,17 +253,19 @@ __global__ void __launch_bounds__(kBatchThreads, 1)
             b0r[jj] = PASS == 1 || PASS == 3 ? b0s[j] : 0u;
         }
         for (int i = 0; i < ntiles; ++i) {
-            const int a = i & 1;
-            const bool got = mbar_wait(&tfull[a], (i >> 1) & 1);
+            const int a = i % Cfg::kAcc;
+            const bool got = mbar_wait(&tfull[a], (i / Cfg::kAcc) & 1);
             if (!__all_sync(0xFFFFFFFFu, got)) break;
             tc_fence_after();
+            // both halves' 16 columns of this warp's queries in flight at once
+            uint32_t rr[G::kEpr][16];
+#pragma unroll
+            for (int u = 0; u < G::kEpr; ++u)
+                tmem_ld16(lane_base + (uint32_t)(a * N + u * QG * HP + sub * QW * HP), rr[u]);
+            tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < G::kEpr; ++u) {
-                // the 16 columns of this warp's queries in half u
-                uint32_t r[16];
-                const uint32_t col = (uint32_t)(a * N + u * QG * HP + sub * QW * HP);
-                tmem_ld16(lane_base + col, r);
-                tmem_wait_ld();
+                const uint32_t(&r)[16] = rr[u];
                 const int64_t tile0 = start + (int64_t)i * tstride * G::kTile;
                 const int64_t t = tile0 + (int64_t)G::kEpr * (quarter * 32 + lane) + u;
                 const int32_t trel = (int32_t)(t - start);  // < chunk
