@@ -314,15 +314,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
         int32_t b = 0, wb = 0, nw = 0, one_page_pt = -1;
         const bool one_page = p.kv.max_pages == 1;
         const uint8_t *swa_seq = nullptr;
-        for (int i = 0; i < n; ++i) {
+        // query u and tile t of the query advance without divisions
+        int64_t u = x0 / p.tpq;
+        int32_t t = (int32_t)(x0 - u * p.tpq);
+        for (int i = 0; i < n; ++i, ++t) {
+            if (t == p.tpq) {
+                t = 0;
+                ++u;
+            }
             const int slot = i % kResRing;
             if (i >= kResRing && !mbar_wait(&res_empty[slot], (uint32_t)((i / kResRing) - 1) & 1u)) break;
-            const int64_t x = x0 + i;
-            const int64_t u = x / p.tpq;
-            const int64_t t = x - u * p.tpq;
             if (u != u_cur) {
                 u_cur = u;
-                b = (int32_t)(u / p.q_per_seq);
+                b = (int32_t)u / p.q_per_seq;
                 wb = p.swa_begin ? p.swa_begin[u] : 0;
                 nw = p.swa_begin ? max(0, p.swa_end[u] - wb) : 0;
                 // a window is a run of ring slots: begin in [0, stride), at most
@@ -402,10 +406,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
             const uint64_t a_o = make_sdesc(kv_addr, 16384, 1024, kSw128);
             const uint64_t b_o = make_sdesc(p_addr, 16, Cfg::kPGroup, Cfg::kPSwizzle);
             bool ok = true;
-            for (int i = 0; i < n && ok; ++i) {
+            int32_t tq = (int32_t)(x0 % p.tpq);  // tile of its query
+            for (int i = 0; i < n && ok; ++i, ++tq) {
+                if (tq == p.tpq) tq = 0;
                 const uint32_t ph = (uint32_t)i & 1u;
-                const int64_t x = x0 + i;
-                const bool first = i == 0 || x % p.tpq == 0;
+                const bool first = i == 0 || tq == 0;
 #pragma unroll 1
                 for (int c = 0; c < 4 && ok; ++c) {
                     if (!mbar_wait(&bar_kv[c], ph)) {
@@ -451,7 +456,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
         raw.kind = 0;
         // tile 0's rows, then Q of its query
         int64_t u_cur = x0 / p.tpq;
-        const uint8_t *swa_seq = p.swa ? p.swa + (u_cur / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
+        int32_t tq0 = (int32_t)(x0 - u_cur * p.tpq);  // tile of its query, advanced without divisions
+        const uint8_t *swa_seq = p.swa ? p.swa + (int64_t)((int32_t)u_cur / p.q_per_seq) * p.swa_seq_stride * CSA2_D
+                                       : nullptr;
         if (n > 0) {
             // Q of the first query does not depend on the resolved rows: its bf16
             // bytes go into the (still unused) KV tile by cp.async first, the first
@@ -481,10 +488,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
             }
             named_bar_sync(kBarWork, kDecWorkThreads);  // the KV tile is free for the first dequantisation
         }
-        for (int i = 0; i < n; ++i) {
+        int64_t u = u_cur;
+        int32_t tq = tq0;
+        for (int i = 0; i < n; ++i, ++tq) {
+            if (tq == p.tpq) {
+                tq = 0;
+                ++u;
+            }
             const int64_t x = x0 + i;
-            const int64_t u = x / p.tpq;
-            const bool last = i == n - 1 || (x + 1) % p.tpq == 0;
+            const bool last = i == n - 1 || tq == p.tpq - 1;
             // 1. dequantise chunk c once the previous tile's P*V on it is done
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -508,8 +520,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&res_empty[slot]);
-                const int64_t un = (x + 1) / p.tpq;
-                const uint8_t *sn = p.swa ? p.swa + (un / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
+                const int64_t un = tq == p.tpq - 1 ? u + 1 : u;
+                const uint8_t *sn =
+                    p.swa ? p.swa + (int64_t)((int32_t)un / p.q_per_seq) * p.swa_seq_stride * CSA2_D : nullptr;
                 gather_row(p, sn, src, kd, m, raw);
             }
             // 3. online softmax: thread = row (TMEM lane), warps 4g..4g+3 take
