@@ -36,7 +36,7 @@
 namespace csa2 {
 
 constexpr int kScanTile = 128;
-constexpr int kScanThreads = 320;  // TMA warp, MMA warp, 8 epilogue warps (two per TMEM lane quarter)
+constexpr int kScanThreads = 192;
 constexpr int kScanN = 16;  // MMA N: indexer heads padded to 16
 constexpr int kHist0Bins = 4096;
 
@@ -58,7 +58,7 @@ struct ScanGeom {
 
 template <int DI>
 struct ScanCfg {
-    static constexpr int kStages = 5;  // two CTAs per SM: 160 KiB of keys in flight per SM
+    static constexpr int kStages = 4;
     static constexpr int kStageBytes = ScanGeom<DI>::kStageBytes;
     static constexpr size_t kSmem = 1024 /*align slack*/ + (size_t)kStages * kStageBytes + 4096 /*q tile*/ +
                                     kHist0Bins * 4 + 256 /*barriers + tmem slot*/ + 4 * 2048 /*page table*/;
@@ -374,8 +374,7 @@ __device__ __forceinline__ void scan_mma_loop(int ntiles, int nstages, const uin
 // all 32 lanes (kEpr calls per tile).
 template <int DI, typename Consume>
 __device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)[kScanN], int hi, uint64_t *tfull,
-                                                   uint64_t *tempty, uint32_t tmem, int quarter, Consume consume,
-                                                   int half = 0, int nhalf = 1) {
+                                                   uint64_t *tempty, uint32_t tmem, int quarter, Consume consume) {
     using G = ScanGeom<DI>;
     const int lane = threadIdx.x & 31;
     const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
@@ -385,46 +384,23 @@ __device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)
         if (!__all_sync(0xFFFFFFFFu, ok)) break;
         tc_fence_after();
         float sc[kScanBatch][G::kEpr];
-        const uint32_t tb = tmem + ((uint32_t)(quarter * 32) << 16) + a * (kScanBatch * G::kN);
-        if (hi <= 4) {
-            // only the real heads' columns, every load of the batch in flight at once
-            uint32_t r[kScanBatch][G::kEpr][4];
 #pragma unroll
-            for (int j = 0; j < kScanBatch; ++j)
-                if (j % nhalf == half)
-#pragma unroll
-                    for (int u = 0; u < G::kEpr; ++u) tmem_ld4(tb + j * G::kN + u * kScanN, r[j][u]);
+        for (int j = 0; j < kScanBatch; ++j) {
+            uint32_t r[G::kN];
+            const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + a * (kScanBatch * G::kN) + j * G::kN;
+            if (G::kN == 32) {
+                tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(r));
+            } else {
+                tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(r));
+            }
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < kScanBatch; ++j)
+            for (int u = 0; u < G::kEpr; ++u) {
+                float v = 0.0f;
 #pragma unroll
-                for (int u = 0; u < G::kEpr; ++u) {
-                    float v = 0.0f;
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        if (h < hi) v = fmaf(wv[h], fmaxf(__uint_as_float(r[j][u][h]), 0.0f), v);
-                    sc[j][u] = v + 0.0f;
-                }
-        } else {
-#pragma unroll
-            for (int j = 0; j < kScanBatch; ++j) {
-                if (j % nhalf != half) continue;
-                uint32_t r[G::kN];
-                const uint32_t ta = tb + j * G::kN;
-                if (G::kN == 32) {
-                    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(r));
-                } else {
-                    tmem_ld16(ta, *reinterpret_cast<uint32_t(*)[16]>(r));
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int u = 0; u < G::kEpr; ++u) {
-                    float v = 0.0f;
-#pragma unroll
-                    for (int h = 0; h < kScanN; ++h)
-                        if (h < hi) v = fmaf(wv[h], fmaxf(__uint_as_float(r[u * kScanN + h]), 0.0f), v);
-                    sc[j][u] = v + 0.0f;
-                }
+                for (int h = 0; h < kScanN; ++h)
+                    if (h < hi) v = fmaf(wv[h], fmaxf(__uint_as_float(r[u * kScanN + h]), 0.0f), v);
+                sc[j][u] = v + 0.0f;
             }
         }
         tc_fence_before();
@@ -434,7 +410,6 @@ __device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)
         for (int j = 0; j < kScanBatch; ++j) {
             const int i = g * kScanBatch + j;
             if (i >= ntiles) break;
-            if (j % nhalf != half) continue;
 #pragma unroll
             for (int u = 0; u < G::kEpr; ++u) consume(i, G::kEpr * (quarter * 32 + lane) + u, score_key(sc[j][u]));
         }
@@ -442,7 +417,7 @@ __device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)
 }
 
 template <int DI>
-__global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
+__global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
     using Cfg = ScanCfg<DI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -478,7 +453,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_con
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], kScanThreads / 32 - 2);
+            mbar_init(&tempty[a], 4);
         }
         fence_mbar_init();
     }
@@ -498,8 +473,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_con
         if (lane == 0)
             scan_mma_loop<DI>(ntiles, Cfg::kStages, stages, smem_u32(qt), full, empty, tfull, tempty, tmem);
     } else {
-        // epilogue: warps 2..9 cover TMEM lane quarters 2, 3, 0, 1 twice; the
-        // first four take the even tiles of each batch, the others the odd
+        // epilogue: warps 2..5 cover TMEM lane quarters 2, 3, 0, 1
         float wv[kScanN];
 #pragma unroll
         for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
@@ -509,7 +483,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_con
             const bool valid = t < limit;
             if (valid) keys[t] = key;
             hist_add_warp(hist, valid ? (key >> 20) : 0xFFFFFFFFu);
-        }, (warp - 2) >> 2, 2);
+        });
     }
     tc_fence_before();
     __syncthreads();
