@@ -278,6 +278,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
     const int n = (int)max((int64_t)0, x1 - x0);
 
     pdl_trigger();
+    if (warp == kDecResWarp && n > 0) {
+        // While the previous kernel finishes: L2 prefetches of what this CTA
+        // reads first and no kernel of this library writes -- q of its
+        // queries and their sequences' page-table rows. A prefetch only warms
+        // L2; every read of them happens after the dependency wait below.
+        const int64_t ua = x0 / p.tpq, ub = (x1 - 1) / p.tpq;
+        for (int64_t u = ua; u <= ub; ++u) {
+            const uint8_t *qb = reinterpret_cast<const uint8_t *>(p.q + u * H * CSA2_D);
+            for (int o = lane * 128; o < H * CSA2_D * 2; o += 32 * 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(qb + o));
+            if (p.kv.max_pages > 1) {
+                const uint8_t *pt = reinterpret_cast<const uint8_t *>(
+                    p.kv.page_table + (int64_t)((int32_t)u / p.q_per_seq) * p.kv.max_pages);
+                for (int64_t o = lane * 128; o < (int64_t)p.kv.max_pages * 4; o += 32 * 128)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(pt + o));
+            }
+        }
+    }
     if (warp == 0) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
