@@ -113,11 +113,12 @@ __device__ __forceinline__ void build_q_tile(uint8_t *qt, const uint8_t *q /*[hi
     }
 }
 
-// Warp-aggregated shared-memory histogram increment (bin 0xFFFFFFFF = skip).
+// Shared-memory histogram increment (bin 0xFFFFFFFF = skip).
 __device__ __forceinline__ void hist_add_warp(uint32_t *hist, uint32_t bin) {
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-    const int lane = threadIdx.x & 31;
-    if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    // a shared-memory atomic per lane: lanes of a warp that hit the same bin
+    // are serialised by the hardware, which measured cheaper than grouping
+    // them with __match_any_sync first
+    if (bin != 0xFFFFFFFFu) atomicAdd(&hist[bin], 1u);
 }
 
 // ---------------------------------------------------------------------------

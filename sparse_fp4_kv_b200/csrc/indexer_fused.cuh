@@ -11,10 +11,10 @@
 // indexer keys by TMA through a deep shared-memory ring into tcgen05 FP8
 // MMAs (as k_index_scan) and keeps every 32-bit score key in shared memory
 // together with a 4096-bin histogram of the keys' top 12 bits. The radix
-// select (digits 12/10/10) then runs on shared memory: each digit's
-// histograms are summed across the cluster over distributed shared memory
-// (CTA r sums one slice of the bins, then every CTA gathers all slices),
-// with hardware cluster barriers between steps. The emission is ordered by
+// select (digits 12/10/10) then runs on shared memory: for each digit every
+// CTA adds its nonzero bins into the first CTA's histogram with distributed
+// shared-memory atomics, the first CTA locates the bins of both target
+// ranks, and every CTA reads them back (three cluster barriers a digit). The emission is ordered by
 // CTA rank and, inside a CTA, by entry, so the output ids are ascending and
 // ties at the threshold go to the lowest ids. No global scratch, no memset,
 // no second launch.
@@ -31,43 +31,47 @@ constexpr int kFusedClusterMax = 16;
 constexpr int kFusedThreads = 256;
 
 
-// Sum the local histograms h[0..nbins) (same shared-memory offset in every
-// CTA of the cluster) over the cluster into full[0..nbins). CTA r first
-// sums bins [r*nbins/C, (r+1)*nbins/C) from every CTA into slice[], then
-// every CTA gathers all slices.
-__device__ __forceinline__ void cluster_hist_sum(uint32_t *h, uint32_t *slice, uint32_t *full, int nbins,
-                                                 uint32_t rank, int CL) {
-    const int per = (nbins + CL - 1) / CL;  // bins summed by each CTA (the last one may sum fewer)
-    const int base = (int)rank * per;
+// Cluster-wide rank bins: every CTA adds its nonzero local bins into the
+// first CTA's accumulator acc (distributed shared-memory atomics, so only
+// the few bins a CTA filled travel); the first CTA finds, for each active
+// target tau, the bin holding rank rem[tau] of the TB bins at
+// acc + hoff[tau] and the rank left inside it, clears acc for the next
+// digit, and every CTA reads the results back. h and acc are at the same
+// shared-memory offsets in every CTA; acc must be zero on entry.
+template <int TB>
+__device__ __forceinline__ void cluster_rank_bins(const uint32_t *h, int nbins, uint32_t *acc, const int (&hoff)[2],
+                                                  const bool (&act)[2], uint32_t (&rem)[2], uint32_t (&bin)[2],
+                                                  uint32_t *scratch, uint32_t *res, uint32_t crank) {
     cluster_sync_all();  // every CTA's local histogram is complete
-    // distributed shared memory loads have a long latency: each thread puts
-    // the loads of all CTAs (reduce) or of four bins (gather) in flight at once
-    for (int i = threadIdx.x; i < per && base + i < nbins; i += kFusedThreads) {
-        uint32_t v[kFusedClusterMax];
-#pragma unroll
-        for (int r = 0; r < kFusedClusterMax; ++r) v[r] = r < CL ? cluster_peer(h, (uint32_t)r)[base + i] : 0u;
-        uint32_t s = 0;
-#pragma unroll
-        for (int r = 0; r < kFusedClusterMax; ++r) s += v[r];
-        slice[i] = s;
+    for (int i = threadIdx.x; i < nbins; i += kFusedThreads) {
+        const uint32_t v = h[i];
+        if (v) asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_smem_addr(acc + i, 0)), "r"(v) : "memory");
     }
-    cluster_sync_all();
-    for (int i0 = threadIdx.x; i0 < nbins; i0 += 4 * kFusedThreads) {
-        uint32_t v[4];
+    cluster_sync_all();  // every addition has landed in the first CTA
+    if (crank == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j * kFusedThreads;
-            const int owner = i / per;
-            v[j] = i < nbins ? cluster_peer(slice, (uint32_t)owner)[i - owner * per] : 0u;
+        for (int tau = 0; tau < 2; ++tau) {
+            if (!act[tau]) continue;
+            uint32_t b, r;
+            find_rank_bin<kFusedThreads, TB / kFusedThreads, false>(acc + hoff[tau], TB, rem[tau], scratch, b, r);
+            if (threadIdx.x == 0) {
+                res[2 * tau] = b;
+                res[2 * tau + 1] = r;
+            }
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (i0 + j * kFusedThreads < nbins) full[i0 + j * kFusedThreads] = v[j];
+        __syncthreads();
+        for (int i = threadIdx.x; i < nbins; i += kFusedThreads) acc[i] = 0u;
     }
-    __syncthreads();
-    // No closing cluster barrier: peers read h only before the second barrier
-    // above, and read slice only before they reach the first barrier of the
-    // next call (or the kernel's final barrier), so both may be rewritten now.
+    cluster_sync_all();  // the results are written
+#pragma unroll
+    for (int tau = 0; tau < 2; ++tau) {
+        if (!act[tau]) continue;
+        uint32_t b, r;
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(b) : "r"(cluster_smem_addr(res + 2 * tau, 0)) : "memory");
+        asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(r) : "r"(cluster_smem_addr(res + 2 * tau + 1, 0)) : "memory");
+        bin[tau] = b;
+        rem[tau] = r;
+    }
 }
 
 struct FusedParams {
@@ -127,7 +131,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---- set-up that reads no global memory ----
     pdl_trigger();
-    for (int i = tid; i < 4096; i += kFusedThreads) hist0[i] = 0u;
+    for (int i = tid; i < 4096; i += kFusedThreads) hist0[i] = full[i] = 0u;
     if (tid == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full_b[s], 1);
@@ -189,11 +193,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         rem[tau] = (uint32_t)max(p.rank[tau], 0);
     }
     // digit 0 (bits 31..20): the histogram built during the scan
-    cluster_hist_sum(hist0, slice, full, 4096, crank, p.csize);
-    #pragma unroll
-    for (int tau = 0; tau < 2; ++tau)
-        if (act[tau]) find_rank_bin<kFusedThreads, 4096 / kFusedThreads, false>(full, 4096, rem[tau], scratch,
-                                                                                b0[tau], rem[tau]);
+    uint32_t *res = words + 96;  // the first CTA's rank bins of a digit
+    {
+        const int hoff[2] = {0, 0};
+        cluster_rank_bins<4096>(hist0, 4096, full, hoff, act, rem, b0, scratch, res, crank);
+    }
     // digits 1 (bits 19..10) and 2 (bits 9..0): each thread takes 4 keys per
     // step (one 16-byte load); most steps hold no key of the threshold bin
     // and cost one ballot
@@ -229,17 +233,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                         hist_add_warp(nh + tau * 1024, m[tau][j] ? (kk[j] >> (shift - 10)) & 1023u : 0xFFFFFFFFu);
         }
         __syncthreads();
-        cluster_hist_sum(nh, slice, full, 2048, crank, p.csize);
+        const int hoff[2] = {0, 1024};
+        uint32_t bin[2] = {0u, 0u};
+        cluster_rank_bins<1024>(nh, 2048, full, hoff, act, rem, bin, scratch, res, crank);
         #pragma unroll
         for (int tau = 0; tau < 2; ++tau) {
             if (!act[tau]) continue;
-            uint32_t bin;
-            find_rank_bin<kFusedThreads, 1024 / kFusedThreads, false>(full + tau * 1024, 1024, rem[tau], scratch,
-                                                                      bin, rem[tau]);
             if (digit == 1) {
-                b1[tau] = bin;
+                b1[tau] = bin[tau];
             } else {
-                T[tau] = (b0[tau] << 20) | (b1[tau] << 10) | bin;
+                T[tau] = (b0[tau] << 20) | (b1[tau] << 10) | bin[tau];
             }
         }
     }
