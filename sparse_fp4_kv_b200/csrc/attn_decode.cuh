@@ -83,7 +83,12 @@ struct DecParams {
     int32_t tpq;    // tiles per query
     int32_t per;    // tiles per CTA
     int32_t nslots;  // partial slots in the workspace
+    // In-kernel merge (queries split over at most kInlineMergeParts CTAs):
+    // the last CTA to finish a part of query u merges all of u's parts.
+    int32_t inline_merge;
+    uint32_t *qcount;  // [nq]: parts of u finished (zeroed before the launch)
 };
+constexpr int kInlineMergeParts = 2;
 
 // ---- the static work split (host and device) -------------------------------
 // CTA g takes tiles [g*per, min((g+1)*per, T)). Its segments are the runs of
@@ -721,6 +726,74 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_attn_decode(DecParams p) {
             }
 #pragma unroll
             for (int j = 0; j < HG; ++j) l_part[j] = 0.0f;
+            if (p.inline_merge && !whole) {
+                // the partial must be visible to the other CTAs of u before this
+                // part is counted: bulk copies complete, every store fenced
+                if (warp == 0) {
+                    bulk_wait_all();
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
+                __threadfence();
+                named_bar_sync(kBarWork, kDecWorkThreads);
+                const int32_t np = sp.owner((u + 1) * p.tpq - 1) - sp.owner(u * p.tpq) + 1;
+                if (tid == 0) {
+                    __threadfence();
+                    const uint32_t done = atomicAdd(p.qcount + u, 1u) + 1u;
+                    part_word[1] = done == (uint32_t)np ? 1 : 0;
+                    __threadfence();
+                }
+                named_bar_sync(kBarWork, kDecWorkThreads);
+                if (part_word[1] != 0 && np <= kInlineMergeParts) {
+                    // the last part of u: weights per head, then o = sum_s w_s o_s
+                    const int32_t s0 = __ldcg(p.qslot + u);
+                    if (s0 < 0 || s0 + np > p.nslots) {
+                        if (tid == 0) set_error(CSA2_DEVERR_SELECT);
+                    } else {
+                        float *wgt = red;  // [H][kInlineMergeParts]
+                        if (tid < H) {
+                            float ls[kInlineMergeParts], mx = -INFINITY;
+#pragma unroll
+                            for (int q = 0; q < kInlineMergeParts; ++q) {
+                                ls[q] = q < np ? __ldcg(p.lse_part + (int64_t)(s0 + q) * H + tid) : -INFINITY;
+                                mx = fmaxf(mx, ls[q]);
+                            }
+                            float L = 0.0f;
+#pragma unroll
+                            for (int q = 0; q < kInlineMergeParts; ++q) {
+                                ls[q] = (mx == -INFINITY || q >= np) ? 0.0f : expf(ls[q] - mx);
+                                L += ls[q];
+                            }
+                            const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+                            for (int q = 0; q < kInlineMergeParts; ++q) wgt[tid * kInlineMergeParts + q] = ls[q] * inv;
+                            if (p.lse) p.lse[u * H + tid] = L > 0.0f ? mx + logf(L) : -INFINITY;
+                        }
+                        named_bar_sync(kBarWork, kDecWorkThreads);
+                        for (int idx = tid; idx < H * (CSA2_D / 4); idx += kDecWorkThreads) {
+                            const int h = idx / (CSA2_D / 4), d4 = idx % (CSA2_D / 4);
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int q = 0; q < kInlineMergeParts; ++q) {
+                                if (q >= np) break;
+                                const float wq = wgt[h * kInlineMergeParts + q];
+                                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                                            p.o_part + ((int64_t)(s0 + q) * H + h) * CSA2_D) + d4);
+                                acc.x = fmaf(wq, v.x, acc.x);
+                                acc.y = fmaf(wq, v.y, acc.y);
+                                acc.z = fmaf(wq, v.z, acc.z);
+                                acc.w = fmaf(wq, v.w, acc.w);
+                            }
+                            if (p.o32) {
+                                *(reinterpret_cast<float4 *>(p.o32 + (u * H + h) * CSA2_D) + d4) = acc;
+                            } else {
+                                const uint32_t lo = (uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16);
+                                const uint32_t hi = (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16);
+                                *reinterpret_cast<uint2 *>(p.o + (u * H + h) * CSA2_D + d4 * 4) = make_uint2(lo, hi);
+                            }
+                        }
+                    }
+                }
+            }
             if (has_next) load_q<H>(p, u + 1, q_tile);
             if (warp == 0) bulk_wait_read();  // the KV tile may be overwritten again
             // m_run is reset, the Q tile rewritten and the staging read before any

@@ -361,7 +361,8 @@ AttnLayout attn_layout(int32_t nq, int32_t h, const AttnPlan &P, bool nvfp4 = fa
 // one SM) and the number of partial slots of the split.
 struct DecPlan {
     int32_t tpq, per, ctas, slots;
-    size_t off_o, off_lse, off_qslot, total;
+    int32_t max_parts;  // CTAs sharing one query, at most
+    size_t off_o, off_lse, off_qslot, off_qcount, total;
 };
 
 DecPlan plan_decode(int32_t nq, int32_t h, int32_t k, int32_t w_max, int sms) {
@@ -376,10 +377,13 @@ DecPlan plan_decode(int32_t nq, int32_t h, int32_t k, int32_t w_max, int sms) {
     const DecSplit sp{T, P.per, P.tpq};
     P.slots = 0;
     for (int32_t g = 0; g < P.ctas; ++g) P.slots += sp.nparts(g);
+    // a query's tiles span at most ceil((tpq - 1) / per) + 1 CTAs
+    P.max_parts = (int32_t)std::min<int64_t>(P.ctas, (P.tpq - 1 + (int64_t)P.per - 1) / P.per + 1);
     P.off_o = 0;
     P.off_lse = align_up((size_t)P.slots * h * CSA2_D * 4, 256);
     P.off_qslot = align_up(P.off_lse + (size_t)P.slots * h * 4, 256);
-    P.total = P.slots > 0 ? align_up(P.off_qslot + (size_t)nq * 4, 256) : 0;
+    P.off_qcount = align_up(P.off_qslot + (size_t)nq * 4, 256);
+    P.total = P.slots > 0 ? align_up(P.off_qcount + (size_t)nq * 4, 256) : 0;
     return P;
 }
 
@@ -983,12 +987,16 @@ template <int H>
 csa2_status launch_decode(const DecParams &dp, const DecPlan &P, bool out_f32, cudaStream_t stream) {
     // the merge reads slot numbers the decode kernel writes: it is not
     // launched after a failed launch of that kernel
+    if (dp.inline_merge && cudaMemsetAsync(dp.qcount, 0, (size_t)dp.nq * 4, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CSA2_ERR_CUDA;
+    }
     if (launch(k_attn_decode<H>, dim3((unsigned)P.ctas), dim3(kDecThreads), DecCfg<H>::kSmem, stream, dp) !=
         cudaSuccess) {
         cudaGetLastError();
         return CSA2_ERR_CUDA;
     }
-    if (P.slots > 0) {
+    if (P.slots > 0 && !dp.inline_merge) {
         const dim3 mgrid((unsigned)H, (unsigned)dp.nq);
         if (out_f32)
             launch(k_attn_merge_parts<H, true>, mgrid, dim3(kMergeThreads), 0, stream, dp);
@@ -1029,6 +1037,12 @@ csa2_status decode_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32
     dp.tpq = P.tpq;
     dp.per = P.per;
     dp.nslots = P.slots;
+    // queries split over at most kInlineMergeParts CTAs are merged inside the
+    // kernel by the CTA that finishes their last part; wider splits by the
+    // merge kernel (CSA2_ATTN_MERGE=kernel forces the merge kernel)
+    const char *mk = std::getenv("CSA2_ATTN_MERGE");
+    dp.inline_merge = P.slots > 0 && P.max_parts <= kInlineMergeParts && !(mk && std::strcmp(mk, "kernel") == 0);
+    dp.qcount = P.slots > 0 ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + P.off_qcount) : nullptr;
     switch (h) {
         case 64:
             if (!smem_attr(k_attn_decode<64>, DecCfg<64>::kSmem)) return CSA2_ERR_CUDA;

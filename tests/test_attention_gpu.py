@@ -205,3 +205,20 @@ def test_query_outside_f16_range_is_reported(B, cuda_device):
     assert B.csa2_device_status() == 8  # CSA2_DEVERR_Q_RANGE
     o0, _ = oracle.sparse_attn(bf16_bits(q[0]), codes, scales, pt[0], ps, topk[0], None, scale)
     assert attn_excess(o.float().cpu().numpy()[0], o0) <= 1.0
+
+
+def test_merge_kernel_path(cuda_device):
+    """Queries split over at most two CTAs are merged inside the attention kernel
+    by the CTA that finishes their last part; wider splits by the merge
+    kernel. This runs the attention tests again with the merge kernel for
+    every split (CSA2_ATTN_MERGE=kernel, read per call; a separate process keeps
+    the environment of this one)."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    env = dict(os.environ, CSA2_ATTN_MERGE="kernel")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        os.path.join(here, "test_attention_gpu.py"), "-k", "not merge_kernel_path"],
+                       env=env, cwd=os.path.dirname(here), capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
