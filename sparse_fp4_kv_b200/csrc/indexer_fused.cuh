@@ -332,26 +332,53 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             pos += wgt[tau * kWarps + ww] + (need > er ? min(need - er, e) : 0u);
             er += e;
         }
-#pragma unroll 4
-        for (int c = 0; c < cpw; ++c) {
-            const uint4 m4 = masks[c];
+        // 32 chunks at a time, lane l holding chunk c0 + l: the equal keys taken
+        // (in entry order, up to the rank left) and the output offsets follow
+        // from warp prefix sums, then the warp writes the chunks one by one
+        for (int c0 = 0; c0 < cpw; c0 += 32) {
+            const int c = c0 + lane;
+            const uint4 m4 = c < cpw ? masks[c] : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t g = tau ? m4.z : m4.x, e = tau ? m4.w : m4.y;
-            if ((g | e) == 0u) continue;
-            uint32_t sm = g;
-            if (e != 0u && er < need) {
-                const bool take = ((e >> lane) & 1u) && er + __popc(e & lt_mask) < need;
-                sm |= __ballot_sync(0xFFFFFFFFu, take);
+            const uint32_t ne = (uint32_t)__popc(e);
+            uint32_t ie = ne;  // inclusive prefix of the equal keys over the group's chunks
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, ie, o);
+                if (lane >= o) ie += y;
             }
-            if ((sm >> lane) & 1u) {
-                const uint32_t at = pos + __popc(sm & lt_mask);
-                if (at < (uint32_t)r_out) {
-                    out[at] = (int32_t)start + w0 + c * 32 + lane;
-                } else {
-                    set_error(CSA2_DEVERR_SELECT);
+            const uint32_t er_c = er + ie - ne;  // equal keys before chunk c
+            uint32_t take = 0u;
+            if (e != 0u && er_c < need) {
+                uint32_t left = min(need - er_c, ne), x = e;
+                for (; left > 0u; --left) {  // the lowest `left` equal keys of the chunk
+                    take |= x & (0u - x);
+                    x &= x - 1u;
                 }
             }
-            pos += __popc(sm);
-            er += __popc(e);
+            const uint32_t sm = g | take;
+            const uint32_t ns = (uint32_t)__popc(sm);
+            uint32_t is = ns;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, is, o);
+                if (lane >= o) is += y;
+            }
+            const uint32_t base_c = pos + is - ns;
+            const int nj = min(32, cpw - c0);
+            for (int j = 0; j < nj; ++j) {
+                const uint32_t smj = __shfl_sync(0xFFFFFFFFu, sm, j);
+                const uint32_t bj = __shfl_sync(0xFFFFFFFFu, base_c, j);
+                if ((smj >> lane) & 1u) {
+                    const uint32_t at = bj + __popc(smj & lt_mask);
+                    if (at < (uint32_t)r_out) {
+                        out[at] = (int32_t)start + w0 + (c0 + j) * 32 + lane;
+                    } else {
+                        set_error(CSA2_DEVERR_SELECT);
+                    }
+                }
+            }
+            pos += __shfl_sync(0xFFFFFFFFu, is, 31);
+            er += __shfl_sync(0xFFFFFFFFu, ie, 31);
         }
     }
     cluster_sync_all();  // peers read cnt[] above; keep this CTA's shared memory alive until they are done
