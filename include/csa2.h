@@ -258,9 +258,11 @@ csa2_status csa2_sparse_attn_decode_static(const void *q_bf16, int32_t nq, int32
  * also uses FP4 quantization": the FP4 values are restored for computation
  * on the chip; here the scores of the selected entries are computed from
  * the FP4 codes directly). Arguments, layouts, workspace rule and errors are
- * those of csa2_sparse_attn_decode, with h = 64 (other head counts are
- * refused with CSA2_ERR_UNSUPPORTED) and the workspace
- * sized by csa2_sparse_attn_nvfp4_workspace_size. What it computes differs
+ * those of csa2_sparse_attn_decode, with h in {16, 32, 64} and the workspace
+ * sized by csa2_sparse_attn_nvfp4_workspace_size. The block-scaled products
+ * run at 64 heads only (their scale-factor layout is established for that
+ * width): 16 and 32 heads run as a 64-head call whose q is padded with zero
+ * heads in the workspace, and the padded heads' outputs are dropped. What it computes differs
  * in one step: q is first quantised to NVFP4 with the cache's own block
  * quantiser (per 16 values one E4M3 scale = RNE(amax / 6), E2M1 codes RNE
  * of x / scale), and that quantised q (exact in f16) is used for the scores
@@ -283,7 +285,8 @@ csa2_status csa2_sparse_attn_decode_nvfp4(const void *q_bf16, int32_t nq, int32_
                                           cudaStream_t stream);
 
 /* Workspace bytes of csa2_sparse_attn_decode_nvfp4 (split partials plus q's
- * FP4 codes and scales); 0 for a head count other than 64. */
+ * FP4 codes and scales; for 16 or 32 heads also the padded q, o and lse);
+ * 0 for a head count other than 16, 32, 64. */
 size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max);
 
 /*

@@ -137,6 +137,33 @@ __global__ void __launch_bounds__(kQuantThreads)
     scales[i] = (uint8_t)sc;
 }
 
+// NVFP4 variant with fewer than 64 heads: the call runs as a 64-head problem
+// (the one shape whose block-scaled products are validated) with q padded by
+// zero heads; the padded heads' outputs are dropped. 16-byte pieces, a
+// thread each.
+__global__ void k_pad_heads(const uint4 *__restrict__ src, int32_t h, int32_t nq, uint4 *__restrict__ dst) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int kPiecesPerHead = CSA2_D * 2 / 16;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // piece of the padded q
+    if (i >= (int64_t)nq * 64 * kPiecesPerHead) return;
+    const int64_t u = i / (64 * kPiecesPerHead);
+    const int hh = (int)((i / kPiecesPerHead) % 64), c = (int)(i % kPiecesPerHead);
+    dst[i] = hh < h ? src[(u * h + hh) * kPiecesPerHead + c] : make_uint4(0u, 0u, 0u, 0u);
+}
+__global__ void k_unpad_heads(const uint4 *__restrict__ src, const float *__restrict__ lse_src, int32_t h, int32_t nq,
+                              uint4 *__restrict__ dst, float *__restrict__ lse_dst) {
+    pdl_trigger();
+    pdl_wait();
+    constexpr int kPiecesPerHead = CSA2_D * 2 / 16;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // piece of the unpadded o
+    if (i >= (int64_t)nq * h * kPiecesPerHead) return;
+    const int64_t u = i / (h * kPiecesPerHead);
+    const int hh = (int)((i / kPiecesPerHead) % h), c = (int)(i % kPiecesPerHead);
+    dst[i] = src[(u * 64 + hh) * kPiecesPerHead + c];
+    if (lse_dst != nullptr && c == 0) lse_dst[u * h + hh] = lse_src[u * 64 + hh];
+}
+
 __device__ __forceinline__ uint32_t kv_chunk_off(int e, int c64) {
     // f16 KV tile: row e, 16-byte chunk c64 (d = 8*c64 .. 8*c64+7)
     return (uint32_t)((c64 >> 3) * 16384 + (e >> 3) * 1024 + (e & 7) * 128 + (((c64 & 7) ^ (e & 7)) << 4));

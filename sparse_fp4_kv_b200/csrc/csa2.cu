@@ -547,7 +547,7 @@ bool prefer_shared(K kernel) {
 bool init_small_kernels() {
     static const char key = 0;
     return once_per_device(&key, [] {
-        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) && prefer_shared(k_batch_sthresh) && prefer_shared(k_batch_thresh) &&
+        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) && prefer_shared(k_pad_heads) && prefer_shared(k_unpad_heads) && prefer_shared(k_batch_sthresh) && prefer_shared(k_batch_thresh) &&
                prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
                prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
                prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
@@ -1060,6 +1060,22 @@ csa2_status decode_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32
     return check_launch();
 }
 
+// Workspace of the NVFP4 variant for fewer than 64 heads: the 64-head call's
+// region, then q padded to 64 heads, its bf16 o and its lse.
+struct NvPad {
+    size_t inner, off_q, off_o, off_lse, total;
+};
+NvPad nvfp4_pad_layout(int32_t nq, int32_t k, int32_t w_max) {
+    NvPad d{};
+    const AttnPlan P = plan_attn_nvfp4(nq, k, w_max, num_sms());
+    d.inner = attn_layout(nq, 64, P, true).total;
+    d.off_q = align_up(d.inner, 256);
+    d.off_o = align_up(d.off_q + (size_t)nq * 64 * CSA2_D * 2, 256);
+    d.off_lse = align_up(d.off_o + (size_t)nq * 64 * CSA2_D * 2, 256);
+    d.total = align_up(d.off_lse + (size_t)nq * 64 * 4, 256);
+    return d;
+}
+
 // Shared body of the decode entry points: o is bf16 (out_f32 false) or the
 // normalised f32 o of this call's rows (out_f32 true, lse required).
 csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t h, const csa2_kv_desc *kv,
@@ -1070,8 +1086,9 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
     if (st != CSA2_OK) return st;
     if (h != 16 && h != 32 && h != 64) return CSA2_ERR_UNSUPPORTED;
     // the block-scaled S product runs at N = 64 only (its scale-factor layout in
-    // TMEM is established for that shape)
-    if (nvfp4 && h != 64) return CSA2_ERR_UNSUPPORTED;
+    // TMEM is established for that shape): 16 and 32 heads run as 64 heads with
+    // q padded by zero heads (the h != 64 branch below)
+    if (nvfp4 && h != 64 && out_f32) return CSA2_ERR_UNSUPPORTED;
     if (nq <= 0 || nq > 65535 || q_per_seq <= 0 || (nq + q_per_seq - 1) / q_per_seq > kv->batch)
         return CSA2_ERR_INVALID_ARG;
     if (k < 0 || w_max < 0 || (k > 0 && !topk) || (topk && !aligned(topk, 4))) return CSA2_ERR_INVALID_ARG;
@@ -1086,6 +1103,27 @@ csa2_status attn_impl(const void *q_bf16, int32_t nq, int32_t q_per_seq, int32_t
     if (!nvfp4) return decode_impl(q_bf16, nq, q_per_seq, h, kv, topk, k, swa, swa_seq_stride, has_swa ? swa_begin : nullptr,
                                    has_swa ? swa_end : nullptr, has_swa ? w_max : 0, softmax_scale, o, out_f32, lse,
                                    ws, ws_bytes, stream);
+    if (h != 64) {
+        // 16 or 32 heads: q padded to 64 heads in the workspace (after the
+        // 64-head call's own region), the padded call, then its first h heads
+        const NvPad pd = nvfp4_pad_layout(nq, k, has_swa ? w_max : 0);
+        if (!ws || ws_bytes < pd.total || !aligned(ws, 256)) return CSA2_ERR_WORKSPACE;
+        if (!init_small_kernels()) return CSA2_ERR_CUDA;
+        uint8_t *wsb = static_cast<uint8_t *>(ws);
+        const int64_t pieces_in = (int64_t)nq * 64 * (CSA2_D * 2 / 16);
+        launch(k_pad_heads, dim3((unsigned)((pieces_in + 255) / 256)), dim3(256), 0, stream,
+               static_cast<const uint4 *>(q_bf16), h, nq, reinterpret_cast<uint4 *>(wsb + pd.off_q));
+        if ((st = check_launch()) != CSA2_OK) return st;
+        st = attn_impl(wsb + pd.off_q, nq, q_per_seq, 64, kv, topk, k, swa, swa_seq_stride, swa_begin, swa_end,
+                       w_max, softmax_scale, wsb + pd.off_o, false, lse ? reinterpret_cast<float *>(wsb + pd.off_lse) : nullptr,
+                       ws, pd.inner, stream, true);
+        if (st != CSA2_OK) return st;
+        const int64_t pieces_out = (int64_t)nq * h * (CSA2_D * 2 / 16);
+        launch(k_unpad_heads, dim3((unsigned)((pieces_out + 255) / 256)), dim3(256), 0, stream,
+               reinterpret_cast<const uint4 *>(wsb + pd.off_o), reinterpret_cast<const float *>(wsb + pd.off_lse), h, nq,
+               static_cast<uint4 *>(o), lse);
+        return check_launch();
+    }
     const AttnPlan P = plan_attn_nvfp4(nq, k, has_swa ? w_max : 0, num_sms());
     const AttnLayout L = attn_layout(nq, h, P, nvfp4);
     if (L.total > 0 && (!ws || ws_bytes < L.total || !aligned(ws, 256))) return CSA2_ERR_WORKSPACE;
@@ -1177,7 +1215,8 @@ csa2_status csa2_sparse_attn_partial(const void *q_bf16, int32_t nq, int32_t q_p
 }
 
 size_t csa2_sparse_attn_nvfp4_workspace_size(int32_t nq, int32_t h, int32_t k, int32_t w_max) {
-    if (nq <= 0 || k < 0 || h != 64) return 0;
+    if (nq <= 0 || k < 0 || (h != 16 && h != 32 && h != 64)) return 0;
+    if (h != 64) return nvfp4_pad_layout(nq, k, w_max).total;
     const AttnPlan P = plan_attn_nvfp4(nq, k, w_max, num_sms());
     return attn_layout(nq, h, P, true).total;
 }

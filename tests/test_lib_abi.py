@@ -109,12 +109,17 @@ def test_host_validation_rejects_before_launch(binding):
 def test_host_validation_of_shard_and_variant_calls(binding):
     L = binding._lib
     kv = _desc(binding)
-    # NVFP4 attention: 64 heads only; a window size without window rows
-    assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 32, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
+    # NVFP4 attention: 16, 32 or 64 heads (16 and 32 padded to 64 in the
+    # workspace, so they need one); a window size without window rows
+    assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 48, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
                                            None, None, 0, None) == 2
+    assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 32, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
+                                           None, None, 0, None) == 3
     assert L.csa2_sparse_attn_decode_nvfp4(0x1000, 1, 1, 64, kv, 0x2000, 8, None, 0, None, None, 16, 0.1, 0x3000,
                                            None, None, 0, None) == 1
-    assert binding.csa2_sparse_attn_nvfp4_workspace_size(1, 32, 256, 0) == 0
+    assert binding.csa2_sparse_attn_nvfp4_workspace_size(1, 48, 256, 0) == 0
+    assert binding.csa2_sparse_attn_nvfp4_workspace_size(1, 32, 256, 0) > \
+        binding.csa2_sparse_attn_nvfp4_workspace_size(1, 64, 256, 0)
     # f32 partials need an lse output
     assert L.csa2_sparse_attn_partial(0x1000, 1, 1, 64, kv, 0x2000, 8, None, 0, None, None, 0, 0.1, 0x3000,
                                       None, None, 0, None) == 1
