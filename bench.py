@@ -766,7 +766,7 @@ def bench_workload(name, args, world, rank, dev, stream, flush, clocks, pk):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rec["cpu_baseline"] = cpu_baseline(recipe)
     extra = {}
-    if name == "stack20" and world == 1 and not args.no_side:
+    if world == 1 and not args.no_side and name != "tiny_full":
         extra["attention_nvfp4"] = time_attn_variants(B, dec)
     del graph
     del dec
@@ -806,7 +806,8 @@ def run_ours(args):
     for name in names:
         rec, ex = bench_workload(name, args, world, rank, dev, stream, flush, clocks, pk)
         records[name] = rec
-        extra.update(ex)
+        for key, val in ex.items():
+            extra.setdefault(key, {})[name] = val
     clocks.stop()
 
     side = world == 1 and not args.no_side
