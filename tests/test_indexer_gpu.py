@@ -101,6 +101,16 @@ def test_full_causal_queries(B, cuda_device):
               shuffle=False)
 
 
+def test_full_empty_sequences_and_many_queries(B, cuda_device):
+    # sequences without entries between others (a query that owns no tile),
+    # and 400 causal queries of one sequence: on the multi-launch path every
+    # CTA then scans the end of one query and the start of the next
+    _run_full(B, cuda_device, [700, 0, 3000, 129, 0, 5000], 64, 64, 4, 100, 300, seed=16)
+    total = 3000
+    _run_full(B, cuda_device, [total], 3072, 64, 4, 150, 0, q_per_seq=400, q_limit=_causal(total, 400), seed=17,
+              shuffle=False)
+
+
 @pytest.mark.parametrize("csize", ["auto", "10", "12", "16"])
 def test_full_long_sequences_ragged(B, cuda_device, monkeypatch, csize):
     # long enough that a query's entries are spread over 8 to 16 CTAs (the
