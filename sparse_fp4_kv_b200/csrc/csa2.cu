@@ -850,49 +850,22 @@ csa2_status csa2_index_full(const uint8_t *qidx, const float *w, int32_t nq, int
     sp.hi = hi;
     sp.box_rows = box_rows;
     const int64_t tiles_max = std::max<int64_t>(1, (n_max + tile_entries - 1) / tile_entries);
-    sp.nq = nq;
-    const bool di64 = kv->di == 64;
-    const size_t scan_smem = di64 ? ScanCfg<64>::kSmem : ScanCfg<128>::kSmem;
-    if (di64 ? !smem_attr(k_index_scan<64>, scan_smem) : !smem_attr(k_index_scan<128>, scan_smem)) return CSA2_ERR_CUDA;
-    // Persistent mode: one CTA per resident slot, each scanning an equal share
-    // of the list of all queries' tiles, so ragged lengths leave no tail of
-    // idle SMs. Admitted when the per-query prefix sums fit the CTA's
-    // histogram words and a share's pages fit its staged page table;
-    // CSA2_SCAN=grid forces grid mode (tests).
-    int per_sm = 0;
-    const cudaError_t oe =
-        di64 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_index_scan<64>, kScanThreads, scan_smem)
-             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_index_scan<128>, kScanThreads, scan_smem);
-    if (oe != cudaSuccess || per_sm < 1) {
-        cudaGetLastError();
-        per_sm = 1;
-    }
-    const int64_t slots = (int64_t)num_sms() * per_sm;
-    const int64_t list_max = (int64_t)nq * tiles_max;  // tiles of the list at most
-    const int64_t share_max = (list_max + slots - 1) / slots;
-    const char *scan_env = std::getenv("CSA2_SCAN");
-    sp.persistent = !(scan_env && std::strcmp(scan_env, "grid") == 0) && nq <= kHist0Bins - 16 &&
-                    list_max < (int64_t(1) << 31) &&
-                    share_max * tile_entries / kv->page_size + 2 <= kMaxScanPages;
-    dim3 sgrid;
-    if (sp.persistent) {
-        sp.chunk_tiles = 0;
-        sgrid = dim3((unsigned)std::min<int64_t>(slots, list_max));
+    // several waves of two resident CTAs per SM when every query had n_max
+    // entries: queries of ragged lengths then leave short CTAs behind instead
+    // of a few long ones, and the hardware scheduler evens the SMs out
+    const int64_t target = (int64_t)num_sms() * 2 * 4;
+    int64_t chunk = std::max<int64_t>(16, ((int64_t)nq * tiles_max + target - 1) / target);
+    chunk = std::min<int64_t>(chunk, 256);
+    chunk = std::min<int64_t>(chunk, std::max<int64_t>(1, ((int64_t)(kMaxScanPages - 2) * kv->page_size) / tile_entries));
+    sp.chunk_tiles = (int32_t)chunk;
+    const dim3 sgrid((unsigned)((tiles_max + chunk - 1) / chunk), (unsigned)nq);
+    if (kv->di == 64) {
+        if (!smem_attr(k_index_scan<64>, ScanCfg<64>::kSmem)) return CSA2_ERR_CUDA;
+        launch(k_index_scan<64>, sgrid, dim3(kScanThreads), ScanCfg<64>::kSmem, stream, tm, sp);
     } else {
-        // several waves of two resident CTAs per SM when every query had n_max
-        // entries: queries of ragged lengths then leave short CTAs behind
-        // instead of a few long ones
-        const int64_t target = (int64_t)num_sms() * 2 * 4;
-        int64_t chunk = std::max<int64_t>(16, ((int64_t)nq * tiles_max + target - 1) / target);
-        chunk = std::min<int64_t>(chunk, 256);
-        chunk = std::min<int64_t>(chunk, std::max<int64_t>(1, ((int64_t)(kMaxScanPages - 2) * kv->page_size) / tile_entries));
-        sp.chunk_tiles = (int32_t)chunk;
-        sgrid = dim3((unsigned)((tiles_max + chunk - 1) / chunk), (unsigned)nq);
+        if (!smem_attr(k_index_scan<128>, ScanCfg<128>::kSmem)) return CSA2_ERR_CUDA;
+        launch(k_index_scan<128>, sgrid, dim3(kScanThreads), ScanCfg<128>::kSmem, stream, tm, sp);
     }
-    if (di64)
-        launch(k_index_scan<64>, sgrid, dim3(kScanThreads), scan_smem, stream, tm, sp);
-    else
-        launch(k_index_scan<128>, sgrid, dim3(kScanThreads), scan_smem, stream, tm, sp);
     if ((st = check_launch()) != CSA2_OK) return st;
 
     // per target (Top-K, then the pool): collect each query's sure ids and

@@ -13,8 +13,7 @@
 //     score(t) = sum_h w_h * max(0, <q_h, kidx_t>)
 // Order: score descending, entry id ascending on ties.
 //
-// Full scan (k_index_scan): per CTA an equal share of all queries' entries
-// (or a chunk of one query's), streamed
+// Full scan (k_index_scan): per CTA a chunk of one query's entries, streamed
 // 128 entries at a time by TMA (64B / 128B swizzle, no multicast) into a
 // shared-memory ring; one thread issues tcgen05.mma kind::f8f6f4
 // (E4M3 x E4M3 -> f32, M = 128 entries, N = 16 padded heads, K = di) into a
@@ -79,8 +78,6 @@ struct ScanParams {
     int32_t chunk_tiles;
     int32_t box_rows;
     int32_t rank[2];   // k, p (0 = no pool)
-    int32_t nq;
-    int32_t persistent;  // 1: one range of the all-query tile list per CTA
 };
 
 // Per-query selection state, per target tau (0 = Top-k, 1 = pool):
@@ -233,15 +230,6 @@ __device__ __forceinline__ int stage_pages(const csa2_kv_desc &kv, int32_t b, in
     return npg;
 }
 
-// Ring position of one role thread (shared-memory stage and its phase, TMEM
-// batch count), carried from one segment of work to the next by a CTA that
-// scans several ranges; a role loop called without one starts afresh.
-struct ScanRing {
-    int s = 0;
-    uint32_t phase = 0;
-    int g = 0;
-};
-
 // TMA producer, run by a whole warp (lane 0 issues): tile i = 128 smem rows =
 // kTile entries, loaded as boxes of box_rows rows. A box never crosses a
 // page (box_rows * kEpr divides the page size), so the page index and the
@@ -249,14 +237,12 @@ struct ScanRing {
 // whose first entry is past the limit are skipped (their rows are not read).
 // Physical rows come from the staged page-table entries.
 template <int DI>
-__device__ __forceinline__ ScanRing scan_tma_loop(const csa2_kv_desc &kv, const int32_t *ptab, int64_t start,
+__device__ __forceinline__ void scan_tma_loop(const csa2_kv_desc &kv, const int32_t *ptab, int64_t start,
                                               int64_t limit, int ntiles, int nstages, int box_rows,
                                               uint8_t *stage_base, const CUtensorMap *tm, uint64_t *full_b,
                                               uint64_t *empty_b, int tile_stride = 1,
-                                              const int32_t *pt_row = nullptr, ScanRing R = ScanRing()) {
+                                              const int32_t *pt_row = nullptr) {
     using G = ScanGeom<DI>;
-    int s = R.s;
-    uint32_t phase = R.phase;
     const bool leader = (threadIdx.x & 31) == 0;
     const int nbox = 128 / box_rows;
     const int32_t step = box_rows * G::kEpr;  // entries per box
@@ -264,9 +250,11 @@ __device__ __forceinline__ ScanRing scan_tma_loop(const csa2_kv_desc &kv, const 
     if (tile_stride > 1) {
         // every tile_stride-th tile from start (a sample of the range): the
         // page of each box is read from the sequence's page-table row
+        int s = 0;
+        uint32_t phase = 0;
         const int64_t lim = limit;
         for (int i = 0; i < ntiles; ++i) {
-            if (!mbar_wait(&empty_b[s], phase ^ 1)) return ScanRing{s, phase, R.g};
+            if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
             const int64_t t0 = start + (int64_t)i * tile_stride * G::kTile;
             int nvalid = 0;
             for (int j = 0; j < nbox; ++j) nvalid += (t0 + (int64_t)j * step < lim);
@@ -289,13 +277,15 @@ __device__ __forceinline__ ScanRing scan_tma_loop(const csa2_kv_desc &kv, const 
                 phase ^= 1u;
             }
         }
-        return ScanRing{s, phase, R.g};
+        return;
     }
     // entry positions fit in 32 bits (sequence lengths are int32)
     int32_t pi = 0, off = (int32_t)(start % ps);
     int32_t t = (int32_t)start;
     const int32_t lim = (int32_t)min(limit, (int64_t)INT32_MAX);
     // ring slot and phase advance without divisions (this loop is latency-bound)
+    int s = 0;
+    uint32_t phase = 0;
     // Fast path: one box per tile and the whole range inside one page (every
     // contiguous cache): consecutive tiles are consecutive rows.
     const int64_t span = (int64_t)ntiles * G::kTile;
@@ -303,7 +293,7 @@ __device__ __forceinline__ ScanRing scan_tma_loop(const csa2_kv_desc &kv, const 
         (int64_t)ptab[0] * ps + off + span <= kv.rows_cap) {
         int32_t y = (int32_t)(((int64_t)ptab[0] * ps + off) / G::kEpr);
         for (int i = 0; i < ntiles; ++i) {
-            if (!mbar_wait(&empty_b[s], phase ^ 1)) return ScanRing{s, phase, R.g};
+            if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
             if (leader) {
                 mbar_arrive_expect_tx(&full_b[s], (uint32_t)G::kStageBytes);
                 tma_load_2d(stage_base + (size_t)s * G::kStageBytes, tm, &full_b[s], 0, y);
@@ -314,56 +304,56 @@ __device__ __forceinline__ ScanRing scan_tma_loop(const csa2_kv_desc &kv, const 
                 phase ^= 1u;
             }
         }
-        return ScanRing{s, phase, R.g};
+        return;
     }
+    // Several boxes per tile: lane j issues box j, so the tile's loads go out
+    // together instead of one after another from a single thread.
+    const int lane = threadIdx.x & 31;
     for (int i = 0; i < ntiles; ++i) {
-        if (!mbar_wait(&empty_b[s], phase ^ 1)) return ScanRing{s, phase, R.g};
+        if (!mbar_wait(&empty_b[s], phase ^ 1)) return;
         int nvalid = 0;
         for (int j = 0; j < nbox; ++j) nvalid += (t + j * step < lim);
         if (leader) mbar_arrive_expect_tx(&full_b[s], (uint32_t)(nvalid * box_rows * 128));
-        for (int j = 0; j < nbox; ++j) {
-            if (j < nvalid && leader) {
-                const int64_t phys = pi < kMaxScanPages ? ptab[pi] : -1;
-                int64_t row = phys * ps + off;
-                if (phys < 0 || row + step > kv.rows_cap) {
-                    set_error(CSA2_DEVERR_BAD_ROW);
-                    row = 0;
-                }
-                tma_load_2d(stage_base + (size_t)s * G::kStageBytes + j * box_rows * 128, tm, &full_b[s], 0,
-                            (int32_t)(row / G::kEpr));
+        __syncwarp();
+        if (lane < nvalid) {
+            const int32_t o = off + lane * step;  // from the start of page pi
+            const int32_t pj = pi + o / ps;
+            const int64_t phys = pj < kMaxScanPages ? ptab[pj] : -1;
+            int64_t row = phys * ps + o % ps;
+            if (phys < 0 || row + step > kv.rows_cap) {
+                set_error(CSA2_DEVERR_BAD_ROW);
+                row = 0;
             }
-            t += step;
-            off += step;
-            if (off == ps) {
-                off = 0;
-                ++pi;
-            }
+            tma_load_2d(stage_base + (size_t)s * G::kStageBytes + lane * box_rows * 128, tm, &full_b[s], 0,
+                        (int32_t)(row / G::kEpr));
         }
+        t += nbox * step;
+        off += nbox * step;
+        pi += off / ps;
+        off %= ps;
         if (++s == nstages) {
             s = 0;
             phase ^= 1u;
         }
     }
-    return ScanRing{s, phase, R.g};
 }
 
 template <int DI>
-__device__ __forceinline__ ScanRing scan_mma_loop(int ntiles, int nstages, const uint8_t *stage_base, uint32_t qaddr,
+__device__ __forceinline__ void scan_mma_loop(int ntiles, int nstages, const uint8_t *stage_base, uint32_t qaddr,
                                               uint64_t *full_b, uint64_t *empty_b, uint64_t *tfull,
-                                              uint64_t *tempty, uint32_t tmem, ScanRing R = ScanRing()) {
+                                              uint64_t *tempty, uint32_t tmem) {
     using G = ScanGeom<DI>;
     const uint32_t idesc = idesc_e4m3_f32(128, G::kN);
     const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
-    int s = R.s;
-    uint32_t phase = R.phase;
-    const int g0 = R.g;
-    for (int g = g0; g < g0 + nbatch; ++g) {
+    int s = 0;
+    uint32_t phase = 0;
+    for (int g = 0; g < nbatch; ++g) {
         const int a = g & 1;
-        if (!mbar_wait(&tempty[a], ((g >> 1) & 1) ^ 1)) return ScanRing{s, phase, g0 + nbatch};
+        if (!mbar_wait(&tempty[a], ((g >> 1) & 1) ^ 1)) return;
         for (int j = 0; j < kScanBatch; ++j) {
-            const int i = (g - g0) * kScanBatch + j;
+            const int i = g * kScanBatch + j;
             if (i >= ntiles) break;
-            if (!mbar_wait(&full_b[s], phase)) return ScanRing{s, phase, g0 + nbatch};
+            if (!mbar_wait(&full_b[s], phase)) return;
             tc_fence_after();
             const uint32_t aaddr = smem_u32(stage_base + (size_t)s * G::kStageBytes);
 #pragma unroll
@@ -380,20 +370,18 @@ __device__ __forceinline__ ScanRing scan_mma_loop(int ntiles, int nstages, const
         }
         tc_commit(&tfull[a]);
     }
-    return ScanRing{s, phase, g0 + nbatch};
 }
 
 // Epilogue of one TMEM lane quarter (a whole warp): for every entry of every
 // tile it computes the score and calls consume(tile, entry_in_tile, key) with
 // all 32 lanes (kEpr calls per tile).
 template <int DI, typename Consume>
-__device__ __forceinline__ int scan_epilogue_loop(int ntiles, const float (&wv)[kScanN], int hi, uint64_t *tfull,
-                                                   uint64_t *tempty, uint32_t tmem, int quarter, Consume consume,
-                                                   int g0 = 0) {
+__device__ __forceinline__ void scan_epilogue_loop(int ntiles, const float (&wv)[kScanN], int hi, uint64_t *tfull,
+                                                   uint64_t *tempty, uint32_t tmem, int quarter, Consume consume) {
     using G = ScanGeom<DI>;
     const int lane = threadIdx.x & 31;
     const int nbatch = (ntiles + kScanBatch - 1) / kScanBatch;
-    for (int g = g0; g < g0 + nbatch; ++g) {
+    for (int g = 0; g < nbatch; ++g) {
         const int a = g & 1;
         const bool ok = mbar_wait(&tfull[a], (g >> 1) & 1);
         if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -423,37 +411,17 @@ __device__ __forceinline__ int scan_epilogue_loop(int ntiles, const float (&wv)[
         if (lane == 0) mbar_arrive(&tempty[a]);
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
-            const int i = (g - g0) * kScanBatch + j;
+            const int i = g * kScanBatch + j;
             if (i >= ntiles) break;
 #pragma unroll
             for (int u = 0; u < G::kEpr; ++u) consume(i, G::kEpr * (quarter * 32 + lane) + u, score_key(sc[j][u]));
         }
     }
-    return g0 + nbatch;
 }
 
-// Tiles of query qi in the scan (kTile entries each, the last one partial).
 template <int DI>
-__device__ __forceinline__ int64_t scan_tiles_of(const ScanParams &p, int32_t qi) {
-    return (query_limit(p.q_limit, p.kv, qi, p.q_per_seq) + ScanGeom<DI>::kTile - 1) / ScanGeom<DI>::kTile;
-}
-
-// Work of one CTA: segments (query qi, its tiles [t0, t1)), scanned in order
-// through one pipeline whose ring and TMEM buffers carry over from segment to
-// segment.
-//  - grid mode (p.persistent == 0): query blockIdx.y, tiles
-//    [blockIdx.x * chunk_tiles, +chunk_tiles); one segment.
-//  - persistent mode: the tiles of all queries, in query order, form one list
-//    that is split into gridDim.x equal ranges (one per resident CTA), so the
-//    SMs finish together whatever the queries' lengths; a range holds the end
-//    of one query, whole queries and the start of another.
-// Per segment the CTA writes the query's keys, adds its shared histogram into
-// the query's global one, and the last CTA to finish a part of the query
-// locates the digit-0 bin of each target rank.
-template <int DI>
-__global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
+__global__ void __launch_bounds__(kScanThreads) k_index_scan(const __grid_constant__ CUtensorMap tm, ScanParams p) {
     using Cfg = ScanCfg<DI>;
-    using G = ScanGeom<DI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
@@ -467,51 +435,20 @@ __global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_con
     int32_t *ptab = reinterpret_cast<int32_t *>(tmem_slot + 2);  // [kMaxScanPages]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int32_t qi = blockIdx.y;
+    const int32_t b = qi / p.q_per_seq;
     pdl_trigger();
     pdl_wait();
-
-    // this CTA's range [ra, rb) of tiles, counted from the first tile of query
-    // q, which is tile pq of the list
-    int64_t ra, rb, pq = 0, per = 0;
-    int32_t q;
-    if (p.persistent) {
-        // exclusive prefix sums of the queries' tile counts in hist[0..nq]
-        // (the host admits this mode only for nq < kHist0Bins - 8 and a total
-        // below 2^31 tiles)
-        const int cnt = (p.nq + kScanThreads - 1) / kScanThreads;
-        const int q0 = tid * cnt;
-        uint32_t loc = 0;
-        for (int j = 0; j < cnt; ++j)
-            if (q0 + j < p.nq) loc += (uint32_t)scan_tiles_of<DI>(p, q0 + j);
-        uint32_t total = 0;
-        uint32_t run = block_excl_scan<kScanThreads>(loc, hist + kHist0Bins - 8, &total);
-        for (int j = 0; j < cnt; ++j)
-            if (q0 + j < p.nq) {
-                hist[q0 + j] = run;
-                run += (uint32_t)scan_tiles_of<DI>(p, q0 + j);
-            }
-        __syncthreads();
-        per = ((int64_t)total + gridDim.x - 1) / gridDim.x;
-        ra = (int64_t)blockIdx.x * per;
-        rb = min(ra + per, (int64_t)total);
-        if (ra >= rb) return;
-        // the query holding tile ra: the last q with prefix[q] <= ra
-        int lo = 0, hi = p.nq - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if ((int64_t)hist[mid] <= ra) lo = mid; else hi = mid - 1;
-        }
-        q = lo;
-        pq = hist[lo];
-        __syncthreads();  // hist is the histogram from here on
-    } else {
-        q = blockIdx.y;
-        ra = (int64_t)blockIdx.x * p.chunk_tiles;
-        rb = min(ra + (int64_t)p.chunk_tiles, scan_tiles_of<DI>(p, q));
-        if (ra >= rb) return;
-    }
+    const int64_t limit = query_limit(p.q_limit, p.kv, qi, p.q_per_seq);
+    using G = ScanGeom<DI>;
+    const int64_t start = (int64_t)blockIdx.x * p.chunk_tiles * G::kTile;
+    if (start >= limit) return;
+    const int64_t rem = limit - start;
+    const int ntiles = (int)min((int64_t)p.chunk_tiles, (rem + G::kTile - 1) / G::kTile);
 
     for (int i = tid; i < kHist0Bins; i += kScanThreads) hist[i] = 0u;
+    build_q_tile<DI>(qt, p.qidx + (int64_t)qi * p.hi * DI, p.hi, kScanThreads);
+    stage_pages(p.kv, b, start, min(rem, (int64_t)ntiles * G::kTile), ptab, kScanThreads);
     if (tid == 0) {
         for (int s = 0; s < Cfg::kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -527,93 +464,54 @@ __global__ void __launch_bounds__(kScanThreads, 2) k_index_scan(const __grid_con
         tmem_alloc(tmem_slot, 2 * kScanBatch * G::kN);
         tmem_relinquish();
     }
-    ScanRing ring;  // this thread's position in the ring (its role's)
-    uint32_t tmem = 0;
-    bool first = true;
-    while (pq < rb) {
-        const int64_t limit = query_limit(p.q_limit, p.kv, q, p.q_per_seq);
-        const int64_t tq = (limit + G::kTile - 1) / G::kTile;
-        if (tq == 0) {  // a query without entries owns no tile
-            ++q;
-            continue;
-        }
-        const int64_t t0 = max(ra, pq) - pq, t1 = min(rb, pq + tq) - pq;
-        const int64_t start = t0 * G::kTile;
-        const int ntiles = (int)(t1 - t0);
-        // CTAs that scan a part of q
-        const uint32_t parts = p.persistent ? (uint32_t)((pq + tq - 1) / per - pq / per + 1)
-                                            : (uint32_t)((tq + p.chunk_tiles - 1) / p.chunk_tiles);
-        const int32_t b = q / p.q_per_seq;
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-        // the previous segment's products and reads are complete (its epilogue
-        // consumed every batch), so the q tile and the page table are free
-        build_q_tile<DI>(qt, p.qidx + (int64_t)q * p.hi * DI, p.hi, kScanThreads);
-        stage_pages(p.kv, b, start, min(limit - start, (int64_t)ntiles * G::kTile), ptab, kScanThreads);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (first) tmem = *tmem_slot;
-        first = false;
-
-        if (warp == 0) {
-            ring = scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, Cfg::kStages, p.box_rows, stages, &tm, full,
-                                     empty, 1, nullptr, ring);
-        } else if (warp == 1) {
-            if (lane == 0)
-                ring = scan_mma_loop<DI>(ntiles, Cfg::kStages, stages, smem_u32(qt), full, empty, tfull, tempty, tmem,
-                                         ring);
-        } else {
-            // epilogue: warps 2..5 cover TMEM lane quarters 2, 3, 0, 1
-            float wv[kScanN];
+    if (warp == 0) {
+        scan_tma_loop<DI>(p.kv, ptab, start, limit, ntiles, Cfg::kStages, p.box_rows, stages, &tm, full, empty);
+    } else if (warp == 1) {
+        if (lane == 0)
+            scan_mma_loop<DI>(ntiles, Cfg::kStages, stages, smem_u32(qt), full, empty, tfull, tempty, tmem);
+    } else {
+        // epilogue: warps 2..5 cover TMEM lane quarters 2, 3, 0, 1
+        float wv[kScanN];
 #pragma unroll
-            for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)q * p.hi + h] : 0.0f;
-            uint32_t *keys = p.keys + (int64_t)q * p.key_stride;
-            ring.g = scan_epilogue_loop<DI>(
-                ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3,
-                [&](int i, int e, uint32_t key) {
-                    const int64_t t = start + (int64_t)i * G::kTile + e;
-                    const bool valid = t < limit;
-                    if (valid) keys[t] = key;
-                    hist_add_warp(hist, valid ? (key >> 20) : 0xFFFFFFFFu);
-                },
-                ring.g);
-        }
-        tc_fence_before();
-        __syncthreads();
-        // the segment's histogram into the query's, leaving the shared one zero
-        for (int i = tid; i < kHist0Bins; i += kScanThreads) {
-            const uint32_t v = hist[i];
-            if (v) {
-                atomicAdd(&p.hist0[(int64_t)q * kHist0Bins + i], v);
-                hist[i] = 0u;
-            }
-        }
-        // the last CTA of this query locates the digit-0 bin of each target rank
-        uint32_t *scratch = hist;  // zero again below
-        if (last_block(&p.state[(int64_t)q * kStateWords + kCtrScan], parts, scratch + 64)) {
-            for (int tau = 0; tau < 2; ++tau) {
-                const int64_t r = p.rank[tau];
-                if (r <= 0 || r >= limit) continue;
-                uint32_t bin, rem;
-                find_rank_bin<kScanThreads, (kHist0Bins + kScanThreads - 1) / kScanThreads, true>(
-                    p.hist0 + (int64_t)q * kHist0Bins, kHist0Bins, (uint32_t)r, scratch, bin, rem);
-                if (tid == 0) {
-                    p.state[(int64_t)q * kStateWords + 8 * tau + 0] = bin;
-                    p.state[(int64_t)q * kStateWords + 8 * tau + 1] = rem;
-                }
-            }
-        }
-        __syncthreads();
-        if (tid <= 64) hist[tid] = 0u;  // the words last_block and find_rank_bin used
-        pq += tq;
-        ++q;
+        for (int h = 0; h < kScanN; ++h) wv[h] = h < p.hi ? p.w[(int64_t)qi * p.hi + h] : 0.0f;
+        uint32_t *keys = p.keys + (int64_t)qi * p.key_stride;
+        scan_epilogue_loop<DI>(ntiles, wv, p.hi, tfull, tempty, tmem, warp & 3, [&](int i, int e, uint32_t key) {
+            const int64_t t = start + (int64_t)i * G::kTile + e;
+            const bool valid = t < limit;
+            if (valid) keys[t] = key;
+            hist_add_warp(hist, valid ? (key >> 20) : 0xFFFFFFFFu);
+        });
     }
     tc_fence_before();
     __syncthreads();
+    for (int i = tid; i < kHist0Bins; i += kScanThreads)
+        if (hist[i]) atomicAdd(&p.hist0[(int64_t)qi * kHist0Bins + i], hist[i]);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 2 * kScanBatch * G::kN);
+    }
+    // the last CTA of this query locates the digit-0 bin of each target rank
+    const int64_t chunk = (int64_t)p.chunk_tiles * G::kTile;
+    uint32_t *scratch = hist;  // the shared histogram is no longer needed
+    if (last_block(&p.state[(int64_t)qi * kStateWords + kCtrScan], (uint32_t)((limit + chunk - 1) / chunk),
+                   scratch + 64)) {
+        for (int tau = 0; tau < 2; ++tau) {
+            const int64_t r = p.rank[tau];
+            if (r <= 0 || r >= limit) continue;
+            uint32_t bin, rem;
+            find_rank_bin<kScanThreads, (kHist0Bins + kScanThreads - 1) / kScanThreads, true>(p.hist0 + (int64_t)qi * kHist0Bins, kHist0Bins, (uint32_t)r, scratch, bin,
+                                        rem);
+            if (tid == 0) {
+                p.state[(int64_t)qi * kStateWords + 8 * tau + 0] = bin;
+                p.state[(int64_t)qi * kStateWords + 8 * tau + 1] = rem;
+            }
+        }
     }
 }
 

@@ -16,14 +16,8 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-@pytest.mark.parametrize("scan", ["persistent", "grid"])
-def test_full_indexer_multipass_path(cuda_device, scan):
-    """The scan in its default persistent form (equal shares of all queries'
-    tiles per resident CTA) and in grid form (CSA2_SCAN=grid: fixed chunks of
-    one query per CTA)."""
+def test_full_indexer_multipass_path(cuda_device):
     env = dict(os.environ, CSA2_FULL_PATH="multipass")
-    if scan == "grid":
-        env["CSA2_SCAN"] = "grid"
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
                         os.path.join(HERE, "test_indexer_gpu.py"), "-k", "full"],
                        env=env, cwd=os.path.dirname(HERE), capture_output=True, text=True, timeout=900)
