@@ -15,7 +15,8 @@ those of the largest single-GPU workload, paged64 (64 paged sequences of
 Metric: decode query-steps per second per layer = sequences * queries *
 layers / step time, with the achieved HBM bandwidth of the step's
 algorithmic bytes. Timing: each workload's step is captured once in a CUDA
-graph; each of the K timed steps is preceded by a 256 MiB L2 flush and
+graph; each of the K timed steps is preceded by an L2 flush (256 MiB written,
+then another 256 MiB read, so no dirty line is left to write back) and
 bracketed by CUDA events on the launching stream; a barrier and a device
 synchronize bracket each workload's timed loop; the reported time is the max
 over ranks. Multi-GPU runs give every rank its own independent sequences
@@ -119,7 +120,7 @@ def time_append_chunk512(B, dev, hbm_gbs, reps=20):
     x = r.latent_rows(0, r.prefill, r.prefill + n, dev).contiguous()
     seq = torch.zeros(n, dtype=torch.int32, device=dev)
     pos = torch.arange(r.prefill, r.prefill + n, dtype=torch.int64, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.Stream(dev)
     for _ in range(3):
         B.csa2_append_fp4(x, seq, pos, kv)
@@ -158,7 +159,7 @@ def time_append_e4m3(B, dev, hbm_gbs, reps=20):
     import torch
     from sparse_fp4_kv_b200 import synth
     n, ring, cap, di = 32768, 32768, 262144, 64
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     xw = synth.normal_bf16(11, 1, 0, n * 512).view(n, 512).to(dev)
     xk = synth.normal_bf16(11, 2, 0, n * di).view(n, di).to(dev)
     swa = torch.zeros((1, ring, 512), dtype=torch.uint8, device=dev)
@@ -200,7 +201,7 @@ def time_attn_variants(B, dec, reps=30):
     import torch
     r = dec.r
     dev = dec.device
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     topk = dec.topk_of(0)
     o = torch.empty_like(dec.o[0])
     lse = torch.empty_like(dec.lse[0])
@@ -254,7 +255,7 @@ def time_sharded_hier1m(dev, world=2, reps=5):
     r = RECIPES["hier1m"]
     shards = [EntryShard(r, off, n, dev) for off, n in shard_ranges(r.n, world)]
     dec = ShardedDecoder(r, shards, LocalGroup(world))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(2):
         dec.step()
     ts = []
@@ -274,6 +275,22 @@ def time_sharded_hier1m(dev, world=2, reps=5):
     return {"workload": "hier1m", "shards": world, "ms_per_step_all_shards_one_gpu": ms,
             "bytes_sent_per_rank_per_step": keys + parts,
             "note": f"shards run sequentially on one GPU; median of {reps} steps (no append in the step)"}
+
+
+class L2Flush:
+    """Clears the 126 MB L2 between timed iterations: fill_() writes a
+    256 MiB buffer, then reads a second 256 MiB buffer, so the timed kernels
+    find neither their inputs nor the flush's dirty lines in L2 (the write-back
+    of those would otherwise land inside the timed region)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
+
+    def fill_(self, v):
+        self.w.fill_(v)
+        self.r.sum()
 
 
 def peaks():
@@ -752,7 +769,7 @@ def bench_workload(name, args, world, rank, dev, stream, flush, clocks, pk):
                       "layers": recipe.layers, "modes": recipe.modes, "entries_max": int(dec.n_max),
                       "entries_total": int(dec.lens.sum()), "topk": recipe.k, "pool": recipe.p, "heads": recipe.h,
                       "window": recipe.w, "indexer": f"{recipe.hi}x{recipe.di}",
-                      "l2": "256 MiB flush before every timed step", "graph": "one CUDA graph per step"},
+                      "l2": "before every timed step 256 MiB written, then another 256 MiB read (inputs and dirty lines out of L2)", "graph": "one CUDA graph per step"},
            "hbm_tbs": by / (ms * 1e-3) / 1e12, "algorithmic_bytes_per_step": by, "algorithmic_flops_per_step": fl,
            "roofline": roofline, "step_roofline": step_rl,
            "breakdown_us_per_call": breakdown, "calls_per_step": calls_per_step,
@@ -792,7 +809,7 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     pk = peaks()
     probe = measure_tc_probe(dev)

@@ -82,6 +82,68 @@ __device__ __forceinline__ uint32_t quantize_block16(const float (&f)[16], uint3
     return s;
 }
 
+// Eight E2M1 codes from eight binary32 quotients: element i in nibble i.
+__device__ __forceinline__ uint32_t e2m1x8_of_f32(const float *q) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
+}
+// Per 16-bit half, the unsigned maximum.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// quantize_block16 on 16 bf16 values as they are loaded (w[i] holds values
+// 2i, 2i+1), with the same results in fewer instructions: the block maximum
+// is taken on the magnitudes' bit patterns two at a time (their integer order
+// is the values' order; 0x7F80 and above mean inf or NaN, which go to the
+// general routine), and the quotients of finite values, which can be neither
+// infinite nor NaN there, are formed two at a time with the same three
+// correctly rounded operations per value.
+__device__ __forceinline__ uint32_t quantize_block16_bf16(const uint32_t (&w)[8], uint32_t (&packed)[2]) {
+    uint32_t m = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 1; i < 8; ++i) m = max_u16x2(m, w[i] & 0x7FFF7FFFu);
+    const uint32_t mm = max(m & 0xFFFFu, m >> 16);
+    if (mm >= 0x7F80u) {
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+        return quantize_block16(f, packed);
+    }
+    const float amax = __uint_as_float(mm << 16);
+    const uint32_t s = f32_to_e4m3_satfinite(quotient_rn(amax, 6.0f, 1.0f / 6.0f));
+    const float sv = __half2float(__ushort_as_half((uint16_t)(e4m3x2_to_f16x2((uint16_t)s) & 0xFFFFu)));
+    packed[0] = packed[1] = 0u;
+    if (sv == 0.0f) return s;
+    const float r = rcp_approx(sv);
+    const float2 r2 = make_float2(r, r), nsv2 = make_float2(-sv, -sv);
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 x = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        const float2 q0 = __fmul2_rn(x, r2);
+        const float2 rem = __ffma2_rn(q0, nsv2, x);  // x - q0 * value(s), exactly as fma(-q0, sv, x)
+        const float2 qq = __ffma2_rn(rem, r2, q0);
+        q[2 * i] = qq.x;
+        q[2 * i + 1] = qq.y;
+    }
+    packed[0] = e2m1x8_of_f32(q);
+    packed[1] = e2m1x8_of_f32(q + 8);
+    return s;
+}
+
 // A warp walks rows r, r + W, r + 2W, ... (W = warps in the grid) in batches
 // of kAppendBatch rows: the input values and destination lookups of a whole
 // batch are issued before any of its rows is quantised and stored, so every
@@ -94,7 +156,7 @@ __device__ __forceinline__ int64_t append_dest(const csa2_kv_desc &kv, const int
     return (b >= 0 && b < kv.batch) ? physical_row(kv, b, pos[r]) : -1;
 }
 
-__global__ void __launch_bounds__(kAppendWarps * 32)
+__global__ void __launch_bounds__(kAppendWarps * 32, 3)
     k_append_fp4(const uint16_t *__restrict__ x, int32_t n, const int32_t *__restrict__ seq,
                  const int64_t *__restrict__ pos, csa2_kv_desc kv) {
     pdl_trigger();
@@ -123,14 +185,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
             }
             const uint32_t wds[8] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w,
                                      v[j][1].x, v[j][1].y, v[j][1].z, v[j][1].w};
-            float f[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                f[2 * i] = __uint_as_float(wds[i] << 16);
-                f[2 * i + 1] = __uint_as_float(wds[i] & 0xFFFF0000u);
-            }
             uint32_t packed[2];
-            const uint32_t s = quantize_block16(f, packed);
+            const uint32_t s = quantize_block16_bf16(wds, packed);
             // codes: 8 bytes per lane (256 contiguous bytes per warp); scales: one
             // byte per lane (the row's 32-byte sector in one warp store)
             *reinterpret_cast<uint2 *>(kv.codes + row[j] * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
