@@ -88,7 +88,7 @@ struct DecParams {
     int32_t inline_merge;
     uint32_t *qcount;  // [nq]: parts of u finished (zeroed before the launch)
 };
-constexpr int kInlineMergeParts = 4;
+constexpr int kInlineMergeParts = 2;
 
 // ---- the static work split (host and device) -------------------------------
 // CTA g takes tiles [g*per, min((g+1)*per, T)). Its segments are the runs of

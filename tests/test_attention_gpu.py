@@ -208,7 +208,7 @@ def test_query_outside_f16_range_is_reported(B, cuda_device):
 
 
 def test_merge_kernel_path(cuda_device):
-    """Queries split over at most four CTAs are merged inside the attention kernel
+    """Queries split over at most two CTAs are merged inside the attention kernel
     by the CTA that finishes their last part; wider splits by the merge
     kernel. This runs the attention tests again with the merge kernel for
     every split (CSA2_ATTN_MERGE=kernel, read per call; a separate process keeps
