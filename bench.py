@@ -864,19 +864,20 @@ def run_e2e(args, dec, stream, flush, world, dev):
     inputs (new latent rows, per-layer queries, indexer queries and weights)
     from pinned host memory to the device and reads every layer's output back.
     The step is one CUDA graph on three streams: the input copies run in layer
-    order on one copy stream, layer l waits only for its own inputs, and layer
-    l's output is copied back on a second copy stream as soon as the layer is
-    done, so the transfers overlap the compute of other layers."""
+    order on one copy stream (per layer the indexer inputs, then q), layer l's
+    indexer call waits only for its indexer inputs and its attention for q as
+    well, and layer l's output is copied back on a second copy stream as soon as
+    the layer is done, so the transfers overlap the compute of other layers."""
     import torch
     r = dec.r
     L = r.layers
-    # each layer's inputs (q, qidx, w) packed into one pinned host buffer and
-    # one device buffer (256-byte aligned parts; the decoder's tensors become
-    # views of it for the measurement), so a layer takes one copy
+    # each layer's indexer inputs (qidx, w) packed into one pinned host buffer
+    # and one device buffer (256-byte aligned parts; the decoder's tensors
+    # become views of it for the measurement), its q in another: the indexer
+    # call waits only for the small pack, the attention for q as well
     saved = (list(dec.q), list(dec.qidx), list(dec.w))
-    packs, hosts = [], []
-    for l in range(L):
-        parts = [dec.q[l], dec.qidx[l], dec.w[l]]
+
+    def pack(parts):
         offs, tot = [], 0
         for t in parts:
             offs.append(tot)
@@ -888,16 +889,22 @@ def run_e2e(args, dec, stream, flush, world, dev):
             nb = t.numel() * t.element_size()
             hbuf[o:o + nb].copy_(t.contiguous().view(-1).cpu().view(torch.uint8))
             views.append(dbuf[o:o + nb].view(t.dtype).view(t.shape))
-        dec.q[l], dec.qidx[l], dec.w[l] = views
-        packs.append(dbuf)
-        hosts.append(hbuf)
+        return dbuf, hbuf, views
+
+    packs, hosts = [], []  # per layer: [indexer pack, q pack]
+    for l in range(L):
+        di, hi, (dec.qidx[l], dec.w[l]) = pack([dec.qidx[l], dec.w[l]])
+        dq, hq, (dec.q[l],) = pack([dec.q[l]])
+        packs.append((di, dq))
+        hosts.append((hi, hq))
     host_x = dec.x_new.cpu().pin_memory()
     host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in dec.o]
-    h2d = host_x.numel() * host_x.element_size() + sum(h.numel() for h in hosts)
+    h2d = host_x.numel() * host_x.element_size() + sum(hi.numel() + hq.numel() for hi, hq in hosts)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev_x = torch.cuda.Event()
     ev_in = [torch.cuda.Event() for _ in range(L)]
+    ev_q = [torch.cuda.Event() for _ in range(L)]
     ev_done = [torch.cuda.Event() for _ in range(L)]
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -907,13 +914,15 @@ def run_e2e(args, dec, stream, flush, world, dev):
             dec.x_new.copy_(host_x, non_blocking=True)
             ev_x.record(s_in)
             for l in range(L):
-                packs[l].copy_(hosts[l], non_blocking=True)
+                packs[l][0].copy_(hosts[l][0], non_blocking=True)
                 ev_in[l].record(s_in)
+                packs[l][1].copy_(hosts[l][1], non_blocking=True)
+                ev_q[l].record(s_in)
         stream.wait_event(ev_x)
         dec.append(stream)
         for l in range(L):
             stream.wait_event(ev_in[l])
-            dec.layer(l, stream)
+            dec.layer(l, stream, before_attention=lambda l=l: stream.wait_event(ev_q[l]))
             ev_done[l].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[l])
@@ -948,9 +957,9 @@ def run_e2e(args, dec, stream, flush, world, dev):
     dec.q, dec.qidx, dec.w = saved
     return {"value": r.nq * r.layers * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "one CUDA graph per step: each layer's inputs (q, qidx, w packed, one copy) copied in layer "
-                    "order on a copy stream, each layer waits for its own inputs, each layer's output copied back "
-                    "as soon as it is done"}
+            "note": "one CUDA graph per step: each layer's inputs copied in layer order on a copy stream as two "
+                    "copies (qidx and w packed, then q), the layer's indexer call waits for the first, its "
+                    "attention for q as well, each layer's output copied back as soon as it is done"}
 
 
 def main():

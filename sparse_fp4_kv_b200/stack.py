@@ -124,7 +124,11 @@ class Csa2Decoder:
         for x, kv in zip(self.x_news, self.kvs):
             B.csa2_append_fp4(x, self.x_seq, self.x_pos, kv, stream)
 
-    def layer(self, l, stream=None):
+    def layer(self, l, stream=None, before_attention=None):
+        """Layer l on `stream`: its indexer call (Full or Reindex; none for
+        Reuse), then attention. before_attention, if given, is called between
+        the two (e.g. to make the stream wait for q alone, which only the
+        attention reads)."""
         r = self.r
         mode, src = self.schedule[l]
         kv = self.kvs[self.cache_of[l]]
@@ -135,6 +139,8 @@ class Csa2Decoder:
         elif mode == "reindex":
             B.csa2_index_reindex(self.qidx[l], self.w[l], r.q_per_seq, self.pool[src], kv, r.k, self.topk[l],
                                  self.ws_reindex, stream)
+        if before_attention is not None:
+            before_attention()
         B.csa2_sparse_attn_decode(self.q[l], r.q_per_seq, kv, self.topk_of(l), self.swa[l],
                                   self.swa[l].shape[1], self.swa_begin, self.swa_end, r.w, self.scale, self.o[l],
                                   self.lse[l], self.ws_attn, stream)
