@@ -103,8 +103,8 @@ def test_full_causal_queries(B, cuda_device):
 
 def test_full_empty_sequences_and_many_queries(B, cuda_device):
     # sequences without entries between others (a query that owns no tile),
-    # and 400 causal queries of one sequence: on the multi-launch path every
-    # CTA then scans the end of one query and the start of the next
+    # and 400 causal queries of one sequence (the batched path by default, the
+    # multi-launch path when it is forced)
     _run_full(B, cuda_device, [700, 0, 3000, 129, 0, 5000], 64, 64, 4, 100, 300, seed=16)
     total = 3000
     _run_full(B, cuda_device, [total], 3072, 64, 4, 150, 0, q_per_seq=400, q_limit=_causal(total, 400), seed=17,
