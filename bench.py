@@ -170,25 +170,36 @@ def time_append_e4m3(B, dev, hbm_gbs, reps=20):
                    torch.full((1,), cap, dtype=torch.int32, device=dev), cap)
     seq = torch.zeros(n, dtype=torch.int32, device=dev)
     pos = torch.arange(cap - n, cap, dtype=torch.int64, device=dev)
+    stream = torch.cuda.Stream(dev)
     out = {}
-    for name, call, by in (("window", lambda: B.csa2_append_swa_e4m3(xw, seq, pos, swa), n * 512 * 3),
-                           ("keys", lambda: B.csa2_append_kidx_e4m3(xk, seq, pos, kv), n * di * 3)):
+    for name, call, by in (("window", lambda s: B.csa2_append_swa_e4m3(xw, seq, pos, swa, s), n * 512 * 3),
+                           ("keys", lambda s: B.csa2_append_kidx_e4m3(xk, seq, pos, kv, s), n * di * 3)):
         for _ in range(3):
-            call()
-        ts = []
-        for i in range(reps):
-            flush.fill_(i & 0xFF)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            call()
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        ts.sort()
-        us = ts[len(ts) // 2]
-        out[name] = {"rows": n, "us_median": us, "algorithmic_bytes": by,
+            call(stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call(stream)
+        res = {}
+        for mode, run in (("eager", lambda: call(stream)), ("graph", g.replay)):
+            ts = []
+            for i in range(reps):
+                with torch.cuda.stream(stream):
+                    flush.fill_(i & 0xFF)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    run()
+                    e1.record(stream)
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            ts.sort()
+            res[mode] = ts[len(ts) // 2]
+        del g
+        us = res["graph"]
+        out[name] = {"rows": n, "us_median_graph": us, "us_median_eager": res["eager"], "algorithmic_bytes": by,
                      "achieved_gbs": by / (us * 1e-6) / 1e9, "frac": by / (us * 1e-6) / 1e9 / hbm_gbs}
-    out["note"] = "bf16 in, E4M3 out; events around the call (launch included), median of %d after an L2 flush" % reps
+    out["note"] = ("bf16 in, E4M3 out; CUDA events around the call, replayed from a CUDA graph (frac) and eager "
+                   "(launch included), median of %d, L2 flushed before each" % reps)
     return out
 
 

@@ -9,7 +9,7 @@
 // x / value(s), ties to the even mantissa, and all-zero codes when value(s)
 // is 0.
 //
-// Layout: one warp per 512-value row. Lane l owns block l (values 16l ..
+// Layout: a warp per 512-value row at a time. Lane l owns block l (values 16l ..
 // 16l+15): it reads 32 contiguous bytes of bf16 input, writes 8 bytes of
 // codes and 1 scale byte, so a warp moves 1 KiB in and 288 B out with fully
 // coalesced 16-byte loads. HBM-bound: 1312 algorithmic bytes per row.
@@ -144,16 +144,47 @@ __device__ __forceinline__ uint32_t quantize_block16_bf16(const uint32_t (&w)[8]
     return s;
 }
 
-// A warp walks rows r, r + W, r + 2W, ... (W = warps in the grid) in batches
-// of kAppendBatch rows: the input values and destination lookups of a whole
-// batch are issued before any of its rows is quantised and stored, so every
-// warp has kAppendBatch rows in flight; the grid is one wave of resident CTAs.
-constexpr int kAppendBatch = 4;
+// One wave of resident CTAs; warp w of the W warps in the grid takes rows
+// w, w + W, w + 2W, ... Two things keep its memory traffic and its
+// arithmetic overlapped:
+//   * destinations are resolved 32 rows at a time, lane j looking up the
+//     physical row of the warp's j-th row of the group (sequence, position,
+//     page table: every lane's chain in flight at once), and handed to the
+//     quantising lanes by a shuffle, so no row waits for its own lookup;
+//   * the bf16 input of kAppendRing - 1 rows is in flight while a row is
+//     quantised: a ring of kAppendRing rows in registers, the slot of the row
+//     just stored refilled with the row kAppendRing - 1 further on.
+// (A grid that loaded a batch of rows, then quantised it, then loaded the
+// next spent its time alternately waiting on memory and on instruction
+// issue.)
+constexpr int kAppendRing = 4;
 
 __device__ __forceinline__ int64_t append_dest(const csa2_kv_desc &kv, const int32_t *__restrict__ seq,
                                                const int64_t *__restrict__ pos, int64_t r) {
     const int32_t b = seq[r];
     return (b >= 0 && b < kv.batch) ? physical_row(kv, b, pos[r]) : -1;
+}
+
+__device__ __forceinline__ void append_load_row(const uint16_t *__restrict__ x, int64_t r, int lane, uint4 (&v)[2]) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16);
+    v[0] = __ldg(src);
+    v[1] = __ldg(src + 1);
+}
+
+// Quantise one row held as lane l's 16 values (block l) and store it at
+// physical row `dest` (< 0: a bad destination, reported and skipped).
+__device__ __forceinline__ void append_store_row(const csa2_kv_desc &kv, int64_t dest, int lane, const uint4 (&v)[2]) {
+    if (dest < 0) {
+        if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
+        return;
+    }
+    const uint32_t wds[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
+    uint32_t packed[2];
+    const uint32_t s = quantize_block16_bf16(wds, packed);
+    // codes: 8 bytes per lane (256 contiguous bytes per warp); scales: one
+    // byte per lane (the row's 32-byte sector in one warp store)
+    *reinterpret_cast<uint2 *>(kv.codes + dest * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
+    kv.scales[dest * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
 }
 
 __global__ void __launch_bounds__(kAppendWarps * 32, 3)
@@ -162,35 +193,30 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3)
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t stride = (int64_t)gridDim.x * kAppendWarps;
-    for (int64_t r0 = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5); r0 < n; r0 += kAppendBatch * stride) {
-        uint4 v[kAppendBatch][2];
-        int64_t row[kAppendBatch];
+    const int64_t W = (int64_t)gridDim.x * kAppendWarps;
+    const int64_t w = (int64_t)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
+    if (w >= n) return;
+    const int64_t rows = (n - w + W - 1) / W;  // rows of this warp: w + k * W, k < rows
+    for (int64_t g0 = 0; g0 < rows; g0 += 32) {
+        const int m = (int)min((int64_t)32, rows - g0);  // rows of this group (warp-uniform)
+        const int64_t first = w + g0 * W;                 // row of group index 0
+        uint4 v[kAppendRing][2];
 #pragma unroll
-        for (int j = 0; j < kAppendBatch; ++j) {
-            const int64_t r = r0 + j * stride;
-            row[j] = -2;  // no row
-            if (r < n) {
-                v[j][0] = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16));
-                v[j][1] = __ldg(reinterpret_cast<const uint4 *>(x + r * CSA2_D + lane * 16) + 1);
-                row[j] = append_dest(kv, seq, pos, r);
-            }
-        }
+        for (int s = 0; s < kAppendRing - 1; ++s)
+            if (s < m) append_load_row(x, first + s * W, lane, v[s]);
+        // lane j: destination of group row j (its lookups overlap the loads above)
+        const int64_t dest_j = lane < m ? append_dest(kv, seq, pos, first + lane * W) : -1;
+        for (int k0 = 0; k0 < m; k0 += kAppendRing) {
 #pragma unroll
-        for (int j = 0; j < kAppendBatch; ++j) {
-            if (row[j] == -2) continue;
-            if (row[j] < 0) {
-                if (lane == 0) set_error(CSA2_DEVERR_BAD_ROW);
-                continue;
+            for (int s = 0; s < kAppendRing; ++s) {
+                const int k = k0 + s;
+                // refill the slot of row k - 1 (stored in the previous step)
+                if (k + kAppendRing - 1 < m)
+                    append_load_row(x, first + (int64_t)(k + kAppendRing - 1) * W, lane,
+                                    v[(s + kAppendRing - 1) % kAppendRing]);
+                const int64_t dest = __shfl_sync(0xFFFFFFFFu, dest_j, k & 31);
+                if (k < m) append_store_row(kv, dest, lane, v[s]);
             }
-            const uint32_t wds[8] = {v[j][0].x, v[j][0].y, v[j][0].z, v[j][0].w,
-                                     v[j][1].x, v[j][1].y, v[j][1].z, v[j][1].w};
-            uint32_t packed[2];
-            const uint32_t s = quantize_block16_bf16(wds, packed);
-            // codes: 8 bytes per lane (256 contiguous bytes per warp); scales: one
-            // byte per lane (the row's 32-byte sector in one warp store)
-            *reinterpret_cast<uint2 *>(kv.codes + row[j] * (CSA2_D / 2) + lane * 8) = make_uint2(packed[0], packed[1]);
-            kv.scales[row[j] * (CSA2_D / CSA2_BLOCK) + lane] = (uint8_t)s;
         }
     }
 }
@@ -204,11 +230,16 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3)
 // nearest even, saturating to +-448, no scale; NaN keeps its sign and becomes
 // the E4M3 NaN code 0x7F.
 //
-// A thread converts 8 consecutive values of a row: one 16-byte load, one
-// 8-byte store. Window rows go to ring slot pos % ring_rows of their
-// sequence; indexer keys go to the physical row of (seq, pos).
+// A thread converts P x 8 consecutive values of one row: P 16-byte loads in
+// flight, one destination lookup, P 8-byte stores. Window rows go to ring
+// slot pos % ring_rows of their sequence (P = kE4m3WindowPieces, so a thread
+// moves 64 bytes in); indexer keys go to the physical row of (seq, pos)
+// (P = 1: keys are short, and more threads keep more of their dependent
+// lookups in flight). P divides the pieces of a row (64 for window rows),
+// so a thread never spans two rows.
 // ---------------------------------------------------------------------------
 constexpr int kE4m3Threads = 256;
+constexpr int kE4m3WindowPieces = 4;
 
 // Two bf16 values (low half first) -> two E4M3 bytes (low byte first).
 __device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w) {
@@ -223,18 +254,21 @@ __device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w) {
 
 // mode 0: window rows (width 512) into swa [batch][ring_rows][512];
 // mode 1: indexer keys (width kv.di) into kv.kidx at the physical row.
+template <int P>
 __global__ void __launch_bounds__(kE4m3Threads)
     k_append_e4m3(const uint16_t *__restrict__ x, int32_t n, int32_t width, const int32_t *__restrict__ seq,
                   const int64_t *__restrict__ pos, int32_t mode, uint8_t *__restrict__ swa, int32_t batch,
                   int64_t ring_rows, csa2_kv_desc kv) {
     pdl_trigger();
     pdl_wait();
-    const int per_row = width / 8;
+    const int groups = width / (8 * P);  // threads per row
     const int64_t t = (int64_t)blockIdx.x * kE4m3Threads + threadIdx.x;
-    if (t >= (int64_t)n * per_row) return;
-    const int64_t r = t / per_row;
-    const int c = (int)(t - r * per_row);
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * width) + c);
+    if (t >= (int64_t)n * groups) return;
+    const int64_t r = t / groups;
+    const int c = (int)(t - r * groups) * P;  // first 8-value piece
+    uint4 v[P];
+#pragma unroll
+    for (int j = 0; j < P; ++j) v[j] = __ldg(reinterpret_cast<const uint4 *>(x + r * width) + c + j);
     const int32_t b = seq[r];
     const int64_t ps = pos[r];
     uint8_t *row = nullptr;
@@ -248,9 +282,12 @@ __global__ void __launch_bounds__(kE4m3Threads)
         if (c == 0) set_error(CSA2_DEVERR_BAD_ROW);
         return;
     }
-    const uint32_t lo = e4m3x2_of_bf16x2(v.x) | (e4m3x2_of_bf16x2(v.y) << 16);
-    const uint32_t hi = e4m3x2_of_bf16x2(v.z) | (e4m3x2_of_bf16x2(v.w) << 16);
-    *reinterpret_cast<uint2 *>(row + c * 8) = make_uint2(lo, hi);
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+        const uint32_t lo = e4m3x2_of_bf16x2(v[j].x) | (e4m3x2_of_bf16x2(v[j].y) << 16);
+        const uint32_t hi = e4m3x2_of_bf16x2(v[j].z) | (e4m3x2_of_bf16x2(v[j].w) << 16);
+        *reinterpret_cast<uint2 *>(row + (c + j) * 8) = make_uint2(lo, hi);
+    }
 }
 
 }  // namespace csa2

@@ -547,7 +547,7 @@ bool prefer_shared(K kernel) {
 bool init_small_kernels() {
     static const char key = 0;
     return once_per_device(&key, [] {
-        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3) && prefer_shared(k_sel_collect) && prefer_shared(k_pad_heads) && prefer_shared(k_unpad_heads) && prefer_shared(k_batch_sthresh) && prefer_shared(k_batch_thresh) &&
+        return prefer_shared(k_append_fp4) && prefer_shared(k_append_e4m3<kE4m3WindowPieces>) && prefer_shared(k_append_e4m3<1>) && prefer_shared(k_sel_collect) && prefer_shared(k_pad_heads) && prefer_shared(k_unpad_heads) && prefer_shared(k_batch_sthresh) && prefer_shared(k_batch_thresh) &&
                prefer_shared(k_reindex_score<64>) && prefer_shared(k_reindex_score<128>) &&
                prefer_shared(k_attn_combine<16, false>) && prefer_shared(k_attn_combine<32, false>) &&
                prefer_shared(k_attn_combine<64, false>) && prefer_shared(k_attn_combine<16, true>) &&
@@ -602,8 +602,8 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
     if (!x_bf16 || !seq || !pos || !aligned(x_bf16, 16) || !aligned(seq, 4) || !aligned(pos, 8))
         return CSA2_ERR_INVALID_ARG;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
-    // one wave of resident CTAs (each warp walks rows with a stride, a batch
-    // of rows in flight at a time), fewer when there are not enough rows
+    // one wave of resident CTAs (each warp walks rows with a stride), fewer
+    // when there are not enough rows for one per warp
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_append_fp4, kAppendWarps * 32, 0) != cudaSuccess ||
         per_sm < 1) {
@@ -611,8 +611,8 @@ csa2_status csa2_append_fp4(const void *x_bf16, int32_t n, const int32_t *seq, c
         per_sm = 1;
     }
     const int64_t want = (int64_t)num_sms() * per_sm;
-    const int64_t rows_per_cta = (int64_t)kAppendWarps * kAppendBatch;
-    const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, ((int64_t)n + rows_per_cta - 1) / rows_per_cta));
+    const unsigned grid =
+        (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, ((int64_t)n + kAppendWarps - 1) / kAppendWarps));
     launch(k_append_fp4, dim3(grid), dim3(kAppendWarps * 32), 0, stream, static_cast<const uint16_t *>(x_bf16), n, seq, pos, *kv);
     return check_launch();
 }
@@ -625,9 +625,9 @@ csa2_status csa2_append_swa_e4m3(const void *x_bf16, int32_t n, const int32_t *s
         !aligned(swa, 8))
         return CSA2_ERR_INVALID_ARG;
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
-    const int64_t threads = (int64_t)n * (CSA2_D / 8);
+    const int64_t threads = (int64_t)n * (CSA2_D / (8 * kE4m3WindowPieces));
     const unsigned grid = (unsigned)((threads + kE4m3Threads - 1) / kE4m3Threads);
-    launch(k_append_e4m3, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
+    launch(k_append_e4m3<kE4m3WindowPieces>, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
            (int32_t)CSA2_D, seq, pos, (int32_t)0, swa, batch, ring_rows, csa2_kv_desc{});
     return check_launch();
 }
@@ -643,7 +643,7 @@ csa2_status csa2_append_kidx_e4m3(const void *x_bf16, int32_t n, const int32_t *
     if (!init_small_kernels()) return CSA2_ERR_CUDA;
     const int64_t threads = (int64_t)n * (kv->di / 8);
     const unsigned grid = (unsigned)((threads + kE4m3Threads - 1) / kE4m3Threads);
-    launch(k_append_e4m3, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
+    launch(k_append_e4m3<1>, dim3(grid), dim3(kE4m3Threads), 0, stream, static_cast<const uint16_t *>(x_bf16), n,
            kv->di, seq, pos, (int32_t)1, static_cast<uint8_t *>(nullptr), (int32_t)0, (int64_t)1, *kv);
     return check_launch();
 }

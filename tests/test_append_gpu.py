@@ -100,6 +100,17 @@ def test_normal_rows_with_outliers_paged(B, cuda_device):
     _check_rows(B, x, cuda_device, ps=64)
 
 
+@pytest.mark.parametrize("n", [1, 17, 4097, 131073])
+def test_ragged_row_counts(B, cuda_device, n):
+    # row counts that leave warps of the grid without rows or with one row
+    # fewer than others; 131073 rows give every warp of a full one-wave grid
+    # (148 SMs x 3 CTAs x 8 warps) more than one group of 32 rows. Rows nobody
+    # writes must stay zero
+    from sparse_fp4_kv_b200 import synth
+    x = synth.normal_bf16(12, 3, 0, n * 512, outlier_p=0.01, outlier_mul=20.0, outlier_stream=6).view(n, 512)
+    _check_rows(B, x, cuda_device, ps=64)
+
+
 def test_scattered_positions_and_bad_rows(B, cuda_device):
     rng = np.random.default_rng(3)
     ps = 32
